@@ -1,0 +1,186 @@
+"""ctypes binding of libkda (``include/kda.h``) for torch tensors.
+
+Argument marshalling only: every step of the computation runs in the CUDA
+kernels of ``libkda.so``. There is no CPU or PyTorch fallback -- if the library
+is missing, or the tensors are not on a CUDA device, the calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libkda.so")
+
+KDA_BF16, KDA_F32 = 0, 1
+ENGINES = {"auto": 0, "generic": 1, "tc": 2}
+_DTYPES = {torch.bfloat16: KDA_BF16, torch.float32: KDA_F32}
+
+_lib = None
+
+
+class KdaError(RuntimeError):
+    def __init__(self, code: int, name: str, detail: str):
+        super().__init__(f"{name} ({code}): {detail}")
+        self.code = code
+        self.name = name
+        self.detail = detail
+
+
+def load():
+    """Load libkda.so (once). Raises if it has not been built."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"libkda.so is not built ({LIB_PATH}); run "
+                           "`python -m gated_delta_rule_116_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    p, i, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+    lib.kda_workspace_bytes.argtypes = [i, i, i, i, i, i, i]
+    lib.kda_workspace_bytes.restype = sz
+    chunk_args = [p, p, p, p, p, p, p, p, i, i, i, i, i, i, i, p, sz, p]
+    lib.kda_chunk_fwd.argtypes = chunk_args
+    lib.kda_chunk_fwd.restype = i
+    lib.kda_chunk_fwd_engine.argtypes = [i] + chunk_args
+    lib.kda_chunk_fwd_engine.restype = i
+    lib.kda_engine_supported.argtypes = [i, i, i, i, i]
+    lib.kda_engine_supported.restype = i
+    lib.kda_recurrent_step.argtypes = [p, p, p, p, p, p, p, p, i, i, i, i, i, p]
+    lib.kda_recurrent_step.restype = i
+    lib.kda_strerror.argtypes = [i]
+    lib.kda_strerror.restype = ctypes.c_char_p
+    lib.kda_last_error_detail.argtypes = []
+    lib.kda_last_error_detail.restype = ctypes.c_char_p
+    lib.kda_device_status.argtypes = [p]
+    lib.kda_device_status.restype = i
+    lib.kda_version.restype = i
+    _lib = lib
+    return lib
+
+
+def _check(rc: int):
+    if rc != 0:
+        lib = load()
+        raise KdaError(rc, lib.kda_strerror(rc).decode(), lib.kda_last_error_detail().decode())
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(device, stream):
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _require(t, name, device, dtype=None, shape=None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.device.type != "cuda":
+        raise ValueError(f"{name} must be on a CUDA device (got {t.device})")
+    if t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype} (got {t.dtype})")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)} (got {tuple(t.shape)})")
+
+
+def engine_supported(engine: str, dk: int, dv: int, chunk: int, dtype=torch.bfloat16) -> bool:
+    return bool(load().kda_engine_supported(ENGINES[engine], dk, dv, chunk, _DTYPES[dtype]))
+
+
+def workspace_bytes(B, T, H, dk, dv, chunk=64, dtype=torch.bfloat16) -> int:
+    return int(load().kda_workspace_bytes(B, T, H, dk, dv, chunk, _DTYPES[dtype]))
+
+
+def chunk_fwd(q, k, v, log_alpha, beta, S0=None, chunk: int = 64, *, out=None, S_T=None,
+              output_final_state: bool = True, engine: str = "auto", workspace=None, stream=None):
+    """Chunked KDA prefill (``kda_chunk_fwd``).
+
+    q, k ``[B,T,H,dk]``, v ``[B,T,H,dv]`` (bf16 or fp32, same dtype);
+    log_alpha ``[B,T,H,dk]`` and beta ``[B,T,H]`` fp32; S0 ``[B,H,dk,dv]`` fp32 or
+    None. Returns ``(out, S_T)``; ``S_T`` is None when ``output_final_state`` is
+    False and no ``S_T`` buffer is given. ``S_T`` may be ``S0`` (in place).
+    """
+    lib = load()
+    device = q.device
+    _require(q, "q", device)
+    if q.dtype not in _DTYPES:
+        raise TypeError(f"q must be bf16 or fp32 (got {q.dtype})")
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    _require(k, "k", device, q.dtype, (B, T, H, dk))
+    _require(v, "v", device, q.dtype, (B, T, H, dv))
+    _require(log_alpha, "log_alpha", device, torch.float32, (B, T, H, dk))
+    _require(beta, "beta", device, torch.float32, (B, T, H))
+    if S0 is not None:
+        _require(S0, "S0", device, torch.float32, (B, H, dk, dv))
+    if out is None:
+        out = torch.empty(B, T, H, dv, device=device, dtype=q.dtype)
+    _require(out, "out", device, q.dtype, (B, T, H, dv))
+    if S_T is None and output_final_state:
+        S_T = torch.empty(B, H, dk, dv, device=device, dtype=torch.float32)
+    if S_T is not None:
+        _require(S_T, "S_T", device, torch.float32, (B, H, dk, dv))
+    need = int(lib.kda_workspace_bytes(B, T, H, dk, dv, chunk, _DTYPES[q.dtype]))
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, device=device, dtype=torch.uint8)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    if engine not in ENGINES:
+        raise ValueError(f"engine must be one of {sorted(ENGINES)}")
+    with torch.cuda.device(device):
+        rc = lib.kda_chunk_fwd_engine(
+            ENGINES[engine], _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(S0),
+            _ptr(out), _ptr(S_T), B, T, H, dk, dv, chunk, _DTYPES[q.dtype], _ptr(workspace),
+            ws_bytes, _stream(device, stream))
+    _check(rc)
+    return out, S_T
+
+
+def recurrent_step(q, k, v, log_alpha, beta, state, slot=None, *, out=None, stream=None):
+    """One decode step (``kda_recurrent_step``); updates ``state`` in place.
+
+    q, k ``[N,H,dk]``, v ``[N,H,dv]`` (bf16 or fp32), log_alpha ``[N,H,dk]`` and
+    beta ``[N,H]`` fp32, state ``[slots,H,dk,dv]`` fp32, slot ``[N]`` int32 or
+    None. Returns ``out [N,H,dv]``.
+    """
+    lib = load()
+    device = q.device
+    _require(q, "q", device)
+    if q.dtype not in _DTYPES:
+        raise TypeError(f"q must be bf16 or fp32 (got {q.dtype})")
+    N, H, dk = q.shape
+    dv = v.shape[-1]
+    _require(k, "k", device, q.dtype, (N, H, dk))
+    _require(v, "v", device, q.dtype, (N, H, dv))
+    _require(log_alpha, "log_alpha", device, torch.float32, (N, H, dk))
+    _require(beta, "beta", device, torch.float32, (N, H))
+    _require(state, "state", device, torch.float32)
+    if state.dim() != 4 or tuple(state.shape[1:]) != (H, dk, dv):
+        raise ValueError(f"state must be [slots,{H},{dk},{dv}] (got {tuple(state.shape)})")
+    if slot is not None:
+        _require(slot, "slot", device, torch.int32, (N,))
+    elif state.shape[0] < N:
+        raise ValueError("state has fewer slots than sequences and no slot map was given")
+    if out is None:
+        out = torch.empty(N, H, dv, device=device, dtype=q.dtype)
+    _require(out, "out", device, q.dtype, (N, H, dv))
+    with torch.cuda.device(device):
+        rc = lib.kda_recurrent_step(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta),
+                                    _ptr(state), _ptr(slot), _ptr(out), N, H, dk, dv,
+                                    _DTYPES[q.dtype], _stream(device, stream))
+    _check(rc)
+    return out
+
+
+def device_status(stream=None, device=None):
+    """Synchronise and raise KdaError if a bounded device wait gave up."""
+    lib = load()
+    device = torch.device("cuda", torch.cuda.current_device()) if device is None else device
+    _check(lib.kda_device_status(_stream(device, stream)))

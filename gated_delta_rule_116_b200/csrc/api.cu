@@ -1,0 +1,202 @@
+// api.cu -- the C ABI of libkda: argument validation, engine choice, launches.
+#include <stdarg.h>
+#include <stdio.h>
+
+#include "kda_internal.cuh"
+
+namespace {
+
+thread_local char g_detail[256] = "";
+
+// Device word a kernel sets when one of its bounded waits gives up.
+__device__ int g_device_error = 0;
+
+int fail(int code, const char *fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_detail, sizeof g_detail, fmt, ap);
+    va_end(ap);
+    return code;
+}
+
+int cuda_fail(cudaError_t e, const char *what) {
+    return fail(KDA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int *device_error_ptr() {
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) return nullptr;
+    return static_cast<int *>(p);
+}
+
+struct Ptr {
+    const void *p;
+    const char *name;
+    bool required;
+};
+
+int check_pointers(const Ptr *ps, int n) {
+    for (int i = 0; i < n; ++i) {
+        if (!ps[i].p) {
+            if (ps[i].required) return fail(KDA_ERR_INVALID_ARG, "%s is NULL", ps[i].name);
+            continue;
+        }
+        if (!aligned16(ps[i].p))
+            return fail(KDA_ERR_ALIGNMENT, "%s is not 16-byte aligned", ps[i].name);
+    }
+    return KDA_OK;
+}
+
+int check_common(int dk, int dv, int dtype) {
+    if (dtype != KDA_BF16 && dtype != KDA_F32)
+        return fail(KDA_ERR_INVALID_ARG, "dtype %d is neither KDA_BF16 nor KDA_F32", dtype);
+    if (dk < 1 || dv < 1) return fail(KDA_ERR_INVALID_ARG, "dk=%d dv=%d must be >= 1", dk, dv);
+    if (dk > 128 || dv > 128)
+        return fail(KDA_ERR_UNSUPPORTED, "dk=%d dv=%d: head dimensions above 128", dk, dv);
+    if (dv % 4 != 0) return fail(KDA_ERR_UNSUPPORTED, "dv=%d is not a multiple of 4", dv);
+    return KDA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int kda_version(void) { return 10000; }
+
+const char *kda_strerror(int code) {
+    switch (code) {
+        case KDA_OK: return "KDA_OK";
+        case KDA_ERR_INVALID_ARG: return "KDA_ERR_INVALID_ARG";
+        case KDA_ERR_UNSUPPORTED: return "KDA_ERR_UNSUPPORTED";
+        case KDA_ERR_ALIGNMENT: return "KDA_ERR_ALIGNMENT";
+        case KDA_ERR_WORKSPACE: return "KDA_ERR_WORKSPACE";
+        case KDA_ERR_CUDA: return "KDA_ERR_CUDA";
+        case KDA_ERR_DEVICE_TIMEOUT: return "KDA_ERR_DEVICE_TIMEOUT";
+        default: return "KDA_ERR_UNKNOWN";
+    }
+}
+
+const char *kda_last_error_detail(void) { return g_detail; }
+
+int kda_engine_supported(int engine, int dk, int dv, int chunk, int dtype) {
+    const bool generic = (dtype == KDA_BF16 || dtype == KDA_F32) && dk >= 1 && dv >= 1 &&
+                         dk <= 128 && dv <= 128 && dv % 4 == 0 &&
+                         (chunk == 16 || chunk == 32 || chunk == 64);
+    switch (engine) {
+        case KDA_ENGINE_AUTO:
+        case KDA_ENGINE_GENERIC: return generic ? 1 : 0;
+        case KDA_ENGINE_TC: return generic && kda::chunk_tc_supported(dk, dv, chunk, dtype) ? 1 : 0;
+        default: return 0;
+    }
+}
+
+size_t kda_workspace_bytes(int B, int T, int H, int dk, int dv, int chunk, int dtype) {
+    if (B <= 0 || T <= 0 || H <= 0) return 0;
+    if (kda::chunk_tc_supported(dk, dv, chunk, dtype)) return kda::chunk_tc_workspace_bytes(B, T, H);
+    return 0;
+}
+
+int kda_chunk_fwd_engine(int engine, const void *q, const void *k, const void *v,
+                         const float *log_alpha, const float *beta, const float *S0, void *out,
+                         float *S_T, int B, int T, int H, int dk, int dv, int chunk, int dtype,
+                         void *workspace, size_t workspace_bytes, void *stream) {
+    g_detail[0] = '\0';
+    if (engine < KDA_ENGINE_AUTO || engine > KDA_ENGINE_TC)
+        return fail(KDA_ERR_INVALID_ARG, "engine %d is not a kda_engine", engine);
+    if (B < 0 || T < 0 || H < 0)
+        return fail(KDA_ERR_INVALID_ARG, "B=%d T=%d H=%d must be >= 0", B, T, H);
+    int rc = check_common(dk, dv, dtype);
+    if (rc != KDA_OK) return rc;
+    if (chunk != 16 && chunk != 32 && chunk != 64)
+        return fail(KDA_ERR_UNSUPPORTED, "chunk=%d is not 16, 32 or 64", chunk);
+    if (B == 0 || H == 0) return KDA_OK;
+    const bool tokens = T > 0;
+    const Ptr ps[] = {{q, "q", tokens},           {k, "k", tokens},       {v, "v", tokens},
+                      {log_alpha, "log_alpha", tokens}, {beta, "beta", tokens}, {out, "out", tokens},
+                      {S0, "S0", false},          {S_T, "S_T", false},    {workspace, "workspace", false}};
+    rc = check_pointers(ps, sizeof ps / sizeof ps[0]);
+    if (rc != KDA_OK) return rc;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+    if (!tokens) {  // S_T = S0 (or zeros)
+        if (!S_T) return KDA_OK;
+        const size_t bytes = static_cast<size_t>(B) * H * dk * dv * sizeof(float);
+        cudaError_t e = S0 ? (S0 == S_T ? cudaSuccess
+                                        : cudaMemcpyAsync(S_T, S0, bytes, cudaMemcpyDeviceToDevice, s))
+                           : cudaMemsetAsync(S_T, 0, bytes, s);
+        return e == cudaSuccess ? KDA_OK : cuda_fail(e, "copying S0 to S_T");
+    }
+
+    const bool tc_ok = kda::chunk_tc_supported(dk, dv, chunk, dtype);
+    bool use_tc = false;
+    if (engine == KDA_ENGINE_TC) {
+        if (!tc_ok)
+            return fail(KDA_ERR_UNSUPPORTED,
+                        "tensor-core engine needs bf16, dk = dv = 128, chunk = 64 (got dtype %d, "
+                        "dk %d, dv %d, chunk %d)", dtype, dk, dv, chunk);
+        use_tc = true;
+    } else if (engine == KDA_ENGINE_AUTO) {
+        use_tc = tc_ok;
+    }
+
+    kda::ChunkArgs a{q, k, v, log_alpha, beta, S0, out, S_T, B, T, H, dk, dv, chunk, dtype,
+                     workspace, workspace_bytes, nullptr};
+    cudaError_t e;
+    if (use_tc) {
+        const size_t need = kda::chunk_tc_workspace_bytes(B, T, H);
+        if (need > 0 && (!workspace || workspace_bytes < need))
+            return fail(KDA_ERR_WORKSPACE, "workspace of %zu bytes given, %zu needed",
+                        workspace ? workspace_bytes : static_cast<size_t>(0), need);
+        a.device_error = device_error_ptr();
+        if (!a.device_error) return fail(KDA_ERR_CUDA, "device error word not addressable");
+        e = kda::launch_chunk_tc(a, s);
+    } else {
+        e = kda::launch_chunk_generic(a, s);
+    }
+    return e == cudaSuccess ? KDA_OK : cuda_fail(e, "launching the prefill kernel");
+}
+
+int kda_chunk_fwd(const void *q, const void *k, const void *v, const float *log_alpha,
+                  const float *beta, const float *S0, void *out, float *S_T, int B, int T, int H,
+                  int dk, int dv, int chunk, int dtype, void *workspace, size_t workspace_bytes,
+                  void *stream) {
+    return kda_chunk_fwd_engine(KDA_ENGINE_AUTO, q, k, v, log_alpha, beta, S0, out, S_T, B, T, H,
+                                dk, dv, chunk, dtype, workspace, workspace_bytes, stream);
+}
+
+int kda_recurrent_step(const void *q, const void *k, const void *v, const float *log_alpha,
+                       const float *beta, float *state, const int32_t *slot, void *out, int N,
+                       int H, int dk, int dv, int dtype, void *stream) {
+    g_detail[0] = '\0';
+    if (N < 0 || H < 0) return fail(KDA_ERR_INVALID_ARG, "N=%d H=%d must be >= 0", N, H);
+    int rc = check_common(dk, dv, dtype);
+    if (rc != KDA_OK) return rc;
+    if (N == 0 || H == 0) return KDA_OK;
+    const Ptr ps[] = {{q, "q", true},       {k, "k", true},         {v, "v", true},
+                      {log_alpha, "log_alpha", true}, {beta, "beta", true}, {state, "state", true},
+                      {out, "out", true},   {slot, "slot", false}};
+    rc = check_pointers(ps, sizeof ps / sizeof ps[0]);
+    if (rc != KDA_OK) return rc;
+    kda::DecodeArgs a{q, k, v, log_alpha, beta, state, slot, out, N, H, dk, dv, dtype};
+    cudaError_t e = kda::launch_decode(a, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? KDA_OK : cuda_fail(e, "launching the decode kernel");
+}
+
+int kda_device_status(void *stream) {
+    g_detail[0] = '\0';
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return cuda_fail(e, "synchronising the stream");
+    int flag = 0;
+    e = cudaMemcpyFromSymbol(&flag, g_device_error, sizeof flag);
+    if (e != cudaSuccess) return cuda_fail(e, "reading the device error word");
+    if (flag == 0) return KDA_OK;
+    const int zero = 0;
+    e = cudaMemcpyToSymbol(g_device_error, &zero, sizeof zero);
+    if (e != cudaSuccess) return cuda_fail(e, "clearing the device error word");
+    return fail(KDA_ERR_DEVICE_TIMEOUT, "a bounded device wait gave up (code %d)", flag);
+}
+
+}  // extern "C"

@@ -1,0 +1,52 @@
+// kda_internal.cuh -- declarations shared by the libkda translation units.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "kda.h"
+
+namespace kda {
+
+template <typename T> __device__ __forceinline__ float to_f32(T x);
+template <> __device__ __forceinline__ float to_f32<float>(float x) { return x; }
+template <> __device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 x) {
+    return __bfloat162float(x);
+}
+
+template <typename T> __device__ __forceinline__ T from_f32(float x);
+template <> __device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
+    return __float2bfloat16_rn(x);
+}
+
+struct ChunkArgs {
+    const void *q, *k, *v;
+    const float *log_alpha, *beta, *S0;
+    void *out;
+    float *S_T;
+    int B, T, H, dk, dv, chunk, dtype;
+    void *workspace;
+    size_t workspace_bytes;
+    int *device_error;  // set to a nonzero code by a kernel whose bounded wait gave up
+};
+
+struct DecodeArgs {
+    const void *q, *k, *v;
+    const float *log_alpha, *beta;
+    float *state;
+    const int32_t *slot;
+    void *out;
+    int N, H, dk, dv, dtype;
+};
+
+// Launchers return cudaSuccess or the launch error. They do no argument checks.
+cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t s);
+cudaError_t launch_chunk_generic(const ChunkArgs &a, cudaStream_t s);
+cudaError_t launch_chunk_tc(const ChunkArgs &a, cudaStream_t s);
+
+bool chunk_tc_supported(int dk, int dv, int chunk, int dtype);
+size_t chunk_tc_workspace_bytes(int B, int T, int H);
+
+}  // namespace kda

@@ -1,0 +1,157 @@
+/*
+ * kda.h -- C ABI of libkda, the B200 (sm_100a) implementation of Kimi Delta
+ * Attention (KDA): chunked prefill and single-token recurrent decode.
+ *
+ * The operator. Per (batch b, head h) a d_k x d_v fp32 state S evolves token by
+ * token as
+ *     S_t = (I - beta_t k_t k_t^T) Diag(alpha_t) S_{t-1} + beta_t k_t v_t^T,
+ *     o_t = S_t^T q_t,        alpha_t = exp(log_alpha_t) in (0,1]^{d_k}.
+ * Kimi Linear summary (es.news.hada.io/topic?id=31936): section "De la atencion
+ * lineal a Gated DeltaNet" gives the delta rule as a rank-1 generalised
+ * Householder update and GDN's forget gate; section "Control fino de memoria en
+ * Kimi Delta Attention" makes the gate diagonal and per channel, a
+ * Diagonal-Plus-Low-Rank transition tied to the key; section "Algoritmo
+ * paralelo por chunks" gives the chunked form that kda_chunk_fwd evaluates.
+ * There is no scale factor on q and no grouped heads: q, k, v all have H heads.
+ *
+ * Conventions for every entry point:
+ *  - All tensor pointers are DEVICE pointers owned by the caller, contiguous,
+ *    16-byte aligned. The library never allocates, frees or keeps a pointer
+ *    after the call returns.
+ *  - Work is enqueued on `stream` (a cudaStream_t passed as void*, NULL = the
+ *    legacy default stream) and the call returns without synchronising.
+ *  - Errors are returned as kda_status codes (never thrown, never trapped).
+ *    Argument errors are detected on the host before anything is enqueued;
+ *    kda_last_error_detail() names the offending argument.
+ *  - Preconditions that are documented but not checked (checking would cost a
+ *    pass over the data): log_alpha <= 0, beta in [0,1], finite inputs, and
+ *    within any chunk the per-channel total decay |sum log_alpha| <= 160
+ *    (the gate factors of the chunked form are anchored at the chunk's
+ *    midpoint and must stay inside the fp32/bf16 exponent range). L2
+ *    normalisation of q and k is the caller's job.
+ */
+#ifndef KDA_H
+#define KDA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    KDA_OK = 0,
+    KDA_ERR_INVALID_ARG = -1,    /* NULL where a pointer is required, negative size, bad enum */
+    KDA_ERR_UNSUPPORTED = -2,    /* shape, chunk or dtype outside what the kernels implement */
+    KDA_ERR_ALIGNMENT = -3,      /* a tensor pointer is not 16-byte aligned */
+    KDA_ERR_WORKSPACE = -4,      /* workspace NULL or smaller than kda_workspace_bytes() */
+    KDA_ERR_CUDA = -5,           /* a CUDA runtime call or kernel launch failed */
+    KDA_ERR_DEVICE_TIMEOUT = -6  /* a bounded device-side wait gave up (kda_device_status) */
+} kda_status;
+
+/* Element type of q, k, v and out. Gates, beta and states are always fp32. */
+typedef enum { KDA_BF16 = 0, KDA_F32 = 1 } kda_dtype;
+
+/* Which prefill engine kda_chunk_fwd_engine runs. */
+typedef enum {
+    KDA_ENGINE_AUTO = 0,     /* tensor-core engine where supported, else the generic one */
+    KDA_ENGINE_GENERIC = 1,  /* fp32 CUDA-core chunked engine: any d_k, d_v <= 128, chunk 16/32/64 */
+    KDA_ENGINE_TC = 2        /* tcgen05/TMEM engine: bf16, d_k = d_v = 128, chunk = 64 */
+} kda_engine;
+
+/*
+ * Bytes of device workspace kda_chunk_fwd needs for this problem (0 when the
+ * chosen engine needs none). Returns 0 for unsupported shapes as well; the
+ * forward call reports those.
+ */
+size_t kda_workspace_bytes(int B, int T, int H, int dk, int dv, int chunk, int dtype);
+
+/*
+ * Chunked prefill over T tokens (Kimi Linear summary, section "Algoritmo
+ * paralelo por chunks": fixed-length chunks, each starting from the previous
+ * chunk's last state; WY/UT form of the rank-1 updates; lower-triangular
+ * inverse by forward substitution; state update in matrix form; output that
+ * combines the inter-chunk recurrent part with the intra-chunk parallel part).
+ *
+ *   q, k       [B,T,H,dk]  dtype        queries and keys
+ *   v          [B,T,H,dv]  dtype        values
+ *   log_alpha  [B,T,H,dk]  fp32         log of the per-channel forget gate
+ *   beta       [B,T,H]     fp32         delta-rule write/erase strength
+ *   S0         [B,H,dk,dv] fp32         initial state; NULL means zeros
+ *   out        [B,T,H,dv]  dtype        o_t (written)
+ *   S_T        [B,H,dk,dv] fp32         final state (written); NULL skips it
+ *   chunk      16, 32 or 64             chunk length C; a ragged last chunk is
+ *                                       padded with identity steps (exact)
+ *   dtype      KDA_BF16 or KDA_F32
+ *   workspace, workspace_bytes          device scratch of at least
+ *                                       kda_workspace_bytes(...) bytes; may be
+ *                                       NULL/0 when that is 0
+ *   stream     cudaStream_t as void*
+ * S0 and S_T may alias (in-place state update). out must not alias inputs.
+ * T = 0 copies S0 (or zeros) to S_T. B = 0 or H = 0 is a no-op.
+ * Supported: dk, dv in [1,128] with dv % 4 == 0 (generic engine); the
+ * tensor-core engine additionally needs bf16, dk = dv = 128, chunk = 64.
+ */
+int kda_chunk_fwd(const void *q, const void *k, const void *v,
+                  const float *log_alpha, const float *beta, const float *S0,
+                  void *out, float *S_T,
+                  int B, int T, int H, int dk, int dv, int chunk, int dtype,
+                  void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * 1 if `engine` (kda_engine) can run a prefill of this shape and dtype, else 0.
+ * KDA_ENGINE_AUTO always can when the generic engine can.
+ */
+int kda_engine_supported(int engine, int dk, int dv, int chunk, int dtype);
+
+/* kda_chunk_fwd with an explicit engine (kda_engine). Same arguments otherwise. */
+int kda_chunk_fwd_engine(int engine, const void *q, const void *k, const void *v,
+                         const float *log_alpha, const float *beta, const float *S0,
+                         void *out, float *S_T,
+                         int B, int T, int H, int dk, int dv, int chunk, int dtype,
+                         void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * One decode step for N sequences against a state cache, in place (the
+ * recurrent form of the same operator; the state is the constant-size cache
+ * that replaces a KV cache, Kimi Linear summary, sections "Hibrido 3:1 de KDA
+ * y MLA" and "Uso de NoPE y resultados de evaluacion").
+ *
+ *   q, k       [N,H,dk]    dtype
+ *   v          [N,H,dv]    dtype
+ *   log_alpha  [N,H,dk]    fp32
+ *   beta       [N,H]       fp32
+ *   state      [slots,H,dk,dv] fp32     read and updated in place
+ *   slot       [N] int32               state row of sequence n; NULL means n.
+ *                                       Entries must be distinct and in
+ *                                       [0, slots) (not checked: device data)
+ *   out        [N,H,dv]    dtype        o = S_new^T q (written)
+ * Supported: dk, dv in [1,128], dv % 4 == 0.
+ */
+int kda_recurrent_step(const void *q, const void *k, const void *v,
+                       const float *log_alpha, const float *beta,
+                       float *state, const int32_t *slot, void *out,
+                       int N, int H, int dk, int dv, int dtype, void *stream);
+
+/* Human-readable name of a kda_status code (static string). */
+const char *kda_strerror(int code);
+
+/* Detail of the last error returned on the calling host thread (static per thread). */
+const char *kda_last_error_detail(void);
+
+/*
+ * Synchronises `stream` and reports whether a kernel of this library gave up
+ * a bounded device-side wait since the previous call (KDA_ERR_DEVICE_TIMEOUT),
+ * clearing the flag; KDA_ERR_CUDA if synchronisation failed; else KDA_OK.
+ */
+int kda_device_status(void *stream);
+
+/* ABI version of this header: major * 10000 + minor * 100 + patch. */
+int kda_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KDA_H */
