@@ -374,7 +374,7 @@ def cpu_baseline(args, seconds_hint=True):
     w = I.WORKLOADS[PREFILL]
     cores = os.cpu_count() or 1
     threads = max(1, min(cores, args.cpu_threads or cores))
-    n_heads = max(1, min(w.H, threads))
+    n_heads = w.H
     T_s = min(w.T, args.cpu_tokens)
     inp = I.prefill_inputs(w, T=T_s, H=n_heads)
     t = time.perf_counter()
@@ -448,7 +448,7 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--decode-steps", type=int, default=1000)
-    ap.add_argument("--cpu-tokens", type=int, default=8192,
+    ap.add_argument("--cpu-tokens", type=int, default=32768,
                     help="tokens per head of the CPU oracle sample")
     ap.add_argument("--cpu-tokens-ref", type=int, default=2048,
                     help="tokens per head per step of the reference arm")
