@@ -88,15 +88,15 @@ def source_hash(*names) -> str:
     return h.hexdigest()[:16]
 
 
-def traffic_from_profiles(kernel_key: str, sources) -> float | None:
-    """DRAM bytes per launch from the committed ncu summary, or None if the kernel
-    source changed since that capture."""
+def traffic_from_profiles(kernel_key: str) -> float | None:
+    """DRAM bytes per launch from the committed ncu summary (profiles/traffic.json),
+    or None if the kernel's sources changed since that capture."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
         return None
     with open(path) as f:
         rec = json.load(f).get(kernel_key)
-    if not rec or rec.get("source_hash") != source_hash(*sources):
+    if not rec or rec.get("source_hash") != source_hash(*rec.get("sources", [])):
         return None
     return float(rec["dram_bytes_per_launch"])
 
@@ -212,8 +212,7 @@ def run_ours(args, rank, world, device):
     hbm, hbm_src = peaks()
     bytes_alg = prefill_bytes(w)
     achieved = bytes_alg / (ms_kernel / 1e3) / 1e9
-    kernel_src = ["chunk_tc.cu"] if engine == "tc" else ["chunk_generic.cu"]
-    traffic = traffic_from_profiles(f"prefill_{engine}", kernel_src)
+    traffic = traffic_from_profiles(f"prefill_{engine}")
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
                 "frac": round(achieved / hbm, 4), "traffic": traffic,
                 "peak_source": hbm_src, "kernel": f"prefill ({engine} engine)",
@@ -330,7 +329,7 @@ def run_decode(kda, args, device, stream, world):
             "frac_of_8TBps": round(gbs / NOMINAL_HBM_GBS, 4),
             "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm, "unit": "GB/s",
                          "frac": round(gbs / hbm, 4), "peak_source": src,
-                         "traffic": traffic_from_profiles("decode", ["decode.cu"])},
+                         "traffic": traffic_from_profiles("decode")},
             "tokens_per_s": round(w.N * world / (ms_total / n_steps / 1e3), 1),
             "launches": n_steps}
 
