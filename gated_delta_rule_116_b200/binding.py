@@ -14,7 +14,7 @@ import torch
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libkda.so")
 
 KDA_BF16, KDA_F32 = 0, 1
-ENGINES = {"auto": 0, "generic": 1, "tc": 2}
+ENGINES = {"auto": 0, "generic": 1, "tc": 2, "tc_cluster": 3}
 _DTYPES = {torch.bfloat16: KDA_BF16, torch.float32: KDA_F32}
 
 _lib = None

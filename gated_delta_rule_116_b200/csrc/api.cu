@@ -88,6 +88,8 @@ int kda_engine_supported(int engine, int dk, int dv, int chunk, int dtype) {
         case KDA_ENGINE_AUTO:
         case KDA_ENGINE_GENERIC: return generic ? 1 : 0;
         case KDA_ENGINE_TC: return generic && kda::chunk_tc_supported(dk, dv, chunk, dtype) ? 1 : 0;
+        case KDA_ENGINE_TC_CLUSTER:
+            return generic && kda::chunk_cluster_supported(dk, dv, chunk, dtype) ? 1 : 0;
         default: return 0;
     }
 }
@@ -103,7 +105,7 @@ int kda_chunk_fwd_engine(int engine, const void *q, const void *k, const void *v
                          float *S_T, int B, int T, int H, int dk, int dv, int chunk, int dtype,
                          void *workspace, size_t workspace_bytes, void *stream) {
     g_detail[0] = '\0';
-    if (engine < KDA_ENGINE_AUTO || engine > KDA_ENGINE_TC)
+    if (engine < KDA_ENGINE_AUTO || engine > KDA_ENGINE_TC_CLUSTER)
         return fail(KDA_ERR_INVALID_ARG, "engine %d is not a kda_engine", engine);
     if (B < 0 || T < 0 || H < 0)
         return fail(KDA_ERR_INVALID_ARG, "B=%d T=%d H=%d must be >= 0", B, T, H);
@@ -130,28 +132,31 @@ int kda_chunk_fwd_engine(int engine, const void *q, const void *k, const void *v
     }
 
     const bool tc_ok = kda::chunk_tc_supported(dk, dv, chunk, dtype);
-    bool use_tc = false;
-    if (engine == KDA_ENGINE_TC) {
-        if (!tc_ok)
+    const bool cl_ok = kda::chunk_cluster_supported(dk, dv, chunk, dtype);
+    bool use_tc = false, use_cluster = false;
+    if (engine == KDA_ENGINE_TC || engine == KDA_ENGINE_TC_CLUSTER) {
+        if (!(engine == KDA_ENGINE_TC ? tc_ok : cl_ok))
             return fail(KDA_ERR_UNSUPPORTED,
-                        "tensor-core engine needs bf16, dk = dv = 128, chunk = 64 (got dtype %d, "
+                        "tensor-core engines need bf16, dk = dv = 128, chunk = 64 (got dtype %d, "
                         "dk %d, dv %d, chunk %d)", dtype, dk, dv, chunk);
-        use_tc = true;
+        use_tc = engine == KDA_ENGINE_TC;
+        use_cluster = engine == KDA_ENGINE_TC_CLUSTER;
     } else if (engine == KDA_ENGINE_AUTO) {
-        use_tc = tc_ok;
+        use_cluster = cl_ok;
+        use_tc = !cl_ok && tc_ok;
     }
 
     kda::ChunkArgs a{q, k, v, log_alpha, beta, S0, out, S_T, B, T, H, dk, dv, chunk, dtype,
                      workspace, workspace_bytes, nullptr};
     cudaError_t e;
-    if (use_tc) {
+    if (use_tc || use_cluster) {
         const size_t need = kda::chunk_tc_workspace_bytes(B, T, H);
         if (need > 0 && (!workspace || workspace_bytes < need))
             return fail(KDA_ERR_WORKSPACE, "workspace of %zu bytes given, %zu needed",
                         workspace ? workspace_bytes : static_cast<size_t>(0), need);
         a.device_error = device_error_ptr();
         if (!a.device_error) return fail(KDA_ERR_CUDA, "device error word not addressable");
-        e = kda::launch_chunk_tc(a, s);
+        e = use_cluster ? kda::launch_chunk_cluster(a, s) : kda::launch_chunk_tc(a, s);
     } else {
         e = kda::launch_chunk_generic(a, s);
     }

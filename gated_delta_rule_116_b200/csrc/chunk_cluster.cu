@@ -1,0 +1,637 @@
+// chunk_cluster.cu -- cluster engine of the chunked KDA prefill on sm_100a
+// (bf16 q/k/v, d_k = d_v = 128, chunk C = 64, fp32 gates and state).
+//
+// Same chunked form and operand precisions as chunk_tc.cu (Kimi Linear
+// summary, es.news.hada.io/topic?id=31936, sections "Algoritmo paralelo por
+// chunks" and "Menor cantidad de operaciones que DPLR general"):
+//   [A;P] = [K*E ; Q*E](K*F)^T (tf32), T = (I + A)^{-1} Diag(beta),
+//   [W | U'] = T [Ks | V] (fp16), then the state chain
+//   X = [Qs ; W] S, U = U' - W S, S <- Diag(e^{g_C}) S + Kb^T U, O = Qs S + P U.
+//
+// The work of one chunk splits into a key-side part that does not depend on
+// the state (everything up to W, U', P, T, Qs, Kb) and the state chain, which
+// is sequential over chunks. One head runs on a cluster of 4 CTAs (4 SMs):
+//   * ranks 0..2 are producers: rank p computes the key-side part of chunks
+//     p, p+3, p+6, ... into a staging image of 82 KB in its shared memory and
+//     bulk-copies it (cp.async.bulk, shared::cta -> shared::cluster) into one
+//     of two slots of the consumer, completing on the slot's mbarrier;
+//   * rank 3 is the consumer: it keeps the 128x128 fp32 state in registers and
+//     runs the chain for every chunk, on all 128 value columns, from the slots.
+//     When it is done with a slot it arms the slot's barrier for the next
+//     chunk and arrives (remotely) on the producer's "slot free" barrier.
+// A producer thus has three chunk periods for the key-side latency, and the
+// consumer's chunk period is the chain alone. Every wait is bounded; after a
+// timeout a CTA records an error in the device error word, stops waiting and
+// still reaches the final cluster barrier and frees its tensor memory.
+#include <cuda.h>
+
+#include "kda_internal.cuh"
+#include "tc_sm100.cuh"
+#include "ut_solve.cuh"
+
+namespace kda {
+namespace {
+
+using tc::fence_proxy_async_smem;
+using tc::mma_f16;
+using tc::mma_tf32;
+using tc::pack_bf16;
+using tc::pack_f16;
+using tc::sw128k_off;
+using tc::tc_fence_after;
+using tc::tc_fence_before;
+using ut::kLD;
+
+constexpr int kC = 64;
+constexpr int kD = 128;
+constexpr int kThreads = 256;
+constexpr int kProducers = 3;
+constexpr int kCluster = kProducers + 1;
+constexpr uint32_t kWaitLimit = 1u << 22;
+
+// ---- slot image: what a producer hands the consumer for one chunk
+constexpr uint32_t SL_QW = 0;          // [Qs ; W] fp16 K-major SW128, 2 K-blocks x 16 KB
+constexpr uint32_t kQWBlk = 16384;
+constexpr uint32_t SL_KB = 32768;      // Kb fp16 [token][channel], 2 blocks x 8 KB
+constexpr uint32_t SL_PT = 49152;      // [P ; T] fp16 K-major SW128, K = 64
+constexpr uint32_t SL_UP = 65536;      // U' fp16 [token][col], 2 blocks x 8 KB
+constexpr uint32_t SL_GAM = 81920;     // e^{g_C} fp32 [128]
+constexpr uint32_t kSlotBytes = 82432;
+constexpr uint32_t kSlotStride = 82944;
+constexpr uint32_t kTokBlk = 8192;
+
+// ---- producer shared memory
+constexpr uint32_t P_KQT = 0;          // [K*E ; Q*E] tf32, 4 K-blocks x 16 KB
+constexpr uint32_t kKQTBlk = 16384;
+constexpr uint32_t P_KHT = 65536;      // K*F tf32, 4 K-blocks x 8 KB
+constexpr uint32_t kKHTBlk = 8192;
+constexpr uint32_t P_AF = 0;           // A (fp32), reuses the tf32 region after the product
+constexpr uint32_t P_XF = 64 * kLD * 4;
+constexpr uint32_t P_STAGE = 98304;    // slot image being built
+constexpr uint32_t P_KSV = P_STAGE + kSlotStride;  // [Ks | V] fp16 [token][col], 4 blocks x 8 KB
+constexpr uint32_t P_VEC = P_KSV + 32768;          // beta[64], psum[4][128]
+constexpr uint32_t P_BAR = P_VEC + (64 + 512) * 4;
+// ---- consumer shared memory
+constexpr uint32_t C_SLOT = 0;         // 2 slots
+constexpr uint32_t C_S16 = 2 * kSlotStride;        // S fp16, MN-major SW128: 2 blocks x 16 KB
+constexpr uint32_t C_U16 = C_S16 + 32768;          // U fp16, MN-major SW128: 2 blocks x 8 KB
+constexpr uint32_t C_BAR = C_U16 + 16384;
+constexpr uint32_t kSmemBytes =
+    (P_BAR > C_BAR ? P_BAR : C_BAR) + 128 + 1024;  // + barriers + alignment slack
+
+// TMEM columns.
+constexpr uint32_t PCOL_AP = 0;        // producer: [A;P] (64 cols)
+constexpr uint32_t PCOL_WU = 64;       // producer: [P;T][Ks|V], lanes 64-127 = [W | U'] (256)
+constexpr uint32_t CCOL_X = 0;         // consumer: 2 x 128 cols ([Qs;W]S (+ [P;T]U))
+constexpr uint32_t CCOL_S = 256;       // consumer: Kb^T U (128 cols)
+constexpr uint32_t kTmemCols = 512;
+
+constexpr uint32_t IDESC_AP = tc::idesc(tc::kFmtTF32, 128, 64, 0, 0);
+constexpr uint32_t IDESC_WU = tc::idesc(tc::kFmtF16, 128, 256, 0, 1);
+constexpr uint32_t IDESC_X = tc::idesc(tc::kFmtF16, 128, 128, 0, 1);   // A K-major, B MN-major
+constexpr uint32_t IDESC_S = tc::idesc(tc::kFmtF16, 128, 128, 1, 1);   // A MN-major, B MN-major
+
+struct Ctl {
+    int *abort;
+    int *err;
+};
+
+__device__ __forceinline__ void fail(const Ctl &k) {
+    *reinterpret_cast<volatile int *>(k.abort) = 1;
+    atomicExch(k.err, 2);
+}
+__device__ __forceinline__ void wait_local(uint64_t *bar, uint32_t parity, const Ctl &k) {
+    if (*reinterpret_cast<volatile int *>(k.abort)) return;
+    if (!tc::mbar_wait(bar, parity, kWaitLimit)) fail(k);
+}
+__device__ __forceinline__ void wait_cluster(uint64_t *bar, uint32_t parity, const Ctl &k) {
+    if (*reinterpret_cast<volatile int *>(k.abort)) return;
+    if (!tc::mbar_wait_cluster(bar, parity, kWaitLimit)) fail(k);
+}
+
+// ============================================================ producer
+__device__ void producer(uint8_t *sm, uint32_t tmem, int rank, const CUtensorMap *tm_q,
+                         const CUtensorMap *tm_k, const CUtensorMap *tm_la,
+                         const CUtensorMap *tm_v, const __nv_bfloat16 *__restrict__ q,
+                         const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *__restrict__ v,
+                         const float *__restrict__ log_alpha, const float *__restrict__ beta,
+                         int T, int H, int h, long ztok, int nchunks, const Ctl &ctl) {
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int quad = warp & 3, half = warp >> 2;
+    const int row = 32 * quad + lane;
+    const uint32_t sbase = tc::smem_u32(sm);
+    float *beta_s = reinterpret_cast<float *>(sm + P_VEC);
+    float *psum = beta_s + 64;
+    float *Af = reinterpret_cast<float *>(sm + P_AF);
+    float *Xf = reinterpret_cast<float *>(sm + P_XF);
+    uint64_t *bar_mma = reinterpret_cast<uint64_t *>(sm + P_BAR);
+    uint64_t *bar_free = bar_mma + 1;
+    uint8_t *st = sm + P_STAGE;
+    uint32_t ph_mma = 0, ph_free = 0;
+
+    const uint64_t d_kqt = tc::smem_desc(sbase + P_KQT, 16, 1024, tc::kSwizzle128);
+    const uint64_t d_kht = tc::smem_desc(sbase + P_KHT, 16, 1024, tc::kSwizzle128);
+    const uint64_t d_pt = tc::smem_desc(sbase + P_STAGE + SL_PT, 16, 1024, tc::kSwizzle128);
+    const uint64_t d_ksv = tc::smem_desc(sbase + P_KSV, kTokBlk, 1024, tc::kSwizzle128);
+    // consumer-side addresses
+    const uint32_t cons = kCluster - 1;
+    const uint32_t c_base = tc::map_to_rank(sbase, cons);
+    const uint32_t c_full = tc::map_to_rank(sbase + C_BAR, cons);  // slot_full[0], [1]
+
+    for (int c = rank; c < nchunks; c += kProducers) {
+        const int t0 = c * kC;
+        const int valid = min(kC, T - t0);
+        const long trow0 = ztok + t0;
+        if (tid == 0) {
+            tc::bulk_wait_read_all();  // the previous image has left the staging area
+            if (c + kProducers < nchunks) {
+                const int z = static_cast<int>(trow0 + kProducers * kC);
+                tc::tma_prefetch_l2_3d(tm_q, 0, h, z);
+                tc::tma_prefetch_l2_3d(tm_k, 0, h, z);
+                tc::tma_prefetch_l2_3d(tm_la, 0, h, z);
+                tc::tma_prefetch_l2_3d(tm_v, 0, h, z);
+            }
+        }
+        __syncthreads();
+
+        // ------------------------------------------------ gates and operands
+        if (tid < kC) beta_s[tid] = tid < valid ? beta[(trow0 + tid) * H + h] : 0.f;
+        {   // V (all 128 columns) -> fp16 columns 128..255 of the [Ks | V] operand
+            const int t = tid >> 2, piece = tid & 3;
+            const uint4 *src = reinterpret_cast<const uint4 *>(v + ((trow0 + t) * H + h) * kD + 32 * piece);
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+                uint4 w = make_uint4(0, 0, 0, 0);
+                if (t < valid) {
+                    const uint4 x = src[m];
+                    w.x = pack_f16(tc::bf16_lo(x.x), tc::bf16_hi(x.x));
+                    w.y = pack_f16(tc::bf16_lo(x.y), tc::bf16_hi(x.y));
+                    w.z = pack_f16(tc::bf16_lo(x.z), tc::bf16_hi(x.z));
+                    w.w = pack_f16(tc::bf16_lo(x.w), tc::bf16_hi(x.w));
+                }
+                *reinterpret_cast<uint4 *>(sm + P_KSV + 2 * kTokBlk +
+                                           sw128k_off(t, 32 * piece + 8 * m, kTokBlk)) = w;
+            }
+        }
+        const int p = tid & 63, qq = tid >> 6;  // channels 2p, 2p+1; tokens 16qq .. 16qq+15
+        float2 lg[16];
+        uint32_t qv[16], kv[16];
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+            const int t = 16 * qq + u;
+            const long o = ((trow0 + t) * H + h) * kD + 2 * p;
+            const bool ok = t < valid;
+            lg[u] = ok ? *reinterpret_cast<const float2 *>(log_alpha + o) : make_float2(0.f, 0.f);
+            qv[u] = ok ? *reinterpret_cast<const uint32_t *>(q + o) : 0u;
+            kv[u] = ok ? *reinterpret_cast<const uint32_t *>(k + o) : 0u;
+        }
+        {
+            float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+            for (int u = 0; u < 16; ++u) { s0 += lg[u].x; s1 += lg[u].y; }
+            psum[qq * 128 + 2 * p] = s0;
+            psum[qq * 128 + 2 * p + 1] = s1;
+        }
+        __syncthreads();
+        {
+            float pre0 = 0.f, pre1 = 0.f, tot0 = 0.f, tot1 = 0.f;
+#pragma unroll
+            for (int q2 = 0; q2 < 4; ++q2) {
+                const float a0 = psum[q2 * 128 + 2 * p], a1 = psum[q2 * 128 + 2 * p + 1];
+                if (q2 < qq) { pre0 += a0; pre1 += a1; }
+                tot0 += a0;
+                tot1 += a1;
+            }
+            const float ga0 = 0.5f * tot0, ga1 = 0.5f * tot1;
+            const float ea0 = expf(ga0), ea1 = expf(ga1);                  // e^{g_a}
+            const float eca0 = expf(tot0 - ga0), eca1 = expf(tot1 - ga1);  // e^{g_C - g_a}
+            if (qq == 0) {
+                float *gam = reinterpret_cast<float *>(st + SL_GAM);
+                gam[2 * p] = expf(tot0);
+                gam[2 * p + 1] = expf(tot1);
+            }
+            constexpr float kLog2e = 1.4426950408889634f;
+            float d0 = (pre0 - ga0) * kLog2e, d1 = (pre1 - ga1) * kLog2e;
+            const uint32_t cc = 2 * p;
+            const uint32_t rowq = qq * 2048u;
+            const uint32_t b32 = (cc & 3u) * 4u + rowq;
+            const uint32_t ch32 = (cc & 31u) >> 2, kb32 = cc >> 5;
+            const uint32_t b16 = (cc & 7u) * 2u + rowq;
+            const uint32_t ch16 = (cc & 63u) >> 3, kb16 = cc >> 6;
+#pragma unroll
+            for (int u = 0; u < 16; ++u) {
+                const uint32_t r = (u >> 3) * 1024u + (u & 7) * 128u;
+                const uint32_t o32 = b32 + r + (((ch32 ^ (u & 7)) & 7u) << 4);
+                const uint32_t o16 = b16 + r + (((ch16 ^ (u & 7)) & 7u) << 4);
+                d0 = fmaf(lg[u].x, kLog2e, d0);
+                d1 = fmaf(lg[u].y, kLog2e, d1);
+                const float q0 = tc::bf16_lo(qv[u]), q1 = tc::bf16_hi(qv[u]);
+                const float k0 = tc::bf16_lo(kv[u]), k1 = tc::bf16_hi(kv[u]);
+                const float E0 = tc::ex2(d0), E1 = tc::ex2(d1);
+                const float F0 = tc::ex2(-d0), F1 = tc::ex2(-d1);
+                const float ke0 = k0 * E0, ke1 = k1 * E1, qe0 = q0 * E0, qe1 = q1 * E1;
+                const float kf0 = k0 * F0, kf1 = k1 * F1;
+                *reinterpret_cast<float2 *>(sm + P_KQT + kb32 * kKQTBlk + o32) = make_float2(ke0, ke1);
+                *reinterpret_cast<float2 *>(sm + P_KQT + kb32 * kKQTBlk + 8192 + o32) = make_float2(qe0, qe1);
+                *reinterpret_cast<float2 *>(sm + P_KHT + kb32 * kKHTBlk + o32) = make_float2(kf0, kf1);
+                *reinterpret_cast<uint32_t *>(st + SL_QW + kb16 * kQWBlk + o16) = pack_f16(qe0 * ea0, qe1 * ea1);
+                *reinterpret_cast<uint32_t *>(sm + P_KSV + kb16 * kTokBlk + o16) = pack_f16(ke0 * ea0, ke1 * ea1);
+                *reinterpret_cast<uint32_t *>(st + SL_KB + kb16 * kTokBlk + o16) = pack_f16(kf0 * eca0, kf1 * eca1);
+            }
+        }
+        fence_proxy_async_smem();
+        __syncthreads();
+
+        // ------------------------------------------------ [A;P] (tf32)
+        if (tid == 0) {
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < 16; ++kk)
+                mma_tf32(tmem + PCOL_AP, d_kqt + (((kk >> 2) * kKQTBlk + (kk & 3) * 32) >> 4),
+                         d_kht + (((kk >> 2) * kKHTBlk + (kk & 3) * 32) >> 4), IDESC_AP, kk > 0);
+            tc::mma_commit(bar_mma);
+        }
+        wait_local(bar_mma, ph_mma, ctl);
+        ph_mma ^= 1;
+        tc_fence_after();
+
+        // ------------------------------------------------ A (fp32), P (fp16), UT solve, T (fp16)
+        {
+            float vv[32];
+            tc::tmem_ld32(tc::tmem_addr(tmem, 32 * quad, PCOL_AP + half * 32), vv);
+            tc::tmem_wait_ld();
+            if (quad < 2) {
+                const int i = row;
+                const float bi = beta_s[i];
+#pragma unroll
+                for (int u = 0; u < 32; ++u) {
+                    const int j = half * 32 + u;
+                    Af[i * kLD + j] = j < i ? bi * vv[u] : 0.f;
+                }
+            } else {
+                const int i = row - 64;
+#pragma unroll
+                for (int u = 0; u < 32; u += 2) {
+                    const int j = half * 32 + u;
+                    const float lo = j <= i ? vv[u] : 0.f, hi = j + 1 <= i ? vv[u + 1] : 0.f;
+                    *reinterpret_cast<uint32_t *>(st + SL_PT + sw128k_off(i, j, 0)) = pack_f16(lo, hi);
+                }
+            }
+        }
+        tc_fence_before();
+        __syncthreads();
+        ut::unit_lower_inverse(Af, Xf, tid);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int e = tid + u * kThreads;
+            const int i = e >> 5, j = (e & 31) * 2;
+            const float lo = j <= i ? Xf[i * kLD + j] * beta_s[j] : 0.f;
+            const float hi = j + 1 <= i ? Xf[i * kLD + j + 1] * beta_s[j + 1] : 0.f;
+            *reinterpret_cast<uint32_t *>(st + SL_PT + 8192 + sw128k_off(i, j, 0)) = pack_f16(lo, hi);
+        }
+        fence_proxy_async_smem();
+        __syncthreads();
+
+        // ------------------------------------------------ [W | U'] = T [Ks | V] (fp16, N = 256)
+        if (tid == 0) {
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+                mma_f16(tmem + PCOL_WU, d_pt + ((kk * 32) >> 4), d_ksv + ((kk * 2048) >> 4), IDESC_WU, kk > 0);
+            tc::mma_commit(bar_mma);
+        }
+        wait_local(bar_mma, ph_mma, ctl);
+        ph_mma ^= 1;
+        tc_fence_after();
+        if (quad >= 2) {
+            const int i = row - 64;
+#pragma unroll
+            for (int part = 0; part < 2; ++part) {   // part 0: W, part 1: U'
+                float w[64];
+                const uint32_t ta = tc::tmem_addr(tmem, 32 * quad, PCOL_WU + part * 128 + half * 64);
+                tc::tmem_ld32(ta, *reinterpret_cast<float(*)[32]>(&w[0]));
+                tc::tmem_ld32(ta + 32, *reinterpret_cast<float(*)[32]>(&w[32]));
+                tc::tmem_wait_ld();
+#pragma unroll
+                for (int u = 0; u < 64; u += 8) {
+                    uint4 x;
+                    x.x = pack_f16(w[u], w[u + 1]);
+                    x.y = pack_f16(w[u + 2], w[u + 3]);
+                    x.z = pack_f16(w[u + 4], w[u + 5]);
+                    x.w = pack_f16(w[u + 6], w[u + 7]);
+                    const int col = half * 64 + u;
+                    const uint32_t off = part == 0 ? SL_QW + sw128k_off(64 + i, col, kQWBlk)
+                                                   : SL_UP + sw128k_off(i, col, kTokBlk);
+                    *reinterpret_cast<uint4 *>(st + off) = x;
+                }
+            }
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+
+        // ------------------------------------------------ hand the image to the consumer
+        if (tid == 0) {
+            wait_cluster(bar_free, ph_free, ctl);
+            const uint32_t s = c & 1;
+            const uint32_t dst = c_base + C_SLOT + s * kSlotStride;
+            const uint32_t full = c_full + s * 8;
+            if (!*reinterpret_cast<volatile int *>(ctl.abort)) {
+                tc::bulk_copy_to_peer(dst + SL_QW, st + SL_QW, 32768, full);
+                tc::bulk_copy_to_peer(dst + SL_KB, st + SL_KB, 16384, full);
+                tc::bulk_copy_to_peer(dst + SL_PT, st + SL_PT, 16384, full);
+                tc::bulk_copy_to_peer(dst + SL_UP, st + SL_UP, kSlotBytes - SL_UP, full);
+                tc::bulk_commit();
+            }
+        }
+        ph_free ^= 1;
+    }
+    if (tid == 0) tc::bulk_wait_read_all();
+}
+
+// ============================================================ consumer
+__device__ void consumer(uint8_t *sm, uint32_t tmem, const float *__restrict__ S0,
+                         __nv_bfloat16 *__restrict__ out, float *__restrict__ S_T, int T, int H,
+                         int h, long bh, long ztok, int nchunks, const Ctl &ctl) {
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int quad = warp & 3, half = warp >> 2;
+    const int row = 32 * quad + lane;   // TMEM lane; state row (key channel)
+    const uint32_t sbase = tc::smem_u32(sm);
+    uint64_t *full = reinterpret_cast<uint64_t *>(sm + C_BAR);  // [2]
+    uint64_t *bar_x = full + 2;
+    uint64_t *bar_s = full + 3;
+    uint64_t *bar_o = full + 4;
+    uint32_t ph_full[2] = {0, 0};
+    uint32_t ph_x = 0, ph_s = 0, ph_o = 0;
+
+    const uint64_t d_s16 = tc::smem_desc(sbase + C_S16, 16384, 1024, tc::kSwizzle128);
+    const uint64_t d_u16 = tc::smem_desc(sbase + C_U16, kTokBlk, 1024, tc::kSwizzle128);
+    const uint32_t p_free = sbase + P_BAR + 8;  // producer's "slot free" barrier (same offset)
+
+    // fp32 state: row `row`, columns half*64 .. +64
+    float S[64];
+#pragma unroll
+    for (int j = 0; j < 64; ++j)
+        S[j] = S0 ? S0[(bh * kD + row) * kD + half * 64 + j] : 0.f;
+    auto write_s16 = [&]() {
+#pragma unroll
+        for (int u = 0; u < 64; u += 8) {
+            uint4 x;
+            x.x = pack_f16(S[u], S[u + 1]);
+            x.y = pack_f16(S[u + 2], S[u + 3]);
+            x.z = pack_f16(S[u + 4], S[u + 5]);
+            x.w = pack_f16(S[u + 6], S[u + 7]);
+            *reinterpret_cast<uint4 *>(sm + C_S16 + half * 16384 + sw128k_off(row, u, 0)) = x;
+        }
+    };
+    write_s16();
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    if (tid == 0) {
+        // slots start free: arm both and release chunks 0 and 1 to their producers
+        for (int s = 0; s < 2 && s < nchunks; ++s) {
+            tc::mbar_arrive_expect_tx(full + s, kSlotBytes);
+            tc::mbar_arrive_remote(tc::map_to_rank(p_free, s % kProducers));
+        }
+    }
+    auto issue_x = [&](int c) {   // X[c&1] = [Qs;W] S16
+        const uint32_t slot = C_SLOT + (c & 1) * kSlotStride;
+        const uint64_t d_qw = tc::smem_desc(sbase + slot + SL_QW, 16, 1024, tc::kSwizzle128);
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+            mma_f16(tmem + CCOL_X + (c & 1) * 128, d_qw + (((kk >> 2) * kQWBlk + (kk & 3) * 32) >> 4),
+                    d_s16 + ((kk * 2048) >> 4), IDESC_X, kk > 0);
+        tc::mma_commit(bar_x);
+    };
+    if (nchunks > 0) {
+        wait_local(full, ph_full[0], ctl);
+        if (tid == 0) issue_x(0);
+    }
+
+    for (int c = 0; c < nchunks; ++c) {
+        const int s = c & 1;
+        const int t0 = c * kC;
+        const int valid = min(kC, T - t0);
+        const uint8_t *slot = sm + C_SLOT + s * kSlotStride;
+        const uint32_t xcol = CCOL_X + s * 128;
+        wait_local(full + s, ph_full[s], ctl);  // (already complete) makes the slot visible
+        ph_full[s] ^= 1;
+        wait_local(bar_x, ph_x, ctl);
+        ph_x ^= 1;
+        tc_fence_after();
+
+        // U = U' - W S  (lanes 64..127 = tokens)
+        if (quad >= 2) {
+            const int i = row - 64;
+            float x[64];
+            const uint32_t ta = tc::tmem_addr(tmem, 32 * quad, xcol + half * 64);
+            tc::tmem_ld32(ta, *reinterpret_cast<float(*)[32]>(&x[0]));
+            tc::tmem_ld32(ta + 32, *reinterpret_cast<float(*)[32]>(&x[32]));
+            tc::tmem_wait_ld();
+#pragma unroll
+            for (int u = 0; u < 64; u += 8) {
+                const uint4 up = *reinterpret_cast<const uint4 *>(slot + SL_UP +
+                                                                  sw128k_off(i, half * 64 + u, kTokBlk));
+                const __half2 *h2 = reinterpret_cast<const __half2 *>(&up);
+                uint4 y;
+                uint32_t *yy = reinterpret_cast<uint32_t *>(&y);
+#pragma unroll
+                for (int m = 0; m < 4; ++m) {
+                    const float2 f = __half22float2(h2[m]);
+                    yy[m] = pack_f16(f.x - x[u + 2 * m], f.y - x[u + 2 * m + 1]);
+                }
+                *reinterpret_cast<uint4 *>(sm + C_U16 + half * kTokBlk + sw128k_off(i, u, 0)) = y;
+            }
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        if (tid == 0) {
+            tc_fence_after();
+            const uint64_t d_kb = tc::smem_desc(sbase + C_SLOT + s * kSlotStride + SL_KB, kTokBlk, 1024,
+                                                tc::kSwizzle128);
+            const uint64_t d_pt = tc::smem_desc(sbase + C_SLOT + s * kSlotStride + SL_PT, 16, 1024,
+                                                tc::kSwizzle128);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+                mma_f16(tmem + CCOL_S, d_kb + ((kk * 2048) >> 4), d_u16 + ((kk * 2048) >> 4), IDESC_S, kk > 0);
+            tc::mma_commit(bar_s);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+                mma_f16(tmem + xcol, d_pt + ((kk * 32) >> 4), d_u16 + ((kk * 2048) >> 4), IDESC_X, 1);
+            tc::mma_commit(bar_o);
+        }
+        // S <- Diag(e^{g_C}) S + Kb^T U
+        wait_local(bar_s, ph_s, ctl);
+        ph_s ^= 1;
+        tc_fence_after();
+        {
+            const float gm = reinterpret_cast<const float *>(slot + SL_GAM)[row];
+            float sv[64];
+            const uint32_t ta = tc::tmem_addr(tmem, 32 * quad, CCOL_S + half * 64);
+            tc::tmem_ld32(ta, *reinterpret_cast<float(*)[32]>(&sv[0]));
+            tc::tmem_ld32(ta + 32, *reinterpret_cast<float(*)[32]>(&sv[32]));
+            tc::tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 64; ++j) S[j] = fmaf(gm, S[j], sv[j]);
+        }
+        write_s16();
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        if (c + 1 < nchunks) {
+            wait_local(full + (s ^ 1), ph_full[s ^ 1], ctl);
+            if (tid == 0) issue_x(c + 1);
+        }
+        // O = Qs S + P U  (lanes 0..63 = tokens)
+        wait_local(bar_o, ph_o, ctl);
+        ph_o ^= 1;
+        tc_fence_after();
+        if (quad < 2) {
+            float o[64];
+            const uint32_t ta = tc::tmem_addr(tmem, 32 * quad, xcol + half * 64);
+            tc::tmem_ld32(ta, *reinterpret_cast<float(*)[32]>(&o[0]));
+            tc::tmem_ld32(ta + 32, *reinterpret_cast<float(*)[32]>(&o[32]));
+            tc::tmem_wait_ld();
+            if (row < valid) {
+                uint4 *dst = reinterpret_cast<uint4 *>(out + ((ztok + t0 + row) * H + h) * kD + half * 64);
+#pragma unroll
+                for (int u = 0; u < 64; u += 8) {
+                    uint4 x;
+                    x.x = pack_bf16(o[u], o[u + 1]);
+                    x.y = pack_bf16(o[u + 2], o[u + 3]);
+                    x.z = pack_bf16(o[u + 4], o[u + 5]);
+                    x.w = pack_bf16(o[u + 6], o[u + 7]);
+                    dst[u / 8] = x;
+                }
+            }
+        }
+        tc_fence_before();
+        __syncthreads();
+        if (tid == 0 && c + 2 < nchunks && !*reinterpret_cast<volatile int *>(ctl.abort)) {
+            tc::mbar_arrive_expect_tx(full + s, kSlotBytes);
+            tc::mbar_arrive_remote(tc::map_to_rank(p_free, (c + 2) % kProducers));
+        }
+    }
+    if (S_T) {
+#pragma unroll
+        for (int j = 0; j < 64; ++j) S_T[(bh * kD + row) * kD + half * 64 + j] = S[j];
+    }
+}
+
+__global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 1)
+chunk_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                     const __grid_constant__ CUtensorMap tm_la, const __grid_constant__ CUtensorMap tm_v,
+                     const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
+                     const __nv_bfloat16 *__restrict__ v, const float *__restrict__ log_alpha,
+                     const float *__restrict__ beta, const float *__restrict__ S0,
+                     __nv_bfloat16 *__restrict__ out, float *__restrict__ S_T, int T, int H, int *err) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                              ~static_cast<uintptr_t>(1023));
+    const int rank = static_cast<int>(tc::cluster_rank());
+    const long bh = blockIdx.x / kCluster;
+    const int b = static_cast<int>(bh / H), h = static_cast<int>(bh - static_cast<long>(b) * H);
+    const long ztok = static_cast<long>(b) * T;
+    const int nchunks = (T + kC - 1) / kC;
+    const bool is_consumer = rank == kCluster - 1;
+    const uint32_t bar_off = is_consumer ? C_BAR : P_BAR;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + bar_off);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + bar_off + 64);
+    int *abort = reinterpret_cast<int *>(sm + bar_off + 68);
+    const int tid = threadIdx.x;
+
+    if (tid == 0) {
+        for (int i = 0; i < 5; ++i) tc::mbar_init(bars + i, 1);
+        *abort = 0;
+        tc::fence_mbar_init();
+    }
+    if ((tid >> 5) == 0) {
+        tc::tmem_alloc(tmem_slot, kTmemCols);
+        tc::tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    tc::cluster_sync();  // every barrier of the cluster is initialised before any remote use
+    const uint32_t tmem = *tmem_slot;
+    const Ctl ctl{abort, err};
+
+    if (is_consumer)
+        consumer(sm, tmem, S0, out, S_T, T, H, h, bh, ztok, nchunks, ctl);
+    else
+        producer(sm, tmem, rank, &tm_q, &tm_k, &tm_la, &tm_v, q, k, v, log_alpha, beta, T, H, h, ztok,
+                 nchunks, ctl);
+
+    tc_fence_before();
+    __syncthreads();
+    tc::cluster_sync();  // no CTA leaves while a peer may still touch its shared memory
+    if ((tid >> 5) == 0) {
+        tc_fence_after();
+        tc::tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult qr;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &qr) ==
+                cudaSuccess &&
+            qr == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    return fn;
+}
+
+// 3-D map over a [B*T, H, 128] tensor with a (128, 1, 64) box, used for L2 prefetches.
+bool make_map(CUtensorMap *m, const void *ptr, CUtensorMapDataType dt, int esize, int H, long tokens) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(kD), static_cast<cuuint64_t>(H),
+                                static_cast<cuuint64_t>(tokens)};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(kD) * esize,
+                                   static_cast<cuuint64_t>(kD) * esize * H};
+    const cuuint32_t box[3] = {static_cast<cuuint32_t>(kD), 1, kC};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return enc(m, dt, 3, const_cast<void *>(ptr), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+bool chunk_cluster_supported(int dk, int dv, int chunk, int dtype) {
+    return dtype == KDA_BF16 && dk == kD && dv == kD && chunk == kC;
+}
+
+cudaError_t launch_chunk_cluster(const ChunkArgs &a, cudaStream_t s) {
+    const long tokens = static_cast<long>(a.B) * a.T;
+    CUtensorMap mq, mk, mla, mv;
+    if (!make_map(&mq, a.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.H, tokens) ||
+        !make_map(&mk, a.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.H, tokens) ||
+        !make_map(&mla, a.log_alpha, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, a.H, tokens) ||
+        !make_map(&mv, a.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.H, tokens))
+        return cudaErrorInvalidValue;
+    cudaError_t e = cudaFuncSetAttribute(chunk_cluster_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(kSmemBytes));
+    if (e != cudaSuccess) return e;
+    const dim3 grid(static_cast<unsigned>(a.B) * a.H * kCluster);
+    chunk_cluster_kernel<<<grid, kThreads, kSmemBytes, s>>>(
+        mq, mk, mla, mv, static_cast<const __nv_bfloat16 *>(a.q),
+        static_cast<const __nv_bfloat16 *>(a.k), static_cast<const __nv_bfloat16 *>(a.v),
+        a.log_alpha, a.beta, a.S0, static_cast<__nv_bfloat16 *>(a.out), a.S_T, a.T, a.H,
+        a.device_error);
+    return cudaGetLastError();
+}
+
+}  // namespace kda

@@ -35,6 +35,7 @@
 
 #include "kda_internal.cuh"
 #include "tc_sm100.cuh"
+#include "ut_solve.cuh"
 
 namespace kda {
 namespace {
@@ -63,7 +64,7 @@ constexpr uint32_t kKQTBlk = 16384;
 constexpr uint32_t OFF_KHT = 65536;       // K*F tf32, 4 K-blocks x 8 KB (64 rows)
 constexpr uint32_t kKHTBlk = 8192;
 // ... then reused for the solve and the [P;T] operand:
-constexpr int kLD = 68;                   // row stride (floats) of A / X (conflict-free fragments)
+using ut::kLD;                            // row stride (floats) of A / X
 constexpr uint32_t OFF_AF = 0;            // A (fp32)
 constexpr uint32_t OFF_XF = 64 * kLD * 4;  // X = (I + A)^{-1} (fp32)
 constexpr uint32_t OFF_PT = 34816;        // [P 8K | T 8K] fp16, K-major, K = 64
@@ -117,122 +118,6 @@ __device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, int *ab
     *reinterpret_cast<volatile int *>(abort) = 1;
     atomicExch(err, 1);
     return false;
-}
-
-// ------------------------------------------------------------------ UT transform
-// X = (I + A)^{-1} for the strictly lower-triangular 64x64 A (row stride kLD),
-// the lower-triangular inverse "row by row by forward substitution" of the
-// chunked algorithm, organised in 16x16 blocks:
-//   1) X_II = (I + A_II)^{-1} for the 4 diagonal blocks: forward substitution,
-//      one column per thread, fp32.
-//   2) R_IJ = A_IJ X_JJ for the 6 blocks below the diagonal (one warp each).
-//   3) block column J, one warp each, top to bottom:
-//      X_IJ = -X_II (R_IJ + sum_{J<K<I} A_IK X_KJ).
-// Block products use warp-level tf32 mma.sync (m16n8k8, fp32 accumulate).
-
-__device__ __forceinline__ uint32_t to_tf32(float x) {
-    uint32_t r;
-    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
-    return r;
-}
-
-// acc[ns][.] += A(16x16) * B(16x16) for one warp; acc holds the two 16x8 halves
-// of the 16x16 result in the m16n8 accumulator layout.
-__device__ __forceinline__ void warp_mm16(float (&acc)[2][4], const float *A, const float *B,
-                                          int lane) {
-    const int g = lane >> 2, t = lane & 3;
-#pragma unroll
-    for (int ks = 0; ks < 2; ++ks) {
-        uint32_t a[4];
-        a[0] = to_tf32(A[g * kLD + 8 * ks + t]);
-        a[1] = to_tf32(A[(g + 8) * kLD + 8 * ks + t]);
-        a[2] = to_tf32(A[g * kLD + 8 * ks + t + 4]);
-        a[3] = to_tf32(A[(g + 8) * kLD + 8 * ks + t + 4]);
-#pragma unroll
-        for (int ns = 0; ns < 2; ++ns) {
-            const uint32_t b0 = to_tf32(B[(8 * ks + t) * kLD + 8 * ns + g]);
-            const uint32_t b1 = to_tf32(B[(8 * ks + t + 4) * kLD + 8 * ns + g]);
-            asm volatile(
-                "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 "
-                "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
-                : "+f"(acc[ns][0]), "+f"(acc[ns][1]), "+f"(acc[ns][2]), "+f"(acc[ns][3])
-                : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-        }
-    }
-}
-__device__ __forceinline__ void acc_load16(float (&acc)[2][4], const float *C, int lane) {
-    const int g = lane >> 2, t = lane & 3;
-#pragma unroll
-    for (int ns = 0; ns < 2; ++ns) {
-        acc[ns][0] = C[g * kLD + 8 * ns + 2 * t];
-        acc[ns][1] = C[g * kLD + 8 * ns + 2 * t + 1];
-        acc[ns][2] = C[(g + 8) * kLD + 8 * ns + 2 * t];
-        acc[ns][3] = C[(g + 8) * kLD + 8 * ns + 2 * t + 1];
-    }
-}
-__device__ __forceinline__ void acc_store16(const float (&acc)[2][4], float *C, float scale,
-                                            int lane) {
-    const int g = lane >> 2, t = lane & 3;
-#pragma unroll
-    for (int ns = 0; ns < 2; ++ns) {
-        C[g * kLD + 8 * ns + 2 * t] = scale * acc[ns][0];
-        C[g * kLD + 8 * ns + 2 * t + 1] = scale * acc[ns][1];
-        C[(g + 8) * kLD + 8 * ns + 2 * t] = scale * acc[ns][2];
-        C[(g + 8) * kLD + 8 * ns + 2 * t + 1] = scale * acc[ns][3];
-    }
-}
-__device__ __forceinline__ const float *blk(const float *M, int I, int J) {
-    return M + 16 * I * kLD + 16 * J;
-}
-__device__ __forceinline__ float *blk(float *M, int I, int J) { return M + 16 * I * kLD + 16 * J; }
-
-__device__ void unit_lower_inverse(const float *A, float *X, int tid) {
-    const int warp = tid >> 5, lane = tid & 31;
-    // 1) diagonal blocks, one column per thread
-    if (tid < 64) {
-        const int I = tid >> 4, jj = tid & 15, base = 16 * I;
-        float x[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            float s0 = 0.f, s1 = 0.f;
-#pragma unroll
-            for (int m = 0; m < i; ++m) {
-                if (m & 1) s1 = fmaf(A[(base + i) * kLD + base + m], x[m], s1);
-                else s0 = fmaf(A[(base + i) * kLD + base + m], x[m], s0);
-            }
-            x[i] = i < jj ? 0.f : (i == jj ? 1.f : -(s0 + s1));
-        }
-#pragma unroll
-        for (int i = 0; i < 16; ++i) X[(base + i) * kLD + base + jj] = x[i];
-    }
-    __syncthreads();
-    // 2) R_IJ = A_IJ X_JJ, stored in X's (I,J) block; warps 0..5
-    if (warp < 6) {
-        const int I = warp < 3 ? warp + 1 : (warp < 5 ? warp - 1 : 3);  // 1,2,3,2,3,3
-        const int J = warp < 3 ? 0 : (warp < 5 ? 1 : 2);                // 0,0,0,1,1,2
-        float acc[2][4] = {};
-        warp_mm16(acc, blk(A, I, J), blk(X, J, J), lane);
-        acc_store16(acc, blk(X, I, J), 1.f, lane);
-    }
-    __syncthreads();
-    // 3) block column J = warp (0..2), top to bottom
-    if (warp < 3) {
-        const int J = warp;
-        for (int I = J + 1; I < 4; ++I) {
-            float acc[2][4];
-            acc_load16(acc, blk(X, I, J), lane);  // R_IJ
-            for (int K = J + 1; K < I; ++K) warp_mm16(acc, blk(A, I, K), blk(X, K, J), lane);
-            __syncwarp();
-            acc_store16(acc, blk(X, I, J), 1.f, lane);  // Y
-            __syncwarp();
-            float out[2][4] = {};
-            warp_mm16(out, blk(X, I, I), blk(X, I, J), lane);
-            __syncwarp();
-            acc_store16(out, blk(X, I, J), -1.f, lane);
-            __syncwarp();
-        }
-    }
-    __syncthreads();
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -449,7 +334,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         tc_fence_before();
         __syncthreads();
         PHASE_MARK(2);
-        unit_lower_inverse(Af, Xf, tid);
+        ut::unit_lower_inverse(Af, Xf, tid);
         PHASE_MARK(3);
 #pragma unroll
         for (int u = 0; u < 8; ++u) {

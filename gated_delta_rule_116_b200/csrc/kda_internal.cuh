@@ -45,8 +45,10 @@ struct DecodeArgs {
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t s);
 cudaError_t launch_chunk_generic(const ChunkArgs &a, cudaStream_t s);
 cudaError_t launch_chunk_tc(const ChunkArgs &a, cudaStream_t s);
+cudaError_t launch_chunk_cluster(const ChunkArgs &a, cudaStream_t s);
 
 bool chunk_tc_supported(int dk, int dv, int chunk, int dtype);
+bool chunk_cluster_supported(int dk, int dv, int chunk, int dtype);
 size_t chunk_tc_workspace_bytes(int B, int T, int H);
 
 }  // namespace kda

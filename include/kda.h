@@ -55,9 +55,13 @@ typedef enum { KDA_BF16 = 0, KDA_F32 = 1 } kda_dtype;
 
 /* Which prefill engine kda_chunk_fwd_engine runs. */
 typedef enum {
-    KDA_ENGINE_AUTO = 0,     /* tensor-core engine where supported, else the generic one */
+    KDA_ENGINE_AUTO = 0,     /* cluster tensor-core engine where supported, else the generic one */
     KDA_ENGINE_GENERIC = 1,  /* fp32 CUDA-core chunked engine: any d_k, d_v <= 128, chunk 16/32/64 */
-    KDA_ENGINE_TC = 2        /* tcgen05/TMEM engine: bf16, d_k = d_v = 128, chunk = 64 */
+    KDA_ENGINE_TC = 2,       /* tcgen05/TMEM engine, one CTA per (b, h, 32 value columns):
+                                bf16, d_k = d_v = 128, chunk = 64 */
+    KDA_ENGINE_TC_CLUSTER = 3 /* tcgen05/TMEM engine, one 4-CTA cluster per (b, h): three
+                                CTAs build chunk operands, one runs the state chain;
+                                bf16, d_k = d_v = 128, chunk = 64 */
 } kda_engine;
 
 /*

@@ -21,7 +21,7 @@ DEV = "cuda"
 
 
 def engines(dtype, dk, dv, chunk):
-    return [e for e in ("generic", "tc") if kda.engine_supported(e, dk, dv, chunk, dtype)]
+    return [e for e in ("generic", "tc", "tc_cluster") if kda.engine_supported(e, dk, dv, chunk, dtype)]
 
 
 def run_gpu(inp, chunk, engine="auto", with_state=True):
