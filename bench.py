@@ -178,7 +178,8 @@ def run_ours(args, rank, world, device):
     w = I.WORKLOADS[PREFILL]
     inp = I.prefill_inputs(w, device=device)
     q, k, v, la, beta, S0 = (inp[x] for x in ("q", "k", "v", "log_alpha", "beta", "S0"))
-    engine = "tc" if kda.engine_supported("tc", w.dk, w.dv, w.chunk, w.dtype) else "generic"
+    engine = next(e for e in ("tc_cluster", "tc", "generic")
+                  if kda.engine_supported(e, w.dk, w.dv, w.chunk, w.dtype))
     out = torch.empty(w.B, w.T, w.H, w.dv, device=device, dtype=w.dtype)
     S_T = torch.empty(w.B, w.H, w.dk, w.dv, device=device, dtype=torch.float32)
     ws_n = kda.workspace_bytes(w.B, w.T, w.H, w.dk, w.dv, w.chunk, w.dtype)
@@ -234,7 +235,7 @@ def run_ours(args, rank, world, device):
             "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "bf16" if engine == "tc" else "f32",
+            "dtype": "f32" if engine == "generic" else "bf16",
             "data": "synthetic (seeded; recipe in kda_inputs.py)",
             "config": {"workload": PREFILL, "B": w.B, "T": w.T, "H": w.H, "dk": w.dk, "dv": w.dv,
                        "chunk": w.chunk, "inputs": "bf16 q/k/v, fp32 gates, fp32 S0/S_T",
@@ -346,7 +347,11 @@ def run_only(args, device):
         q, k, v, la, beta, S0 = (inp[x] for x in ("q", "k", "v", "log_alpha", "beta", "S0"))
         out = torch.empty(w.B, w.T, w.H, w.dv, device=device, dtype=w.dtype)
         S_T = torch.empty(w.B, w.H, w.dk, w.dv, device=device, dtype=torch.float32)
-        fn = lambda: kda.chunk_fwd(q, k, v, la, beta, S0, w.chunk, out=out, S_T=S_T, stream=stream)
+        ws_n = kda.workspace_bytes(w.B, w.T, w.H, w.dk, w.dv, w.chunk, w.dtype)
+        ws = torch.empty(max(ws_n, 1), device=device, dtype=torch.uint8) if ws_n else None
+        eng = args.engine or "auto"
+        fn = lambda: kda.chunk_fwd(q, k, v, la, beta, S0, w.chunk, out=out, S_T=S_T, engine=eng,
+                                   workspace=ws, stream=stream)
     else:
         w = I.WORKLOADS[DECODE]
         state = I.decode_state(w, device=device)
@@ -456,6 +461,8 @@ def main(argv=None):
     ap.add_argument("--only", choices=["prefill", "decode"],
                     help="profiling mode: run just this kernel's workload (warm-up + steps), "
                          "print its time, no JSON line")
+    ap.add_argument("--engine", default=None, choices=["auto", "generic", "tc", "tc_cluster"],
+                    help="with --only prefill: the prefill engine (default auto)")
     ap.add_argument("--workload", default=None,
                     help="with --only prefill: the prefill workload to run (default prefill_32k)")
     args = ap.parse_args(argv)

@@ -96,6 +96,8 @@ int kda_engine_supported(int engine, int dk, int dv, int chunk, int dtype) {
 
 size_t kda_workspace_bytes(int B, int T, int H, int dk, int dv, int chunk, int dtype) {
     if (B <= 0 || T <= 0 || H <= 0) return 0;
+    if (kda::chunk_cluster_supported(dk, dv, chunk, dtype))
+        return kda::chunk_cluster_workspace_bytes(B, H);
     if (kda::chunk_tc_supported(dk, dv, chunk, dtype)) return kda::chunk_tc_workspace_bytes(B, T, H);
     return 0;
 }
@@ -150,7 +152,8 @@ int kda_chunk_fwd_engine(int engine, const void *q, const void *k, const void *v
                      workspace, workspace_bytes, nullptr};
     cudaError_t e;
     if (use_tc || use_cluster) {
-        const size_t need = kda::chunk_tc_workspace_bytes(B, T, H);
+        const size_t need = use_cluster ? kda::chunk_cluster_workspace_bytes(B, H)
+                                        : kda::chunk_tc_workspace_bytes(B, T, H);
         if (need > 0 && (!workspace || workspace_bytes < need))
             return fail(KDA_ERR_WORKSPACE, "workspace of %zu bytes given, %zu needed",
                         workspace ? workspace_bytes : static_cast<size_t>(0), need);

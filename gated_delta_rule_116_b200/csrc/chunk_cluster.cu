@@ -12,13 +12,17 @@
 // the state (everything up to W, U', P, T, Qs, Kb) and the state chain, which
 // is sequential over chunks. One head runs on a cluster of 4 CTAs (4 SMs):
 //   * ranks 0..2 are producers: rank p computes the key-side part of chunks
-//     p, p+3, p+6, ... into a staging image of 82 KB in its shared memory and
-//     bulk-copies it (cp.async.bulk, shared::cta -> shared::cluster) into one
-//     of two slots of the consumer, completing on the slot's mbarrier;
+//     p, p+3, p+6, ... into an 82 KB image in its shared memory, bulk-stores
+//     it (cp.async.bulk shared -> global) into its own slot of a small ring in
+//     the workspace (it stays in L2) and arrives, across the cluster, on the
+//     consumer's "ready" barrier for that producer;
 //   * rank 3 is the consumer: it keeps the 128x128 fp32 state in registers and
-//     runs the chain for every chunk, on all 128 value columns, from the slots.
-//     When it is done with a slot it arms the slot's barrier for the next
-//     chunk and arrives (remotely) on the producer's "slot free" barrier.
+//     runs the chain for every chunk, on all 128 value columns. Its thread 0
+//     pulls published images into two shared-memory slots (bulk global ->
+//     shared loads) as soon as a slot is free, and tells the producer (its
+//     "loaded" barrier) that the ring slot may be reused.
+// The ring goes through L2 because a DSMEM bulk copy moves only ~20 B/cycle
+// between two SMs, whereas an L2 bulk load of the same 82 KB takes ~1K cycles.
 // A producer thus has three chunk periods for the key-side latency, and the
 // consumer's chunk period is the chain alone. Every wait is bounded; after a
 // timeout a CTA records an error in the device error word, stops waiting and
@@ -47,6 +51,7 @@ constexpr int kD = 128;
 constexpr int kThreads = 256;
 constexpr int kProducers = 3;
 constexpr int kCluster = kProducers + 1;
+constexpr int kRingSlots = 2 * kProducers;
 constexpr uint32_t kWaitLimit = 1u << 22;
 
 // ---- slot image: what a producer hands the consumer for one chunk
@@ -67,6 +72,12 @@ constexpr uint32_t P_KHT = 65536;      // K*F tf32, 4 K-blocks x 8 KB
 constexpr uint32_t kKHTBlk = 8192;
 constexpr uint32_t P_AF = 0;           // A (fp32), reuses the tf32 region after the product
 constexpr uint32_t P_XF = 64 * kLD * 4;
+// ... and after the UT solve, holds the TMA-loaded inputs of the producer's next chunk:
+constexpr uint32_t P_IN_Q = 0;         // q  [64 tokens][128] bf16
+constexpr uint32_t P_IN_K = 16384;     // k
+constexpr uint32_t P_IN_LA = 32768;    // log alpha [64][128] fp32
+constexpr uint32_t P_IN_V = 65536;     // v  [64][128] bf16
+constexpr uint32_t kInBytes = 81920;
 constexpr uint32_t P_STAGE = 98304;    // slot image being built
 constexpr uint32_t P_KSV = P_STAGE + kSlotStride;  // [Ks | V] fp16 [token][col], 4 blocks x 8 KB
 constexpr uint32_t P_VEC = P_KSV + 32768;          // beta[64], psum[4][128]
@@ -91,6 +102,26 @@ constexpr uint32_t IDESC_WU = tc::idesc(tc::kFmtF16, 128, 256, 0, 1);
 constexpr uint32_t IDESC_X = tc::idesc(tc::kFmtF16, 128, 128, 0, 1);   // A K-major, B MN-major
 constexpr uint32_t IDESC_S = tc::idesc(tc::kFmtF16, 128, 128, 1, 1);   // A MN-major, B MN-major
 
+#ifdef KDA_PHASE_TIMING
+// Debug builds only: cycles per phase summed over chunks, for cluster 0
+// (slots 0..9 producer rank 0, slots 16..23 the consumer).
+__device__ unsigned long long g_cluster_cycles[32];
+#define CMARK(idx)                                                        \
+    do {                                                                  \
+        if (blockIdx.x < kCluster && threadIdx.x == 0 && (idx) < 32) {    \
+            const unsigned long long now_ = clock64();                    \
+            g_cluster_cycles[idx] += now_ - t_prev_;                      \
+            t_prev_ = now_;                                               \
+        }                                                                 \
+    } while (0)
+#define CMARK_INIT unsigned long long t_prev_ = clock64()
+#else
+#define CMARK(idx) \
+    do {           \
+    } while (0)
+#define CMARK_INIT
+#endif
+
 struct Ctl {
     int *abort;
     int *err;
@@ -110,7 +141,7 @@ __device__ __forceinline__ void wait_cluster(uint64_t *bar, uint32_t parity, con
 }
 
 // ============================================================ producer
-__device__ void producer(uint8_t *sm, uint32_t tmem, int rank, const CUtensorMap *tm_q,
+__device__ void producer(uint8_t *sm, uint32_t tmem, int rank, uint8_t *ring, const CUtensorMap *tm_q,
                          const CUtensorMap *tm_k, const CUtensorMap *tm_la,
                          const CUtensorMap *tm_v, const __nv_bfloat16 *__restrict__ q,
                          const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *__restrict__ v,
@@ -125,40 +156,51 @@ __device__ void producer(uint8_t *sm, uint32_t tmem, int rank, const CUtensorMap
     float *Af = reinterpret_cast<float *>(sm + P_AF);
     float *Xf = reinterpret_cast<float *>(sm + P_XF);
     uint64_t *bar_mma = reinterpret_cast<uint64_t *>(sm + P_BAR);
-    uint64_t *bar_free = bar_mma + 1;
+    uint64_t *bar_loaded = bar_mma + 1;  // [2]: one per ring slot of this producer
     uint8_t *st = sm + P_STAGE;
-    uint32_t ph_mma = 0, ph_free = 0;
+    uint32_t ph_mma = 0;
+    int img = 0;  // index of this producer's next image
 
     const uint64_t d_kqt = tc::smem_desc(sbase + P_KQT, 16, 1024, tc::kSwizzle128);
     const uint64_t d_kht = tc::smem_desc(sbase + P_KHT, 16, 1024, tc::kSwizzle128);
     const uint64_t d_pt = tc::smem_desc(sbase + P_STAGE + SL_PT, 16, 1024, tc::kSwizzle128);
     const uint64_t d_ksv = tc::smem_desc(sbase + P_KSV, kTokBlk, 1024, tc::kSwizzle128);
-    // consumer-side addresses
-    const uint32_t cons = kCluster - 1;
-    const uint32_t c_base = tc::map_to_rank(sbase, cons);
-    const uint32_t c_full = tc::map_to_rank(sbase + C_BAR, cons);  // slot_full[0], [1]
+    // the consumer's "ready" barriers for this producer's two ring slots
+    const uint32_t c_ready = tc::map_to_rank(sbase + C_BAR + 40 + 16 * rank, kCluster - 1);
 
+    CMARK_INIT;
+    const int mk = rank == 0 ? 0 : 64;  // only rank 0 records (slots 0..8)
+    uint64_t *bar_in = bar_mma + 3;
+    uint32_t ph_in = 0;
+    auto load_inputs = [&](int cc) {   // TMA: the 64-token chunk cc of head h (all channels)
+        const int z = static_cast<int>(ztok + static_cast<long>(cc) * kC);
+        tc::mbar_arrive_expect_tx(bar_in, kInBytes);
+        tc::tma_load_3d(sm + P_IN_Q, tm_q, bar_in, 0, h, z);
+        tc::tma_load_3d(sm + P_IN_K, tm_k, bar_in, 0, h, z);
+        tc::tma_load_3d(sm + P_IN_LA, tm_la, bar_in, 0, h, z);
+        tc::tma_load_3d(sm + P_IN_V, tm_v, bar_in, 0, h, z);
+    };
+    if (tid == 0 && rank < nchunks) load_inputs(rank);
     for (int c = rank; c < nchunks; c += kProducers) {
         const int t0 = c * kC;
         const int valid = min(kC, T - t0);
         const long trow0 = ztok + t0;
-        if (tid == 0) {
-            tc::bulk_wait_read_all();  // the previous image has left the staging area
-            if (c + kProducers < nchunks) {
-                const int z = static_cast<int>(trow0 + kProducers * kC);
-                tc::tma_prefetch_l2_3d(tm_q, 0, h, z);
-                tc::tma_prefetch_l2_3d(tm_k, 0, h, z);
-                tc::tma_prefetch_l2_3d(tm_la, 0, h, z);
-                tc::tma_prefetch_l2_3d(tm_v, 0, h, z);
-            }
+        if (tid == 0 && c + 2 * kProducers < nchunks) {
+            const int z = static_cast<int>(trow0 + 2 * kProducers * kC);
+            tc::tma_prefetch_l2_3d(tm_q, 0, h, z);
+            tc::tma_prefetch_l2_3d(tm_k, 0, h, z);
+            tc::tma_prefetch_l2_3d(tm_la, 0, h, z);
+            tc::tma_prefetch_l2_3d(tm_v, 0, h, z);
         }
-        __syncthreads();
+        wait_local(bar_in, ph_in, ctl);
+        ph_in ^= 1;
+        CMARK(mk + 0);
 
         // ------------------------------------------------ gates and operands
         if (tid < kC) beta_s[tid] = tid < valid ? beta[(trow0 + tid) * H + h] : 0.f;
         {   // V (all 128 columns) -> fp16 columns 128..255 of the [Ks | V] operand
             const int t = tid >> 2, piece = tid & 3;
-            const uint4 *src = reinterpret_cast<const uint4 *>(v + ((trow0 + t) * H + h) * kD + 32 * piece);
+            const uint4 *src = reinterpret_cast<const uint4 *>(sm + P_IN_V + t * 256 + 64 * piece);
 #pragma unroll
             for (int m = 0; m < 4; ++m) {
                 uint4 w = make_uint4(0, 0, 0, 0);
@@ -179,11 +221,11 @@ __device__ void producer(uint8_t *sm, uint32_t tmem, int rank, const CUtensorMap
 #pragma unroll
         for (int u = 0; u < 16; ++u) {
             const int t = 16 * qq + u;
-            const long o = ((trow0 + t) * H + h) * kD + 2 * p;
             const bool ok = t < valid;
-            lg[u] = ok ? *reinterpret_cast<const float2 *>(log_alpha + o) : make_float2(0.f, 0.f);
-            qv[u] = ok ? *reinterpret_cast<const uint32_t *>(q + o) : 0u;
-            kv[u] = ok ? *reinterpret_cast<const uint32_t *>(k + o) : 0u;
+            lg[u] = ok ? *reinterpret_cast<const float2 *>(sm + P_IN_LA + t * 512 + 8 * p)
+                       : make_float2(0.f, 0.f);
+            qv[u] = ok ? *reinterpret_cast<const uint32_t *>(sm + P_IN_Q + t * 256 + 4 * p) : 0u;
+            kv[u] = ok ? *reinterpret_cast<const uint32_t *>(sm + P_IN_K + t * 256 + 4 * p) : 0u;
         }
         {
             float s0 = 0.f, s1 = 0.f;
@@ -192,7 +234,8 @@ __device__ void producer(uint8_t *sm, uint32_t tmem, int rank, const CUtensorMap
             psum[qq * 128 + 2 * p] = s0;
             psum[qq * 128 + 2 * p + 1] = s1;
         }
-        __syncthreads();
+        if (tid == 0) tc::bulk_wait_read_all();  // the previous image has left the staging area
+        __syncthreads();  // inputs are in registers: the tf32 tiles may now overwrite them
         {
             float pre0 = 0.f, pre1 = 0.f, tot0 = 0.f, tot1 = 0.f;
 #pragma unroll
@@ -241,6 +284,7 @@ __device__ void producer(uint8_t *sm, uint32_t tmem, int rank, const CUtensorMap
         }
         fence_proxy_async_smem();
         __syncthreads();
+        CMARK(mk + 1);
 
         // ------------------------------------------------ [A;P] (tf32)
         if (tid == 0) {
@@ -254,6 +298,7 @@ __device__ void producer(uint8_t *sm, uint32_t tmem, int rank, const CUtensorMap
         wait_local(bar_mma, ph_mma, ctl);
         ph_mma ^= 1;
         tc_fence_after();
+        CMARK(mk + 2);
 
         // ------------------------------------------------ A (fp32), P (fp16), UT solve, T (fp16)
         {
@@ -280,7 +325,9 @@ __device__ void producer(uint8_t *sm, uint32_t tmem, int rank, const CUtensorMap
         }
         tc_fence_before();
         __syncthreads();
+        CMARK(mk + 3);
         ut::unit_lower_inverse(Af, Xf, tid);
+        CMARK(mk + 4);
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
             const int e = tid + u * kThreads;
@@ -291,6 +338,9 @@ __device__ void producer(uint8_t *sm, uint32_t tmem, int rank, const CUtensorMap
         }
         fence_proxy_async_smem();
         __syncthreads();
+        // the tf32 region (tiles, A, X) is dead until the next chunk: stage its inputs there
+        if (tid == 0 && c + kProducers < nchunks) load_inputs(c + kProducers);
+        CMARK(mk + 5);
 
         // ------------------------------------------------ [W | U'] = T [Ks | V] (fp16, N = 256)
         if (tid == 0) {
@@ -303,6 +353,7 @@ __device__ void producer(uint8_t *sm, uint32_t tmem, int rank, const CUtensorMap
         wait_local(bar_mma, ph_mma, ctl);
         ph_mma ^= 1;
         tc_fence_after();
+        CMARK(mk + 6);
         if (quad >= 2) {
             const int i = row - 64;
 #pragma unroll
@@ -329,28 +380,29 @@ __device__ void producer(uint8_t *sm, uint32_t tmem, int rank, const CUtensorMap
         fence_proxy_async_smem();
         tc_fence_before();
         __syncthreads();
+        CMARK(mk + 7);
 
-        // ------------------------------------------------ hand the image to the consumer
+        // ------------------------------------------------ publish the image through L2
         if (tid == 0) {
-            wait_cluster(bar_free, ph_free, ctl);
-            const uint32_t s = c & 1;
-            const uint32_t dst = c_base + C_SLOT + s * kSlotStride;
-            const uint32_t full = c_full + s * 8;
+            const int b = img & 1;  // ring slot of this image; image img-2 used it before
+            if (img >= 2) wait_cluster(bar_loaded + b, ((img >> 1) - 1) & 1, ctl);
+            CMARK(mk + 9);
             if (!*reinterpret_cast<volatile int *>(ctl.abort)) {
-                tc::bulk_copy_to_peer(dst + SL_QW, st + SL_QW, 32768, full);
-                tc::bulk_copy_to_peer(dst + SL_KB, st + SL_KB, 16384, full);
-                tc::bulk_copy_to_peer(dst + SL_PT, st + SL_PT, 16384, full);
-                tc::bulk_copy_to_peer(dst + SL_UP, st + SL_UP, kSlotBytes - SL_UP, full);
+                tc::bulk_store_global(ring + (2 * rank + b) * kSlotStride, st, kSlotBytes);
                 tc::bulk_commit();
+                tc::bulk_wait_all();
+                tc::fence_proxy_async_global();
+                tc::mbar_arrive_remote(c_ready + 8 * b);
             }
         }
-        ph_free ^= 1;
+        CMARK(mk + 8);
+        ++img;
     }
     if (tid == 0) tc::bulk_wait_read_all();
 }
 
 // ============================================================ consumer
-__device__ void consumer(uint8_t *sm, uint32_t tmem, const float *__restrict__ S0,
+__device__ void consumer(uint8_t *sm, uint32_t tmem, const uint8_t *ring, const float *__restrict__ S0,
                          __nv_bfloat16 *__restrict__ out, float *__restrict__ S_T, int T, int H,
                          int h, long bh, long ztok, int nchunks, const Ctl &ctl) {
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -361,12 +413,42 @@ __device__ void consumer(uint8_t *sm, uint32_t tmem, const float *__restrict__ S
     uint64_t *bar_x = full + 2;
     uint64_t *bar_s = full + 3;
     uint64_t *bar_o = full + 4;
+    uint64_t *ready = full + 5;  // [6]: producer p, ring slot b at ready[2p + b]
     uint32_t ph_full[2] = {0, 0};
     uint32_t ph_x = 0, ph_s = 0, ph_o = 0;
 
     const uint64_t d_s16 = tc::smem_desc(sbase + C_S16, 16384, 1024, tc::kSwizzle128);
     const uint64_t d_u16 = tc::smem_desc(sbase + C_U16, kTokBlk, 1024, tc::kSwizzle128);
-    const uint32_t p_free = sbase + P_BAR + 8;  // producer's "slot free" barrier (same offset)
+    uint64_t d_qw[2], d_kb[2], d_pt[2];
+#pragma unroll
+    for (int s = 0; s < 2; ++s) {
+        const uint32_t sl = sbase + C_SLOT + s * kSlotStride;
+        d_qw[s] = tc::smem_desc(sl + SL_QW, 16, 1024, tc::kSwizzle128);
+        d_kb[s] = tc::smem_desc(sl + SL_KB, kTokBlk, 1024, tc::kSwizzle128);
+        d_pt[s] = tc::smem_desc(sl + SL_PT, 16, 1024, tc::kSwizzle128);
+    }
+    const uint32_t p_loaded = sbase + P_BAR + 8;  // producers' "loaded" barrier (same offset)
+
+    // Thread 0 pulls published images: chunks next_load .. limit (their slots are free).
+    int next_load = 0;
+    auto pull = [&](int limit, bool block) {
+        while (next_load <= limit && next_load < nchunks) {
+            const int pc = next_load % kProducers, j = next_load / kProducers;
+            const int rs = 2 * pc + (j & 1);  // ring slot (and its ready barrier)
+            const uint32_t par = (j >> 1) & 1;
+            if (block)
+                wait_cluster(ready + rs, par, ctl);
+            else if (!tc::mbar_test_cluster(ready + rs, par))
+                return;
+            if (*reinterpret_cast<volatile int *>(ctl.abort)) return;
+            tc::fence_proxy_async_global();
+            const int sl = next_load & 1;
+            tc::mbar_arrive_expect_tx(full + sl, kSlotBytes);
+            tc::bulk_load_global(sm + C_SLOT + sl * kSlotStride, ring + rs * kSlotStride, kSlotBytes,
+                                 full + sl);
+            ++next_load;
+        }
+    };
 
     // fp32 state: row `row`, columns half*64 .. +64
     float S[64];
@@ -384,32 +466,25 @@ __device__ void consumer(uint8_t *sm, uint32_t tmem, const float *__restrict__ S
             *reinterpret_cast<uint4 *>(sm + C_S16 + half * 16384 + sw128k_off(row, u, 0)) = x;
         }
     };
+    auto issue_x = [&](int c) {   // X[c&1] = [Qs;W] S16
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+            mma_f16(tmem + CCOL_X + (c & 1) * 128, d_qw[c & 1] + (((kk >> 2) * kQWBlk + (kk & 3) * 32) >> 4),
+                    d_s16 + ((kk * 2048) >> 4), IDESC_X, kk > 0);
+        tc::mma_commit(bar_x);
+    };
     write_s16();
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
-    if (tid == 0) {
-        // slots start free: arm both and release chunks 0 and 1 to their producers
-        for (int s = 0; s < 2 && s < nchunks; ++s) {
-            tc::mbar_arrive_expect_tx(full + s, kSlotBytes);
-            tc::mbar_arrive_remote(tc::map_to_rank(p_free, s % kProducers));
-        }
-    }
-    auto issue_x = [&](int c) {   // X[c&1] = [Qs;W] S16
-        const uint32_t slot = C_SLOT + (c & 1) * kSlotStride;
-        const uint64_t d_qw = tc::smem_desc(sbase + slot + SL_QW, 16, 1024, tc::kSwizzle128);
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-            mma_f16(tmem + CCOL_X + (c & 1) * 128, d_qw + (((kk >> 2) * kQWBlk + (kk & 3) * 32) >> 4),
-                    d_s16 + ((kk * 2048) >> 4), IDESC_X, kk > 0);
-        tc::mma_commit(bar_x);
-    };
+    if (tid == 0) pull(0, true);
     if (nchunks > 0) {
         wait_local(full, ph_full[0], ctl);
         if (tid == 0) issue_x(0);
     }
 
+    CMARK_INIT;
     for (int c = 0; c < nchunks; ++c) {
         const int s = c & 1;
         const int t0 = c * kC;
@@ -418,9 +493,19 @@ __device__ void consumer(uint8_t *sm, uint32_t tmem, const float *__restrict__ S
         const uint32_t xcol = CCOL_X + s * 128;
         wait_local(full + s, ph_full[s], ctl);  // (already complete) makes the slot visible
         ph_full[s] ^= 1;
+        if (tid == 0 && c + 2 * kProducers < nchunks)  // the ring slot of chunk c is reusable
+            tc::mbar_arrive_remote(tc::map_to_rank(p_loaded + 8 * ((c / kProducers) & 1), c % kProducers));
+        CMARK(16);
+#ifdef KDA_PHASE_TIMING
+        const unsigned long long w0_ = clock64();
+#endif
         wait_local(bar_x, ph_x, ctl);
         ph_x ^= 1;
         tc_fence_after();
+#ifndef KDA_NO_EARLY_PULL
+        if (tid == 0) pull(c + 1, false);
+#endif
+        CMARK(17);
 
         // U = U' - W S  (lanes 64..127 = tokens)
         if (quad >= 2) {
@@ -447,26 +532,29 @@ __device__ void consumer(uint8_t *sm, uint32_t tmem, const float *__restrict__ S
         }
         fence_proxy_async_smem();
         tc_fence_before();
+#ifdef KDA_PHASE_TIMING
+        if (blockIdx.x == kCluster - 1 && (threadIdx.x & 31) == 0)
+            atomicAdd(&g_cluster_cycles[24 + (threadIdx.x >> 5)], clock64() - w0_);
+#endif
         __syncthreads();
+        CMARK(18);
         if (tid == 0) {
             tc_fence_after();
-            const uint64_t d_kb = tc::smem_desc(sbase + C_SLOT + s * kSlotStride + SL_KB, kTokBlk, 1024,
-                                                tc::kSwizzle128);
-            const uint64_t d_pt = tc::smem_desc(sbase + C_SLOT + s * kSlotStride + SL_PT, 16, 1024,
-                                                tc::kSwizzle128);
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
-                mma_f16(tmem + CCOL_S, d_kb + ((kk * 2048) >> 4), d_u16 + ((kk * 2048) >> 4), IDESC_S, kk > 0);
+                mma_f16(tmem + CCOL_S, d_kb[s] + ((kk * 2048) >> 4), d_u16 + ((kk * 2048) >> 4), IDESC_S, kk > 0);
             tc::mma_commit(bar_s);
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
-                mma_f16(tmem + xcol, d_pt + ((kk * 32) >> 4), d_u16 + ((kk * 2048) >> 4), IDESC_X, 1);
+                mma_f16(tmem + xcol, d_pt[s] + ((kk * 32) >> 4), d_u16 + ((kk * 2048) >> 4), IDESC_X, 1);
             tc::mma_commit(bar_o);
+            pull(c + 1, false);
         }
         // S <- Diag(e^{g_C}) S + Kb^T U
         wait_local(bar_s, ph_s, ctl);
         ph_s ^= 1;
         tc_fence_after();
+        CMARK(19);
         {
             const float gm = reinterpret_cast<const float *>(slot + SL_GAM)[row];
             float sv[64];
@@ -481,14 +569,18 @@ __device__ void consumer(uint8_t *sm, uint32_t tmem, const float *__restrict__ S
         fence_proxy_async_smem();
         tc_fence_before();
         __syncthreads();
+        CMARK(20);
         if (c + 1 < nchunks) {
+            if (tid == 0) pull(c + 1, true);
             wait_local(full + (s ^ 1), ph_full[s ^ 1], ctl);
             if (tid == 0) issue_x(c + 1);
         }
+        CMARK(21);
         // O = Qs S + P U  (lanes 0..63 = tokens)
         wait_local(bar_o, ph_o, ctl);
         ph_o ^= 1;
         tc_fence_after();
+        CMARK(22);
         if (quad < 2) {
             float o[64];
             const uint32_t ta = tc::tmem_addr(tmem, 32 * quad, xcol + half * 64);
@@ -510,10 +602,8 @@ __device__ void consumer(uint8_t *sm, uint32_t tmem, const float *__restrict__ S
         }
         tc_fence_before();
         __syncthreads();
-        if (tid == 0 && c + 2 < nchunks && !*reinterpret_cast<volatile int *>(ctl.abort)) {
-            tc::mbar_arrive_expect_tx(full + s, kSlotBytes);
-            tc::mbar_arrive_remote(tc::map_to_rank(p_free, (c + 2) % kProducers));
-        }
+        if (tid == 0) pull(c + 2, false);  // the slot of chunk c is free
+        CMARK(23);
     }
     if (S_T) {
 #pragma unroll
@@ -527,7 +617,8 @@ chunk_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                      const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
                      const __nv_bfloat16 *__restrict__ v, const float *__restrict__ log_alpha,
                      const float *__restrict__ beta, const float *__restrict__ S0,
-                     __nv_bfloat16 *__restrict__ out, float *__restrict__ S_T, int T, int H, int *err) {
+                     __nv_bfloat16 *__restrict__ out, float *__restrict__ S_T, uint8_t *__restrict__ ws,
+                     int T, int H, int *err) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~static_cast<uintptr_t>(1023));
@@ -539,12 +630,12 @@ chunk_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     const bool is_consumer = rank == kCluster - 1;
     const uint32_t bar_off = is_consumer ? C_BAR : P_BAR;
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + bar_off);
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + bar_off + 64);
-    int *abort = reinterpret_cast<int *>(sm + bar_off + 68);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + bar_off + 96);
+    int *abort = reinterpret_cast<int *>(sm + bar_off + 100);
     const int tid = threadIdx.x;
 
     if (tid == 0) {
-        for (int i = 0; i < 5; ++i) tc::mbar_init(bars + i, 1);
+        for (int i = 0; i < 11; ++i) tc::mbar_init(bars + i, 1);
         *abort = 0;
         tc::fence_mbar_init();
     }
@@ -559,11 +650,12 @@ chunk_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     const uint32_t tmem = *tmem_slot;
     const Ctl ctl{abort, err};
 
+    uint8_t *ring = ws + bh * kRingSlots * kSlotStride;  // this head's ring: two slots per producer
     if (is_consumer)
-        consumer(sm, tmem, S0, out, S_T, T, H, h, bh, ztok, nchunks, ctl);
+        consumer(sm, tmem, ring, S0, out, S_T, T, H, h, bh, ztok, nchunks, ctl);
     else
-        producer(sm, tmem, rank, &tm_q, &tm_k, &tm_la, &tm_v, q, k, v, log_alpha, beta, T, H, h, ztok,
-                 nchunks, ctl);
+        producer(sm, tmem, rank, ring, &tm_q, &tm_k, &tm_la, &tm_v, q, k, v, log_alpha, beta, T, H, h,
+                 ztok, nchunks, ctl);
 
     tc_fence_before();
     __syncthreads();
@@ -609,8 +701,23 @@ bool make_map(CUtensorMap *m, const void *ptr, CUtensorMapDataType dt, int esize
 
 }  // namespace
 
+#ifdef KDA_PHASE_TIMING
+extern "C" int kda_debug_cluster_cycles(unsigned long long *out32, int reset) {
+    cudaError_t e = cudaMemcpyFromSymbol(out32, g_cluster_cycles, sizeof(unsigned long long) * 32);
+    if (reset) {
+        unsigned long long z[32] = {0};
+        cudaMemcpyToSymbol(g_cluster_cycles, z, sizeof z);
+    }
+    return e == cudaSuccess ? 0 : -1;
+}
+#endif
+
 bool chunk_cluster_supported(int dk, int dv, int chunk, int dtype) {
     return dtype == KDA_BF16 && dk == kD && dv == kD && chunk == kC;
+}
+
+size_t chunk_cluster_workspace_bytes(int B, int H) {
+    return static_cast<size_t>(B) * H * kRingSlots * kSlotStride;
 }
 
 cudaError_t launch_chunk_cluster(const ChunkArgs &a, cudaStream_t s) {
@@ -629,8 +736,8 @@ cudaError_t launch_chunk_cluster(const ChunkArgs &a, cudaStream_t s) {
     chunk_cluster_kernel<<<grid, kThreads, kSmemBytes, s>>>(
         mq, mk, mla, mv, static_cast<const __nv_bfloat16 *>(a.q),
         static_cast<const __nv_bfloat16 *>(a.k), static_cast<const __nv_bfloat16 *>(a.v),
-        a.log_alpha, a.beta, a.S0, static_cast<__nv_bfloat16 *>(a.out), a.S_T, a.T, a.H,
-        a.device_error);
+        a.log_alpha, a.beta, a.S0, static_cast<__nv_bfloat16 *>(a.out), a.S_T,
+        static_cast<uint8_t *>(a.workspace), a.T, a.H, a.device_error);
     return cudaGetLastError();
 }
 

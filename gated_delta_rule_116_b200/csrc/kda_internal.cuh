@@ -50,5 +50,6 @@ cudaError_t launch_chunk_cluster(const ChunkArgs &a, cudaStream_t s);
 bool chunk_tc_supported(int dk, int dv, int chunk, int dtype);
 bool chunk_cluster_supported(int dk, int dv, int chunk, int dtype);
 size_t chunk_tc_workspace_bytes(int B, int T, int H);
+size_t chunk_cluster_workspace_bytes(int B, int H);
 
 }  // namespace kda
