@@ -61,6 +61,17 @@ int check_common(int dk, int dv, int dtype) {
 
 }  // namespace
 
+namespace kda {
+int set_error_detail(int code, const char *fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_detail, sizeof g_detail, fmt, ap);
+    va_end(ap);
+    return code;
+}
+int *device_error_word() { return device_error_ptr(); }
+}  // namespace kda
+
 extern "C" {
 
 int kda_version(void) { return 10000; }

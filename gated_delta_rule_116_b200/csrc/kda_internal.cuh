@@ -47,6 +47,11 @@ cudaError_t launch_chunk_generic(const ChunkArgs &a, cudaStream_t s);
 cudaError_t launch_chunk_tc(const ChunkArgs &a, cudaStream_t s);
 cudaError_t launch_chunk_cluster(const ChunkArgs &a, cudaStream_t s);
 
+// Records `fmt` as the calling thread's kda_last_error_detail() and returns code.
+int set_error_detail(int code, const char *fmt, ...);
+// Device address of the word kernels set when a bounded wait gives up (nullptr on error).
+int *device_error_word();
+
 bool chunk_tc_supported(int dk, int dv, int chunk, int dtype);
 bool chunk_cluster_supported(int dk, int dv, int chunk, int dtype);
 size_t chunk_tc_workspace_bytes(int B, int T, int H);

@@ -138,6 +138,29 @@ int kda_recurrent_step(const void *q, const void *k, const void *v,
                        float *state, const int32_t *slot, void *out,
                        int N, int H, int dk, int dv, int dtype, void *stream);
 
+/*
+ * Chunked prefill that allocates nothing and takes no workspace: the same
+ * computation as kda_chunk_fwd_engine(KDA_ENGINE_TC_CLUSTER, ...), whose
+ * scratch (the ring of per-chunk operand images) lives in a fixed device
+ * array of this library. The pages have no counterpart of this call; it exists
+ * for callers that cannot allocate device memory at call time, e.g. a serving
+ * process whose pool allocator owns all free memory, or a plug-in inside a
+ * framework that owns every allocation.
+ *   Arguments as kda_chunk_fwd without the workspace; supported: bf16,
+ *   dk = dv = 128, chunk = 64, and B * H <= 32 heads (larger problems return
+ *   KDA_ERR_UNSUPPORTED and must use kda_chunk_fwd).
+ *   Every GPU that loads the library holds the array (15.2 MiB) until exit.
+ *   The first call on a device looks up the array's address with that device
+ *   current; make it before any stream capture. All calls share the array:
+ *   calls that overlap on the GPU race and must be serialised by the caller.
+ *   No cudaMalloc, cudaFree or allocating library routine is called.
+ */
+int kda_chunk_fwd_static(const void *q, const void *k, const void *v,
+                         const float *log_alpha, const float *beta, const float *S0,
+                         void *out, float *S_T,
+                         int B, int T, int H, int dk, int dv, int chunk, int dtype,
+                         void *stream);
+
 /* Human-readable name of a kda_status code (static string). */
 const char *kda_strerror(int code);
 
