@@ -202,12 +202,8 @@ def run_ours(args, rank, world, device):
         t1.record(stream)
         torch.cuda.synchronize(device)
     barrier(world)
-    ms_total = t0.elapsed_time(t1)
     ms_kernel = statistics.mean(s.elapsed_time(e) for s, e in evs)
-    ms_total = max_over_ranks(ms_total, world, device)
-    ms_step = ms_total / args.steps
-    tokens = w.tokens * world
-    value = tokens / (ms_total / args.steps / 1e3)
+    value, ms_step = weak_scaling_rate(w.tokens, t0.elapsed_time(t1), world, device, args.steps)
 
     # roofline of the dominant kernel (the prefill kernel; one launch per step)
     hbm, hbm_src = peaks()
@@ -280,8 +276,8 @@ def run_e2e(kda, w, inp, engine, ws, args, device, stream, world):
         step()
     t1.record(stream)
     torch.cuda.synchronize(device)
-    ms = max_over_ranks(t0.elapsed_time(t1), world, device) / n
-    return {"value": round(w.tokens * world / (ms / 1e3), 1), "unit": "tokens/s",
+    rate, ms = weak_scaling_rate(w.tokens, t0.elapsed_time(t1), world, device, n)
+    return {"value": round(rate, 1), "unit": "tokens/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(ms, 3),
             "steps": n}
 
@@ -316,7 +312,7 @@ def run_decode(kda, args, device, stream, world):
         per.append((a, b))
     t1.record(stream)
     torch.cuda.synchronize(device)
-    ms_total = max_over_ranks(t0.elapsed_time(t1), world, device)
+    tok_rate, ms_loop = weak_scaling_rate(w.N, t0.elapsed_time(t1), world, device, n_steps)
     kern = sorted(a.elapsed_time(b) for a, b in per)
     med = kern[len(kern) // 2]
     hbm, src = peaks()
@@ -325,13 +321,13 @@ def run_decode(kda, args, device, stream, world):
     return {"workload": DECODE, "steps": n_steps, "us_per_step_median": round(med * 1e3, 2),
             "us_per_step_p10": round(kern[len(kern) // 10] * 1e3, 2),
             "us_per_step_p90": round(kern[(9 * len(kern)) // 10] * 1e3, 2),
-            "us_per_step_loop": round(ms_total / n_steps * 1e3, 2),
+            "us_per_step_loop": round(ms_loop * 1e3, 2),
             "state_bytes_per_step": bytes_step, "state_GBps": round(gbs, 1),
             "frac_of_8TBps": round(gbs / NOMINAL_HBM_GBS, 4),
             "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm, "unit": "GB/s",
                          "frac": round(gbs / hbm, 4), "peak_source": src,
                          "traffic": traffic_from_profiles("decode")},
-            "tokens_per_s": round(w.N * world / (ms_total / n_steps / 1e3), 1),
+            "tokens_per_s": round(tok_rate, 1),
             "launches": n_steps}
 
 
@@ -443,6 +439,13 @@ def max_over_ranks(x, world, device):
     t = torch.tensor([x], device=device, dtype=torch.float64)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
+
+
+def weak_scaling_rate(units_per_rank, ms_local, world, device, steps=1):
+    """Whole-job rate when every rank does the same work: the units of all ranks
+    over the slowest rank's time. Returns (units per second, slowest ms per step)."""
+    ms_step = max_over_ranks(ms_local, world, device) / steps
+    return units_per_rank * world / (ms_step / 1e3), ms_step
 
 
 def main(argv=None):
