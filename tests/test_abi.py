@@ -85,6 +85,18 @@ def test_chunk_rejects(lib, kw, code):
     assert detail(lib)
 
 
+@pytest.mark.parametrize("engine", [0, 3])
+def test_chunk_workspace_missing_or_short(lib, engine):
+    """The cluster engine (also what engine 0 picks for this shape) needs a workspace of
+    kda_workspace_bytes(); without one, or with fewer bytes, the call fails on the
+    host with KDA_ERR_WORKSPACE before any launch."""
+    need = lib.kda_workspace_bytes(1, 64, 2, 128, 128, 64, 0)
+    assert need > 0
+    assert chunk(lib, engine=engine) == -4
+    assert "workspace" in detail(lib)
+    assert chunk(lib, engine=engine, ws=FAKE, wsb=need - 16) == -4
+
+
 def test_chunk_empty_batch_is_noop(lib):
     assert chunk(lib, B=0, q=None, k=None, v=None, la=None, beta=None, out=None) == 0
     assert chunk(lib, H=0, q=None, k=None, v=None, la=None, beta=None, out=None) == 0

@@ -121,6 +121,20 @@ def test_bf16_chunk_size_invariance(chunk):
         compare(inp, out, st, *ref)
 
 
+def test_bf16_initial_state_in_place():
+    """S_T may alias S0: each engine reads a head's initial state before writing its final one."""
+    inp = I.prefill_inputs("prefill_32k", T=150, H=3, B=2)
+    ref_out, ref_st = run_oracle(inp)
+    for eng in engines(torch.bfloat16, 128, 128, 64):
+        g = {k: (v.to(DEV) if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
+        state = g["S0"].clone()
+        out, st = kda.chunk_fwd(g["q"], g["k"], g["v"], g["log_alpha"], g["beta"], state,
+                                chunk=64, engine=eng, S_T=state)
+        torch.cuda.synchronize()
+        assert st.data_ptr() == state.data_ptr()
+        compare(inp, out, st, ref_out, ref_st)
+
+
 def test_zero_length_copies_state():
     inp = I.prefill_inputs("fp32_small", T=0, s0_std=1.0)
     out, st = run_gpu(inp, 16)
