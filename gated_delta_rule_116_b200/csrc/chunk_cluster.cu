@@ -493,8 +493,12 @@ __device__ void consumer(uint8_t *sm, uint32_t tmem, const uint8_t *ring, const 
         const uint32_t xcol = CCOL_X + s * 128;
         wait_local(full + s, ph_full[s], ctl);  // (already complete) makes the slot visible
         ph_full[s] ^= 1;
-        if (tid == 0 && c + 2 * kProducers < nchunks)  // the ring slot of chunk c is reusable
-            tc::mbar_arrive_remote(tc::map_to_rank(p_loaded + 8 * ((c / kProducers) & 1), c % kProducers));
+        if (tid == 0 && c + 2 * kProducers < nchunks) {  // the ring slot of chunk c is reusable
+            // relaxed: the slot's bulk load has completed (observed above); no writes of
+            // this thread need to be ordered before the producer's reuse of the slot
+            const uint32_t rb = tc::map_to_rank(p_loaded + 8 * ((c / kProducers) & 1), c % kProducers);
+            asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(rb) : "memory");
+        }
         CMARK(16);
 #ifdef KDA_PHASE_TIMING
         const unsigned long long w0_ = clock64();
