@@ -414,19 +414,18 @@ __device__ void consumer(uint8_t *sm, uint32_t tmem, const uint8_t *ring, const 
     uint64_t *bar_s = full + 3;
     uint64_t *bar_o = full + 4;
     uint64_t *ready = full + 5;  // [6]: producer p, ring slot b at ready[2p + b]
-    uint32_t ph_full[2] = {0, 0};
+    uint32_t ph_full = 0;   // bit s: parity of slot s's next fill
     uint32_t ph_x = 0, ph_s = 0, ph_o = 0;
 
     const uint64_t d_s16 = tc::smem_desc(sbase + C_S16, 16384, 1024, tc::kSwizzle128);
     const uint64_t d_u16 = tc::smem_desc(sbase + C_U16, kTokBlk, 1024, tc::kSwizzle128);
-    uint64_t d_qw[2], d_kb[2], d_pt[2];
-#pragma unroll
-    for (int s = 0; s < 2; ++s) {
-        const uint32_t sl = sbase + C_SLOT + s * kSlotStride;
-        d_qw[s] = tc::smem_desc(sl + SL_QW, 16, 1024, tc::kSwizzle128);
-        d_kb[s] = tc::smem_desc(sl + SL_KB, kTokBlk, 1024, tc::kSwizzle128);
-        d_pt[s] = tc::smem_desc(sl + SL_PT, 16, 1024, tc::kSwizzle128);
-    }
+    // Operand descriptors of slot 0; slot 1 is kSlotStride bytes further. They are
+    // selected arithmetically so that they stay in registers (an array indexed by the
+    // slot would live in local memory and be reloaded before every MMA).
+    const uint64_t d_qw0 = tc::smem_desc(sbase + C_SLOT + SL_QW, 16, 1024, tc::kSwizzle128);
+    const uint64_t d_kb0 = tc::smem_desc(sbase + C_SLOT + SL_KB, kTokBlk, 1024, tc::kSwizzle128);
+    const uint64_t d_pt0 = tc::smem_desc(sbase + C_SLOT + SL_PT, 16, 1024, tc::kSwizzle128);
+    constexpr uint64_t kSlotDesc = kSlotStride >> 4;   // slot stride in descriptor units
     const uint32_t p_loaded = sbase + P_BAR + 8;  // producers' "loaded" barrier (same offset)
 
     // Thread 0 pulls published images: chunks next_load .. limit (their slots are free).
@@ -470,7 +469,7 @@ __device__ void consumer(uint8_t *sm, uint32_t tmem, const uint8_t *ring, const 
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-            mma_f16(tmem + CCOL_X + (c & 1) * 128, d_qw[c & 1] + (((kk >> 2) * kQWBlk + (kk & 3) * 32) >> 4),
+            mma_f16(tmem + CCOL_X + (c & 1) * 128, d_qw0 + (c & 1) * kSlotDesc + (((kk >> 2) * kQWBlk + (kk & 3) * 32) >> 4),
                     d_s16 + ((kk * 2048) >> 4), IDESC_X, kk > 0);
         tc::mma_commit(bar_x);
     };
@@ -480,7 +479,7 @@ __device__ void consumer(uint8_t *sm, uint32_t tmem, const uint8_t *ring, const 
     __syncthreads();
     if (tid == 0) pull(0, true);
     if (nchunks > 0) {
-        wait_local(full, ph_full[0], ctl);
+        wait_local(full, ph_full & 1, ctl);
         if (tid == 0) issue_x(0);
     }
 
@@ -491,8 +490,8 @@ __device__ void consumer(uint8_t *sm, uint32_t tmem, const uint8_t *ring, const 
         const int valid = min(kC, T - t0);
         const uint8_t *slot = sm + C_SLOT + s * kSlotStride;
         const uint32_t xcol = CCOL_X + s * 128;
-        wait_local(full + s, ph_full[s], ctl);  // (already complete) makes the slot visible
-        ph_full[s] ^= 1;
+        wait_local(full + s, (ph_full >> s) & 1, ctl);  // (already complete) makes the slot visible
+        ph_full ^= 1u << s;
         if (tid == 0 && c + 2 * kProducers < nchunks) {  // the ring slot of chunk c is reusable
             // relaxed: the slot's bulk load has completed (observed above); no writes of
             // this thread need to be ordered before the producer's reuse of the slot
@@ -546,11 +545,11 @@ __device__ void consumer(uint8_t *sm, uint32_t tmem, const uint8_t *ring, const 
             tc_fence_after();
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
-                mma_f16(tmem + CCOL_S, d_kb[s] + ((kk * 2048) >> 4), d_u16 + ((kk * 2048) >> 4), IDESC_S, kk > 0);
+                mma_f16(tmem + CCOL_S, d_kb0 + s * kSlotDesc + ((kk * 2048) >> 4), d_u16 + ((kk * 2048) >> 4), IDESC_S, kk > 0);
             tc::mma_commit(bar_s);
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
-                mma_f16(tmem + xcol, d_pt[s] + ((kk * 32) >> 4), d_u16 + ((kk * 2048) >> 4), IDESC_X, 1);
+                mma_f16(tmem + xcol, d_pt0 + s * kSlotDesc + ((kk * 32) >> 4), d_u16 + ((kk * 2048) >> 4), IDESC_X, 1);
             tc::mma_commit(bar_o);
             pull(c + 1, false);
         }
@@ -576,7 +575,7 @@ __device__ void consumer(uint8_t *sm, uint32_t tmem, const uint8_t *ring, const 
         CMARK(20);
         if (c + 1 < nchunks) {
             if (tid == 0) pull(c + 1, true);
-            wait_local(full + (s ^ 1), ph_full[s ^ 1], ctl);
+            wait_local(full + (s ^ 1), (ph_full >> (s ^ 1)) & 1, ctl);
             if (tid == 0) issue_x(c + 1);
         }
         CMARK(21);
