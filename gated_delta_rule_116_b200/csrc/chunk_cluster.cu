@@ -12,10 +12,14 @@
 // the state (everything up to W, U', P, T, Qs, Kb) and the state chain, which
 // is sequential over chunks. One head runs on a cluster of 4 CTAs (4 SMs):
 //   * ranks 0..2 are producers: rank p computes the key-side part of chunks
-//     p, p+3, p+6, ... into an 82 KB image in its shared memory, bulk-stores
-//     it (cp.async.bulk shared -> global) into its own slot of a small ring in
-//     the workspace (it stays in L2) and arrives, across the cluster, on the
-//     consumer's "ready" barrier for that producer;
+//     p, p+3, p+6, ... as an 82 KB image and writes it into one of its three
+//     slots of a small ring in the workspace (it stays in L2): Qs, Kb and
+//     e^{g_C} straight from registers in the gate prologue; [P;T] (an operand
+//     of its own MMA), W and U' staged in shared memory and bulk-stored
+//     (cp.async.bulk shared -> global), [P;T] as soon as T is formed. Once the
+//     stores are complete, thread 0 arrives (release, cluster scope; the
+//     generic stores of all threads precede it through a CTA barrier) on the
+//     consumer's "ready" barrier of that slot;
 //   * rank 3 is the consumer: it keeps the 128x128 fp32 state in registers and
 //     runs the chain for every chunk, on all 128 value columns. Its thread 0
 //     pulls published images into two shared-memory slots (bulk global ->
@@ -23,6 +27,9 @@
 //     "loaded" barrier) that the ring slot may be reused.
 // The ring goes through L2 because a DSMEM bulk copy moves only ~20 B/cycle
 // between two SMs, whereas an L2 bulk load of the same 82 KB takes ~1K cycles.
+// The producers set the pace of the cluster, so their image stores are kept
+// short: writing Qs and Kb from registers and storing [P;T] early leaves only
+// W and U' (32 KB) to store and wait for at the end of an image.
 // A producer thus has three chunk periods for the key-side latency, and the
 // consumer's chunk period is the chain alone. Every wait is bounded; after a
 // timeout a CTA records an error in the device error word, stops waiting and
@@ -51,7 +58,8 @@ constexpr int kD = 128;
 constexpr int kThreads = 256;
 constexpr int kProducers = 3;
 constexpr int kCluster = kProducers + 1;
-constexpr int kRingSlots = 2 * kProducers;
+constexpr int kRingDepth = 3;   // ring slots per producer
+constexpr int kRingSlots = kRingDepth * kProducers;
 constexpr uint32_t kWaitLimit = 1u << 22;
 
 // ---- slot image: what a producer hands the consumer for one chunk
@@ -64,6 +72,7 @@ constexpr uint32_t SL_GAM = 81920;     // e^{g_C} fp32 [128]
 constexpr uint32_t kSlotBytes = 82432;
 constexpr uint32_t kSlotStride = 82944;
 constexpr uint32_t kTokBlk = 8192;
+static_assert(kRingSlots * kSlotStride == kClusterRingBytesPerHead, "ring size");
 
 // ---- producer shared memory
 constexpr uint32_t P_KQT = 0;          // [K*E ; Q*E] tf32, 4 K-blocks x 16 KB
@@ -78,7 +87,7 @@ constexpr uint32_t P_IN_K = 16384;     // k
 constexpr uint32_t P_IN_LA = 32768;    // log alpha [64][128] fp32
 constexpr uint32_t P_IN_V = 65536;     // v  [64][128] bf16
 constexpr uint32_t kInBytes = 81920;
-constexpr uint32_t P_STAGE = 98304;    // slot image being built
+constexpr uint32_t P_STAGE = 98304;    // image-sized area: [P;T], W and U' are staged here
 constexpr uint32_t P_KSV = P_STAGE + kSlotStride;  // [Ks | V] fp16 [token][col], 4 blocks x 8 KB
 constexpr uint32_t P_VEC = P_KSV + 32768;          // beta[64], psum[4][128]
 constexpr uint32_t P_BAR = P_VEC + (64 + 512) * 4;
@@ -88,7 +97,7 @@ constexpr uint32_t C_S16 = 2 * kSlotStride;        // S fp16, MN-major SW128: 2 
 constexpr uint32_t C_U16 = C_S16 + 32768;          // U fp16, MN-major SW128: 2 blocks x 8 KB
 constexpr uint32_t C_BAR = C_U16 + 16384;
 constexpr uint32_t kSmemBytes =
-    (P_BAR > C_BAR ? P_BAR : C_BAR) + 128 + 1024;  // + barriers + alignment slack
+    (P_BAR > C_BAR ? P_BAR : C_BAR) + 192 + 1024;  // + barriers + alignment slack
 
 // TMEM columns.
 constexpr uint32_t PCOL_AP = 0;        // producer: [A;P] (64 cols)
@@ -156,7 +165,7 @@ __device__ void producer(uint8_t *sm, uint32_t tmem, int rank, uint8_t *ring, co
     float *Af = reinterpret_cast<float *>(sm + P_AF);
     float *Xf = reinterpret_cast<float *>(sm + P_XF);
     uint64_t *bar_mma = reinterpret_cast<uint64_t *>(sm + P_BAR);
-    uint64_t *bar_loaded = bar_mma + 1;  // [2]: one per ring slot of this producer
+    uint64_t *bar_loaded = bar_mma + 1;  // [kRingDepth]: one per ring slot of this producer
     uint8_t *st = sm + P_STAGE;
     uint32_t ph_mma = 0;
     int img = 0;  // index of this producer's next image
@@ -165,12 +174,12 @@ __device__ void producer(uint8_t *sm, uint32_t tmem, int rank, uint8_t *ring, co
     const uint64_t d_kht = tc::smem_desc(sbase + P_KHT, 16, 1024, tc::kSwizzle128);
     const uint64_t d_pt = tc::smem_desc(sbase + P_STAGE + SL_PT, 16, 1024, tc::kSwizzle128);
     const uint64_t d_ksv = tc::smem_desc(sbase + P_KSV, kTokBlk, 1024, tc::kSwizzle128);
-    // the consumer's "ready" barriers for this producer's two ring slots
-    const uint32_t c_ready = tc::map_to_rank(sbase + C_BAR + 40 + 16 * rank, kCluster - 1);
+    // the consumer's "ready" barriers for this producer's ring slots
+    const uint32_t c_ready = tc::map_to_rank(sbase + C_BAR + 40 + 8 * kRingDepth * rank, kCluster - 1);
 
     CMARK_INIT;
     const int mk = rank == 0 ? 0 : 64;  // only rank 0 records (slots 0..8)
-    uint64_t *bar_in = bar_mma + 3;
+    uint64_t *bar_in = bar_mma + 1 + kRingDepth;
     uint32_t ph_in = 0;
     auto load_inputs = [&](int cc) {   // TMA: the 64-token chunk cc of head h (all channels)
         const int z = static_cast<int>(ztok + static_cast<long>(cc) * kC);
@@ -234,7 +243,12 @@ __device__ void producer(uint8_t *sm, uint32_t tmem, int rank, uint8_t *ring, co
             psum[qq * 128 + 2 * p] = s0;
             psum[qq * 128 + 2 * p + 1] = s1;
         }
-        if (tid == 0) tc::bulk_wait_read_all();  // the previous image has left the staging area
+        const int rb = img % kRingDepth;  // ring slot of this image; image img-kRingDepth used it before
+        uint8_t *gs = ring + (kRingDepth * rank + rb) * kSlotStride;
+        if (tid == 0) {
+            tc::bulk_wait_read_all();  // the previous [P;T] has left the staging area
+            if (img >= kRingDepth) wait_cluster(bar_loaded + rb, ((img / kRingDepth) - 1) & 1, ctl);
+        }
         __syncthreads();  // inputs are in registers: the tf32 tiles may now overwrite them
         {
             float pre0 = 0.f, pre1 = 0.f, tot0 = 0.f, tot1 = 0.f;
@@ -249,7 +263,7 @@ __device__ void producer(uint8_t *sm, uint32_t tmem, int rank, uint8_t *ring, co
             const float ea0 = expf(ga0), ea1 = expf(ga1);                  // e^{g_a}
             const float eca0 = expf(tot0 - ga0), eca1 = expf(tot1 - ga1);  // e^{g_C - g_a}
             if (qq == 0) {
-                float *gam = reinterpret_cast<float *>(st + SL_GAM);
+                float *gam = reinterpret_cast<float *>(gs + SL_GAM);
                 gam[2 * p] = expf(tot0);
                 gam[2 * p + 1] = expf(tot1);
             }
@@ -277,9 +291,9 @@ __device__ void producer(uint8_t *sm, uint32_t tmem, int rank, uint8_t *ring, co
                 *reinterpret_cast<float2 *>(sm + P_KQT + kb32 * kKQTBlk + o32) = make_float2(ke0, ke1);
                 *reinterpret_cast<float2 *>(sm + P_KQT + kb32 * kKQTBlk + 8192 + o32) = make_float2(qe0, qe1);
                 *reinterpret_cast<float2 *>(sm + P_KHT + kb32 * kKHTBlk + o32) = make_float2(kf0, kf1);
-                *reinterpret_cast<uint32_t *>(st + SL_QW + kb16 * kQWBlk + o16) = pack_f16(qe0 * ea0, qe1 * ea1);
+                *reinterpret_cast<uint32_t *>(gs + SL_QW + kb16 * kQWBlk + o16) = pack_f16(qe0 * ea0, qe1 * ea1);
                 *reinterpret_cast<uint32_t *>(sm + P_KSV + kb16 * kTokBlk + o16) = pack_f16(ke0 * ea0, ke1 * ea1);
-                *reinterpret_cast<uint32_t *>(st + SL_KB + kb16 * kTokBlk + o16) = pack_f16(kf0 * eca0, kf1 * eca1);
+                *reinterpret_cast<uint32_t *>(gs + SL_KB + kb16 * kTokBlk + o16) = pack_f16(kf0 * eca0, kf1 * eca1);
             }
         }
         fence_proxy_async_smem();
@@ -339,7 +353,11 @@ __device__ void producer(uint8_t *sm, uint32_t tmem, int rank, uint8_t *ring, co
         fence_proxy_async_smem();
         __syncthreads();
         // the tf32 region (tiles, A, X) is dead until the next chunk: stage its inputs there
-        if (tid == 0 && c + kProducers < nchunks) load_inputs(c + kProducers);
+        if (tid == 0) {
+            if (c + kProducers < nchunks) load_inputs(c + kProducers);
+            tc::bulk_store_global(gs + SL_PT, st + SL_PT, 16384);   // [P;T] to the ring slot
+            tc::bulk_commit();
+        }
         CMARK(mk + 5);
 
         // ------------------------------------------------ [W | U'] = T [Ks | V] (fp16, N = 256)
@@ -383,17 +401,17 @@ __device__ void producer(uint8_t *sm, uint32_t tmem, int rank, uint8_t *ring, co
         CMARK(mk + 7);
 
         // ------------------------------------------------ publish the image through L2
+        // Every thread's generic stores into the slot (Qs, Kb, e^{g_C}) precede thread 0's
+        // release through the CTA barrier above; the release is cumulative.
         if (tid == 0) {
-            const int b = img & 1;  // ring slot of this image; image img-2 used it before
-            if (img >= 2) wait_cluster(bar_loaded + b, ((img >> 1) - 1) & 1, ctl);
             CMARK(mk + 9);
-            if (!*reinterpret_cast<volatile int *>(ctl.abort)) {
-                tc::bulk_store_global(ring + (2 * rank + b) * kSlotStride, st, kSlotBytes);
-                tc::bulk_commit();
-                tc::bulk_wait_all();
-                tc::fence_proxy_async_global();
-                tc::mbar_arrive_remote(c_ready + 8 * b);
-            }
+            tc::bulk_store_global(gs + SL_QW + 8192, st + SL_QW + 8192, 8192);   // W, K-block 0
+            tc::bulk_store_global(gs + SL_QW + kQWBlk + 8192, st + SL_QW + kQWBlk + 8192, 8192);
+            tc::bulk_store_global(gs + SL_UP, st + SL_UP, 16384);                  // U'
+            tc::bulk_commit();
+            tc::bulk_wait_all();   // [P;T], W and U' have reached the slot
+            tc::fence_proxy_async_global();
+            if (!*reinterpret_cast<volatile int *>(ctl.abort)) tc::mbar_arrive_remote(c_ready + 8 * rb);
         }
         CMARK(mk + 8);
         ++img;
@@ -413,7 +431,7 @@ __device__ void consumer(uint8_t *sm, uint32_t tmem, const uint8_t *ring, const 
     uint64_t *bar_x = full + 2;
     uint64_t *bar_s = full + 3;
     uint64_t *bar_o = full + 4;
-    uint64_t *ready = full + 5;  // [6]: producer p, ring slot b at ready[2p + b]
+    uint64_t *ready = full + 5;  // [kRingSlots]: producer p, ring slot b at ready[kRingDepth p + b]
     uint32_t ph_full = 0;   // bit s: parity of slot s's next fill
     uint32_t ph_x = 0, ph_s = 0, ph_o = 0;
 
@@ -433,8 +451,8 @@ __device__ void consumer(uint8_t *sm, uint32_t tmem, const uint8_t *ring, const 
     auto pull = [&](int limit, bool block) {
         while (next_load <= limit && next_load < nchunks) {
             const int pc = next_load % kProducers, j = next_load / kProducers;
-            const int rs = 2 * pc + (j & 1);  // ring slot (and its ready barrier)
-            const uint32_t par = (j >> 1) & 1;
+            const int rs = kRingDepth * pc + j % kRingDepth;  // ring slot (and its ready barrier)
+            const uint32_t par = (j / kRingDepth) & 1;
             if (block)
                 wait_cluster(ready + rs, par, ctl);
             else if (!tc::mbar_test_cluster(ready + rs, par))
@@ -492,10 +510,10 @@ __device__ void consumer(uint8_t *sm, uint32_t tmem, const uint8_t *ring, const 
         const uint32_t xcol = CCOL_X + s * 128;
         wait_local(full + s, (ph_full >> s) & 1, ctl);  // (already complete) makes the slot visible
         ph_full ^= 1u << s;
-        if (tid == 0 && c + 2 * kProducers < nchunks) {  // the ring slot of chunk c is reusable
+        if (tid == 0 && c + kRingSlots < nchunks) {  // the ring slot of chunk c is reusable
             // relaxed: the slot's bulk load has completed (observed above); no writes of
             // this thread need to be ordered before the producer's reuse of the slot
-            const uint32_t rb = tc::map_to_rank(p_loaded + 8 * ((c / kProducers) & 1), c % kProducers);
+            const uint32_t rb = tc::map_to_rank(p_loaded + 8 * ((c / kProducers) % kRingDepth), c % kProducers);
             asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(rb) : "memory");
         }
         CMARK(16);
@@ -633,12 +651,12 @@ chunk_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     const bool is_consumer = rank == kCluster - 1;
     const uint32_t bar_off = is_consumer ? C_BAR : P_BAR;
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + bar_off);
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + bar_off + 96);
-    int *abort = reinterpret_cast<int *>(sm + bar_off + 100);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + bar_off + 128);
+    int *abort = reinterpret_cast<int *>(sm + bar_off + 132);
     const int tid = threadIdx.x;
 
     if (tid == 0) {
-        for (int i = 0; i < 11; ++i) tc::mbar_init(bars + i, 1);
+        for (int i = 0; i < 14; ++i) tc::mbar_init(bars + i, 1);
         *abort = 0;
         tc::fence_mbar_init();
     }
@@ -653,7 +671,7 @@ chunk_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     const uint32_t tmem = *tmem_slot;
     const Ctl ctl{abort, err};
 
-    uint8_t *ring = ws + bh * kRingSlots * kSlotStride;  // this head's ring: two slots per producer
+    uint8_t *ring = ws + bh * kRingSlots * kSlotStride;  // this head's ring: kRingDepth slots per producer
     if (is_consumer)
         consumer(sm, tmem, ring, S0, out, S_T, T, H, h, bh, ztok, nchunks, ctl);
     else

@@ -35,8 +35,7 @@ namespace kda {
 namespace {
 
 constexpr int kMaxHeads = 32;                       // limit on B * H
-constexpr size_t kRingBytesPerHead = 6ull * 82944;  // 6 ring slots of 81 KB per head
-constexpr size_t kStaticBytes = kMaxHeads * kRingBytesPerHead;
+constexpr size_t kStaticBytes = kMaxHeads * kClusterRingBytesPerHead;
 constexpr int kMaxDevices = 64;
 
 static __device__ __align__(256) uint8_t g_static_ring[kStaticBytes];

@@ -56,5 +56,7 @@ bool chunk_tc_supported(int dk, int dv, int chunk, int dtype);
 bool chunk_cluster_supported(int dk, int dv, int chunk, int dtype);
 size_t chunk_tc_workspace_bytes(int B, int T, int H);
 size_t chunk_cluster_workspace_bytes(int B, int H);
+// Ring of operand images of the cluster engine: 3 producers x 3 slots of 81 KB per head.
+constexpr size_t kClusterRingBytesPerHead = 9ull * 82944;
 
 }  // namespace kda
