@@ -16,7 +16,8 @@
 //     slots of a small ring in the workspace (it stays in L2): Qs, Kb and
 //     e^{g_C} straight from registers in the gate prologue; [P;T] (an operand
 //     of its own MMA), W and U' staged in shared memory and bulk-stored
-//     (cp.async.bulk shared -> global), [P;T] as soon as T is formed. Once the
+//     (cp.async.bulk shared -> global), [P;T] as soon as T is formed and W
+//     while U' is formed. Once the
 //     stores are complete, thread 0 arrives (release, cluster scope; the
 //     generic stores of all threads precede it through a CTA barrier) on the
 //     consumer's "ready" barrier of that slot;
@@ -28,8 +29,8 @@
 // The ring goes through L2 because a DSMEM bulk copy moves only ~20 B/cycle
 // between two SMs, whereas an L2 bulk load of the same 82 KB takes ~1K cycles.
 // The producers set the pace of the cluster, so their image stores are kept
-// short: writing Qs and Kb from registers and storing [P;T] early leaves only
-// W and U' (32 KB) to store and wait for at the end of an image.
+// short: writing Qs and Kb from registers and storing [P;T] and W early
+// leaves only U' (16 KB) to store and wait for at the end of an image.
 // A producer thus has three chunk periods for the key-side latency, and the
 // consumer's chunk period is the chain alone. Every wait is bounded; after a
 // timeout a CTA records an error in the device error word, stops waiting and
@@ -96,8 +97,13 @@ constexpr uint32_t C_SLOT = 0;         // 2 slots
 constexpr uint32_t C_S16 = 2 * kSlotStride;        // S fp16, MN-major SW128: 2 blocks x 16 KB
 constexpr uint32_t C_U16 = C_S16 + 32768;          // U fp16, MN-major SW128: 2 blocks x 8 KB
 constexpr uint32_t C_BAR = C_U16 + 16384;
+#ifdef KDA_PHASE_TIMING
+constexpr uint32_t kDbgBytes = 256;    // per-phase cycle accumulators, after the barriers
+#else
+constexpr uint32_t kDbgBytes = 0;
+#endif
 constexpr uint32_t kSmemBytes =
-    (P_BAR > C_BAR ? P_BAR : C_BAR) + 192 + 1024;  // + barriers + alignment slack
+    (P_BAR > C_BAR ? P_BAR : C_BAR) + 192 + kDbgBytes + 1024;  // + barriers + alignment slack
 
 // TMEM columns.
 constexpr uint32_t PCOL_AP = 0;        // producer: [A;P] (64 cols)
@@ -113,22 +119,36 @@ constexpr uint32_t IDESC_S = tc::idesc(tc::kFmtF16, 128, 128, 1, 1);   // A MN-m
 
 #ifdef KDA_PHASE_TIMING
 // Debug builds only: cycles per phase summed over chunks, for cluster 0
-// (slots 0..9 producer rank 0, slots 16..23 the consumer).
+// (slots 0..9 producer rank 0, slots 16..23 the consumer). Thread 0 of each CTA
+// accumulates in shared memory (a global read-modify-write per mark would cost
+// ~1K cycles and distort the phases) and adds its slots to the global array once.
 __device__ unsigned long long g_cluster_cycles[32];
 #define CMARK(idx)                                                        \
     do {                                                                  \
-        if (blockIdx.x < kCluster && threadIdx.x == 0 && (idx) < 32) {    \
+        if (threadIdx.x == 0 && (idx) < 32) {                             \
             const unsigned long long now_ = clock64();                    \
-            g_cluster_cycles[idx] += now_ - t_prev_;                      \
+            t_acc_[idx] += now_ - t_prev_;                                \
             t_prev_ = now_;                                               \
         }                                                                 \
     } while (0)
-#define CMARK_INIT unsigned long long t_prev_ = clock64()
+#define CMARK_INIT(bar_off)                                                                 \
+    unsigned long long *t_acc_ = reinterpret_cast<unsigned long long *>(sm + (bar_off) + 192); \
+    if (threadIdx.x == 0)                                                                   \
+        for (int i_ = 0; i_ < 32; ++i_) t_acc_[i_] = 0;                                     \
+    unsigned long long t_prev_ = clock64()
+#define CMARK_FLUSH(lo, hi)                                                               \
+    do {                                                                                  \
+        if (blockIdx.x < kCluster && threadIdx.x == 0)                                    \
+            for (int i_ = (lo); i_ < (hi); ++i_) atomicAdd(&g_cluster_cycles[i_], t_acc_[i_]); \
+    } while (0)
 #else
 #define CMARK(idx) \
     do {           \
     } while (0)
-#define CMARK_INIT
+#define CMARK_INIT(bar_off)
+#define CMARK_FLUSH(lo, hi) \
+    do {                    \
+    } while (0)
 #endif
 
 struct Ctl {
@@ -177,7 +197,7 @@ __device__ void producer(uint8_t *sm, uint32_t tmem, int rank, uint8_t *ring, co
     // the consumer's "ready" barriers for this producer's ring slots
     const uint32_t c_ready = tc::map_to_rank(sbase + C_BAR + 40 + 8 * kRingDepth * rank, kCluster - 1);
 
-    CMARK_INIT;
+    CMARK_INIT(P_BAR);
     const int mk = rank == 0 ? 0 : 64;  // only rank 0 records (slots 0..8)
     uint64_t *bar_in = bar_mma + 1 + kRingDepth;
     uint32_t ph_in = 0;
@@ -207,22 +227,12 @@ __device__ void producer(uint8_t *sm, uint32_t tmem, int rank, uint8_t *ring, co
 
         // ------------------------------------------------ gates and operands
         if (tid < kC) beta_s[tid] = tid < valid ? beta[(trow0 + tid) * H + h] : 0.f;
-        {   // V (all 128 columns) -> fp16 columns 128..255 of the [Ks | V] operand
+        uint4 vin[4];   // V row tid/4, columns 32 (tid%4) .. +32 (bf16); stored while [A;P] runs
+        {
             const int t = tid >> 2, piece = tid & 3;
             const uint4 *src = reinterpret_cast<const uint4 *>(sm + P_IN_V + t * 256 + 64 * piece);
 #pragma unroll
-            for (int m = 0; m < 4; ++m) {
-                uint4 w = make_uint4(0, 0, 0, 0);
-                if (t < valid) {
-                    const uint4 x = src[m];
-                    w.x = pack_f16(tc::bf16_lo(x.x), tc::bf16_hi(x.x));
-                    w.y = pack_f16(tc::bf16_lo(x.y), tc::bf16_hi(x.y));
-                    w.z = pack_f16(tc::bf16_lo(x.z), tc::bf16_hi(x.z));
-                    w.w = pack_f16(tc::bf16_lo(x.w), tc::bf16_hi(x.w));
-                }
-                *reinterpret_cast<uint4 *>(sm + P_KSV + 2 * kTokBlk +
-                                           sw128k_off(t, 32 * piece + 8 * m, kTokBlk)) = w;
-            }
+            for (int m = 0; m < 4; ++m) vin[m] = t < valid ? src[m] : make_uint4(0, 0, 0, 0);
         }
         const int p = tid & 63, qq = tid >> 6;  // channels 2p, 2p+1; tokens 16qq .. 16qq+15
         float2 lg[16];
@@ -309,6 +319,19 @@ __device__ void producer(uint8_t *sm, uint32_t tmem, int rank, uint8_t *ring, co
                          d_kht + (((kk >> 2) * kKHTBlk + (kk & 3) * 32) >> 4), IDESC_AP, kk > 0);
             tc::mma_commit(bar_mma);
         }
+        {   // V -> fp16 columns 128..255 of the [Ks | V] operand (read by [W | U'] only)
+            const int t = tid >> 2, piece = tid & 3;
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+                uint4 w;
+                w.x = pack_f16(tc::bf16_lo(vin[m].x), tc::bf16_hi(vin[m].x));
+                w.y = pack_f16(tc::bf16_lo(vin[m].y), tc::bf16_hi(vin[m].y));
+                w.z = pack_f16(tc::bf16_lo(vin[m].z), tc::bf16_hi(vin[m].z));
+                w.w = pack_f16(tc::bf16_lo(vin[m].w), tc::bf16_hi(vin[m].w));
+                *reinterpret_cast<uint4 *>(sm + P_KSV + 2 * kTokBlk +
+                                           sw128k_off(t, 32 * piece + 8 * m, kTokBlk)) = w;
+            }
+        }
         wait_local(bar_mma, ph_mma, ctl);
         ph_mma ^= 1;
         tc_fence_after();
@@ -372,10 +395,10 @@ __device__ void producer(uint8_t *sm, uint32_t tmem, int rank, uint8_t *ring, co
         ph_mma ^= 1;
         tc_fence_after();
         CMARK(mk + 6);
-        if (quad >= 2) {
-            const int i = row - 64;
 #pragma unroll
-            for (int part = 0; part < 2; ++part) {   // part 0: W, part 1: U'
+        for (int part = 0; part < 2; ++part) {   // part 0: W, part 1: U'
+            if (quad >= 2) {
+                const int i = row - 64;
                 float w[64];
                 const uint32_t ta = tc::tmem_addr(tmem, 32 * quad, PCOL_WU + part * 128 + half * 64);
                 tc::tmem_ld32(ta, *reinterpret_cast<float(*)[32]>(&w[0]));
@@ -394,8 +417,16 @@ __device__ void producer(uint8_t *sm, uint32_t tmem, int rank, uint8_t *ring, co
                     *reinterpret_cast<uint4 *>(st + off) = x;
                 }
             }
+            fence_proxy_async_smem();
+            if (part == 0) {   // W leaves while U' is formed
+                __syncthreads();
+                if (tid == 0) {
+                    tc::bulk_store_global(gs + SL_QW + 8192, st + SL_QW + 8192, 8192);   // W, K-block 0
+                    tc::bulk_store_global(gs + SL_QW + kQWBlk + 8192, st + SL_QW + kQWBlk + 8192, 8192);
+                    tc::bulk_commit();
+                }
+            }
         }
-        fence_proxy_async_smem();
         tc_fence_before();
         __syncthreads();
         CMARK(mk + 7);
@@ -405,8 +436,6 @@ __device__ void producer(uint8_t *sm, uint32_t tmem, int rank, uint8_t *ring, co
         // release through the CTA barrier above; the release is cumulative.
         if (tid == 0) {
             CMARK(mk + 9);
-            tc::bulk_store_global(gs + SL_QW + 8192, st + SL_QW + 8192, 8192);   // W, K-block 0
-            tc::bulk_store_global(gs + SL_QW + kQWBlk + 8192, st + SL_QW + kQWBlk + 8192, 8192);
             tc::bulk_store_global(gs + SL_UP, st + SL_UP, 16384);                  // U'
             tc::bulk_commit();
             tc::bulk_wait_all();   // [P;T], W and U' have reached the slot
@@ -417,6 +446,7 @@ __device__ void producer(uint8_t *sm, uint32_t tmem, int rank, uint8_t *ring, co
         ++img;
     }
     if (tid == 0) tc::bulk_wait_read_all();
+    CMARK_FLUSH(0, 10);
 }
 
 // ============================================================ consumer
@@ -501,7 +531,7 @@ __device__ void consumer(uint8_t *sm, uint32_t tmem, const uint8_t *ring, const 
         if (tid == 0) issue_x(0);
     }
 
-    CMARK_INIT;
+    CMARK_INIT(C_BAR);
     for (int c = 0; c < nchunks; ++c) {
         const int s = c & 1;
         const int t0 = c * kC;
@@ -630,6 +660,7 @@ __device__ void consumer(uint8_t *sm, uint32_t tmem, const uint8_t *ring, const 
 #pragma unroll
         for (int j = 0; j < 64; ++j) S_T[(bh * kD + row) * kD + half * 64 + j] = S[j];
     }
+    CMARK_FLUSH(16, 24);
 }
 
 __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 1)
