@@ -1,4 +1,5 @@
 // api.cu -- the C ABI of libkda: argument validation, engine choice, launches.
+#include <limits.h>
 #include <stdarg.h>
 #include <stdio.h>
 
@@ -126,6 +127,13 @@ int kda_chunk_fwd_engine(int engine, const void *q, const void *k, const void *v
     if (rc != KDA_OK) return rc;
     if (chunk != 16 && chunk != 32 && chunk != 64)
         return fail(KDA_ERR_UNSUPPORTED, "chunk=%d is not 16, 32 or 64", chunk);
+    // Token rows are 32-bit tensor-map coordinates; a head is up to 4 CTAs of a 1-D grid.
+    if (static_cast<long long>(B) * T > INT_MAX)
+        return fail(KDA_ERR_UNSUPPORTED, "B*T = %lld tokens: more than 2^31 - 1; split the batch",
+                    static_cast<long long>(B) * T);
+    if (static_cast<long long>(B) * H > INT_MAX / 4)
+        return fail(KDA_ERR_UNSUPPORTED, "B*H = %lld heads: more than 2^29 - 1; split the batch",
+                    static_cast<long long>(B) * H);
     if (B == 0 || H == 0) return KDA_OK;
     const bool tokens = T > 0;
     const Ptr ps[] = {{q, "q", tokens},           {k, "k", tokens},       {v, "v", tokens},
@@ -192,6 +200,10 @@ int kda_recurrent_step(const void *q, const void *k, const void *v, const float 
     if (N < 0 || H < 0) return fail(KDA_ERR_INVALID_ARG, "N=%d H=%d must be >= 0", N, H);
     int rc = check_common(dk, dv, dtype);
     if (rc != KDA_OK) return rc;
+    // A (sequence, head) is up to 2 CTAs of a 1-D grid.
+    if (static_cast<long long>(N) * H > INT_MAX / 2)
+        return fail(KDA_ERR_UNSUPPORTED, "N*H = %lld heads: more than 2^30 - 1; split the batch",
+                    static_cast<long long>(N) * H);
     if (N == 0 || H == 0) return KDA_OK;
     const Ptr ps[] = {{q, "q", true},       {k, "k", true},         {v, "v", true},
                       {log_alpha, "log_alpha", true}, {beta, "beta", true}, {state, "state", true},

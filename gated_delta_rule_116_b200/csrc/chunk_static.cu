@@ -12,7 +12,7 @@
 // lives in g_static_ring below, sized for at most kMaxHeads heads (B*H).
 //
 // Properties a caller has to know:
-//  * every GPU that loads this library holds kStaticBytes (15.2 MiB) of device
+//  * every GPU that loads this library holds kStaticBytes (22.8 MiB) of device
 //    memory for the array until the process exits;
 //  * the first call on each device looks up the array's device address
 //    (cudaGetSymbolAddress, with that device current); make that first call

@@ -96,6 +96,8 @@ size_t kda_workspace_bytes(int B, int T, int H, int dk, int dv, int chunk, int d
  * T = 0 copies S0 (or zeros) to S_T. B = 0 or H = 0 is a no-op.
  * Supported: dk, dv in [1,128] with dv % 4 == 0 (generic engine); the
  * tensor-core engine additionally needs bf16, dk = dv = 128, chunk = 64.
+ * Limits: B*T <= 2^31 - 1 tokens and B*H <= 2^29 - 1 heads; larger problems
+ * return KDA_ERR_UNSUPPORTED (split the batch).
  */
 int kda_chunk_fwd(const void *q, const void *k, const void *v,
                   const float *log_alpha, const float *beta, const float *S0,
@@ -131,7 +133,8 @@ int kda_chunk_fwd_engine(int engine, const void *q, const void *k, const void *v
  *                                       Entries must be distinct and in
  *                                       [0, slots) (not checked: device data)
  *   out        [N,H,dv]    dtype        o = S_new^T q (written)
- * Supported: dk, dv in [1,128], dv % 4 == 0.
+ * Supported: dk, dv in [1,128], dv % 4 == 0; N*H <= 2^30 - 1 (larger batches
+ * return KDA_ERR_UNSUPPORTED).
  */
 int kda_recurrent_step(const void *q, const void *k, const void *v,
                        const float *log_alpha, const float *beta,
@@ -149,7 +152,7 @@ int kda_recurrent_step(const void *q, const void *k, const void *v,
  *   Arguments as kda_chunk_fwd without the workspace; supported: bf16,
  *   dk = dv = 128, chunk = 64, and B * H <= 32 heads (larger problems return
  *   KDA_ERR_UNSUPPORTED and must use kda_chunk_fwd).
- *   Every GPU that loads the library holds the array (15.2 MiB) until exit.
+ *   Every GPU that loads the library holds the array (22.8 MiB) until exit.
  *   The first call on a device looks up the array's address with that device
  *   current; make it before any stream capture. All calls share the array:
  *   calls that overlap on the GPU race and must be serialised by the caller.

@@ -79,6 +79,7 @@ def test_chunk_misaligned_pointer(lib, field):
     (dict(dk=256), -2), (dict(dv=130), -2), (dict(dv=6), -2), (dict(C=48), -2),
     (dict(C=128), -2), (dict(engine=9), -1), (dict(engine=3, C=16), -2), (dict(engine=3, dtype=1), -2),
     (dict(engine=2, dtype=1), -2), (dict(engine=2, dk=64), -2), (dict(engine=2, C=32), -2),
+    (dict(B=2, T=2**30), -2), (dict(B=2**15, H=2**15), -2), (dict(engine=1, B=3, T=2**30), -2),
 ])
 def test_chunk_rejects(lib, kw, code):
     assert chunk(lib, **kw) == code
@@ -114,7 +115,7 @@ def test_step_null_pointer(lib, field):
 
 @pytest.mark.parametrize("kw,code", [
     (dict(state=FAKE + 4), -3), (dict(slot=FAKE + 8), -3), (dict(dtype=2), -1), (dict(N=-1), -1),
-    (dict(dk=129), -2), (dict(dv=10), -2),
+    (dict(dk=129), -2), (dict(dv=10), -2), (dict(N=2**16, H=2**14), -2),
 ])
 def test_step_rejects(lib, kw, code):
     assert step(lib, **kw) == code
