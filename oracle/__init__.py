@@ -13,7 +13,8 @@ as the Kimi Linear summary (es.news.hada.io/topic?id=31936) describes it in its
 sections "De la atencion lineal a Gated DeltaNet" (delta rule, scalar-gated
 GDN) and "Control fino de memoria en Kimi Delta Attention" (per-channel
 diagonal gate). ``decode_step`` is one step of the same recurrence applied to a
-slot-indexed state cache.
+slot-indexed state cache. ``oracle.grad`` holds the backward pass of the same
+recurrence (fp64 numpy).
 """
 from __future__ import annotations
 
