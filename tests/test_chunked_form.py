@@ -1,0 +1,145 @@
+"""The chunked equations, checked against the oracle in fp64 (CPU).
+
+The CUDA prefill engines implement the chunked form of the recurrence (Kimi
+Linear summary, es.news.hada.io/topic?id=31936, section "Algoritmo paralelo
+por chunks": fixed-length chunks that start from the previous chunk's last
+state, the WY representation of the rank-1 updates, the UT transform with the
+lower-triangular inverse taken row by row by forward substitution, a matrix
+state update per chunk, and outputs that add the inter-chunk recurrent part to
+the intra-chunk parallel part). This file writes those equations out in plain
+NumPy, in exact (un-anchored) form, and checks that they reach the oracle's
+result: the forward against ``oracle.forward``, and the chunked backward --
+the same chunks in reverse, with the state gradient as the sequential chain --
+against ``oracle.grad.backward``. It shares no code with the CUDA sources.
+
+Per chunk (g = in-chunk prefix sum of log alpha, gamma = e^{g_C}):
+    A_ij = beta_i k_i.(k_j e^{g_i - g_j}) (j < i),  P_ij = q_i.(k_j e^{g_i - g_j}) (j <= i)
+    T = (I + A)^{-1} Diag(beta),  W = T (K e^{g}),  U' = T V
+    U = U' - W S,  O = (Q e^{g}) S + P U,  S <- Diag(gamma) S + (K e^{g_C - g})^T U
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from oracle import grad
+
+
+def unit_lower_inverse(A):
+    """(I + A)^{-1} for strictly lower-triangular A, row by row by forward substitution."""
+    n = A.shape[0]
+    X = np.zeros((n, n))
+    for i in range(n):
+        X[i, i] = 1.0
+        X[i, :i] = -A[i, :i] @ X[:i, :i]
+    return X
+
+
+def chunk_terms(qc, kc, vc, lc, bc):
+    n = qc.shape[0]
+    g = np.cumsum(lc, axis=0)
+    D = np.exp(g[:, None, :] - g[None, :, :])                     # e^{g_i - g_j}, [i, j, channel]
+    lower, lower_eq = np.tril(np.ones((n, n)), -1), np.tril(np.ones((n, n)))
+    At = np.einsum("ic,jc,ijc->ij", kc, kc, D) * lower
+    P = np.einsum("ic,jc,ijc->ij", qc, kc, D) * lower_eq
+    X = unit_lower_inverse(At * bc[:, None])
+    Tm = X * bc[None, :]
+    Ks, Qs, Kb = kc * np.exp(g), qc * np.exp(g), kc * np.exp(g[-1] - g)
+    return dict(g=g, At=At, P=P, X=X, T=Tm, Ks=Ks, Qs=Qs, Kb=Kb, W=Tm @ Ks, Up=Tm @ vc,
+                gamma=np.exp(g[-1]), lower=lower, lower_eq=lower_eq)
+
+
+def chunked_forward(q, k, v, la, be, S0, C):
+    S = S0.copy()
+    out = np.zeros((q.shape[0], v.shape[1]))
+    states = []
+    for t0 in range(0, q.shape[0], C):
+        sl = slice(t0, min(t0 + C, q.shape[0]))
+        c = chunk_terms(q[sl], k[sl], v[sl], la[sl], be[sl])
+        states.append(S.copy())
+        U = c["Up"] - c["W"] @ S
+        out[sl] = c["Qs"] @ S + c["P"] @ U
+        S = c["gamma"][:, None] * S + c["Kb"].T @ U
+    return out, S, states
+
+
+def chunked_backward(q, k, v, la, be, S0, dO, dST, C):
+    _, _, states = chunked_forward(q, k, v, la, be, S0, C)
+    res = {n: np.zeros_like(a) for n, a in (("dq", q), ("dk", k), ("dv", v), ("dlog_alpha", la),
+                                             ("dbeta", be))}
+    dS = dST.copy()                                     # gradient of the state leaving the chunk
+    starts = list(range(0, q.shape[0], C))
+    for ci in reversed(range(len(starts))):
+        sl = slice(starts[ci], min(starts[ci] + C, q.shape[0]))
+        S, c = states[ci], chunk_terms(q[sl], k[sl], v[sl], la[sl], be[sl])
+        vc, do = v[sl], dO[sl]
+        U = c["Up"] - c["W"] @ S
+        # the sequential part: the state gradient through one chunk
+        dU = c["P"].T @ do + c["Kb"] @ dS
+        dS_in = c["Qs"].T @ do + c["gamma"][:, None] * dS - c["W"].T @ dU
+        # everything else is local to the chunk once dU, dS and S are known
+        dQs, dP, dKb = do @ S.T, (do @ U.T) * c["lower_eq"], U @ dS.T
+        dW = -dU @ S.T
+        dT = dW @ c["Ks"].T + dU @ vc.T
+        dKs = c["T"].T @ dW
+        res["dv"][sl] = c["T"].T @ dU
+        dX = dT * be[sl][None, :]
+        dA = -(c["X"].T @ dX @ c["X"].T) * c["lower"]
+        res["dbeta"][sl] = np.sum(dT * c["X"], axis=0) + np.sum(dA * c["At"], axis=1)
+        dAt = dA * be[sl][:, None]
+        g = c["g"]
+        Kt, Kh, Qt = k[sl] * np.exp(g), k[sl] * np.exp(-g), q[sl] * np.exp(g)
+        dKt, dQt = dAt @ Kh, dP @ Kh
+        dKh = dAt.T @ Kt + dP.T @ Qt
+        res["dk"][sl] = dKt * np.exp(g) + dKh * np.exp(-g) + dKs * np.exp(g) + dKb * np.exp(g[-1] - g)
+        res["dq"][sl] = dQt * np.exp(g) + dQs * np.exp(g)
+        dg = (dKt * Kt - dKh * Kh + dQt * Qt + dKs * c["Ks"] + dQs * c["Qs"] - dKb * c["Kb"])
+        dg[-1] += np.sum(dS * S, axis=1) * c["gamma"] + np.sum(dKb * c["Kb"], axis=0)
+        res["dlog_alpha"][sl] = np.cumsum(dg[::-1], axis=0)[::-1]
+        dS = dS_in
+    res["dS0"] = dS
+    return res
+
+
+def head_problem(T, d, dv, seed):
+    rng = np.random.default_rng(seed)
+    f32 = lambda a: a.astype(np.float32).astype(np.float64)      # inputs the C oracle reads exactly
+    q = f32(rng.standard_normal((T, d)))
+    k = rng.standard_normal((T, d))
+    k = f32(k / np.linalg.norm(k, axis=1, keepdims=True))
+    v = f32(rng.standard_normal((T, dv)))
+    la = f32(-np.log1p(np.exp(rng.standard_normal((T, d)))))
+    be = f32(1.0 / (1.0 + np.exp(-rng.standard_normal(T))))
+    S0 = 0.3 * rng.standard_normal((d, dv))
+    return q, k, v, la, be, S0, rng.standard_normal((T, dv)), rng.standard_normal((d, dv))
+
+
+CASES = [(64, 8, 6, 16, 0), (50, 8, 6, 16, 1), (130, 16, 8, 64, 2), (97, 12, 4, 32, 3), (5, 4, 4, 64, 4)]
+
+
+@pytest.mark.parametrize("T,d,dv,C,seed", CASES)
+def test_chunked_forward_equals_the_recurrence(T, d, dv, C, seed):
+    q, k, v, la, be, S0, _, _ = head_problem(T, d, dv, seed)
+    out, ST, _ = chunked_forward(q, k, v, la, be, S0, C)
+    t = lambda a: torch.from_numpy(a[None, :, None].astype(np.float32))
+    ref_o, ref_s = oracle.forward(t(q), t(k), t(v), t(la), torch.from_numpy(be[None, :, None].astype(np.float32)),
+                                  torch.from_numpy(S0[None, None]))
+    np.testing.assert_allclose(out, ref_o[0, :, 0], rtol=1e-9, atol=1e-10)
+    np.testing.assert_allclose(ST, ref_s[0, 0], rtol=1e-9, atol=1e-10)
+
+
+@pytest.mark.parametrize("T,d,dv,C,seed", CASES)
+def test_chunked_backward_equals_the_reverse_recurrence(T, d, dv, C, seed):
+    q, k, v, la, be, S0, dO, dST = head_problem(T, d, dv, seed)
+    mine = chunked_backward(q, k, v, la, be, S0, dO, dST, C)
+    e = lambda a: a[None, :, None]
+    ref = grad.backward(e(q), e(k), e(v), e(la), e(be), e(dO), S0=S0[None, None], dS_T=dST[None, None])
+    for n in ["dq", "dk", "dv", "dlog_alpha", "dbeta"]:
+        np.testing.assert_allclose(mine[n], ref[n][0, :, 0], rtol=1e-9, atol=1e-10, err_msg=n)
+    np.testing.assert_allclose(mine["dS0"], ref["dS0"][0, 0], rtol=1e-9, atol=1e-10)
+
+
+def test_forward_substitution_inverts():
+    rng = np.random.default_rng(0)
+    A = np.tril(rng.standard_normal((20, 20)), -1)
+    np.testing.assert_allclose(unit_lower_inverse(A) @ (np.eye(20) + A), np.eye(20), atol=1e-10)
