@@ -143,3 +143,41 @@ def test_forward_substitution_inverts():
     rng = np.random.default_rng(0)
     A = np.tril(rng.standard_normal((20, 20)), -1)
     np.testing.assert_allclose(unit_lower_inverse(A) @ (np.eye(20) + A), np.eye(20), atol=1e-10)
+
+
+def chunked_chain(q, k, v, la, be, S_init, C):
+    """The chunked chain from S_init; returns outputs and final state (columns of
+    S_init evolve independently, so S_init may be any d x n matrix)."""
+    out, S, _ = chunked_forward(q, k, v, la, be, S_init, C)
+    return out, S
+
+
+@pytest.mark.parametrize("T,split,C,seed", [(256, 128, 64, 0), (200, 64, 32, 1), (131, 64, 64, 2)])
+def test_sequence_split_with_output_correction(T, split, C, seed):
+    """Two segments of one head computed independently, then joined.
+
+    The second segment runs its chain twice, side by side: from a zero state
+    with values V (outputs O0, final state S0_end), and from the identity with
+    zero values (its "outputs" are Y = Qs M - P W M, with M the transition
+    product up to each chunk, and its final state is M_end). With the first
+    segment's final state S_mid:
+        O = O0 + Y S_mid,     S_T = S0_end + M_end S_mid.
+    Both halves of the augmented state [0 | I] (values [V | 0]) are value
+    columns of one chain, so each is the engine's chain as it stands."""
+    d, dv = 8, 6
+    q, k, v, la, be, S0, _, _ = head_problem(T, d, dv, seed)
+    first = slice(0, split)
+    second = slice(split, T)
+    o1, S_mid = chunked_chain(q[first], k[first], v[first], la[first], be[first], S0, C)
+    aug = np.concatenate([np.zeros((d, dv)), np.eye(d)], axis=1)          # [0 | I]
+    v_aug = np.concatenate([v[second], np.zeros((T - split, d))], axis=1)   # [V | 0]
+    o_aug, S_aug = chunked_chain(q[second], k[second], v_aug, la[second], be[second], aug, C)
+    O0, Y = o_aug[:, :dv], o_aug[:, dv:]
+    o2 = O0 + Y @ S_mid
+    ST = S_aug[:, :dv] + S_aug[:, dv:] @ S_mid
+    out = np.concatenate([o1, o2])
+    t = lambda a: torch.from_numpy(a[None, :, None].astype(np.float32))
+    ref_o, ref_s = oracle.forward(t(q), t(k), t(v), t(la), torch.from_numpy(be[None, :, None].astype(np.float32)),
+                                  torch.from_numpy(S0[None, None]))
+    np.testing.assert_allclose(out, ref_o[0, :, 0], rtol=1e-9, atol=1e-10)
+    np.testing.assert_allclose(ST, ref_s[0, 0], rtol=1e-9, atol=1e-10)
