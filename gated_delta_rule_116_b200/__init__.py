@@ -1,14 +1,15 @@
-"""B200 (sm_100a) Kimi Delta Attention: chunked prefill and recurrent decode.
+"""B200 (sm_100a) Kimi Delta Attention: chunked prefill, its backward pass and
+recurrent decode.
 
 The compute runs in ``libkda.so`` (hand-written CUDA, C ABI in
 ``include/kda.h``); this package is its thin Python binding.
 
     out, S_T = chunk_fwd(q, k, v, log_alpha, beta, S0, chunk=64)
+    grads = chunk_bwd(q, k, v, log_alpha, beta, grad_out, S0, grad_S_T)
     out = recurrent_step(q, k, v, log_alpha, beta, state, slot)
 """
-from .binding import (ENGINES, KDA_BF16, KDA_F32, LIB_PATH, KdaError, chunk_fwd, device_status,
-                      engine_supported,
-                      load, recurrent_step, workspace_bytes)
+from .binding import (ENGINES, KDA_BF16, KDA_F32, LIB_PATH, KdaError, chunk_bwd, chunk_fwd,
+                      device_status, engine_supported, load, recurrent_step, workspace_bytes)
 
-__all__ = ["chunk_fwd", "recurrent_step", "workspace_bytes", "device_status", "engine_supported", "load", "KdaError",
-           "ENGINES", "KDA_BF16", "KDA_F32", "LIB_PATH"]
+__all__ = ["chunk_fwd", "chunk_bwd", "recurrent_step", "workspace_bytes", "device_status",
+           "engine_supported", "load", "KdaError", "ENGINES", "KDA_BF16", "KDA_F32", "LIB_PATH"]

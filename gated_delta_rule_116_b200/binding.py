@@ -47,6 +47,10 @@ def load():
     lib.kda_chunk_fwd_engine.restype = i
     lib.kda_engine_supported.argtypes = [i, i, i, i, i]
     lib.kda_engine_supported.restype = i
+    lib.kda_chunk_bwd.argtypes = [p] * 14 + [i, i, i, i, i, i, p, sz, p]
+    lib.kda_chunk_bwd.restype = i
+    lib.kda_bwd_workspace_bytes.argtypes = [i, i, i, i, i, i]
+    lib.kda_bwd_workspace_bytes.restype = sz
     lib.kda_recurrent_step.argtypes = [p, p, p, p, p, p, p, p, i, i, i, i, i, p]
     lib.kda_recurrent_step.restype = i
     lib.kda_strerror.argtypes = [i]
@@ -141,6 +145,48 @@ def chunk_fwd(q, k, v, log_alpha, beta, S0=None, chunk: int = 64, *, out=None, S
             ws_bytes, _stream(device, stream))
     _check(rc)
     return out, S_T
+
+
+def chunk_bwd(q, k, v, log_alpha, beta, grad_out, S0=None, grad_S_T=None, *, workspace=None,
+              stream=None):
+    """Backward pass of ``chunk_fwd`` (``kda_chunk_bwd``).
+
+    Inputs as ``chunk_fwd``; ``grad_out`` ``[B,T,H,dv]`` in the input dtype and
+    ``grad_S_T`` ``[B,H,dk,dv]`` fp32 (or None) are dL/d(out) and dL/d(S_T).
+    Returns a dict with ``q``, ``k``, ``v`` (input dtype), ``log_alpha``,
+    ``beta`` and ``S0`` (fp32) gradients.
+    """
+    lib = load()
+    device = q.device
+    _require(q, "q", device)
+    if q.dtype not in _DTYPES:
+        raise TypeError(f"q must be bf16 or fp32 (got {q.dtype})")
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    _require(k, "k", device, q.dtype, (B, T, H, dk))
+    _require(v, "v", device, q.dtype, (B, T, H, dv))
+    _require(log_alpha, "log_alpha", device, torch.float32, (B, T, H, dk))
+    _require(beta, "beta", device, torch.float32, (B, T, H))
+    _require(grad_out, "grad_out", device, q.dtype, (B, T, H, dv))
+    if S0 is not None:
+        _require(S0, "S0", device, torch.float32, (B, H, dk, dv))
+    if grad_S_T is not None:
+        _require(grad_S_T, "grad_S_T", device, torch.float32, (B, H, dk, dv))
+    g = dict(q=torch.empty_like(q), k=torch.empty_like(k), v=torch.empty_like(v),
+             log_alpha=torch.empty_like(log_alpha), beta=torch.empty_like(beta),
+             S0=torch.empty(B, H, dk, dv, device=device, dtype=torch.float32))
+    need = int(lib.kda_bwd_workspace_bytes(B, T, H, dk, dv, _DTYPES[q.dtype]))
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, device=device, dtype=torch.uint8)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    with torch.cuda.device(device):
+        rc = lib.kda_chunk_bwd(
+            _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(S0), _ptr(grad_out),
+            _ptr(grad_S_T), _ptr(g["q"]), _ptr(g["k"]), _ptr(g["v"]), _ptr(g["log_alpha"]),
+            _ptr(g["beta"]), _ptr(g["S0"]), B, T, H, dk, dv, _DTYPES[q.dtype], _ptr(workspace),
+            ws_bytes, _stream(device, stream))
+    _check(rc)
+    return g
 
 
 def recurrent_step(q, k, v, log_alpha, beta, state, slot=None, *, out=None, stream=None):

@@ -215,6 +215,62 @@ int kda_recurrent_step(const void *q, const void *k, const void *v, const float 
     return e == cudaSuccess ? KDA_OK : cuda_fail(e, "launching the decode kernel");
 }
 
+size_t kda_bwd_workspace_bytes(int B, int T, int H, int dk, int dv, int dtype) {
+    if (B <= 0 || T <= 0 || H <= 0 || dk < 1 || dv < 1 || dk > 128 || dv > 128) return 0;
+    if (dtype != KDA_BF16 && dtype != KDA_F32) return 0;
+    return kda::chunk_bwd_workspace_bytes(B, T, H, dk, dv);
+}
+
+int kda_chunk_bwd(const void *q, const void *k, const void *v, const float *log_alpha,
+                  const float *beta, const float *S0, const void *grad_out, const float *grad_S_T,
+                  void *grad_q, void *grad_k, void *grad_v, float *grad_log_alpha, float *grad_beta,
+                  float *grad_S0, int B, int T, int H, int dk, int dv, int dtype, void *workspace,
+                  size_t workspace_bytes, void *stream) {
+    g_detail[0] = '\0';
+    if (dtype != KDA_BF16 && dtype != KDA_F32)
+        return fail(KDA_ERR_INVALID_ARG, "dtype %d is neither KDA_BF16 nor KDA_F32", dtype);
+    if (B < 0 || T < 0 || H < 0)
+        return fail(KDA_ERR_INVALID_ARG, "B=%d T=%d H=%d must be >= 0", B, T, H);
+    if (dk < 1 || dv < 1) return fail(KDA_ERR_INVALID_ARG, "dk=%d dv=%d must be >= 1", dk, dv);
+    if (dk > 128 || dv > 128)
+        return fail(KDA_ERR_UNSUPPORTED, "dk=%d dv=%d: head dimensions above 128", dk, dv);
+    if (static_cast<long long>(B) * T > INT_MAX)
+        return fail(KDA_ERR_UNSUPPORTED, "B*T = %lld tokens: more than 2^31 - 1; split the batch",
+                    static_cast<long long>(B) * T);
+    if (static_cast<long long>(B) * H > INT_MAX / 4)
+        return fail(KDA_ERR_UNSUPPORTED, "B*H = %lld heads: more than 2^29 - 1; split the batch",
+                    static_cast<long long>(B) * H);
+    if (B == 0 || H == 0) return KDA_OK;
+    const bool tokens = T > 0;
+    const Ptr ps[] = {{q, "q", tokens}, {k, "k", tokens}, {v, "v", tokens},
+                      {log_alpha, "log_alpha", tokens}, {beta, "beta", tokens},
+                      {grad_out, "grad_out", tokens}, {grad_q, "grad_q", tokens},
+                      {grad_k, "grad_k", tokens}, {grad_v, "grad_v", tokens},
+                      {grad_log_alpha, "grad_log_alpha", tokens}, {grad_beta, "grad_beta", tokens},
+                      {S0, "S0", false}, {grad_S_T, "grad_S_T", false}, {grad_S0, "grad_S0", false},
+                      {workspace, "workspace", false}};
+    int rc = check_pointers(ps, sizeof ps / sizeof ps[0]);
+    if (rc != KDA_OK) return rc;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (!tokens) {  // grad_S0 = grad_S_T (or zeros)
+        if (!grad_S0) return KDA_OK;
+        const size_t bytes = static_cast<size_t>(B) * H * dk * dv * sizeof(float);
+        cudaError_t e = grad_S_T ? (grad_S_T == grad_S0 ? cudaSuccess
+                                                        : cudaMemcpyAsync(grad_S0, grad_S_T, bytes,
+                                                                          cudaMemcpyDeviceToDevice, s))
+                                 : cudaMemsetAsync(grad_S0, 0, bytes, s);
+        return e == cudaSuccess ? KDA_OK : cuda_fail(e, "copying grad_S_T to grad_S0");
+    }
+    const size_t need = kda::chunk_bwd_workspace_bytes(B, T, H, dk, dv);
+    if (!workspace || workspace_bytes < need)
+        return fail(KDA_ERR_WORKSPACE, "workspace of %zu bytes given, %zu needed",
+                    workspace ? workspace_bytes : static_cast<size_t>(0), need);
+    cudaError_t e = kda::launch_chunk_bwd(q, k, v, log_alpha, beta, S0, grad_out, grad_S_T, grad_q,
+                                          grad_k, grad_v, grad_log_alpha, grad_beta, grad_S0, B, T, H,
+                                          dk, dv, dtype, workspace, s);
+    return e == cudaSuccess ? KDA_OK : cuda_fail(e, "launching the backward kernels");
+}
+
 int kda_device_status(void *stream) {
     g_detail[0] = '\0';
     cudaStream_t s = static_cast<cudaStream_t>(stream);

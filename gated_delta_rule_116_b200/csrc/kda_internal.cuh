@@ -56,6 +56,12 @@ bool chunk_tc_supported(int dk, int dv, int chunk, int dtype);
 bool chunk_cluster_supported(int dk, int dv, int chunk, int dtype);
 size_t chunk_tc_workspace_bytes(int B, int T, int H);
 size_t chunk_cluster_workspace_bytes(int B, int H);
+// Backward pass (chunk_bwd.cu).
+size_t chunk_bwd_workspace_bytes(int B, int T, int H, int dk, int dv);
+cudaError_t launch_chunk_bwd(const void *q, const void *k, const void *v, const float *la,
+                             const float *beta, const float *S0, const void *dout, const float *dS_T,
+                             void *dq, void *dk_, void *dv_, float *dla, float *dbeta, float *dS0, int B,
+                             int T, int H, int dk, int dv, int dtype, void *ws, cudaStream_t s);
 // Ring of operand images of the cluster engine: 3 producers x 3 slots of 81 KB per head.
 constexpr size_t kClusterRingBytesPerHead = 9ull * 82944;
 

@@ -142,6 +142,40 @@ int kda_recurrent_step(const void *q, const void *k, const void *v,
                        int N, int H, int dk, int dv, int dtype, void *stream);
 
 /*
+ * Backward pass of kda_chunk_fwd: the gradients of a scalar loss L with respect
+ * to q, k, v, log_alpha, beta and S0, given dL/d(out) and dL/d(S_T). The pages
+ * print no backward pass; this is the derivative of the same recurrence, in
+ * the same chunked (WY/UT) form as the prefill, visited last chunk to first.
+ *
+ *   q, k, v, log_alpha, beta, S0        as kda_chunk_fwd (S0 NULL means zeros)
+ *   grad_out   [B,T,H,dv]  dtype        dL/d(out)
+ *   grad_S_T   [B,H,dk,dv] fp32         dL/d(S_T); NULL means zeros
+ *   grad_q, grad_k [B,T,H,dk] dtype     written
+ *   grad_v     [B,T,H,dv]  dtype        written
+ *   grad_log_alpha [B,T,H,dk] fp32      written
+ *   grad_beta  [B,T,H]     fp32         written
+ *   grad_S0    [B,H,dk,dv] fp32         written; NULL skips it
+ *   workspace, workspace_bytes          device scratch of at least
+ *                                       kda_bwd_workspace_bytes(...) bytes: the
+ *                                       entry state of every 16-token chunk plus
+ *                                       fp32 accumulators for grad_q and grad_k
+ * Outputs must not alias inputs. Computes in fp32 on CUDA cores.
+ * T = 0 copies grad_S_T (or zeros) to grad_S0. B = 0 or H = 0 is a no-op.
+ * Supported: dtype KDA_BF16 or KDA_F32, dk and dv in [1,128]; the same B*T and
+ * B*H limits as kda_chunk_fwd.
+ */
+int kda_chunk_bwd(const void *q, const void *k, const void *v,
+                  const float *log_alpha, const float *beta, const float *S0,
+                  const void *grad_out, const float *grad_S_T,
+                  void *grad_q, void *grad_k, void *grad_v,
+                  float *grad_log_alpha, float *grad_beta, float *grad_S0,
+                  int B, int T, int H, int dk, int dv, int dtype,
+                  void *workspace, size_t workspace_bytes, void *stream);
+
+/* Workspace bytes kda_chunk_bwd needs for this shape (0 for empty or unsupported shapes). */
+size_t kda_bwd_workspace_bytes(int B, int T, int H, int dk, int dv, int dtype);
+
+/*
  * Chunked prefill that allocates nothing and takes no workspace: the same
  * computation as kda_chunk_fwd_engine(KDA_ENGINE_TC_CLUSTER, ...), whose
  * scratch (the ring of per-chunk operand images) lives in a fixed device

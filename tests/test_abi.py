@@ -135,3 +135,41 @@ def test_binding_refuses_cpu_tensors():
     x = torch.zeros(1, 4, 1, 16)
     with pytest.raises(ValueError, match="CUDA"):
         kda.chunk_fwd(x, x, x, x, torch.zeros(1, 4, 1), chunk=16)
+
+
+def bwd(lib, q=FAKE, k=FAKE, v=FAKE, la=FAKE, beta=FAKE, S0=None, go=FAKE, gST=None, gq=FAKE,
+        gk=FAKE, gv=FAKE, gla=FAKE, gb=FAKE, gS0=None, B=1, T=32, H=2, dk=128, dv=128, dtype=0,
+        ws=None, wsb=0):
+    return lib.kda_chunk_bwd(q, k, v, la, beta, S0, go, gST, gq, gk, gv, gla, gb, gS0, B, T, H, dk,
+                             dv, dtype, ws, wsb, None)
+
+
+@pytest.mark.parametrize("field", ["q", "k", "v", "la", "beta", "go", "gq", "gk", "gv", "gla", "gb"])
+def test_bwd_null_pointer(lib, field):
+    assert bwd(lib, **{field: None}) == -1
+    assert detail(lib)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(gq=FAKE + 4), -3), (dict(gS0=FAKE + 8), -3), (dict(dtype=3), -1), (dict(B=-1), -1),
+    (dict(dk=0), -1), (dict(dk=129), -2), (dict(dv=200), -2), (dict(B=2, T=2**30), -2),
+])
+def test_bwd_rejects(lib, kw, code):
+    assert bwd(lib, **kw) == code
+    assert detail(lib)
+
+
+def test_bwd_workspace_missing_or_short(lib):
+    need = lib.kda_bwd_workspace_bytes(1, 32, 2, 128, 128, 0)
+    # two 16-token chunks of 128 x 128 fp32 entry states per head, plus fp32 dq and dk
+    assert need == (2 * 2 * 128 * 128 + 2 * 32 * 2 * 128) * 4
+    assert bwd(lib) == -4 and "workspace" in detail(lib)
+    assert bwd(lib, ws=FAKE, wsb=need - 16) == -4
+
+
+def test_bwd_empty_batch_is_noop(lib):
+    none = dict(q=None, k=None, v=None, la=None, beta=None, go=None, gq=None, gk=None, gv=None,
+                gla=None, gb=None)
+    assert bwd(lib, B=0, **none) == 0
+    assert bwd(lib, H=0, **none) == 0
+    assert lib.kda_bwd_workspace_bytes(0, 32, 2, 128, 128, 0) == 0
