@@ -173,3 +173,12 @@ def test_bwd_empty_batch_is_noop(lib):
     assert bwd(lib, B=0, **none) == 0
     assert bwd(lib, H=0, **none) == 0
     assert lib.kda_bwd_workspace_bytes(0, 32, 2, 128, 128, 0) == 0
+
+
+def test_binding_backward_refuses_cpu_tensors():
+    import torch
+    x = torch.zeros(1, 4, 1, 16)
+    la = torch.zeros(1, 4, 1, 16)
+    b = torch.zeros(1, 4, 1)
+    with pytest.raises(ValueError, match="CUDA"):
+        kda.chunk_bwd(x, x, x, la, b, x)
