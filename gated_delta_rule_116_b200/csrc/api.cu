@@ -271,6 +271,37 @@ int kda_chunk_bwd(const void *q, const void *k, const void *v, const float *log_
     return e == cudaSuccess ? KDA_OK : cuda_fail(e, "launching the backward kernels");
 }
 
+int kda_chunk_fwd_varlen(const void *q, const void *k, const void *v, const float *log_alpha,
+                         const float *beta, const int32_t *cu_seqlens, const float *S0, void *out,
+                         float *S_T, int N, int total_T, int H, int dk, int dv, int dtype,
+                         void *stream) {
+    g_detail[0] = '\0';
+    if (dtype != KDA_BF16 && dtype != KDA_F32)
+        return fail(KDA_ERR_INVALID_ARG, "dtype %d is neither KDA_BF16 nor KDA_F32", dtype);
+    if (N < 0 || total_T < 0 || H < 0)
+        return fail(KDA_ERR_INVALID_ARG, "N=%d total_T=%d H=%d must be >= 0", N, total_T, H);
+    if (dk < 1 || dv < 1) return fail(KDA_ERR_INVALID_ARG, "dk=%d dv=%d must be >= 1", dk, dv);
+    if (dk > 128 || dv > 128)
+        return fail(KDA_ERR_UNSUPPORTED, "dk=%d dv=%d: head dimensions above 128", dk, dv);
+    if (static_cast<long long>(N) * H > INT_MAX / 4)
+        return fail(KDA_ERR_UNSUPPORTED, "N*H = %lld heads: more than 2^29 - 1; split the batch",
+                    static_cast<long long>(N) * H);
+    if (N == 0 || H == 0) return KDA_OK;
+    if (!cu_seqlens) return fail(KDA_ERR_INVALID_ARG, "cu_seqlens is NULL");
+    if ((reinterpret_cast<uintptr_t>(cu_seqlens) & 3u) != 0)
+        return fail(KDA_ERR_ALIGNMENT, "cu_seqlens is not 4-byte aligned");
+    const bool tokens = total_T > 0;
+    const Ptr ps[] = {{q, "q", tokens}, {k, "k", tokens}, {v, "v", tokens},
+                      {log_alpha, "log_alpha", tokens}, {beta, "beta", tokens}, {out, "out", tokens},
+                      {S0, "S0", false}, {S_T, "S_T", false}};
+    int rc = check_pointers(ps, sizeof ps / sizeof ps[0]);
+    if (rc != KDA_OK) return rc;
+    cudaError_t e = kda::launch_chunk_varlen(q, k, v, log_alpha, beta, cu_seqlens, S0, out, S_T, N,
+                                             total_T, H, dk, dv, dtype,
+                                             static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? KDA_OK : cuda_fail(e, "launching the variable-length prefill");
+}
+
 int kda_device_status(void *stream) {
     g_detail[0] = '\0';
     cudaStream_t s = static_cast<cudaStream_t>(stream);

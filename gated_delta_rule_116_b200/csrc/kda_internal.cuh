@@ -62,6 +62,11 @@ cudaError_t launch_chunk_bwd(const void *q, const void *k, const void *v, const 
                              const float *beta, const float *S0, const void *dout, const float *dS_T,
                              void *dq, void *dk_, void *dv_, float *dla, float *dbeta, float *dS0, int B,
                              int T, int H, int dk, int dv, int dtype, void *ws, cudaStream_t s);
+// Variable-length prefill (chunk_varlen.cu).
+cudaError_t launch_chunk_varlen(const void *q, const void *k, const void *v, const float *la,
+                                const float *beta, const int32_t *cu_seqlens, const float *S0,
+                                void *out, float *S_T, int N, int total_T, int H, int dk, int dv,
+                                int dtype, cudaStream_t s);
 // Ring of operand images of the cluster engine: 3 producers x 3 slots of 81 KB per head.
 constexpr size_t kClusterRingBytesPerHead = 9ull * 82944;
 

@@ -142,6 +142,36 @@ int kda_recurrent_step(const void *q, const void *k, const void *v,
                        int N, int H, int dk, int dv, int dtype, void *stream);
 
 /*
+ * Chunked prefill of a packed batch of N sequences of different lengths.
+ * Sequence n is tokens cu_seqlens[n] .. cu_seqlens[n+1]-1 of the packed
+ * tensors and starts from S0[n] (or zeros); no state crosses a sequence
+ * boundary. Computes in fp32 on CUDA cores with 16-token chunks.
+ *
+ *   q, k       [total_T,H,dk]  dtype     (packed over sequences)
+ *   v          [total_T,H,dv]  dtype
+ *   log_alpha  [total_T,H,dk]  fp32
+ *   beta       [total_T,H]     fp32
+ *   cu_seqlens [N+1]       int32 (device) nondecreasing token offsets, usually
+ *                                       cu_seqlens[0] = 0 and cu_seqlens[N] =
+ *                                       total_T. Offsets are device data and
+ *                                       are not checked; the kernel clamps them
+ *                                       to [0, total_T], so no access leaves the
+ *                                       tensors. Tokens outside every sequence
+ *                                       keep their previous out values.
+ *   S0         [N,H,dk,dv] fp32         NULL means zeros
+ *   out        [total_T,H,dv] dtype     written for every token of a sequence
+ *   S_T        [N,H,dk,dv] fp32         final state per sequence; NULL skips it
+ * N = 0 or H = 0 is a no-op. Supported: dtype KDA_BF16 or KDA_F32, dk and dv
+ * in [1,128], N*H <= 2^29 - 1.
+ */
+int kda_chunk_fwd_varlen(const void *q, const void *k, const void *v,
+                         const float *log_alpha, const float *beta,
+                         const int32_t *cu_seqlens, const float *S0,
+                         void *out, float *S_T,
+                         int N, int total_T, int H, int dk, int dv, int dtype,
+                         void *stream);
+
+/*
  * Backward pass of kda_chunk_fwd: the gradients of a scalar loss L with respect
  * to q, k, v, log_alpha, beta and S0, given dL/d(out) and dL/d(S_T). The pages
  * print no backward pass; this is the derivative of the same recurrence, in

@@ -182,3 +182,23 @@ def test_binding_backward_refuses_cpu_tensors():
     b = torch.zeros(1, 4, 1)
     with pytest.raises(ValueError, match="CUDA"):
         kda.chunk_bwd(x, x, x, la, b, x)
+
+
+def varlen(lib, q=FAKE, k=FAKE, v=FAKE, la=FAKE, beta=FAKE, cu=FAKE, S0=None, out=FAKE, ST=None,
+           N=2, TT=64, H=2, dk=128, dv=128, dtype=0):
+    return lib.kda_chunk_fwd_varlen(q, k, v, la, beta, cu, S0, out, ST, N, TT, H, dk, dv, dtype, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(cu=None), -1), (dict(cu=FAKE + 2), -3), (dict(q=None), -1), (dict(out=FAKE + 8), -3),
+    (dict(dtype=2), -1), (dict(N=-1), -1), (dict(TT=-1), -1), (dict(dk=0), -1), (dict(dv=129), -2),
+    (dict(N=2**15, H=2**15), -2),
+])
+def test_varlen_rejects(lib, kw, code):
+    assert varlen(lib, **kw) == code
+    assert detail(lib)
+
+
+def test_varlen_empty_is_noop(lib):
+    assert varlen(lib, N=0, cu=None, q=None, k=None, v=None, la=None, beta=None, out=None) == 0
+    assert varlen(lib, H=0, cu=None, q=None, k=None, v=None, la=None, beta=None, out=None) == 0
