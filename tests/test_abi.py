@@ -40,6 +40,20 @@ def test_every_declared_symbol_is_exported(lib):
         assert hasattr(lib, name), f"{name} declared in kda.h but not exported"
 
 
+def test_every_exported_entry_point_is_declared():
+    """The library's exported C entry points (``kda_*``, from its dynamic symbol
+    table) are exactly those the header documents; debug counters exist only in
+    debug builds."""
+    import subprocess
+    nm = subprocess.run(["nm", "-D", "--defined-only", kda.LIB_PATH], capture_output=True, text=True)
+    if nm.returncode != 0:
+        pytest.skip("nm is not available")
+    exported = {line.split()[-1] for line in nm.stdout.splitlines()
+                if line.split() and line.split()[-1].startswith("kda_")}
+    exported = {n for n in exported if not n.startswith("kda_debug_")}
+    assert exported == set(declared_functions())
+
+
 def test_status_names(lib):
     expect = {0: "KDA_OK", -1: "KDA_ERR_INVALID_ARG", -2: "KDA_ERR_UNSUPPORTED",
               -3: "KDA_ERR_ALIGNMENT", -4: "KDA_ERR_WORKSPACE", -5: "KDA_ERR_CUDA",
