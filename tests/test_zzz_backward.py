@@ -84,3 +84,19 @@ def test_zero_length_copies_the_state_cotangent():
     got = kda.chunk_bwd(q, q, q, la, beta, q, None, dST)
     torch.cuda.synchronize()
     assert torch.equal(got["S0"], dST)
+
+
+def test_autograd_through_the_library():
+    """kda_prefill: torch.autograd gradients through chunk_fwd and chunk_bwd on the GPU."""
+    x = I.prefill_inputs("fp32_small", T=40)
+    x["S0"] = 0.1 * torch.randn(1, 2, 16, 16, generator=torch.Generator().manual_seed(4))
+    t = {n: x[n].to(DEV).requires_grad_(True) for n in NAMES}
+    out, S_T = kda.kda_prefill(t["q"], t["k"], t["v"], t["log_alpha"], t["beta"], t["S0"], chunk=16)
+    g = torch.Generator().manual_seed(5)
+    W1, W2 = torch.randn(tuple(out.shape), generator=g), torch.randn(tuple(S_T.shape), generator=g)
+    ((out * W1.to(DEV)).sum() + (S_T * W2.to(DEV)).sum()).backward()
+    torch.cuda.synchronize()
+    ref = grad.backward(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], W1, S0=x["S0"], dS_T=W2)
+    for n in NAMES:
+        r = ref["d" + n]
+        assert_close(t[n].grad, r, 1e-4 * max(1.0, float(np.abs(r).max())), 0.0, f"grad {n}")
