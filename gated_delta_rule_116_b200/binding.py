@@ -47,7 +47,7 @@ def load():
     lib.kda_chunk_fwd_engine.restype = i
     lib.kda_engine_supported.argtypes = [i, i, i, i, i]
     lib.kda_engine_supported.restype = i
-    lib.kda_chunk_fwd_varlen.argtypes = [p] * 9 + [i, i, i, i, i, i, p]
+    lib.kda_chunk_fwd_varlen.argtypes = [p] * 10 + [i, i, i, i, i, i, p]
     lib.kda_chunk_fwd_varlen.restype = i
     lib.kda_chunk_bwd.argtypes = [p] * 14 + [i, i, i, i, i, i, p, sz, p]
     lib.kda_chunk_bwd.restype = i
@@ -149,14 +149,16 @@ def chunk_fwd(q, k, v, log_alpha, beta, S0=None, chunk: int = 64, *, out=None, S
     return out, S_T
 
 
-def chunk_fwd_varlen(q, k, v, log_alpha, beta, cu_seqlens, S0=None, *, out=None, S_T=None,
-                     output_final_state: bool = True, stream=None):
+def chunk_fwd_varlen(q, k, v, log_alpha, beta, cu_seqlens, S0=None, *, slot=None, out=None,
+                     S_T=None, output_final_state: bool = True, stream=None):
     """Chunked prefill of packed variable-length sequences (``kda_chunk_fwd_varlen``).
 
     q, k ``[total_T,H,dk]``, v ``[total_T,H,dv]`` (bf16 or fp32), log_alpha
     ``[total_T,H,dk]`` and beta ``[total_T,H]`` fp32, cu_seqlens ``[N+1]`` int32
-    token offsets on the device, S0 ``[N,H,dk,dv]`` fp32 or None. Returns
-    ``(out, S_T)``.
+    token offsets on the device. Without ``slot``, S0 and S_T are ``[N,H,dk,dv]``.
+    With ``slot`` (``[N]`` int32), they are a state cache ``[slots,H,dk,dv]``
+    (the decode step's) and sequence n uses row ``slot[n]``; S_T then defaults
+    to S0, updated in place. Returns ``(out, S_T)``.
     """
     lib = load()
     device = q.device
@@ -173,19 +175,32 @@ def chunk_fwd_varlen(q, k, v, log_alpha, beta, cu_seqlens, S0=None, *, out=None,
     if cu_seqlens.dim() != 1 or cu_seqlens.numel() < 1:
         raise ValueError("cu_seqlens must be a 1-D tensor of N+1 offsets")
     N = cu_seqlens.numel() - 1
-    if S0 is not None:
-        _require(S0, "S0", device, torch.float32, (N, H, dk, dv))
+    if slot is not None:
+        _require(slot, "slot", device, torch.int32, (N,))
+        if S_T is None and output_final_state:
+            if S0 is None:
+                raise ValueError("with a slot map, give the state cache as S0 or S_T")
+            S_T = S0
+        for t, name in ((S0, "S0"), (S_T, "S_T")):
+            if t is not None:
+                _require(t, name, device, torch.float32)
+                if t.dim() != 4 or tuple(t.shape[1:]) != (H, dk, dv):
+                    raise ValueError(f"{name} must be [slots,{H},{dk},{dv}] (got {tuple(t.shape)})")
+    else:
+        if S0 is not None:
+            _require(S0, "S0", device, torch.float32, (N, H, dk, dv))
+        if S_T is None and output_final_state:
+            S_T = torch.empty(N, H, dk, dv, device=device, dtype=torch.float32)
+        if S_T is not None:
+            _require(S_T, "S_T", device, torch.float32, (N, H, dk, dv))
     if out is None:
         out = torch.empty(TT, H, dv, device=device, dtype=q.dtype)
     _require(out, "out", device, q.dtype, (TT, H, dv))
-    if S_T is None and output_final_state:
-        S_T = torch.empty(N, H, dk, dv, device=device, dtype=torch.float32)
-    if S_T is not None:
-        _require(S_T, "S_T", device, torch.float32, (N, H, dk, dv))
     with torch.cuda.device(device):
         rc = lib.kda_chunk_fwd_varlen(
-            _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(cu_seqlens), _ptr(S0),
-            _ptr(out), _ptr(S_T), N, TT, H, dk, dv, _DTYPES[q.dtype], _stream(device, stream))
+            _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(cu_seqlens), _ptr(slot),
+            _ptr(S0), _ptr(out), _ptr(S_T), N, TT, H, dk, dv, _DTYPES[q.dtype],
+            _stream(device, stream))
     _check(rc)
     return out, S_T
 

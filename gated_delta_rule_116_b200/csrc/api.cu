@@ -272,9 +272,9 @@ int kda_chunk_bwd(const void *q, const void *k, const void *v, const float *log_
 }
 
 int kda_chunk_fwd_varlen(const void *q, const void *k, const void *v, const float *log_alpha,
-                         const float *beta, const int32_t *cu_seqlens, const float *S0, void *out,
-                         float *S_T, int N, int total_T, int H, int dk, int dv, int dtype,
-                         void *stream) {
+                         const float *beta, const int32_t *cu_seqlens, const int32_t *slot,
+                         const float *S0, void *out, float *S_T, int N, int total_T, int H, int dk,
+                         int dv, int dtype, void *stream) {
     g_detail[0] = '\0';
     if (dtype != KDA_BF16 && dtype != KDA_F32)
         return fail(KDA_ERR_INVALID_ARG, "dtype %d is neither KDA_BF16 nor KDA_F32", dtype);
@@ -290,14 +290,16 @@ int kda_chunk_fwd_varlen(const void *q, const void *k, const void *v, const floa
     if (!cu_seqlens) return fail(KDA_ERR_INVALID_ARG, "cu_seqlens is NULL");
     if ((reinterpret_cast<uintptr_t>(cu_seqlens) & 3u) != 0)
         return fail(KDA_ERR_ALIGNMENT, "cu_seqlens is not 4-byte aligned");
+    if ((reinterpret_cast<uintptr_t>(slot) & 3u) != 0)
+        return fail(KDA_ERR_ALIGNMENT, "slot is not 4-byte aligned");
     const bool tokens = total_T > 0;
     const Ptr ps[] = {{q, "q", tokens}, {k, "k", tokens}, {v, "v", tokens},
                       {log_alpha, "log_alpha", tokens}, {beta, "beta", tokens}, {out, "out", tokens},
                       {S0, "S0", false}, {S_T, "S_T", false}};
     int rc = check_pointers(ps, sizeof ps / sizeof ps[0]);
     if (rc != KDA_OK) return rc;
-    cudaError_t e = kda::launch_chunk_varlen(q, k, v, log_alpha, beta, cu_seqlens, S0, out, S_T, N,
-                                             total_T, H, dk, dv, dtype,
+    cudaError_t e = kda::launch_chunk_varlen(q, k, v, log_alpha, beta, cu_seqlens, slot, S0, out,
+                                             S_T, N, total_T, H, dk, dv, dtype,
                                              static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? KDA_OK : cuda_fail(e, "launching the variable-length prefill");
 }

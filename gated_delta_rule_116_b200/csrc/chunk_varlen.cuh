@@ -2,8 +2,11 @@
 // sequences, fp32 on CUDA cores (bodies; kernels and launch in chunk_varlen.cu).
 //
 // Sequence n occupies tokens cu_seqlens[n] .. cu_seqlens[n+1]-1 of packed
-// [total_T, H, d] tensors and starts from its own state S0[n] (or zeros); the
-// recurrence never crosses a sequence boundary. Per sequence this is the
+// [total_T, H, d] tensors and starts from its own state (or zeros); the
+// recurrence never crosses a sequence boundary. With a slot map, sequence n's
+// initial and final states are row slot[n] of state caches [slots, H, dk, dv]
+// (the layout of the decode step's cache, so a prefill can fill the rows that
+// decode steps then continue, in place); without one, row n. Per sequence this is the
 // chunked form of the prefill (Kimi Linear summary, es.news.hada.io/topic?id=31936,
 // section "Algoritmo paralelo por chunks"): fixed-length chunks starting from
 // the previous chunk's last state, the WY/UT form, and outputs that add the
@@ -20,8 +23,9 @@ using kbwd::kThreads;
 
 template <typename Tin>
 __device__ void varlen_body(float *sm, const Tin *q, const Tin *k, const Tin *v, const float *log_alpha,
-                            const float *beta, const int32_t *cu_seqlens, const float *S0, Tin *out,
-                            float *S_T, int total_T, int H, int dk, int dv) {
+                            const float *beta, const int32_t *cu_seqlens, const int32_t *slot,
+                            const float *S0, Tin *out, float *S_T, int total_T, int H, int dk,
+                            int dv) {
     const kbwd::Layout L(dk, kNV);
     kbwd::Tiles s(sm, L);
     const int tid = threadIdx.x, LD = L.LD, LC = L.LC, NV = L.NV;
@@ -31,9 +35,10 @@ __device__ void varlen_body(float *sm, const Tin *q, const Tin *k, const Tin *v,
     const int start = min(max(cu_seqlens[n], 0), total_T);
     const int end = min(max(cu_seqlens[n + 1], start), total_T);
     const int len = end - start;
+    const long row = (slot ? static_cast<long>(slot[n]) : static_cast<long>(n)) * H + h;   // state row
     for (int e = tid; e < dk * NV; e += kThreads) {
         const int c = e / NV, j = e - c * NV;
-        s.S[e] = (S0 && j < nv) ? S0[(static_cast<long>(nh) * dk + c) * dv + n0 + j] : 0.f;
+        s.S[e] = (S0 && j < nv) ? S0[(row * dk + c) * dv + n0 + j] : 0.f;
     }
     const int nchunks = (len + kC - 1) / kC;
     for (int ch = 0; ch < nchunks; ++ch) {
@@ -68,7 +73,7 @@ __device__ void varlen_body(float *sm, const Tin *q, const Tin *k, const Tin *v,
     if (S_T)
         for (int e = tid; e < dk * NV; e += kThreads) {
             const int c = e / NV, j = e - c * NV;
-            if (j < nv) S_T[(static_cast<long>(nh) * dk + c) * dv + n0 + j] = s.S[e];
+            if (j < nv) S_T[(row * dk + c) * dv + n0 + j] = s.S[e];
         }
 }
 

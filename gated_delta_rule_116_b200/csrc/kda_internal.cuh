@@ -64,9 +64,9 @@ cudaError_t launch_chunk_bwd(const void *q, const void *k, const void *v, const 
                              int T, int H, int dk, int dv, int dtype, void *ws, cudaStream_t s);
 // Variable-length prefill (chunk_varlen.cu).
 cudaError_t launch_chunk_varlen(const void *q, const void *k, const void *v, const float *la,
-                                const float *beta, const int32_t *cu_seqlens, const float *S0,
-                                void *out, float *S_T, int N, int total_T, int H, int dk, int dv,
-                                int dtype, cudaStream_t s);
+                                const float *beta, const int32_t *cu_seqlens, const int32_t *slot,
+                                const float *S0, void *out, float *S_T, int N, int total_T, int H,
+                                int dk, int dv, int dtype, cudaStream_t s);
 // Ring of operand images of the cluster engine: 3 producers x 3 slots of 81 KB per head.
 constexpr size_t kClusterRingBytesPerHead = 9ull * 82944;
 

@@ -144,8 +144,11 @@ int kda_recurrent_step(const void *q, const void *k, const void *v,
 /*
  * Chunked prefill of a packed batch of N sequences of different lengths.
  * Sequence n is tokens cu_seqlens[n] .. cu_seqlens[n+1]-1 of the packed
- * tensors and starts from S0[n] (or zeros); no state crosses a sequence
- * boundary. Computes in fp32 on CUDA cores with 16-token chunks.
+ * tensors and starts from its own initial state (or zeros); no state crosses a
+ * sequence boundary. With a slot map the states live in a state cache of the
+ * decode step's layout: a prefill reads and writes row slot[n], and
+ * kda_recurrent_step continues from the same rows. Computes in fp32 on CUDA
+ * cores with 16-token chunks.
  *
  *   q, k       [total_T,H,dk]  dtype     (packed over sequences)
  *   v          [total_T,H,dv]  dtype
@@ -158,16 +161,21 @@ int kda_recurrent_step(const void *q, const void *k, const void *v,
  *                                       to [0, total_T], so no access leaves the
  *                                       tensors. Tokens outside every sequence
  *                                       keep their previous out values.
- *   S0         [N,H,dk,dv] fp32         NULL means zeros
+ *   slot       [N] int32 (device)       state row of sequence n; NULL means n.
+ *                                       Entries must be distinct and in
+ *                                       [0, slots) (not checked: device data)
+ *   S0         [rows,H,dk,dv] fp32      initial states (rows = slots, or N
+ *                                       without a slot map); NULL means zeros
  *   out        [total_T,H,dv] dtype     written for every token of a sequence
- *   S_T        [N,H,dk,dv] fp32         final state per sequence; NULL skips it
+ *   S_T        [rows,H,dk,dv] fp32      final states; NULL skips them. S_T may
+ *                                       be S0 (the state cache, in place)
  * N = 0 or H = 0 is a no-op. Supported: dtype KDA_BF16 or KDA_F32, dk and dv
  * in [1,128], N*H <= 2^29 - 1.
  */
 int kda_chunk_fwd_varlen(const void *q, const void *k, const void *v,
                          const float *log_alpha, const float *beta,
-                         const int32_t *cu_seqlens, const float *S0,
-                         void *out, float *S_T,
+                         const int32_t *cu_seqlens, const int32_t *slot,
+                         const float *S0, void *out, float *S_T,
                          int N, int total_T, int H, int dk, int dv, int dtype,
                          void *stream);
 

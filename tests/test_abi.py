@@ -198,13 +198,15 @@ def test_binding_backward_refuses_cpu_tensors():
         kda.chunk_bwd(x, x, x, la, b, x)
 
 
-def varlen(lib, q=FAKE, k=FAKE, v=FAKE, la=FAKE, beta=FAKE, cu=FAKE, S0=None, out=FAKE, ST=None,
-           N=2, TT=64, H=2, dk=128, dv=128, dtype=0):
-    return lib.kda_chunk_fwd_varlen(q, k, v, la, beta, cu, S0, out, ST, N, TT, H, dk, dv, dtype, None)
+def varlen(lib, q=FAKE, k=FAKE, v=FAKE, la=FAKE, beta=FAKE, cu=FAKE, slot=None, S0=None, out=FAKE,
+           ST=None, N=2, TT=64, H=2, dk=128, dv=128, dtype=0):
+    return lib.kda_chunk_fwd_varlen(q, k, v, la, beta, cu, slot, S0, out, ST, N, TT, H, dk, dv, dtype,
+                                    None)
 
 
 @pytest.mark.parametrize("kw,code", [
-    (dict(cu=None), -1), (dict(cu=FAKE + 2), -3), (dict(q=None), -1), (dict(out=FAKE + 8), -3),
+    (dict(cu=None), -1), (dict(cu=FAKE + 2), -3), (dict(slot=FAKE + 2), -3), (dict(q=None), -1),
+    (dict(out=FAKE + 8), -3),
     (dict(dtype=2), -1), (dict(N=-1), -1), (dict(TT=-1), -1), (dict(dk=0), -1), (dict(dv=129), -2),
     (dict(N=2**15, H=2**15), -2),
 ])

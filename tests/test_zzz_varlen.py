@@ -60,3 +60,35 @@ def test_fp32_other_sizes_no_state():
 def test_bf16_head_size_128():
     flat, S0, cu = packed("prefill_4k", [50, 0, 70], H=2, seed=3)
     check(flat, S0, cu)
+
+
+def test_paged_prefill_then_decode():
+    """Prefill packed sequences into rows of a state cache (slot map, in place), then
+    one decode step from the same rows: the serving handoff. Each sequence's
+    outputs, its decode output and its cache row equal the oracle run on that
+    sequence plus its next token; rows outside the map are untouched."""
+    lens, slots, H = [20, 0, 37], [3, 0, 4], 2
+    flat, _, cu = packed("fp32_small", lens, H=H, seed=6)
+    g = torch.Generator().manual_seed(7)
+    cache0 = 0.1 * torch.randn(5, H, 16, 16, generator=g)
+    nxt = I.prefill_inputs("fp32_small", B=1, T=len(lens), H=H, seed=9)   # one new token per sequence
+    step = {n: nxt[n][0].contiguous() for n in ("q", "k", "v", "log_alpha", "beta")}
+    cache = cache0.to(DEV)
+    slot = torch.tensor(slots, dtype=torch.int32, device=DEV)
+    dev = {n: t.to(DEV) for n, t in flat.items()}
+    out, ST = kda.chunk_fwd_varlen(dev["q"], dev["k"], dev["v"], dev["log_alpha"], dev["beta"],
+                                   cu.to(DEV), cache, slot=slot)
+    assert ST.data_ptr() == cache.data_ptr()
+    o1 = kda.recurrent_step(*(step[n].to(DEV) for n in ("q", "k", "v", "log_alpha", "beta")), cache, slot)
+    torch.cuda.synchronize()
+    out, o1, cache = out.cpu(), o1.cpu(), cache.cpu()
+    atol, rtol = tol_for(torch.float32)
+    for n, r in enumerate(slots):
+        a, b = int(cu[n]), int(cu[n + 1])
+        cat = lambda name: torch.cat([flat[name][a:b], step[name][n:n + 1]])[None]
+        ref_o, ref_s = oracle.forward(cat("q"), cat("k"), cat("v"), cat("log_alpha"), cat("beta"), cache0[r][None])
+        assert_close(out[a:b], ref_o[0, :-1], atol, rtol, f"prefill out of sequence {n}")
+        assert_close(o1[n], ref_o[0, -1], atol, rtol, f"decode out of sequence {n}")
+        assert_close(cache[r], ref_s[0], atol, rtol, f"cache row {r}")
+    for r in (1, 2):
+        assert torch.equal(cache[r], cache0[r])
