@@ -24,6 +24,8 @@
 //    results; serialise them;
 //  * nothing here allocates: no cudaMalloc, no cudaFree, no library routine
 //    that allocates.
+#include <cuda.h>
+#include <limits.h>
 #include <stdarg.h>
 #include <stdio.h>
 
@@ -41,20 +43,47 @@ constexpr int kMaxDevices = 64;
 static __device__ __align__(256) uint8_t g_static_ring[kStaticBytes];
 
 std::mutex g_setup_mutex;
-void *g_ring_address[kMaxDevices];  // device address of g_static_ring, per device
+// Device address of g_static_ring per device, and the context it was looked up
+// in: after a device reset (or a released and re-created primary context) the
+// module is loaded again and the address must be looked up again.
+void *g_ring_address[kMaxDevices];
+CUcontext g_ring_context[kMaxDevices];
 
-// Device address of the array on the current device, looked up once per device.
+// cuCtxGetCurrent through the runtime's driver entry point (the library does not
+// link the driver library directly, so it still loads where no driver exists).
+typedef CUresult (*CtxGetCurrentFn)(CUcontext *);
+CUcontext current_context() {
+    static CtxGetCurrentFn fn = nullptr;
+    if (!fn) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult qr;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &qr) != cudaSuccess ||
+            qr != cudaDriverEntryPointSuccess)
+            return nullptr;
+        fn = reinterpret_cast<CtxGetCurrentFn>(p);
+    }
+    CUcontext ctx = nullptr;
+    return fn(&ctx) == CUDA_SUCCESS ? ctx : nullptr;
+}
+
+// Device address of the array on the current device, looked up once per device
+// and context. cudaGetSymbolAddress makes the device's primary context current
+// on its first use, so the context is read again after it.
 cudaError_t ring_address(void **out) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    CUcontext ctx = current_context();
     std::lock_guard<std::mutex> lock(g_setup_mutex);
-    if (!g_ring_address[dev]) {
+    if (!ctx || !g_ring_address[dev] || g_ring_context[dev] != ctx) {
         void *p = nullptr;
         e = cudaGetSymbolAddress(&p, g_static_ring);
         if (e != cudaSuccess) return e;
+        ctx = current_context();
+        if (!ctx) return cudaErrorDeviceUninitialized;
         g_ring_address[dev] = p;
+        g_ring_context[dev] = ctx;
     }
     *out = g_ring_address[dev];
     return cudaSuccess;
@@ -77,6 +106,11 @@ extern "C" int kda_chunk_fwd_static(const void *q, const void *k, const void *v,
                                 "kda_chunk_fwd_static runs the cluster engine only: bf16, "
                                 "dk = dv = 128, chunk = 64 (got dtype %d, dk %d, dv %d, chunk %d)",
                                 dtype, dk, dv, chunk);
+    // Token rows are 32-bit tensor-map coordinates, as in kda_chunk_fwd.
+    if (static_cast<long long>(B) * T > INT_MAX)
+        return set_error_detail(KDA_ERR_UNSUPPORTED,
+                                "B*T = %lld tokens: more than 2^31 - 1; split the batch",
+                                static_cast<long long>(B) * T);
     if (static_cast<long>(B) * H > kMaxHeads)
         return set_error_detail(KDA_ERR_UNSUPPORTED,
                                 "B*H = %ld heads exceed the %d heads kda_chunk_fwd_static's fixed "

@@ -222,11 +222,12 @@ size_t kda_bwd_workspace_bytes(int B, int T, int H, int dk, int dv, int dtype);
  * process whose pool allocator owns all free memory, or a plug-in inside a
  * framework that owns every allocation.
  *   Arguments as kda_chunk_fwd without the workspace; supported: bf16,
- *   dk = dv = 128, chunk = 64, and B * H <= 32 heads (larger problems return
- *   KDA_ERR_UNSUPPORTED and must use kda_chunk_fwd).
+ *   dk = dv = 128, chunk = 64, B * H <= 32 heads and B * T <= 2^31 - 1 tokens
+ *   (larger problems return KDA_ERR_UNSUPPORTED; they must use kda_chunk_fwd).
  *   Every GPU that loads the library holds the array (22.8 MiB) until exit.
  *   The first call on a device looks up the array's address with that device
- *   current; make it before any stream capture. All calls share the array:
+ *   current (again after a device reset re-creates the context); make it
+ *   before any stream capture. All calls share the array:
  *   calls that overlap on the GPU race and must be serialised by the caller.
  *   No cudaMalloc, cudaFree or allocating library routine is called.
  */

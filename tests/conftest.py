@@ -24,3 +24,20 @@ def pytest_collection_modifyitems(config, items):
     for item in items:
         if "gpu" in item.keywords:
             item.add_marker(skip)
+
+
+def pytest_terminal_summary(terminalreporter):
+    """Margins of every CUDA-vs-oracle comparison of this run (worst first)."""
+    try:
+        from kda_check import RECORDS
+    except ImportError:  # pragma: no cover
+        return
+    if not RECORDS:
+        return
+    rows = sorted(RECORDS, key=lambda r: -r[3])
+    tr = terminalreporter
+    tr.section("parity margins (error / bound; 1.0 = at the tolerance)")
+    tr.write_line(f"{'comparison':60s} {'max_abs':>10s} {'max_rel':>10s} {'err/bound':>9s}")
+    for what, ma, mr, ratio in rows[:40]:
+        tr.write_line(f"{what[:60]:60s} {ma:10.3e} {mr:10.3e} {ratio:9.3f}")
+    tr.write_line(f"{len(rows)} comparisons; worst error/bound {rows[0][3]:.3f} ({rows[0][0]})")

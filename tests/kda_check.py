@@ -5,6 +5,10 @@ Tolerances (written here once, used by every parity test):
 * bf16 q/k/v with fp32 gates and state: |x - ref| <= 2e-3 + 1e-2 * |ref| for
   every element of ``out`` and ``S_T`` (max-abs 2e-3, relative 1e-2).
 * fp32 q/k/v: |x - ref| <= 1e-4 for every element.
+
+Every comparison records its margin (max-abs error, max-rel error and the
+worst error / bound ratio) in ``RECORDS``; ``tests/conftest.py`` prints the
+table at the end of the run, so a passing run shows how much room is left.
 """
 import numpy as np
 import torch
@@ -15,6 +19,9 @@ F32_ATOL, F32_RTOL = 1e-4, 0.0
 
 def tol_for(dtype):
     return (F32_ATOL, F32_RTOL) if dtype == torch.float32 else (BF16_ATOL, BF16_RTOL)
+
+
+RECORDS = []   # (what, max_abs, max_rel, worst error / bound)
 
 
 def to_np(x):
@@ -34,9 +41,12 @@ def assert_close(x, ref, atol, rtol, what=""):
     bound = atol + rtol * np.abs(ref)
     worst = np.unravel_index(np.argmax(err - bound), err.shape)
     stats = {"max_abs": float(err.max()),
-             "max_rel": float((err / np.maximum(np.abs(ref), 1e-30)).max())}
+             "max_rel": float((err / np.maximum(np.abs(ref), 1e-30)).max()),
+             "ratio": float((err / bound).max())}
+    RECORDS.append((what, stats["max_abs"], stats["max_rel"], stats["ratio"]))
     assert (err <= bound).all(), (
         f"{what}: {int((err > bound).sum())} of {err.size} elements out of tolerance "
-        f"(atol {atol}, rtol {rtol}); max_abs {stats['max_abs']:.3e}; worst at {worst}: "
+        f"(atol {atol}, rtol {rtol}); max_abs {stats['max_abs']:.3e}, error/bound "
+        f"{stats['ratio']:.3f}; worst at {worst}: "
         f"got {x[worst]:.6e}, want {ref[worst]:.6e}")
     return stats

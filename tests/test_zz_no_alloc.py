@@ -8,9 +8,12 @@ and kda_chunk_fwd_static takes only inputs and outputs.
 
 The GPU test calls it twice in a row through the C ABI, on different problems
 queued back to back on one stream (the second reuses the array the first
-left behind), and checks both against kda_chunk_fwd with a workspace, within
-the bf16 tolerance of the parity tests. The file is named to be collected last,
-so a run that stops at its first failure has run every other test before it.
+left behind). Both calls run the same deterministic kernel as kda_chunk_fwd
+with a workspace, so their results must be bit-for-bit equal to that call's;
+the second problem is also compared with the fp64 oracle within the bf16
+tolerance of the parity tests, and no bounded device wait may have given up.
+The file is named to be collected last, so a run that stops at its first
+failure has run every other test before it.
 """
 import ctypes
 
@@ -18,6 +21,7 @@ import pytest
 import torch
 
 import kda_inputs as I
+import oracle
 from kda_check import BF16_ATOL, BF16_RTOL, assert_close
 from gated_delta_rule_116_b200 import binding
 
@@ -37,6 +41,8 @@ def lib():
     lib.kda_workspace_bytes.argtypes = [i, i, i, i, i, i, i]
     lib.kda_workspace_bytes.restype = sz
     lib.kda_last_error_detail.restype = ctypes.c_char_p
+    lib.kda_device_status.argtypes = [p]
+    lib.kda_device_status.restype = i
     return lib
 
 
@@ -86,6 +92,11 @@ def test_static_rejects_more_heads_than_the_array_holds():
     rc = L.kda_chunk_fwd_static(fake, fake, fake, fake, fake, None, fake, None,
                                  1, 64, 2, 64, 128, 64, KDA_BF16, None)
     assert rc == -2
+    # more tokens than 32-bit token rows address (B*T = 2^31 + 2), within the head limit
+    rc = L.kda_chunk_fwd_static(fake, fake, fake, fake, fake, None, fake, None,
+                                 2, 2**30 + 1, 2, 128, 128, 64, KDA_BF16, None)
+    assert rc == -2
+    assert "2^31" in L.kda_last_error_detail().decode()
 
 
 @pytest.mark.gpu
@@ -101,8 +112,14 @@ def test_static_matches_workspace_entry_point_on_two_calls_in_a_row():
         rc = call_static(L, pb, stream)
         assert rc == 0, L.kda_last_error_detail().decode()
     torch.cuda.synchronize()
+    assert L.kda_device_status(ctypes.c_void_p(stream.cuda_stream)) == 0, "a device wait gave up"
     for name, pb in (("first", first), ("second", second)):
         ref_out, ref_st = call_with_workspace(L, pb, stream)
         torch.cuda.synchronize()
-        assert_close(pb["out"].float(), ref_out.float(), BF16_ATOL, BF16_RTOL, f"{name} out")
-        assert_close(pb["S_T"], ref_st, BF16_ATOL, BF16_RTOL, f"{name} S_T")
+        assert torch.equal(pb["out"], ref_out), f"{name} out differs from kda_chunk_fwd"
+        assert torch.equal(pb["S_T"], ref_st), f"{name} S_T differs from kda_chunk_fwd"
+    # the second problem (it ran on the array the first one left behind) against the oracle
+    cpu = {k: (v.cpu() if isinstance(v, torch.Tensor) else v) for k, v in second.items()}
+    o_ref, s_ref = oracle.forward(cpu["q"], cpu["k"], cpu["v"], cpu["la"], cpu["beta"], None)
+    assert_close(second["out"], o_ref, BF16_ATOL, BF16_RTOL, "second out vs oracle")
+    assert_close(second["S_T"], s_ref, BF16_ATOL, BF16_RTOL, "second S_T vs oracle")
