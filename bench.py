@@ -178,7 +178,7 @@ def run_ours(args, rank, world, device):
     w = I.WORKLOADS[PREFILL]
     inp = I.prefill_inputs(w, device=device)
     q, k, v, la, beta, S0 = (inp[x] for x in ("q", "k", "v", "log_alpha", "beta", "S0"))
-    engine = next(e for e in ("tc_cluster", "tc", "generic")
+    engine = next(e for e in ("tc_cluster", "generic")
                   if kda.engine_supported(e, w.dk, w.dv, w.chunk, w.dtype))
     out = torch.empty(w.B, w.T, w.H, w.dv, device=device, dtype=w.dtype)
     S_T = torch.empty(w.B, w.H, w.dk, w.dv, device=device, dtype=torch.float32)
@@ -217,14 +217,15 @@ def run_ours(args, rank, world, device):
                 "flops_per_launch": prefill_flops(w),
                 "tensor_tflops_achieved": round(prefill_flops(w) / (ms_kernel / 1e3) / 1e12, 2)}
 
+    fused = run_fused(kda, w, ws, args, device, stream) if engine == "tc_cluster" else None
     e2e = run_e2e(kda, w, inp, engine, ws, args, device, stream, world)
     decode = run_decode(kda, args, device, stream, world)
     clocks = clk.summary()
-    launches = args.steps  # one prefill kernel per step
+    launches = args.steps  # one prefill kernel per step (the fused leg's launches are outside the timed region)
 
     cpu = None
     if rank == 0 and world == 1 and not args.skip_cpu_baseline:
-        cpu = cpu_baseline(args)
+        cpu = cpu_baseline(args, gpu_inputs=inp, gpu_out=out, gpu_st=S_T)
 
     if rank == 0:
         line = {
@@ -238,9 +239,38 @@ def run_ours(args, rank, world, device):
                        "engine": engine, "per_rank": "one full workload per GPU",
                        "l2": f"inputs larger than L2 ({bytes_alg / 1e9:.2f} GB moved per step)"},
             "roofline": roofline, "e2e": e2e, "gpu_launches": launches + decode.pop("launches"),
-            "clocks": clocks, "decode": decode, "cpu_baseline": cpu,
+            "clocks": clocks, "decode": decode, "fused_prologue": fused, "cpu_baseline": cpu,
         }
         print(json.dumps(line), flush=True)
+
+
+def run_fused(kda, w, ws, args, device, stream):
+    """The same prefill with the layer prologue fused in (kda_chunk_fwd_fused): raw q, k
+    and the gate's pre-activation (bf16) instead of unit q, k and fp32 log alpha. Its
+    algorithmic bytes per token-head are 3*2*d + 2*d + 4 + 2*d = 1284 at d = 128."""
+    lw = I.prefill_layer_inputs(w, device=device)
+    out = torch.empty(w.B, w.T, w.H, w.dv, device=device, dtype=w.dtype)
+    S_T = torch.empty(w.B, w.H, w.dk, w.dv, device=device, dtype=torch.float32)
+
+    def step():
+        kda.chunk_fwd_fused(lw["q"], lw["k"], lw["v"], lw["gate"], lw["beta"], lw["S0"], w.chunk,
+                            out=out, S_T=S_T, workspace=ws, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(device)
+    evs = time_events(step, args.steps, stream)
+    torch.cuda.synchronize(device)
+    ms = statistics.mean(s.elapsed_time(e) for s, e in evs)
+    e = 2 if w.dtype == torch.bfloat16 else 4
+    bytes_alg = (w.B * w.T * w.H * (2 * w.dk * e + w.dv * e + w.dk * e + 4 + w.dv * e)
+                 + w.B * w.H * 4 * w.dk * w.dv * (2 if w.s0_std > 0 else 1))
+    hbm, src = peaks()
+    gbs = bytes_alg / (ms / 1e3) / 1e9
+    return {"entry": "kda_chunk_fwd_fused", "kernel_ms": round(ms, 4),
+            "tokens_per_s": round(w.tokens / (ms / 1e3), 1), "bytes_per_launch": bytes_alg,
+            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm, "unit": "GB/s",
+                         "frac": round(gbs / hbm, 4), "peak_source": src}}
 
 
 def run_e2e(kda, w, inp, engine, ws, args, device, stream, world):
@@ -367,8 +397,15 @@ def run_only(args, device):
 
 # ---------------------------------------------------------------------------- CPU oracle
 
-def cpu_baseline(args, seconds_hint=True):
-    """The fp64 oracle, as it stands, on a bounded sample of prefill_32k."""
+def cpu_baseline(args, gpu_inputs=None, gpu_out=None, gpu_st=None):
+    """The fp64 oracle, as it stands, on a bounded sample of prefill_32k.
+
+    With the bench's own device inputs and results, the oracle runs on exactly
+    those inputs (copied to the host) and its output is compared element by
+    element with the GPU's over the whole sample: the line then reports the
+    parity margin of the timed workload itself (max-abs, max-rel and worst
+    error / bound for the bf16 bound |x - ref| <= 2e-3 + 1e-2 |ref|)."""
+    import numpy as np
     import oracle
 
     w = I.WORKLOADS[PREFILL]
@@ -376,17 +413,35 @@ def cpu_baseline(args, seconds_hint=True):
     threads = max(1, min(cores, args.cpu_threads or cores))
     n_heads = w.H
     T_s = min(w.T, args.cpu_tokens)
-    inp = I.prefill_inputs(w, T=T_s, H=n_heads)
+    if gpu_inputs is not None:
+        cut = lambda x: None if x is None else x[:, :T_s].cpu()
+        inp = {n: cut(gpu_inputs[n]) for n in ("q", "k", "v", "log_alpha", "beta")}
+        inp["S0"] = None if gpu_inputs["S0"] is None else gpu_inputs["S0"].cpu()
+    else:
+        inp = I.prefill_inputs(w, T=T_s, H=n_heads)
     t = time.perf_counter()
-    oracle.forward(inp["q"], inp["k"], inp["v"], inp["log_alpha"], inp["beta"], inp["S0"],
-                   nthreads=threads)
+    ref_o, ref_s = oracle.forward(inp["q"], inp["k"], inp["v"], inp["log_alpha"], inp["beta"],
+                                  inp["S0"], nthreads=threads)
     dt = time.perf_counter() - t
     tok_s = T_s * (n_heads / w.H) / dt
     used = min(threads, n_heads)
-    return {"value": round(tok_s, 2), "unit": "tokens/s", "cores": used, "kind": "oracle",
-            "sample": f"fp64 oracle on {n_heads} of {w.H} heads x first {T_s} tokens of {PREFILL} "
-                      f"({dt:.1f} s); tokens/s scaled by heads/{w.H}",
-            "host_cores": cores}
+    res = {"value": round(tok_s, 2), "unit": "tokens/s", "cores": used, "kind": "oracle",
+           "sample": f"fp64 oracle on {n_heads} of {w.H} heads x first {T_s} tokens of {PREFILL} "
+                     f"({dt:.1f} s); tokens/s scaled by heads/{w.H}",
+           "host_cores": cores}
+    if gpu_out is not None:
+        def margin(x, ref):
+            x = x.double().cpu().numpy()
+            err = np.abs(x - ref)
+            return {"max_abs": float(err.max()),
+                    "max_rel": float((err / np.maximum(np.abs(ref), 1e-30)).max()),
+                    "worst_err_over_bound": float((err / (2e-3 + 1e-2 * np.abs(ref))).max())}
+        par = {"out": margin(gpu_out[:, :T_s], ref_o), "elements": int(ref_o.size)}
+        if T_s == w.T:
+            par["S_T"] = margin(gpu_st, ref_s)
+        par["bound"] = "|x - ref| <= 2e-3 + 1e-2 |ref| (bf16 inputs, fp32 state)"
+        res["parity"] = par
+    return res
 
 
 def run_reference(args, rank, world):
@@ -464,7 +519,7 @@ def main(argv=None):
     ap.add_argument("--only", choices=["prefill", "decode"],
                     help="profiling mode: run just this kernel's workload (warm-up + steps), "
                          "print its time, no JSON line")
-    ap.add_argument("--engine", default=None, choices=["auto", "generic", "tc", "tc_cluster"],
+    ap.add_argument("--engine", default=None, choices=["auto", "generic", "tc_cluster"],
                     help="with --only prefill: the prefill engine (default auto)")
     ap.add_argument("--workload", default=None,
                     help="with --only prefill: the prefill workload to run (default prefill_32k)")

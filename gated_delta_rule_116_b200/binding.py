@@ -14,7 +14,7 @@ import torch
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libkda.so")
 
 KDA_BF16, KDA_F32 = 0, 1
-ENGINES = {"auto": 0, "generic": 1, "tc": 2, "tc_cluster": 3}
+ENGINES = {"auto": 0, "generic": 1, "tc_cluster": 3}
 _DTYPES = {torch.bfloat16: KDA_BF16, torch.float32: KDA_F32}
 
 _lib = None
@@ -44,6 +44,8 @@ def load():
     lib.kda_chunk_fwd.argtypes = chunk_args
     lib.kda_chunk_fwd.restype = i
     lib.kda_chunk_fwd_engine.argtypes = [i] + chunk_args
+    lib.kda_chunk_fwd_fused.argtypes = chunk_args
+    lib.kda_chunk_fwd_fused.restype = i
     lib.kda_chunk_fwd_engine.restype = i
     lib.kda_engine_supported.argtypes = [i, i, i, i, i]
     lib.kda_engine_supported.restype = i
@@ -60,6 +62,8 @@ def load():
     lib.kda_last_error_detail.argtypes = []
     lib.kda_last_error_detail.restype = ctypes.c_char_p
     lib.kda_device_status.argtypes = [p]
+    lib.kda_test_inject_wait_timeout.argtypes = [i]
+    lib.kda_test_inject_wait_timeout.restype = i
     lib.kda_device_status.restype = i
     lib.kda_version.restype = i
     _lib = lib
@@ -145,6 +149,45 @@ def chunk_fwd(q, k, v, log_alpha, beta, S0=None, chunk: int = 64, *, out=None, S
             ENGINES[engine], _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(S0),
             _ptr(out), _ptr(S_T), B, T, H, dk, dv, chunk, _DTYPES[q.dtype], _ptr(workspace),
             ws_bytes, _stream(device, stream))
+    _check(rc)
+    return out, S_T
+
+
+def chunk_fwd_fused(q, k, v, gate, beta, S0=None, chunk: int = 64, *, out=None, S_T=None,
+                    output_final_state: bool = True, workspace=None, stream=None):
+    """Chunked prefill with the layer prologue fused in (``kda_chunk_fwd_fused``):
+    q and k are L2-normalised and log_alpha = -softplus(gate) inside the kernel.
+
+    q, k ``[B,T,H,128]`` (un-normalised), v ``[B,T,H,128]`` and gate ``[B,T,H,128]``
+    (the gate's pre-activation), all bf16; beta ``[B,T,H]`` fp32; S0 as ``chunk_fwd``.
+    Returns ``(out, S_T)`` like ``chunk_fwd``.
+    """
+    lib = load()
+    device = q.device
+    _require(q, "q", device, torch.bfloat16)
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    _require(k, "k", device, torch.bfloat16, (B, T, H, dk))
+    _require(v, "v", device, torch.bfloat16, (B, T, H, dv))
+    _require(gate, "gate", device, torch.bfloat16, (B, T, H, dk))
+    _require(beta, "beta", device, torch.float32, (B, T, H))
+    if S0 is not None:
+        _require(S0, "S0", device, torch.float32, (B, H, dk, dv))
+    if out is None:
+        out = torch.empty(B, T, H, dv, device=device, dtype=torch.bfloat16)
+    _require(out, "out", device, torch.bfloat16, (B, T, H, dv))
+    if S_T is None and output_final_state:
+        S_T = torch.empty(B, H, dk, dv, device=device, dtype=torch.float32)
+    if S_T is not None:
+        _require(S_T, "S_T", device, torch.float32, (B, H, dk, dv))
+    need = int(lib.kda_workspace_bytes(B, T, H, dk, dv, chunk, KDA_BF16))
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, device=device, dtype=torch.uint8)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    with torch.cuda.device(device):
+        rc = lib.kda_chunk_fwd_fused(
+            _ptr(q), _ptr(k), _ptr(v), _ptr(gate), _ptr(beta), _ptr(S0), _ptr(out), _ptr(S_T),
+            B, T, H, dk, dv, chunk, KDA_BF16, _ptr(workspace), ws_bytes, _stream(device, stream))
     _check(rc)
     return out, S_T
 
@@ -281,6 +324,13 @@ def recurrent_step(q, k, v, log_alpha, beta, state, slot=None, *, out=None, stre
                                     _DTYPES[q.dtype], _stream(device, stream))
     _check(rc)
     return out
+
+
+def test_inject_wait_timeout(on: bool) -> bool:
+    """Test hook of the prefill engine's give-up path (``kda_test_inject_wait_timeout``):
+    while on, cluster-engine launches run out a bounded device wait on purpose (no
+    fault, no trap) and ``device_status`` reports it. Returns the previous setting."""
+    return bool(load().kda_test_inject_wait_timeout(1 if on else 0))
 
 
 def device_status(stream=None, device=None):

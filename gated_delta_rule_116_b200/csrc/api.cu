@@ -75,7 +75,7 @@ int *device_error_word() { return device_error_ptr(); }
 
 extern "C" {
 
-int kda_version(void) { return 10000; }
+int kda_version(void) { return 20000; }
 
 const char *kda_strerror(int code) {
     switch (code) {
@@ -92,6 +92,8 @@ const char *kda_strerror(int code) {
 
 const char *kda_last_error_detail(void) { return g_detail; }
 
+int kda_test_inject_wait_timeout(int on) { return kda::set_test_timeout(on); }
+
 int kda_engine_supported(int engine, int dk, int dv, int chunk, int dtype) {
     const bool generic = (dtype == KDA_BF16 || dtype == KDA_F32) && dk >= 1 && dv >= 1 &&
                          dk <= 128 && dv <= 128 && dv % 4 == 0 &&
@@ -99,7 +101,6 @@ int kda_engine_supported(int engine, int dk, int dv, int chunk, int dtype) {
     switch (engine) {
         case KDA_ENGINE_AUTO:
         case KDA_ENGINE_GENERIC: return generic ? 1 : 0;
-        case KDA_ENGINE_TC: return generic && kda::chunk_tc_supported(dk, dv, chunk, dtype) ? 1 : 0;
         case KDA_ENGINE_TC_CLUSTER:
             return generic && kda::chunk_cluster_supported(dk, dv, chunk, dtype) ? 1 : 0;
         default: return 0;
@@ -110,7 +111,6 @@ size_t kda_workspace_bytes(int B, int T, int H, int dk, int dv, int chunk, int d
     if (B <= 0 || T <= 0 || H <= 0) return 0;
     if (kda::chunk_cluster_supported(dk, dv, chunk, dtype))
         return kda::chunk_cluster_workspace_bytes(B, H);
-    if (kda::chunk_tc_supported(dk, dv, chunk, dtype)) return kda::chunk_tc_workspace_bytes(B, T, H);
     return 0;
 }
 
@@ -119,7 +119,7 @@ int kda_chunk_fwd_engine(int engine, const void *q, const void *k, const void *v
                          float *S_T, int B, int T, int H, int dk, int dv, int chunk, int dtype,
                          void *workspace, size_t workspace_bytes, void *stream) {
     g_detail[0] = '\0';
-    if (engine < KDA_ENGINE_AUTO || engine > KDA_ENGINE_TC_CLUSTER)
+    if (engine != KDA_ENGINE_AUTO && engine != KDA_ENGINE_GENERIC && engine != KDA_ENGINE_TC_CLUSTER)
         return fail(KDA_ERR_INVALID_ARG, "engine %d is not a kda_engine", engine);
     if (B < 0 || T < 0 || H < 0)
         return fail(KDA_ERR_INVALID_ARG, "B=%d T=%d H=%d must be >= 0", B, T, H);
@@ -152,36 +152,78 @@ int kda_chunk_fwd_engine(int engine, const void *q, const void *k, const void *v
         return e == cudaSuccess ? KDA_OK : cuda_fail(e, "copying S0 to S_T");
     }
 
-    const bool tc_ok = kda::chunk_tc_supported(dk, dv, chunk, dtype);
     const bool cl_ok = kda::chunk_cluster_supported(dk, dv, chunk, dtype);
-    bool use_tc = false, use_cluster = false;
-    if (engine == KDA_ENGINE_TC || engine == KDA_ENGINE_TC_CLUSTER) {
-        if (!(engine == KDA_ENGINE_TC ? tc_ok : cl_ok))
+    bool use_cluster = false;
+    if (engine == KDA_ENGINE_TC_CLUSTER) {
+        if (!cl_ok)
             return fail(KDA_ERR_UNSUPPORTED,
-                        "tensor-core engines need bf16, dk = dv = 128, chunk = 64 (got dtype %d, "
+                        "the tensor-core engine needs bf16, dk = dv = 128, chunk = 64 (got dtype %d, "
                         "dk %d, dv %d, chunk %d)", dtype, dk, dv, chunk);
-        use_tc = engine == KDA_ENGINE_TC;
-        use_cluster = engine == KDA_ENGINE_TC_CLUSTER;
+        use_cluster = true;
     } else if (engine == KDA_ENGINE_AUTO) {
         use_cluster = cl_ok;
-        use_tc = !cl_ok && tc_ok;
     }
 
     kda::ChunkArgs a{q, k, v, log_alpha, beta, S0, out, S_T, B, T, H, dk, dv, chunk, dtype,
                      workspace, workspace_bytes, nullptr};
     cudaError_t e;
-    if (use_tc || use_cluster) {
-        const size_t need = use_cluster ? kda::chunk_cluster_workspace_bytes(B, H)
-                                        : kda::chunk_tc_workspace_bytes(B, T, H);
+    if (use_cluster) {
+        const size_t need = kda::chunk_cluster_workspace_bytes(B, H);
         if (need > 0 && (!workspace || workspace_bytes < need))
             return fail(KDA_ERR_WORKSPACE, "workspace of %zu bytes given, %zu needed",
                         workspace ? workspace_bytes : static_cast<size_t>(0), need);
         a.device_error = device_error_ptr();
         if (!a.device_error) return fail(KDA_ERR_CUDA, "device error word not addressable");
-        e = use_cluster ? kda::launch_chunk_cluster(a, s) : kda::launch_chunk_tc(a, s);
+        e = kda::launch_chunk_cluster(a, s);
     } else {
         e = kda::launch_chunk_generic(a, s);
     }
+    return e == cudaSuccess ? KDA_OK : cuda_fail(e, "launching the prefill kernel");
+}
+
+int kda_chunk_fwd_fused(const void *q, const void *k, const void *v, const void *gate,
+                        const float *beta, const float *S0, void *out, float *S_T, int B, int T,
+                        int H, int dk, int dv, int chunk, int dtype, void *workspace,
+                        size_t workspace_bytes, void *stream) {
+    g_detail[0] = '\0';
+    if (B < 0 || T < 0 || H < 0)
+        return fail(KDA_ERR_INVALID_ARG, "B=%d T=%d H=%d must be >= 0", B, T, H);
+    int rc = check_common(dk, dv, dtype);
+    if (rc != KDA_OK) return rc;
+    if (!kda::chunk_cluster_supported(dk, dv, chunk, dtype))
+        return fail(KDA_ERR_UNSUPPORTED,
+                    "the fused prologue runs on the tensor-core engine: bf16, dk = dv = 128, chunk = 64 "
+                    "(got dtype %d, dk %d, dv %d, chunk %d)", dtype, dk, dv, chunk);
+    if (static_cast<long long>(B) * T > INT_MAX)
+        return fail(KDA_ERR_UNSUPPORTED, "B*T = %lld tokens: more than 2^31 - 1; split the batch",
+                    static_cast<long long>(B) * T);
+    if (static_cast<long long>(B) * H > INT_MAX / 4)
+        return fail(KDA_ERR_UNSUPPORTED, "B*H = %lld heads: more than 2^29 - 1; split the batch",
+                    static_cast<long long>(B) * H);
+    if (B == 0 || H == 0) return KDA_OK;
+    const bool tokens = T > 0;
+    const Ptr ps[] = {{q, "q", tokens},       {k, "k", tokens},   {v, "v", tokens},
+                      {gate, "gate", tokens}, {beta, "beta", tokens}, {out, "out", tokens},
+                      {S0, "S0", false},      {S_T, "S_T", false}, {workspace, "workspace", false}};
+    rc = check_pointers(ps, sizeof ps / sizeof ps[0]);
+    if (rc != KDA_OK) return rc;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (!tokens) {  // S_T = S0 (or zeros)
+        if (!S_T) return KDA_OK;
+        const size_t bytes = static_cast<size_t>(B) * H * dk * dv * sizeof(float);
+        cudaError_t e = S0 ? (S0 == S_T ? cudaSuccess
+                                        : cudaMemcpyAsync(S_T, S0, bytes, cudaMemcpyDeviceToDevice, s))
+                           : cudaMemsetAsync(S_T, 0, bytes, s);
+        return e == cudaSuccess ? KDA_OK : cuda_fail(e, "copying S0 to S_T");
+    }
+    const size_t need = kda::chunk_cluster_workspace_bytes(B, H);
+    if (!workspace || workspace_bytes < need)
+        return fail(KDA_ERR_WORKSPACE, "workspace of %zu bytes given, %zu needed",
+                    workspace ? workspace_bytes : static_cast<size_t>(0), need);
+    kda::ChunkArgs a{q, k, v, nullptr, beta, S0, out, S_T, B, T, H, dk, dv, chunk, dtype,
+                     workspace, workspace_bytes, device_error_ptr(), gate};
+    if (!a.device_error) return fail(KDA_ERR_CUDA, "device error word not addressable");
+    const cudaError_t e = kda::launch_chunk_cluster(a, s);
     return e == cudaSuccess ? KDA_OK : cuda_fail(e, "launching the prefill kernel");
 }
 

@@ -33,35 +33,37 @@ constexpr int kNV = 32;
 struct Layout {
     int dk, NV, LD, LC;
     __host__ __device__ Layout(int dk_, int NV_) : dk(dk_), NV(NV_), LD(dk_ + 1), LC(kC + 1) {}
-    // 10 [C][LD] tiles, 7 [C][LC], 5 [C][NV], 3 [dk][NV], vectors
+    // 12 [C][LD] tiles, 7 [C][LC], 5 [C][NV], 3 [dk][NV], vectors
     __host__ __device__ size_t floats() const {
-        return 10ull * kC * LD + 7ull * kC * LC + 5ull * kC * NV + 3ull * dk * NV + 6ull * dk + 3ull * kC;
+        return 12ull * kC * LD + 7ull * kC * LC + 5ull * kC * NV + 3ull * dk * NV + 3ull * dk + 3ull * kC;
     }
 };
 
 struct Tiles {
-    float *Qt, *Kt, *Kh, *G, *W, *dQs, *dKb, *dW, *dKs, *dQt;   // [C][LD]
+    // Qt, Kt: q and k; Qs = q e^{g}, Ks = k e^{g}, Kh = Kb = k e^{g_C - g}; G: prefix sums g
+    float *Qt, *Kt, *Kh, *G, *W, *dQs, *dKb, *dW, *dKs, *dQt, *Qs, *Ks;   // [C][LD]
     float *At, *P, *X, *Tm, *dT, *dA, *dP;                      // [C][LC]
     float *V, *Up, *U, *dO, *dU;                                 // [C][NV]
     float *S, *dS, *dSn;                                         // [dk][NV]
-    float *ga, *e_a, *e_ca, *gam, *dgam, *gsum;                  // [dk]
+    float *gam, *dgam, *gsum;                                    // [dk]
     float *bt, *dbt, *pad;                                       // [C]
     __device__ Tiles(float *sm, const Layout &L) {
         const int CD = kC * L.LD, CC = kC * L.LC, CN = kC * L.NV, DN = L.dk * L.NV;
         float *p = sm;
         Qt = p; p += CD; Kt = p; p += CD; Kh = p; p += CD; G = p; p += CD; W = p; p += CD;
         dQs = p; p += CD; dKb = p; p += CD; dW = p; p += CD; dKs = p; p += CD; dQt = p; p += CD;
+        Qs = p; p += CD; Ks = p; p += CD;
         At = p; p += CC; P = p; p += CC; X = p; p += CC; Tm = p; p += CC; dT = p; p += CC;
         dA = p; p += CC; dP = p; p += CC;
         V = p; p += CN; Up = p; p += CN; U = p; p += CN; dO = p; p += CN; dU = p; p += CN;
         S = p; p += DN; dS = p; p += DN; dSn = p; p += DN;
-        ga = p; p += L.dk; e_a = p; p += L.dk; e_ca = p; p += L.dk; gam = p; p += L.dk;
+        gam = p; p += L.dk;
         dgam = p; p += L.dk; gsum = p; p += L.dk;
         bt = p; p += kC; dbt = p; p += kC; pad = p;
     }
 };
 
-// The state-independent terms of one chunk: g, the anchored factors, At, P,
+// The state-independent terms of one chunk: g, Qs, Ks, Kb, At, P,
 // X = (I + A)^{-1}, T, W = T Ks, U' = T V. Loads q, k, log alpha, v (slice), beta.
 template <typename Tin>
 __device__ void chunk_terms(Tiles &s, const Layout &L, const Tin *q, const Tin *k, const Tin *v,
@@ -90,37 +92,34 @@ __device__ void chunk_terms(Tiles &s, const Layout &L, const Tin *q, const Tin *
     for (int t = tid; t < kC; t += kThreads)
         s.bt[t] = t < valid ? beta[(static_cast<long>(b) * T + t0 + t) * H + h] : 0.f;
     __syncthreads();
-    for (int c = tid; c < dk; c += kThreads) {   // prefix sums; anchor g_a = g_C / 2
+    for (int c = tid; c < dk; c += kThreads) {   // prefix sums
         float acc = 0.f;
         for (int t = 0; t < kC; ++t) {
             acc += s.G[t * LD + c];
             s.G[t * LD + c] = acc;
         }
         s.gsum[c] = acc;
-        s.ga[c] = 0.5f * acc;
-        s.e_a[c] = expf(0.5f * acc);
-        s.e_ca[c] = expf(acc - 0.5f * acc);
         s.gam[c] = expf(acc);
     }
     __syncthreads();
-    for (int e = tid; e < kC * dk; e += kThreads) {   // q~ = q e^{g - g_a}, k~ = k e^{g - g_a}, k^ = k e^{g_a - g}
+    for (int e = tid; e < kC * dk; e += kThreads) {   // Qs = q e^{g}, Ks = k e^{g}, Kb = k e^{g_C - g}
         const int t = e / dk, c = e - t * dk;
-        const float d = s.G[t * LD + c] - s.ga[c];
-        const float E = expf(d), F = expf(-d);
+        const float gv = s.G[t * LD + c];
+        const float up = expf(gv), down = expf(s.gsum[c] - gv);
         const float kv = s.Kt[t * LD + c];
-        s.Qt[t * LD + c] *= E;
-        s.Kt[t * LD + c] = kv * E;
-        s.Kh[t * LD + c] = kv * F;
+        s.Qs[t * LD + c] = s.Qt[t * LD + c] * up;
+        s.Ks[t * LD + c] = kv * up;
+        s.Kh[t * LD + c] = kv * down;
     }
-    __syncthreads();
     for (int e = tid; e < 2 * kC * kC; e += kThreads) {   // At (strict lower), P (lower)
         const int which = e / (kC * kC), r = e - which * kC * kC;
         const int i = r / kC, j = r - i * kC;
         float acc = 0.f;
         if (which == 0 ? j < i : (need_p && j <= i)) {
             const float *x = (which == 0 ? s.Kt : s.Qt) + i * LD;
-            const float *y = s.Kh + j * LD;
-            for (int c = 0; c < dk; ++c) acc = fmaf(x[c], y[c], acc);
+            const float *y = s.Kt + j * LD;
+            const float *gi = s.G + i * LD, *gj = s.G + j * LD;
+            for (int c = 0; c < dk; ++c) acc = fmaf(x[c], y[c] * expf(gi[c] - gj[c]), acc);
         }
         (which == 0 ? s.At : s.P)[i * LC + j] = acc;
     }
@@ -143,8 +142,8 @@ __device__ void chunk_terms(Tiles &s, const Layout &L, const Tin *q, const Tin *
         if (e < kC * dk) {
             const int i = e / dk, c = e - i * dk;
             float acc = 0.f;
-            for (int j = 0; j <= i; ++j) acc = fmaf(s.Tm[i * LC + j], s.Kt[j * LD + c], acc);
-            s.W[i * LD + c] = acc * s.e_a[c];
+            for (int j = 0; j <= i; ++j) acc = fmaf(s.Tm[i * LC + j], s.Ks[j * LD + c], acc);
+            s.W[i * LD + c] = acc;
         } else {
             const int r = e - kC * dk, i = r / NV, n = r - i * NV;
             float acc = 0.f;
@@ -189,8 +188,7 @@ __device__ void states_body(float *sm, const Tin *q, const Tin *k, const Tin *v,
         for (int e = tid; e < dk * NV; e += kThreads) {   // S <- Diag(gamma) S + Kb^T U
             const int c = e / NV, n = e - c * NV;
             float acc = s.gam[c] * s.S[e];
-            const float eca = s.e_ca[c];
-            for (int t = 0; t < kC; ++t) acc = fmaf(s.Kh[t * LD + c] * eca, s.U[t * NV + n], acc);
+            for (int t = 0; t < kC; ++t) acc = fmaf(s.Kh[t * LD + c], s.U[t * NV + n], acc);
             s.S[e] = acc;
         }
     }
@@ -242,7 +240,7 @@ __device__ void bwd_body(float *sm, const Tin *q, const Tin *k, const Tin *v, co
             const int j = e / NV, n = e - j * NV;
             float acc = 0.f;
             for (int i = j; i < kC; ++i) acc = fmaf(s.P[i * LC + j], s.dO[i * NV + n], acc);
-            for (int c = 0; c < dk; ++c) acc = fmaf(s.Kh[j * LD + c] * s.e_ca[c], s.dS[c * NV + n], acc);
+            for (int c = 0; c < dk; ++c) acc = fmaf(s.Kh[j * LD + c], s.dS[c * NV + n], acc);
             s.dU[e] = acc;
         }
         __syncthreads();
@@ -250,9 +248,8 @@ __device__ void bwd_body(float *sm, const Tin *q, const Tin *k, const Tin *v, co
         for (int e = tid; e < dk * NV; e += kThreads) {   // dSn = Qs^T dO + Diag(gamma) dS - W^T dU
             const int c = e / NV, n = e - c * NV;
             float acc = s.gam[c] * s.dS[e];
-            const float ea = s.e_a[c];
             for (int i = 0; i < kC; ++i) {
-                acc = fmaf(s.Qt[i * LD + c] * ea, s.dO[i * NV + n], acc);
+                acc = fmaf(s.Qs[i * LD + c], s.dO[i * NV + n], acc);
                 acc = fmaf(-s.W[i * LD + c], s.dU[i * NV + n], acc);
             }
             s.dSn[e] = acc;
@@ -298,7 +295,7 @@ __device__ void bwd_body(float *sm, const Tin *q, const Tin *k, const Tin *v, co
                 const int i = e / kC, j = e - i * kC;
                 float acc = 0.f;
                 if (j <= i) {
-                    for (int c = 0; c < dk; ++c) acc = fmaf(s.dW[i * LD + c], s.Kt[j * LD + c] * s.e_a[c], acc);
+                    for (int c = 0; c < dk; ++c) acc = fmaf(s.dW[i * LD + c], s.Ks[j * LD + c], acc);
                     for (int n = 0; n < NV; ++n) acc = fmaf(s.dU[i * NV + n], s.V[j * NV + n], acc);
                 }
                 s.dT[i * LC + j] = acc;
@@ -346,18 +343,27 @@ __device__ void bwd_body(float *sm, const Tin *q, const Tin *k, const Tin *v, co
             s.dT[(i)*LC + (e - i * kC)] *= s.bt[i];
         }
         __syncthreads();
-        // dKt = dAt Kh (into dW), dKh = dAt^T Kt + dP^T Qt (into W), dQt = dP Kh
+        // The intra-chunk products, term by term (E_ij = e^{g_i - g_j} per channel):
+        //   R_i  = sum_{j<i}  dAt_ij k_j E_ij             (row side of A,   into dW)
+        //   Cc_j = sum_{i>j}  dAt_ij k_i E_ij
+        //        + sum_{i>=j} dP_ij  q_i E_ij             (column side,     into W)
+        //   Rq_i = sum_{j<=i} dP_ij  k_j E_ij             (row side of P,   into dQt)
         for (int e = tid; e < 3 * kC * dk; e += kThreads) {
             const int which = e / (kC * dk), r = e - which * kC * dk;
             const int i = r / dk, c = r - i * dk;
+            const float gi = s.G[i * LD + c];
             float acc = 0.f;
             if (which == 0) {
-                for (int j = 0; j < i; ++j) acc = fmaf(s.dT[i * LC + j], s.Kh[j * LD + c], acc);
+                for (int j = 0; j < i; ++j)
+                    acc = fmaf(s.dT[i * LC + j], s.Kt[j * LD + c] * expf(gi - s.G[j * LD + c]), acc);
             } else if (which == 1) {
-                for (int a = i + 1; a < kC; ++a) acc = fmaf(s.dT[a * LC + i], s.Kt[a * LD + c], acc);
-                for (int a = i; a < kC; ++a) acc = fmaf(s.dP[a * LC + i], s.Qt[a * LD + c], acc);
+                for (int a = i + 1; a < kC; ++a)
+                    acc = fmaf(s.dT[a * LC + i], s.Kt[a * LD + c] * expf(s.G[a * LD + c] - gi), acc);
+                for (int a = i; a < kC; ++a)
+                    acc = fmaf(s.dP[a * LC + i], s.Qt[a * LD + c] * expf(s.G[a * LD + c] - gi), acc);
             } else {
-                for (int j = 0; j <= i; ++j) acc = fmaf(s.dP[i * LC + j], s.Kh[j * LD + c], acc);
+                for (int j = 0; j <= i; ++j)
+                    acc = fmaf(s.dP[i * LC + j], s.Kt[j * LD + c] * expf(gi - s.G[j * LD + c]), acc);
             }
             (which == 0 ? s.dW : (which == 1 ? s.W : s.dQt))[i * LD + c] = acc;
         }
@@ -365,15 +371,15 @@ __device__ void bwd_body(float *sm, const Tin *q, const Tin *k, const Tin *v, co
         // dk, dq; dg per token and channel (into dKs, after its use)
         for (int e = tid; e < kC * dk; e += kThreads) {
             const int t = e / dk, c = e - t * dk;
-            const float d = s.G[t * LD + c] - s.ga[c];
-            const float E = expf(d), F = expf(-d);
-            const float ea = s.e_a[c], eca = s.e_ca[c];
-            const float kt = s.Kt[t * LD + c], kh = s.Kh[t * LD + c], qt = s.Qt[t * LD + c];
-            const float dkt = s.dW[t * LD + c], dkh = s.W[t * LD + c], dqt = s.dQt[t * LD + c];
+            const float gv = s.G[t * LD + c];
+            const float up = expf(gv), down = expf(s.gsum[c] - gv);
+            const float kv = s.Kt[t * LD + c], qv = s.Qt[t * LD + c];
+            const float rk = s.dW[t * LD + c], cc = s.W[t * LD + c], rq = s.dQt[t * LD + c];
             const float dks = s.dKs[t * LD + c], dkb = s.dKb[t * LD + c], dqs = s.dQs[t * LD + c];
-            const float dk_v = dkt * E + dkh * F + dks * E * ea + dkb * F * eca;
-            const float dq_v = dqt * E + dqs * E * ea;
-            const float dg = dkt * kt - dkh * kh + dqt * qt + dks * kt * ea + dqs * qt * ea - dkb * kh * eca;
+            const float dk_v = rk + cc + dks * up + dkb * down;
+            const float dq_v = rq + dqs * up;
+            const float dg = kv * (rk - cc) + qv * rq + dks * s.Ks[t * LD + c] + dqs * s.Qs[t * LD + c] -
+                             dkb * s.Kh[t * LD + c];
             s.dKs[t * LD + c] = dg;
             if (t < valid) {
                 const long o = ((static_cast<long>(b) * T + t0 + t) * H + h) * dk + c;
@@ -384,8 +390,7 @@ __device__ void bwd_body(float *sm, const Tin *q, const Tin *k, const Tin *v, co
         __syncthreads();
         for (int c = tid; c < dk; c += kThreads) {   // g_C's own terms, then the in-chunk suffix sums
             float gc = s.dgam[c];
-            const float eca = s.e_ca[c];
-            for (int t = 0; t < kC; ++t) gc = fmaf(s.dKb[t * LD + c], s.Kh[t * LD + c] * eca, gc);
+            for (int t = 0; t < kC; ++t) gc = fmaf(s.dKb[t * LD + c], s.Kh[t * LD + c], gc);
             float acc = gc;
             for (int t = kC - 1; t >= 0; --t) {
                 acc += s.dKs[t * LD + c];

@@ -1,12 +1,30 @@
 // chunk_cluster.cu -- cluster engine of the chunked KDA prefill on sm_100a
 // (bf16 q/k/v, d_k = d_v = 128, chunk C = 64, fp32 gates and state).
 //
-// Same chunked form and operand precisions as chunk_tc.cu (Kimi Linear
-// summary, es.news.hada.io/topic?id=31936, sections "Algoritmo paralelo por
-// chunks" and "Menor cantidad de operaciones que DPLR general"):
-//   [A;P] = [K*E ; Q*E](K*F)^T (tf32), T = (I + A)^{-1} Diag(beta),
-//   [W | U'] = T [Ks | V] (fp16), then the state chain
-//   X = [Qs ; W] S, U = U' - W S, S <- Diag(e^{g_C}) S + Kb^T U, O = Qs S + P U.
+// Chunked form (Kimi Linear summary, es.news.hada.io/topic?id=31936, sections
+// "Algoritmo paralelo por chunks" and "Menor cantidad de operaciones que DPLR
+// general"). Per chunk, with g the in-chunk inclusive prefix sum of log alpha:
+//   A = Diag(beta) strict_lower(K~ K^T),  P = lower(Q~ K^T)   (entries carry e^{g_i - g_j})
+//   T = (I + A)^{-1} Diag(beta),  [W | U'] = T [Ks | V]       (Ks = K e^{g})
+//   state chain: X = [Qs ; W] S, U = U' - W S, O = Qs S + P U,
+//                S <- Diag(e^{g_C}) S + Kb^T U                 (Qs = Q e^{g}, Kb = K e^{g_C - g})
+//
+// The two intra-chunk products are built from 16-token sub-chunks (the
+// summary's secondary chunking for fine-grained decay), so that no gate factor
+// leaves the floating-point range whatever the decay:
+//   * a block (I, J) below the diagonal (row sub-chunk I, column sub-chunk
+//     J < I) uses e^{g_i - g_j} = e^{g_i - G_I} e^{G_I - G_{J+1}} e^{G_{J+1} - g_j},
+//     G_I = g at the end of sub-chunk I-1: all three factors are <= 1. The row
+//     operand (with the middle factor, per channel) stays in the registers of
+//     the warp that owns sub-chunk I; the column operand K e^{G_{J+1} - g} is
+//     written once to shared memory; tf32 mma.sync, like the diagonal blocks;
+//   * a diagonal block (I, I) anchors both factors at the sub-chunk's 8th token
+//     m: e^{g_i - g_m} e^{g_m - g_j}, each within e^{87} whenever the
+//     sub-chunk's total decay is within e^{-87}; computed in tf32 with
+//     warp-level mma.sync from registers. A channel whose sub-chunk decays
+//     further takes its factors from log alpha clamped at -10 per token: every
+//     product that changes is then below e^-10 before and after, a change
+//     (< 4.6e-5) below the tf32 rounding of the same factor (2^-11).
 //
 // The work of one chunk splits into a key-side part that does not depend on
 // the state (everything up to W, U', P, T, Qs, Kb) and the state chain, which
@@ -14,10 +32,9 @@
 //   * ranks 0..2 are producers: rank p computes the key-side part of chunks
 //     p, p+3, p+6, ... as an 82 KB image and writes it into one of its three
 //     slots of a small ring in the workspace (it stays in L2): Qs, Kb and
-//     e^{g_C} straight from registers in the gate prologue; [P;T] (an operand
-//     of its own MMA), W and U' staged in shared memory and bulk-stored
-//     (cp.async.bulk shared -> global), [P;T] as soon as T is formed and W
-//     while U' is formed. Once the
+//     e^{g_C} straight from registers; [P;T] (an operand of its own MMA), W and
+//     U' staged in shared memory and bulk-stored (cp.async.bulk shared ->
+//     global), [P;T] as soon as T is formed and W while U' is formed. Once the
 //     stores are complete, thread 0 arrives (release, cluster scope; the
 //     generic stores of all threads precede it through a CTA barrier) on the
 //     consumer's "ready" barrier of that slot;
@@ -28,13 +45,9 @@
 //     "loaded" barrier) that the ring slot may be reused.
 // The ring goes through L2 because a DSMEM bulk copy moves only ~20 B/cycle
 // between two SMs, whereas an L2 bulk load of the same 82 KB takes ~1K cycles.
-// The producers set the pace of the cluster, so their image stores are kept
-// short: writing Qs and Kb from registers and storing [P;T] and W early
-// leaves only U' (16 KB) to store and wait for at the end of an image.
-// A producer thus has three chunk periods for the key-side latency, and the
-// consumer's chunk period is the chain alone. Every wait is bounded; after a
-// timeout a CTA records an error in the device error word, stops waiting and
-// still reaches the final cluster barrier and frees its tensor memory.
+// Every wait is bounded; after a timeout a CTA records an error in the device
+// error word, stops waiting and still reaches the final cluster barrier and
+// frees its tensor memory.
 #include <cuda.h>
 
 #include "kda_internal.cuh"
@@ -46,7 +59,6 @@ namespace {
 
 using tc::fence_proxy_async_smem;
 using tc::mma_f16;
-using tc::mma_tf32;
 using tc::pack_bf16;
 using tc::pack_f16;
 using tc::sw128k_off;
@@ -62,6 +74,10 @@ constexpr int kCluster = kProducers + 1;
 constexpr int kRingDepth = 3;   // ring slots per producer
 constexpr int kRingSlots = kRingDepth * kProducers;
 constexpr uint32_t kWaitLimit = 1u << 22;
+constexpr uint32_t kTestWaitLimit = 1u << 12;   // polls of a bounded wait under the test hook
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kRangeLog = -87.f;   // e^-87 ~ 1.6e-38: factors of a sub-chunk stay normal above it
+constexpr float kClampLog = -10.f;   // per-token clamp of log alpha for the fallback factors
 
 // ---- slot image: what a producer hands the consumer for one chunk
 constexpr uint32_t SL_QW = 0;          // [Qs ; W] fp16 K-major SW128, 2 K-blocks x 16 KB
@@ -76,141 +92,238 @@ constexpr uint32_t kTokBlk = 8192;
 static_assert(kRingSlots * kSlotStride == kClusterRingBytesPerHead, "ring size");
 
 // ---- producer shared memory
-constexpr uint32_t P_KQT = 0;          // [K*E ; Q*E] tf32, 4 K-blocks x 16 KB
-constexpr uint32_t kKQTBlk = 16384;
-constexpr uint32_t P_KHT = 65536;      // K*F tf32, 4 K-blocks x 8 KB
-constexpr uint32_t kKHTBlk = 8192;
-constexpr uint32_t P_AF = 0;           // A (fp32), reuses the tf32 region after the product
-constexpr uint32_t P_XF = 64 * kLD * 4;
-// ... and after the UT solve, holds the TMA-loaded inputs of the producer's next chunk:
-constexpr uint32_t P_IN_Q = 0;         // q  [64 tokens][128] bf16
-constexpr uint32_t P_IN_K = 16384;     // k
-constexpr uint32_t P_IN_LA = 32768;    // log alpha [64][128] fp32
-constexpr uint32_t P_IN_V = 65536;     // v  [64][128] bf16
+// Inputs of a chunk (TMA). q, k and log alpha come as 128-byte rows in the
+// 128-byte swizzle (16-byte piece p of token row r stored at piece p ^ (r % 8)),
+// so that the prologue's fragment-ordered reads are free of bank conflicts.
+constexpr uint32_t P_IN_Q = 0;         // q: 2 boxes (64 channels each) x [64 tokens][128 B]
+constexpr uint32_t P_IN_K = 16384;     // k: same
+constexpr uint32_t P_IN_LA = 32768;    // log alpha: 4 boxes (32 channels each) x [64][128 B]
+constexpr uint32_t P_IN_V = 65536;     // v [64][128] bf16, plain rows
+constexpr uint32_t kBoxBytes = 8192;
 constexpr uint32_t kInBytes = 81920;
-constexpr uint32_t P_STAGE = 98304;    // image-sized area: [P;T], W and U' are staged here
-constexpr uint32_t P_KSV = P_STAGE + kSlotStride;  // [Ks | V] fp16 [token][col], 4 blocks x 8 KB
-constexpr uint32_t P_VEC = P_KSV + 32768;          // beta[64], psum[4][128]
-constexpr uint32_t P_BAR = P_VEC + (64 + 512) * 4;
+// ... or, for the fused layer prologue (raw q, k and the gate's pre-activation x):
+constexpr uint32_t P_IN_X = 32768;     // x: 2 boxes (64 channels each, bf16) x [64][128 B]
+constexpr uint32_t P_IN_VF = 49152;    // v
+constexpr uint32_t kInBytesF = 65536;
+// ... and once the prologue has read them, the same region holds:
+constexpr uint32_t P_AF = 0;                   // A fp32 [64][kLD]
+constexpr uint32_t P_XF = 64 * kLD * 4;        // X = (I + A)^{-1} fp32 [64][kLD]
+constexpr uint32_t P_DX = 2 * 64 * kLD * 4;    // diagonal-block partials of channels 64..127 (8 KB)
+constexpr uint32_t P_PX = P_DX + 8192;         // off-diagonal-block partials, both halves: 2 x 6 x 2 KB
+// K e^{G_{J+1} - g} (fp32), the column operand of the off-diagonal blocks, in the
+// swizzled layout of log alpha; then Kb staged for the ring (image layout)
+constexpr uint32_t P_KSIG = 81920;
+constexpr uint32_t P_KBS = P_KSIG + 32768;
+constexpr uint32_t P_STAGE = 131072;   // [P;T] 16 KB, W 2 x 8 KB, U' 16 KB (bulk-stored to the ring)
+constexpr uint32_t ST_PT = 0;
+constexpr uint32_t ST_W = 16384;
+constexpr uint32_t ST_UP = 32768;
+constexpr uint32_t ST_GL = ST_W;       // before W and U' exist: g^L in the layout of log alpha (32 KB),
+constexpr uint32_t ST_QS = ST_W;       // then Qs staged for the ring: 2 K-blocks x 8 KB (image layout)
+constexpr uint32_t P_KSV = 180224;     // [Ks | V] fp16 [token][col], 4 blocks x 8 KB
+// beta of two chunks [2][64] (the next one arrives by cp.async during this one); per
+// sub-chunk I and channel c ([4][128] each): tot = total log alpha of the sub-chunk,
+// e^{-g_m}, e^{g_m - tot} (g_m = g^L at its 8th token) and e^{tot}; a flag
+constexpr uint32_t P_VEC = 212992;
+constexpr uint32_t V_TOT = 128, V_EM = V_TOT + 512, V_EC = V_EM + 512, V_P = V_EC + 512, V_FLAG = V_P + 512;
+constexpr uint32_t V_INV = V_FLAG + 4;   // fused prologue: 1 / ||q_t||, 1 / ||k_t|| ([2][64])
+constexpr uint32_t P_BAR = P_VEC + (V_INV + 128) * 4;
 // ---- consumer shared memory
 constexpr uint32_t C_SLOT = 0;         // 2 slots
 constexpr uint32_t C_S16 = 2 * kSlotStride;        // S fp16, MN-major SW128: 2 blocks x 16 KB
 constexpr uint32_t C_U16 = C_S16 + 32768;          // U fp16, MN-major SW128: 2 blocks x 8 KB
 constexpr uint32_t C_BAR = C_U16 + 16384;
-#ifdef KDA_PHASE_TIMING
-constexpr uint32_t kDbgBytes = 256;    // per-phase cycle accumulators, after the barriers
-#else
-constexpr uint32_t kDbgBytes = 0;
-#endif
 constexpr uint32_t kSmemBytes =
-    (P_BAR > C_BAR ? P_BAR : C_BAR) + 192 + kDbgBytes + 1024;  // + barriers + alignment slack
+    (P_BAR > C_BAR ? P_BAR : C_BAR) + 192 + 1024;  // + barriers + alignment slack
+static_assert(P_PX + 2 * 6 * 2048 <= P_KSIG, "producer layout");
+static_assert(P_KBS + 16384 <= P_STAGE, "producer layout");
 
 // TMEM columns.
-constexpr uint32_t PCOL_AP = 0;        // producer: [A;P] (64 cols)
-constexpr uint32_t PCOL_WU = 64;       // producer: [P;T][Ks|V], lanes 64-127 = [W | U'] (256)
+constexpr uint32_t PCOL_WU = 128;      // producer: [P;T][Ks|V], lanes 64-127 = [W | U'] (256)
 constexpr uint32_t CCOL_X = 0;         // consumer: 2 x 128 cols ([Qs;W]S (+ [P;T]U))
 constexpr uint32_t CCOL_S = 256;       // consumer: Kb^T U (128 cols)
 constexpr uint32_t kTmemCols = 512;
 
-constexpr uint32_t IDESC_AP = tc::idesc(tc::kFmtTF32, 128, 64, 0, 0);
 constexpr uint32_t IDESC_WU = tc::idesc(tc::kFmtF16, 128, 256, 0, 1);
 constexpr uint32_t IDESC_X = tc::idesc(tc::kFmtF16, 128, 128, 0, 1);   // A K-major, B MN-major
 constexpr uint32_t IDESC_S = tc::idesc(tc::kFmtF16, 128, 128, 1, 1);   // A MN-major, B MN-major
 
-#ifdef KDA_PHASE_TIMING
-// Debug builds only: cycles per phase summed over chunks, for cluster 0
-// (slots 0..9 producer rank 0, slots 16..23 the consumer). Thread 0 of each CTA
-// accumulates in shared memory (a global read-modify-write per mark would cost
-// ~1K cycles and distort the phases) and adds its slots to the global array once.
-__device__ unsigned long long g_cluster_cycles[32];
-#define CMARK(idx)                                                        \
-    do {                                                                  \
-        if (threadIdx.x == 0 && (idx) < 32) {                             \
-            const unsigned long long now_ = clock64();                    \
-            t_acc_[idx] += now_ - t_prev_;                                \
-            t_prev_ = now_;                                               \
-        }                                                                 \
-    } while (0)
-#define CMARK_INIT(bar_off)                                                                 \
-    unsigned long long *t_acc_ = reinterpret_cast<unsigned long long *>(sm + (bar_off) + 192); \
-    if (threadIdx.x == 0)                                                                   \
-        for (int i_ = 0; i_ < 32; ++i_) t_acc_[i_] = 0;                                     \
-    unsigned long long t_prev_ = clock64()
-#define CMARK_FLUSH(lo, hi)                                                               \
-    do {                                                                                  \
-        if (blockIdx.x < kCluster && threadIdx.x == 0)                                    \
-            for (int i_ = (lo); i_ < (hi); ++i_) atomicAdd(&g_cluster_cycles[i_], t_acc_[i_]); \
-    } while (0)
-#else
-#define CMARK(idx) \
-    do {           \
-    } while (0)
-#define CMARK_INIT(bar_off)
-#define CMARK_FLUSH(lo, hi) \
-    do {                    \
-    } while (0)
-#endif
-
+// Give-up protocol. Every wait on a peer or on an asynchronous operation is bounded
+// (`limit` polls). A thread whose wait runs out records KDA_ERR_DEVICE_TIMEOUT in the
+// device error word and sets the abort flag of every CTA of the cluster; any wait that
+// sees the flag stops waiting. From then on no thread issues a new TMA load, MMA, bulk
+// copy or remote arrive; each CTA leaves its chunk loop at the next uniform check,
+// waits (bounded again) for the asynchronous operations it has issued and not yet
+// seen complete -- those complete by themselves -- and then reaches the final cluster
+// barrier and frees its tensor memory. At most one operation per barrier is ever in
+// flight, so "pending" is a flag and the parity to drain is the next expected one.
 struct Ctl {
-    int *abort;
-    int *err;
+    int *abort;              // this CTA's abort flag (shared memory)
+    int *err;                // device error word
+    uint32_t peer_abort[4];  // the abort flag of every CTA of the cluster (shared::cluster)
+    uint32_t limit;          // polls of a bounded wait
 };
 
+__device__ __forceinline__ bool aborted(const Ctl &k) { return *reinterpret_cast<volatile int *>(k.abort) != 0; }
 __device__ __forceinline__ void fail(const Ctl &k) {
-    *reinterpret_cast<volatile int *>(k.abort) = 1;
     atomicExch(k.err, 2);
+#pragma unroll
+    for (int r = 0; r < 4; ++r)
+        asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(k.peer_abort[r]), "r"(1) : "memory");
 }
-__device__ __forceinline__ void wait_local(uint64_t *bar, uint32_t parity, const Ctl &k) {
-    if (*reinterpret_cast<volatile int *>(k.abort)) return;
-    if (!tc::mbar_wait(bar, parity, kWaitLimit)) fail(k);
+// Waits for the phase `parity` of `bar`; false if the cluster gave up (now or earlier).
+__device__ __forceinline__ bool wait_local(uint64_t *bar, uint32_t parity, const Ctl &k) {
+    for (uint32_t i = 0; i < k.limit; ++i) {
+        if (tc::mbar_try_wait(bar, parity)) return true;
+        if ((i & 63) == 0 && aborted(k)) return false;
+    }
+    fail(k);
+    return false;
 }
-__device__ __forceinline__ void wait_cluster(uint64_t *bar, uint32_t parity, const Ctl &k) {
-    if (*reinterpret_cast<volatile int *>(k.abort)) return;
-    if (!tc::mbar_wait_cluster(bar, parity, kWaitLimit)) fail(k);
+// The same with acquire at cluster scope (barriers that peers arrive on).
+__device__ __forceinline__ bool wait_cluster(uint64_t *bar, uint32_t parity, const Ctl &k) {
+    for (uint32_t i = 0; i < k.limit; ++i) {
+        if (tc::mbar_try_wait_cluster(bar, parity)) return true;
+        if ((i & 63) == 0 && aborted(k)) return false;
+    }
+    fail(k);
+    return false;
+}
+// Drain: waits (bounded, regardless of the abort flag) for an operation this thread
+// issued; they complete by themselves.
+__device__ __forceinline__ void drain(uint64_t *bar, uint32_t parity, const Ctl &k) {
+    if (!tc::mbar_wait(bar, parity, kWaitLimit)) atomicExch(k.err, 2);
 }
 
+// 4-byte asynchronous copy global -> shared (completion by cp.async.wait_group).
+__device__ __forceinline__ void cp_async4(void *dst, const void *src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(tc::smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_prev() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
+
+// log alpha = -softplus(x) = -(max(x, 0) + log(1 + e^{-|x|})) for the gate's pre-activation x
+// (Kimi Linear summary, section "Configuracion del modelo Kimi Linear": a data-dependent
+// per-channel decay gate like GDN's and Mamba's). For e^{-|x|} < 1e-3 the logarithm is
+// its series e - e^2/2, exact to e^3/3, where 1 + e would lose e's digits in fp32.
+__device__ __forceinline__ float neg_softplus(float x) {
+    constexpr float kLn2 = 0.6931471805599453f;
+    const float e = tc::ex2(-fabsf(x) * kLog2e);
+    const float l = e < 1e-3f ? e * (1.f - 0.5f * e) : tc::lg2(1.f + e) * kLn2;
+    return -(fmaxf(x, 0.f) + l);
+}
+
+// Inclusive prefix sum over the 8 lanes 4g + t (g = 0..7) that share t.
+__device__ __forceinline__ float scan8(float x, int g) {
+    float y = __shfl_up_sync(0xffffffffu, x, 4);
+    if (g >= 1) x += y;
+    y = __shfl_up_sync(0xffffffffu, x, 8);
+    if (g >= 2) x += y;
+    y = __shfl_up_sync(0xffffffffu, x, 16);
+    if (g >= 4) x += y;
+    return x;
+}
+
+// Index of the off-diagonal block (I, J), J < I, among the six: (1,0) (2,0) (2,1) (3,0) (3,1) (3,2).
+__device__ __forceinline__ int pair_index(int I, int J) { return I * (I - 1) / 2 + J; }
+
 // ============================================================ producer
-__device__ void producer(uint8_t *sm, uint32_t tmem, int rank, uint8_t *ring, const CUtensorMap *tm_q,
-                         const CUtensorMap *tm_k, const CUtensorMap *tm_la,
-                         const CUtensorMap *tm_v, const __nv_bfloat16 *__restrict__ q,
-                         const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *__restrict__ v,
-                         const float *__restrict__ log_alpha, const float *__restrict__ beta,
-                         int T, int H, int h, long ztok, int nchunks, const Ctl &ctl) {
+// Thread mapping of the gate prologue: warp w handles sub-chunk I = w % 4 (16
+// tokens) and channel half w / 4 (64 channels); lane (g, t) = (lane / 4, lane % 4)
+// holds tokens 16 I + g and 16 I + g + 8 and, for s = 0..7, the channel pair
+// 8 s + 2 t, 8 s + 2 t + 1 of its half -- exactly the elements of the tf32
+// mma.sync fragments of the diagonal block (k-step s: channel 8 s + 2 t is
+// fragment column t, channel 8 s + 2 t + 1 is column t + 4), so the diagonal
+// products need no shared-memory round trip.
+template <bool kFused>
+__device__ void producer(uint8_t *sm, uint32_t tmem, int rank, uint8_t *ring,
+                         const CUtensorMap *tm_q, const CUtensorMap *tm_k, const CUtensorMap *tm_la,
+                         const CUtensorMap *tm_v, const CUtensorMap *tm_qs, const CUtensorMap *tm_ks,
+                         const CUtensorMap *tm_las, const float *__restrict__ beta, int T, int H,
+                         int h, long ztok, int nchunks, const Ctl &ctl, int test_timeout) {
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int quad = warp & 3, half = warp >> 2;
     const int row = 32 * quad + lane;
+    // sub-chunk of this warp: warps w and w + 4 share a scheduler, and sub-chunk I writes
+    // 3 - I copies of the off-diagonal columns, so a scheduler gets sub-chunks I and 3 - I
+    const int I = half == 0 ? quad : 3 - quad, g = lane >> 2, t4 = lane & 3;
+    const int ta = 16 * I + g, tb = ta + 8;
     const uint32_t sbase = tc::smem_u32(sm);
-    float *beta_s = reinterpret_cast<float *>(sm + P_VEC);
-    float *psum = beta_s + 64;
+    float *vec = reinterpret_cast<float *>(sm + P_VEC);   // beta buffers and per-channel tables
+    // beta of chunk cc (token rows of this head) into buffer b, by threads 0..63; tokens past
+    // T are identity steps (beta = 0)
+    auto load_beta = [&](int cc, int b) {
+        if (tid < kC && cc < nchunks) {
+            const int t = cc * kC + tid;
+            if (t < T) cp_async4(vec + 64 * b + tid, beta + (ztok + t) * H + h);
+            else vec[64 * b + tid] = 0.f;
+        }
+        cp_async_commit();
+    };
     float *Af = reinterpret_cast<float *>(sm + P_AF);
     float *Xf = reinterpret_cast<float *>(sm + P_XF);
     uint64_t *bar_mma = reinterpret_cast<uint64_t *>(sm + P_BAR);
     uint64_t *bar_loaded = bar_mma + 1;  // [kRingDepth]: one per ring slot of this producer
+    uint64_t *bar_in = bar_mma + 1 + kRingDepth;
     uint8_t *st = sm + P_STAGE;
-    uint32_t ph_mma = 0;
+    uint32_t ph_mma = 0, ph_in = 0;
+    bool pend_in = false, pend_mma = false;   // thread 0: a TMA input batch / an MMA group in flight
     int img = 0;  // index of this producer's next image
 
-    const uint64_t d_kqt = tc::smem_desc(sbase + P_KQT, 16, 1024, tc::kSwizzle128);
-    const uint64_t d_kht = tc::smem_desc(sbase + P_KHT, 16, 1024, tc::kSwizzle128);
-    const uint64_t d_pt = tc::smem_desc(sbase + P_STAGE + SL_PT, 16, 1024, tc::kSwizzle128);
+    const uint64_t d_pt = tc::smem_desc(sbase + P_STAGE + ST_PT, 16, 1024, tc::kSwizzle128);
     const uint64_t d_ksv = tc::smem_desc(sbase + P_KSV, kTokBlk, 1024, tc::kSwizzle128);
     // the consumer's "ready" barriers for this producer's ring slots
     const uint32_t c_ready = tc::map_to_rank(sbase + C_BAR + 40 + 8 * kRingDepth * rank, kCluster - 1);
 
-    CMARK_INIT(P_BAR);
-    const int mk = rank == 0 ? 0 : 64;  // only rank 0 records (slots 0..8)
-    uint64_t *bar_in = bar_mma + 1 + kRingDepth;
-    uint32_t ph_in = 0;
+    // P's blocks above the diagonal are zero in every image; nothing else writes them
+    for (int e = tid; e < 64 * 32; e += kThreads) {
+        const int i = e >> 5, j = 2 * (e & 31);
+        if (j >= 16 * ((i >> 4) + 1))
+            *reinterpret_cast<uint32_t *>(st + ST_PT + sw128k_off(i, j, 0)) = 0u;
+    }
+    if (tid == 0) *reinterpret_cast<volatile int *>(vec + V_FLAG) = 0;
+    __syncthreads();
+
     auto load_inputs = [&](int cc) {   // TMA: the 64-token chunk cc of head h (all channels)
+        if (aborted(ctl)) return;
+        pend_in = true;
         const int z = static_cast<int>(ztok + static_cast<long>(cc) * kC);
-        tc::mbar_arrive_expect_tx(bar_in, kInBytes);
-        tc::tma_load_3d(sm + P_IN_Q, tm_q, bar_in, 0, h, z);
-        tc::tma_load_3d(sm + P_IN_K, tm_k, bar_in, 0, h, z);
-        tc::tma_load_3d(sm + P_IN_LA, tm_la, bar_in, 0, h, z);
-        tc::tma_load_3d(sm + P_IN_V, tm_v, bar_in, 0, h, z);
+        tc::mbar_arrive_expect_tx(bar_in, kFused ? kInBytesF : kInBytes);
+        tc::tma_load_3d(sm + P_IN_Q, tm_qs, bar_in, 0, h, z);
+        tc::tma_load_3d(sm + P_IN_Q + kBoxBytes, tm_qs, bar_in, 64, h, z);
+        tc::tma_load_3d(sm + P_IN_K, tm_ks, bar_in, 0, h, z);
+        tc::tma_load_3d(sm + P_IN_K + kBoxBytes, tm_ks, bar_in, 64, h, z);
+        if (kFused) {   // tm_las maps the gate's pre-activation x (bf16, 64-channel boxes)
+            tc::tma_load_3d(sm + P_IN_X, tm_las, bar_in, 0, h, z);
+            tc::tma_load_3d(sm + P_IN_X + kBoxBytes, tm_las, bar_in, 64, h, z);
+            tc::tma_load_3d(sm + P_IN_VF, tm_v, bar_in, 0, h, z);
+        } else {
+#pragma unroll
+            for (int b = 0; b < 4; ++b)
+                tc::tma_load_3d(sm + P_IN_LA + b * kBoxBytes, tm_las, bar_in, 32 * b, h, z);
+            tc::tma_load_3d(sm + P_IN_V, tm_v, bar_in, 0, h, z);
+        }
+    };
+    // Publication of an image: thread 0 waits until all its bulk stores (Qs, Kb, [P;T], W,
+    // U' of that image) are complete, then arrives (release, cluster scope; the generic
+    // stores of other threads into the slot precede it through CTA barriers) on the
+    // consumer's "ready" barrier of the image's ring slot.
+    // (A test hook withholds producer 0's first "ready", so that the consumer's wait runs out.)
+    int pending = -1, pending_img = 0;
+    auto publish = [&]() {
+        if (tid == 0 && pending >= 0) {
+            tc::bulk_wait_all();
+            tc::fence_proxy_async_global();
+            const bool withheld = test_timeout && rank == 0 && pending_img == 0;
+            if (!aborted(ctl) && !withheld) tc::mbar_arrive_remote(c_ready + 8 * pending);
+        }
+        pending = -1;
     };
     if (tid == 0 && rank < nchunks) load_inputs(rank);
+    load_beta(rank, 0);
     for (int c = rank; c < nchunks; c += kProducers) {
+        if (__syncthreads_or(aborted(ctl))) break;   // uniform: the cluster gave up
+        const float *beta_s = vec + 64 * (img & 1);
         const int t0 = c * kC;
         const int valid = min(kC, T - t0);
         const long trow0 = ztok + t0;
@@ -221,188 +334,358 @@ __device__ void producer(uint8_t *sm, uint32_t tmem, int rank, uint8_t *ring, co
             tc::tma_prefetch_l2_3d(tm_la, 0, h, z);
             tc::tma_prefetch_l2_3d(tm_v, 0, h, z);
         }
-        wait_local(bar_in, ph_in, ctl);
-        ph_in ^= 1;
-        CMARK(mk + 0);
+        if (wait_local(bar_in, ph_in, ctl)) {
+            ph_in ^= 1;
+            pend_in = false;
+        }
 
-        // ------------------------------------------------ gates and operands
-        if (tid < kC) beta_s[tid] = tid < valid ? beta[(trow0 + tid) * H + h] : 0.f;
-        uint4 vin[4];   // V row tid/4, columns 32 (tid%4) .. +32 (bf16); stored while [A;P] runs
-        {
-            const int t = tid >> 2, piece = tid & 3;
-            const uint4 *src = reinterpret_cast<const uint4 *>(sm + P_IN_V + t * 256 + 64 * piece);
-#pragma unroll
-            for (int m = 0; m < 4; ++m) vin[m] = t < valid ? src[m] : make_uint4(0, 0, 0, 0);
-        }
-        const int p = tid & 63, qq = tid >> 6;  // channels 2p, 2p+1; tokens 16qq .. 16qq+15
-        float2 lg[16];
-        uint32_t qv[16], kv[16];
-#pragma unroll
-        for (int u = 0; u < 16; ++u) {
-            const int t = 16 * qq + u;
-            const bool ok = t < valid;
-            lg[u] = ok ? *reinterpret_cast<const float2 *>(sm + P_IN_LA + t * 512 + 8 * p)
-                       : make_float2(0.f, 0.f);
-            qv[u] = ok ? *reinterpret_cast<const uint32_t *>(sm + P_IN_Q + t * 256 + 4 * p) : 0u;
-            kv[u] = ok ? *reinterpret_cast<const uint32_t *>(sm + P_IN_K + t * 256 + 4 * p) : 0u;
-        }
-        {
-            float s0 = 0.f, s1 = 0.f;
-#pragma unroll
-            for (int u = 0; u < 16; ++u) { s0 += lg[u].x; s1 += lg[u].y; }
-            psum[qq * 128 + 2 * p] = s0;
-            psum[qq * 128 + 2 * p + 1] = s1;
-        }
-        const int rb = img % kRingDepth;  // ring slot of this image; image img-kRingDepth used it before
-        uint8_t *gs = ring + (kRingDepth * rank + rb) * kSlotStride;
-        if (tid == 0) {
-            tc::bulk_wait_read_all();  // the previous [P;T] has left the staging area
-            if (img >= kRingDepth) wait_cluster(bar_loaded + rb, ((img / kRingDepth) - 1) & 1, ctl);
-        }
-        __syncthreads();  // inputs are in registers: the tf32 tiles may now overwrite them
-        {
-            float pre0 = 0.f, pre1 = 0.f, tot0 = 0.f, tot1 = 0.f;
-#pragma unroll
-            for (int q2 = 0; q2 < 4; ++q2) {
-                const float a0 = psum[q2 * 128 + 2 * p], a1 = psum[q2 * 128 + 2 * p + 1];
-                if (q2 < qq) { pre0 += a0; pre1 += a1; }
-                tot0 += a0;
-                tot1 += a1;
-            }
-            const float ga0 = 0.5f * tot0, ga1 = 0.5f * tot1;
-            const float ea0 = expf(ga0), ea1 = expf(ga1);                  // e^{g_a}
-            const float eca0 = expf(tot0 - ga0), eca1 = expf(tot1 - ga1);  // e^{g_C - g_a}
-            if (qq == 0) {
-                float *gam = reinterpret_cast<float *>(gs + SL_GAM);
-                gam[2 * p] = expf(tot0);
-                gam[2 * p + 1] = expf(tot1);
-            }
-            constexpr float kLog2e = 1.4426950408889634f;
-            float d0 = (pre0 - ga0) * kLog2e, d1 = (pre1 - ga1) * kLog2e;
-            const uint32_t cc = 2 * p;
-            const uint32_t rowq = qq * 2048u;
-            const uint32_t b32 = (cc & 3u) * 4u + rowq;
-            const uint32_t ch32 = (cc & 31u) >> 2, kb32 = cc >> 5;
-            const uint32_t b16 = (cc & 7u) * 2u + rowq;
-            const uint32_t ch16 = (cc & 63u) >> 3, kb16 = cc >> 6;
-#pragma unroll
-            for (int u = 0; u < 16; ++u) {
-                const uint32_t r = (u >> 3) * 1024u + (u & 7) * 128u;
-                const uint32_t o32 = b32 + r + (((ch32 ^ (u & 7)) & 7u) << 4);
-                const uint32_t o16 = b16 + r + (((ch16 ^ (u & 7)) & 7u) << 4);
-                d0 = fmaf(lg[u].x, kLog2e, d0);
-                d1 = fmaf(lg[u].y, kLog2e, d1);
-                const float q0 = tc::bf16_lo(qv[u]), q1 = tc::bf16_hi(qv[u]);
-                const float k0 = tc::bf16_lo(kv[u]), k1 = tc::bf16_hi(kv[u]);
-                const float E0 = tc::ex2(d0), E1 = tc::ex2(d1);
-                const float F0 = tc::ex2(-d0), F1 = tc::ex2(-d1);
-                const float ke0 = k0 * E0, ke1 = k1 * E1, qe0 = q0 * E0, qe1 = q1 * E1;
-                const float kf0 = k0 * F0, kf1 = k1 * F1;
-                *reinterpret_cast<float2 *>(sm + P_KQT + kb32 * kKQTBlk + o32) = make_float2(ke0, ke1);
-                *reinterpret_cast<float2 *>(sm + P_KQT + kb32 * kKQTBlk + 8192 + o32) = make_float2(qe0, qe1);
-                *reinterpret_cast<float2 *>(sm + P_KHT + kb32 * kKHTBlk + o32) = make_float2(kf0, kf1);
-                *reinterpret_cast<uint32_t *>(gs + SL_QW + kb16 * kQWBlk + o16) = pack_f16(qe0 * ea0, qe1 * ea1);
-                *reinterpret_cast<uint32_t *>(sm + P_KSV + kb16 * kTokBlk + o16) = pack_f16(ke0 * ea0, ke1 * ea1);
-                *reinterpret_cast<uint32_t *>(gs + SL_KB + kb16 * kTokBlk + o16) = pack_f16(kf0 * eca0, kf1 * eca1);
-            }
-        }
-        fence_proxy_async_smem();
-        __syncthreads();
-        CMARK(mk + 1);
-
-        // ------------------------------------------------ [A;P] (tf32)
-        if (tid == 0) {
-            tc_fence_after();
-#pragma unroll
-            for (int kk = 0; kk < 16; ++kk)
-                mma_tf32(tmem + PCOL_AP, d_kqt + (((kk >> 2) * kKQTBlk + (kk & 3) * 32) >> 4),
-                         d_kht + (((kk >> 2) * kKHTBlk + (kk & 3) * 32) >> 4), IDESC_AP, kk > 0);
-            tc::mma_commit(bar_mma);
-        }
+        load_beta(c + kProducers, (img + 1) & 1);   // the next image's beta, one image ahead
         {   // V -> fp16 columns 128..255 of the [Ks | V] operand (read by [W | U'] only)
             const int t = tid >> 2, piece = tid & 3;
+            const uint4 *src = reinterpret_cast<const uint4 *>(sm + (kFused ? P_IN_VF : P_IN_V) + t * 256 + 64 * piece);
 #pragma unroll
             for (int m = 0; m < 4; ++m) {
+                const uint4 vin = t < valid ? src[m] : make_uint4(0, 0, 0, 0);
                 uint4 w;
-                w.x = pack_f16(tc::bf16_lo(vin[m].x), tc::bf16_hi(vin[m].x));
-                w.y = pack_f16(tc::bf16_lo(vin[m].y), tc::bf16_hi(vin[m].y));
-                w.z = pack_f16(tc::bf16_lo(vin[m].z), tc::bf16_hi(vin[m].z));
-                w.w = pack_f16(tc::bf16_lo(vin[m].w), tc::bf16_hi(vin[m].w));
+                w.x = pack_f16(tc::bf16_lo(vin.x), tc::bf16_hi(vin.x));
+                w.y = pack_f16(tc::bf16_lo(vin.y), tc::bf16_hi(vin.y));
+                w.z = pack_f16(tc::bf16_lo(vin.z), tc::bf16_hi(vin.z));
+                w.w = pack_f16(tc::bf16_lo(vin.w), tc::bf16_hi(vin.w));
                 *reinterpret_cast<uint4 *>(sm + P_KSV + 2 * kTokBlk +
                                            sw128k_off(t, 32 * piece + 8 * m, kTokBlk)) = w;
             }
         }
-        wait_local(bar_mma, ph_mma, ctl);
-        ph_mma ^= 1;
-        tc_fence_after();
-        CMARK(mk + 2);
 
-        // ------------------------------------------------ A (fp32), P (fp16), UT solve, T (fp16)
-        {
-            float vv[32];
-            tc::tmem_ld32(tc::tmem_addr(tmem, 32 * quad, PCOL_AP + half * 32), vv);
-            tc::tmem_wait_ld();
-            if (quad < 2) {
-                const int i = row;
-                const float bi = beta_s[i];
+        // ------------------------------------------------ phase 1a: in-sub-chunk prefix sums
+        // Thread (p, I) = (tid % 64, tid / 64) runs channels 2p, 2p + 1 of sub-chunk I token by
+        // token: g^L into ST_GL (the swizzled layout of log alpha), and the per-channel table.
+        if (kFused) {   // 1 / ||q_t|| and 1 / ||k_t|| over the 128 channels (a zero row stays zero)
+            const int t = tid >> 2, which = (tid >> 1) & 1, hf = tid & 1;
+            const uint8_t *rowp = sm + (which ? P_IN_K : P_IN_Q) + hf * kBoxBytes + t * 128;
+            float ss = 0.f;
 #pragma unroll
-                for (int u = 0; u < 32; ++u) {
-                    const int j = half * 32 + u;
-                    Af[i * kLD + j] = j < i ? bi * vv[u] : 0.f;
+            for (int c = 0; c < 8; ++c) {
+                const uint4 x = *reinterpret_cast<const uint4 *>(rowp + (((c ^ (t & 7)) & 7) << 4));
+                const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+                for (int m = 0; m < 4; ++m) {
+                    const float lo = tc::bf16_lo(w[m]), hi = tc::bf16_hi(w[m]);
+                    ss = fmaf(lo, lo, fmaf(hi, hi, ss));
                 }
-            } else {
-                const int i = row - 64;
+            }
+            ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+            if (hf == 0) vec[V_INV + which * 64 + t] = ss > 0.f ? rsqrtf(ss) : 0.f;
+        }
+        {
+            const int p = tid & 63, Ib = tid >> 6, cp = 2 * p;
+            const uint32_t off = (cp >> 5) * kBoxBytes + (cp & 3) * 4;
+            const uint32_t ch = (cp & 31) >> 2;
+            float s0 = 0.f, s1 = 0.f, m0 = 0.f, m1 = 0.f;
 #pragma unroll
-                for (int u = 0; u < 32; u += 2) {
-                    const int j = half * 32 + u;
-                    const float lo = j <= i ? vv[u] : 0.f, hi = j + 1 <= i ? vv[u + 1] : 0.f;
-                    *reinterpret_cast<uint32_t *>(st + SL_PT + sw128k_off(i, j, 0)) = pack_f16(lo, hi);
+            for (int u = 0; u < 16; ++u) {
+                const int t = 16 * Ib + u;
+                const uint32_t o = off + t * 128u + (((ch ^ (t & 7)) & 7u) << 4);
+                float2 x = make_float2(0.f, 0.f);
+                if (t < valid) {
+                    if (kFused) {   // log alpha = -softplus(x), x from its bf16 box
+                        const uint32_t xo = (cp >> 6) * kBoxBytes + t * 128u +
+                                            (((((cp & 63) >> 3) ^ (t & 7)) & 7u) << 4) + (cp & 7) * 2;
+                        const uint32_t xv = *reinterpret_cast<const uint32_t *>(sm + P_IN_X + xo);
+                        x = make_float2(neg_softplus(tc::bf16_lo(xv)), neg_softplus(tc::bf16_hi(xv)));
+                    } else {
+                        x = *reinterpret_cast<const float2 *>(sm + P_IN_LA + o);
+                    }
+                }
+                s0 += x.x;
+                s1 += x.y;
+                *reinterpret_cast<float2 *>(st + ST_GL + o) = make_float2(s0, s1);
+                if (u == 7) { m0 = s0; m1 = s1; }
+            }
+            const int e = Ib * 128 + cp;
+            *reinterpret_cast<float2 *>(vec + V_TOT + e) = make_float2(s0, s1);
+            *reinterpret_cast<float2 *>(vec + V_EM + e) =
+                make_float2(tc::ex2(-m0 * kLog2e), tc::ex2(-m1 * kLog2e));
+            *reinterpret_cast<float2 *>(vec + V_EC + e) =
+                make_float2(tc::ex2((m0 - s0) * kLog2e), tc::ex2((m1 - s1) * kLog2e));
+            *reinterpret_cast<float2 *>(vec + V_P + e) =
+                make_float2(tc::ex2(s0 * kLog2e), tc::ex2(s1 * kLog2e));
+            if (s0 < kRangeLog || s1 < kRangeLog) *reinterpret_cast<volatile int *>(vec + V_FLAG) = 1;
+        }
+        publish();   // the previous image (its stores have had phase 1a to land)
+        __syncthreads();
+        const bool far_decay = *reinterpret_cast<volatile int *>(vec + V_FLAG) != 0;
+
+        // ------------------------------------------------ phase 1b: diagonal blocks (tf32
+        // mma.sync, fragments straight from registers), rows of the off-diagonal blocks
+        const bool va = ta < valid, vb = tb < valid;
+        // the fused prologue's L2 normalisation, applied where q and k are unpacked
+        const float nqa = kFused ? vec[V_INV + ta] : 1.f, nqb = kFused ? vec[V_INV + tb] : 1.f;
+        const float nka = kFused ? vec[V_INV + 64 + ta] : 1.f, nkb = kFused ? vec[V_INV + 64 + tb] : 1.f;
+        uint32_t qA[8], qB[8], kA[8], kB[8];
+        float rA[8][2], rB[8][2], sA[8][2], sB[8][2];   // e^{g^L}, e^{tot - g^L} of tokens a, b
+        float accA[2][4] = {}, accP[2][4] = {};
+        const uint32_t rowa = static_cast<uint32_t>(ta) * 128u, rowb = static_cast<uint32_t>(tb) * 128u;
+#pragma unroll
+        for (int s = 0; s < 8; ++s) {
+            const int c0 = 64 * half + 8 * s + 2 * t4;
+            const uint32_t qk_off = half * kBoxBytes + ((s ^ g) << 4) + 4 * t4;
+            const uint32_t la_off = (c0 >> 5) * kBoxBytes + (((((c0 & 31) >> 2) ^ g) & 7) << 4) + 8 * (t4 & 1);
+            qA[s] = va ? *reinterpret_cast<const uint32_t *>(sm + P_IN_Q + rowa + qk_off) : 0u;
+            qB[s] = vb ? *reinterpret_cast<const uint32_t *>(sm + P_IN_Q + rowb + qk_off) : 0u;
+            kA[s] = va ? *reinterpret_cast<const uint32_t *>(sm + P_IN_K + rowa + qk_off) : 0u;
+            kB[s] = vb ? *reinterpret_cast<const uint32_t *>(sm + P_IN_K + rowb + qk_off) : 0u;
+            const float2 xa = *reinterpret_cast<const float2 *>(st + ST_GL + rowa + la_off);
+            const float2 xb = *reinterpret_cast<const float2 *>(st + ST_GL + rowb + la_off);
+            const int e = I * 128 + c0;
+            const float2 tot = *reinterpret_cast<const float2 *>(vec + V_TOT + e);
+            const float2 em = *reinterpret_cast<const float2 *>(vec + V_EM + e);
+            const float2 ec = *reinterpret_cast<const float2 *>(vec + V_EC + e);
+            // factors anchored at the sub-chunk's start (rho) and end (sigma), both <= 1
+            rA[s][0] = tc::ex2(xa.x * kLog2e);
+            rA[s][1] = tc::ex2(xa.y * kLog2e);
+            rB[s][0] = tc::ex2(xb.x * kLog2e);
+            rB[s][1] = tc::ex2(xb.y * kLog2e);
+            sA[s][0] = tc::ex2((tot.x - xa.x) * kLog2e);
+            sA[s][1] = tc::ex2((tot.y - xa.y) * kLog2e);
+            sB[s][0] = tc::ex2((tot.x - xb.x) * kLog2e);
+            sB[s][1] = tc::ex2((tot.y - xb.y) * kLog2e);
+            // diagonal-block factors around token 7: rows e^{g_i - g_m} = rho_i e^{-g_m},
+            // columns e^{g_m - g_j} = sigma_j e^{g_m - tot}
+            float ra0 = rA[s][0] * em.x, ra1 = rA[s][1] * em.y, rb0 = rB[s][0] * em.x, rb1 = rB[s][1] * em.y;
+            float ca0 = sA[s][0] * ec.x, ca1 = sA[s][1] * ec.y, cb0 = sB[s][0] * ec.x, cb1 = sB[s][1] * ec.y;
+            if (far_decay) {
+                // some channel of the chunk decays by more than e^-87 inside one sub-chunk: such a
+                // channel takes its diagonal factors from log alpha clamped at -10 per token
+                const bool f0 = tot.x >= kRangeLog, f1 = tot.y >= kRangeLog;
+                float2 la = make_float2(0.f, 0.f), lb = make_float2(0.f, 0.f);
+                if (kFused) {
+                    const uint32_t xa2 = va ? *reinterpret_cast<const uint32_t *>(sm + P_IN_X + rowa + qk_off) : 0u;
+                    const uint32_t xb2 = vb ? *reinterpret_cast<const uint32_t *>(sm + P_IN_X + rowb + qk_off) : 0u;
+                    if (va) la = make_float2(neg_softplus(tc::bf16_lo(xa2)), neg_softplus(tc::bf16_hi(xa2)));
+                    if (vb) lb = make_float2(neg_softplus(tc::bf16_lo(xb2)), neg_softplus(tc::bf16_hi(xb2)));
+                } else {
+                    if (va) la = *reinterpret_cast<const float2 *>(sm + P_IN_LA + rowa + la_off);
+                    if (vb) lb = *reinterpret_cast<const float2 *>(sm + P_IN_LA + rowb + la_off);
+                }
+                float ya0 = scan8(fmaxf(la.x, kClampLog), g), ya1 = scan8(fmaxf(la.y, kClampLog), g);
+                float yb0 = scan8(fmaxf(lb.x, kClampLog), g), yb1 = scan8(fmaxf(lb.y, kClampLog), g);
+                const float ym0 = __shfl_sync(0xffffffffu, ya0, 28 + t4);   // at token 7
+                const float ym1 = __shfl_sync(0xffffffffu, ya1, 28 + t4);
+                yb0 += ym0;
+                yb1 += ym1;
+                if (!f0) {
+                    ra0 = tc::ex2((ya0 - ym0) * kLog2e);
+                    rb0 = tc::ex2((yb0 - ym0) * kLog2e);
+                    ca0 = tc::ex2((ym0 - ya0) * kLog2e);
+                    cb0 = tc::ex2((ym0 - yb0) * kLog2e);
+                }
+                if (!f1) {
+                    ra1 = tc::ex2((ya1 - ym1) * kLog2e);
+                    rb1 = tc::ex2((yb1 - ym1) * kLog2e);
+                    ca1 = tc::ex2((ym1 - ya1) * kLog2e);
+                    cb1 = tc::ex2((ym1 - yb1) * kLog2e);
+                }
+            }
+            const float qa0 = tc::bf16_lo(qA[s]) * nqa, qa1 = tc::bf16_hi(qA[s]) * nqa;
+            const float qb0 = tc::bf16_lo(qB[s]) * nqb, qb1 = tc::bf16_hi(qB[s]) * nqb;
+            const float ka0 = tc::bf16_lo(kA[s]) * nka, ka1 = tc::bf16_hi(kA[s]) * nka;
+            const float kb0 = tc::bf16_lo(kB[s]) * nkb, kb1 = tc::bf16_hi(kB[s]) * nkb;
+            {   // diagonal block: A^d += K~ K^^T, P^d += Q~ K^^T over this k-step's 8 channels
+                // (fp32 operands; the tensor cores read them as tf32)
+                const uint32_t ak[4] = {__float_as_uint(ka0 * ra0), __float_as_uint(kb0 * rb0),
+                                        __float_as_uint(ka1 * ra1), __float_as_uint(kb1 * rb1)};
+                const uint32_t aq[4] = {__float_as_uint(qa0 * ra0), __float_as_uint(qb0 * rb0),
+                                        __float_as_uint(qa1 * ra1), __float_as_uint(qb1 * rb1)};
+                const uint32_t b00 = __float_as_uint(ka0 * ca0), b01 = __float_as_uint(ka1 * ca1);  // column token g
+                const uint32_t b10 = __float_as_uint(kb0 * cb0), b11 = __float_as_uint(kb1 * cb1);  // column token g + 8
+                tc::mma_16x8x8_tf32(accA[0], ak, b00, b01);
+                tc::mma_16x8x8_tf32(accA[1], ak, b10, b11);
+                tc::mma_16x8x8_tf32(accP[0], aq, b00, b01);
+                tc::mma_16x8x8_tf32(accP[1], aq, b10, b11);
+            }
+            // column operand of the off-diagonal blocks: K e^{G_{J+1} - g_j} for this sub-chunk J = I
+            *reinterpret_cast<float2 *>(sm + P_KSIG + rowa + la_off) = make_float2(ka0 * sA[s][0], ka1 * sA[s][1]);
+            *reinterpret_cast<float2 *>(sm + P_KSIG + rowb + la_off) = make_float2(kb0 * sB[s][0], kb1 * sB[s][1]);
+        }
+
+        const int rb = img % kRingDepth;  // ring slot of this image; image img-kRingDepth used it before
+        uint8_t *gs = ring + (kRingDepth * rank + rb) * kSlotStride;
+        if (tid == 0) {
+            tc::bulk_wait_read_all();  // the previous image's staged parts have left shared memory
+            if (img >= kRingDepth) wait_cluster(bar_loaded + rb, ((img / kRingDepth) - 1) & 1, ctl);
+        }
+        cp_async_wait_prev();   // this image's beta (all but the group just issued)
+        __syncthreads();   // the inputs and g^L are dead; every thread has read the flag
+        if (tid == 0) *reinterpret_cast<volatile int *>(vec + V_FLAG) = 0;   // for the next image
+
+        // ------------------------------------------------ phase 2: chunk-level factors
+        // (products of the sub-chunks' e^{tot}: e^{G_I}, e^{g_C - G_{I+1}}) and the off-diagonal blocks
+        if (half == 1) {   // diagonal partials of channels 64..127 for the half-0 warp of sub-chunk I
+            float4 *dx = reinterpret_cast<float4 *>(sm + P_DX) + (I * 32 + lane) * 4;
+            dx[0] = make_float4(accA[0][0], accA[0][1], accA[0][2], accA[0][3]);
+            dx[1] = make_float4(accA[1][0], accA[1][1], accA[1][2], accA[1][3]);
+            dx[2] = make_float4(accP[0][0], accP[0][1], accP[0][2], accP[0][3]);
+            dx[3] = make_float4(accP[1][0], accP[1][1], accP[1][2], accP[1][3]);
+        }
+        const uint32_t row_a = half * 8192u + (ta >> 3) * 1024u + g * 128u + 4u * t4;   // token a, no swizzle term
+#pragma unroll
+        for (int s = 0; s < 8; ++s) {
+            const int c0 = 64 * half + 8 * s + 2 * t4;
+            float2 pj[4];   // e^{tot_J} of the four sub-chunks
+#pragma unroll
+            for (int J = 0; J < 4; ++J) pj[J] = *reinterpret_cast<const float2 *>(vec + V_P + J * 128 + c0);
+            float eG0 = 1.f, eG1 = 1.f, eK0 = 1.f, eK1 = 1.f;
+#pragma unroll
+            for (int J = 0; J < 4; ++J) {
+                if (J < I) { eG0 *= pj[J].x; eG1 *= pj[J].y; }
+                if (J > I) { eK0 *= pj[J].x; eK1 *= pj[J].y; }
+            }
+            const float qa0 = tc::bf16_lo(qA[s]) * nqa, qa1 = tc::bf16_hi(qA[s]) * nqa;
+            const float qb0 = tc::bf16_lo(qB[s]) * nqb, qb1 = tc::bf16_hi(qB[s]) * nqb;
+            const float ka0 = tc::bf16_lo(kA[s]) * nka, ka1 = tc::bf16_hi(kA[s]) * nka;
+            const float kb0 = tc::bf16_lo(kB[s]) * nkb, kb1 = tc::bf16_hi(kB[s]) * nkb;
+            const float fa0 = rA[s][0] * eG0, fa1 = rA[s][1] * eG1, fb0 = rB[s][0] * eG0, fb1 = rB[s][1] * eG1;
+            // Qs = Q e^{g} and Kb = K e^{g_C - g} (staged for the ring slot), Ks = K e^{g} into [Ks | V];
+            // all three are [token][channel] tiles with 64-channel blocks 8 KB apart
+            const uint32_t oa = row_a + (((s ^ g) & 7) << 4), ob = oa + 1024;
+            *reinterpret_cast<uint32_t *>(st + ST_QS + oa) = pack_f16(qa0 * fa0, qa1 * fa1);
+            *reinterpret_cast<uint32_t *>(st + ST_QS + ob) = pack_f16(qb0 * fb0, qb1 * fb1);
+            *reinterpret_cast<uint32_t *>(sm + P_KSV + oa) = pack_f16(ka0 * fa0, ka1 * fa1);
+            *reinterpret_cast<uint32_t *>(sm + P_KSV + ob) = pack_f16(kb0 * fb0, kb1 * fb1);
+            *reinterpret_cast<uint32_t *>(sm + P_KBS + oa) = pack_f16(ka0 * sA[s][0] * eK0, ka1 * sA[s][1] * eK1);
+            *reinterpret_cast<uint32_t *>(sm + P_KBS + ob) = pack_f16(kb0 * sB[s][0] * eK0, kb1 * sB[s][1] * eK1);
+            if (I == 0 && g == 0)
+                *reinterpret_cast<float2 *>(gs + SL_GAM + 4 * c0) =
+                    make_float2(pj[0].x * pj[1].x * pj[2].x * pj[3].x, pj[0].y * pj[1].y * pj[2].y * pj[3].y);
+        }
+        // Off-diagonal blocks (I, J), J < I, over this warp's 64 channels:
+        //   A^o += [K e^{g - G_I} Diag(e^{G_I - G_{J+1}})] (K e^{G_{J+1} - g})^T, P^o likewise with Q;
+        // partials of both channel halves go to shared memory, summed by the half-1 warp below.
+        for (int J = 0; J < I; ++J) {
+            float oA[2][4] = {}, oP[2][4] = {};
+#pragma unroll
+            for (int s = 0; s < 8; ++s) {
+                const int c0 = 64 * half + 8 * s + 2 * t4;
+                float D0 = 1.f, D1 = 1.f;   // e^{G_I - G_{J+1}}: the sub-chunks strictly between J and I
+#pragma unroll
+                for (int Jm = 1; Jm < 3; ++Jm)
+                    if (Jm > J && Jm < I) {
+                        const float2 pm = *reinterpret_cast<const float2 *>(vec + V_P + Jm * 128 + c0);
+                        D0 *= pm.x;
+                        D1 *= pm.y;
+                    }
+                const float ra0 = rA[s][0] * D0, ra1 = rA[s][1] * D1, rb0 = rB[s][0] * D0, rb1 = rB[s][1] * D1;
+                const uint32_t ak[4] = {__float_as_uint(tc::bf16_lo(kA[s]) * nka * ra0), __float_as_uint(tc::bf16_lo(kB[s]) * nkb * rb0),
+                                        __float_as_uint(tc::bf16_hi(kA[s]) * nka * ra1), __float_as_uint(tc::bf16_hi(kB[s]) * nkb * rb1)};
+                const uint32_t aq[4] = {__float_as_uint(tc::bf16_lo(qA[s]) * nqa * ra0), __float_as_uint(tc::bf16_lo(qB[s]) * nqb * rb0),
+                                        __float_as_uint(tc::bf16_hi(qA[s]) * nqa * ra1), __float_as_uint(tc::bf16_hi(qB[s]) * nqb * rb1)};
+                const uint32_t la_off = (c0 >> 5) * kBoxBytes + (((((c0 & 31) >> 2) ^ g) & 7) << 4) + 8 * (t4 & 1);
+                const uint32_t rj = static_cast<uint32_t>(16 * J + g) * 128u;   // column token g of sub-chunk J
+                const float2 y0 = *reinterpret_cast<const float2 *>(sm + P_KSIG + rj + la_off);
+                const float2 y1 = *reinterpret_cast<const float2 *>(sm + P_KSIG + rj + 1024 + la_off);  // token g + 8
+                tc::mma_16x8x8_tf32(oA[0], ak, __float_as_uint(y0.x), __float_as_uint(y0.y));
+                tc::mma_16x8x8_tf32(oA[1], ak, __float_as_uint(y1.x), __float_as_uint(y1.y));
+                tc::mma_16x8x8_tf32(oP[0], aq, __float_as_uint(y0.x), __float_as_uint(y0.y));
+                tc::mma_16x8x8_tf32(oP[1], aq, __float_as_uint(y1.x), __float_as_uint(y1.y));
+            }
+            float4 *px = reinterpret_cast<float4 *>(sm + P_PX) + ((half * 6 + pair_index(I, J)) * 32 + lane) * 4;
+            px[0] = make_float4(oA[0][0], oA[0][1], oA[0][2], oA[0][3]);
+            px[1] = make_float4(oA[1][0], oA[1][1], oA[1][2], oA[1][3]);
+            px[2] = make_float4(oP[0][0], oP[0][1], oP[0][2], oP[0][3]);
+            px[3] = make_float4(oP[1][0], oP[1][1], oP[1][2], oP[1][3]);
+        }
+        fence_proxy_async_smem();   // Ks and the staged Qs, Kb reach the async proxy
+        __syncthreads();
+
+        if (tid == 0 && !aborted(ctl)) {
+            tc::bulk_store_global(gs + SL_QW, st + ST_QS, 8192);                 // Qs, K-block 0
+            tc::bulk_store_global(gs + SL_QW + kQWBlk, st + ST_QS + 8192, 8192); // Qs, K-block 1
+            tc::bulk_store_global(gs + SL_KB, sm + P_KBS, 16384);                // Kb
+            tc::bulk_commit();
+        }
+        const float ba = beta_s[ta], bb = beta_s[tb];
+        if (half == 0) {
+            // diagonal blocks of A (times beta, strictly lower) and P (lower), both channel halves summed
+            const float4 *dx = reinterpret_cast<const float4 *>(sm + P_DX) + (I * 32 + lane) * 4;
+            const float4 x0 = dx[0], x1 = dx[1], x2 = dx[2], x3 = dx[3];
+            accA[0][0] += x0.x; accA[0][1] += x0.y; accA[0][2] += x0.z; accA[0][3] += x0.w;
+            accA[1][0] += x1.x; accA[1][1] += x1.y; accA[1][2] += x1.z; accA[1][3] += x1.w;
+            accP[0][0] += x2.x; accP[0][1] += x2.y; accP[0][2] += x2.z; accP[0][3] += x2.w;
+            accP[1][0] += x3.x; accP[1][1] += x3.y; accP[1][2] += x3.z; accP[1][3] += x3.w;
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt) {
+                const int jl = 8 * nt + 2 * t4, j = 16 * I + jl;
+                *reinterpret_cast<float2 *>(Af + ta * kLD + j) =
+                    make_float2(jl < g ? ba * accA[nt][0] : 0.f, jl + 1 < g ? ba * accA[nt][1] : 0.f);
+                *reinterpret_cast<float2 *>(Af + tb * kLD + j) =
+                    make_float2(jl < g + 8 ? bb * accA[nt][2] : 0.f, jl + 1 < g + 8 ? bb * accA[nt][3] : 0.f);
+                *reinterpret_cast<uint32_t *>(st + ST_PT + sw128k_off(ta, j, 0)) =
+                    pack_f16(jl <= g ? accP[nt][0] : 0.f, jl + 1 <= g ? accP[nt][1] : 0.f);
+                *reinterpret_cast<uint32_t *>(st + ST_PT + sw128k_off(tb, j, 0)) =
+                    pack_f16(jl <= g + 8 ? accP[nt][2] : 0.f, jl + 1 <= g + 8 ? accP[nt][3] : 0.f);
+            }
+        } else {
+            // off-diagonal blocks (I, J) of A and P, both channel halves summed
+            for (int J = 0; J < I; ++J) {
+                const float4 *p0 = reinterpret_cast<const float4 *>(sm + P_PX) + (pair_index(I, J) * 32 + lane) * 4;
+                const float4 *p1 = p0 + 6 * 32 * 4;
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt) {
+                    const float4 a0 = p0[nt], a1 = p1[nt], q0 = p0[2 + nt], q1 = p1[2 + nt];
+                    const int j = 16 * J + 8 * nt + 2 * t4;
+                    *reinterpret_cast<float2 *>(Af + ta * kLD + j) = make_float2(ba * (a0.x + a1.x), ba * (a0.y + a1.y));
+                    *reinterpret_cast<float2 *>(Af + tb * kLD + j) = make_float2(bb * (a0.z + a1.z), bb * (a0.w + a1.w));
+                    *reinterpret_cast<uint32_t *>(st + ST_PT + sw128k_off(ta, j, 0)) = pack_f16(q0.x + q1.x, q0.y + q1.y);
+                    *reinterpret_cast<uint32_t *>(st + ST_PT + sw128k_off(tb, j, 0)) = pack_f16(q0.z + q1.z, q0.w + q1.w);
                 }
             }
         }
-        tc_fence_before();
         __syncthreads();
-        CMARK(mk + 3);
+
+        // ------------------------------------------------ UT solve, T (fp16)
         ut::unit_lower_inverse(Af, Xf, tid);
-        CMARK(mk + 4);
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
             const int e = tid + u * kThreads;
             const int i = e >> 5, j = (e & 31) * 2;
             const float lo = j <= i ? Xf[i * kLD + j] * beta_s[j] : 0.f;
             const float hi = j + 1 <= i ? Xf[i * kLD + j + 1] * beta_s[j + 1] : 0.f;
-            *reinterpret_cast<uint32_t *>(st + SL_PT + 8192 + sw128k_off(i, j, 0)) = pack_f16(lo, hi);
+            *reinterpret_cast<uint32_t *>(st + ST_PT + 8192 + sw128k_off(i, j, 0)) = pack_f16(lo, hi);
         }
         fence_proxy_async_smem();
         __syncthreads();
-        // the tf32 region (tiles, A, X) is dead until the next chunk: stage its inputs there
+        // the input region (A, X) is dead until the next chunk: stage its inputs there
         if (tid == 0) {
+            tc::bulk_wait_read_all();   // the staged Qs and Kb have left the input region
             if (c + kProducers < nchunks) load_inputs(c + kProducers);
-            tc::bulk_store_global(gs + SL_PT, st + SL_PT, 16384);   // [P;T] to the ring slot
-            tc::bulk_commit();
+            if (!aborted(ctl)) {
+                tc::bulk_store_global(gs + SL_PT, st + ST_PT, 16384);   // [P;T] to the ring slot
+                tc::bulk_commit();
+            }
         }
-        CMARK(mk + 5);
 
         // ------------------------------------------------ [W | U'] = T [Ks | V] (fp16, N = 256)
-        if (tid == 0) {
+        if (tid == 0 && !aborted(ctl)) {
             tc_fence_after();
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
                 mma_f16(tmem + PCOL_WU, d_pt + ((kk * 32) >> 4), d_ksv + ((kk * 2048) >> 4), IDESC_WU, kk > 0);
             tc::mma_commit(bar_mma);
+            pend_mma = true;
         }
-        wait_local(bar_mma, ph_mma, ctl);
-        ph_mma ^= 1;
+        if (wait_local(bar_mma, ph_mma, ctl)) {
+            ph_mma ^= 1;
+            pend_mma = false;
+        }
         tc_fence_after();
-        CMARK(mk + 6);
 #pragma unroll
         for (int part = 0; part < 2; ++part) {   // part 0: W, part 1: U'
             if (quad >= 2) {
                 const int i = row - 64;
                 float w[64];
-                const uint32_t ta = tc::tmem_addr(tmem, 32 * quad, PCOL_WU + part * 128 + half * 64);
-                tc::tmem_ld32(ta, *reinterpret_cast<float(*)[32]>(&w[0]));
-                tc::tmem_ld32(ta + 32, *reinterpret_cast<float(*)[32]>(&w[32]));
+                const uint32_t taddr = tc::tmem_addr(tmem, 32 * quad, PCOL_WU + part * 128 + half * 64);
+                tc::tmem_ld32(taddr, *reinterpret_cast<float(*)[32]>(&w[0]));
+                tc::tmem_ld32(taddr + 32, *reinterpret_cast<float(*)[32]>(&w[32]));
                 tc::tmem_wait_ld();
 #pragma unroll
                 for (int u = 0; u < 64; u += 8) {
@@ -412,43 +695,50 @@ __device__ void producer(uint8_t *sm, uint32_t tmem, int rank, uint8_t *ring, co
                     x.z = pack_f16(w[u + 4], w[u + 5]);
                     x.w = pack_f16(w[u + 6], w[u + 7]);
                     const int col = half * 64 + u;
-                    const uint32_t off = part == 0 ? SL_QW + sw128k_off(64 + i, col, kQWBlk)
-                                                   : SL_UP + sw128k_off(i, col, kTokBlk);
+                    const uint32_t off = part == 0 ? ST_W + sw128k_off(i, col, 8192)
+                                                   : ST_UP + sw128k_off(i, col, kTokBlk);
                     *reinterpret_cast<uint4 *>(st + off) = x;
                 }
             }
             fence_proxy_async_smem();
             if (part == 0) {   // W leaves while U' is formed
                 __syncthreads();
-                if (tid == 0) {
-                    tc::bulk_store_global(gs + SL_QW + 8192, st + SL_QW + 8192, 8192);   // W, K-block 0
-                    tc::bulk_store_global(gs + SL_QW + kQWBlk + 8192, st + SL_QW + kQWBlk + 8192, 8192);
+                if (tid == 0 && !aborted(ctl)) {
+                    tc::bulk_store_global(gs + SL_QW + 8192, st + ST_W, 8192);   // W, K-block 0
+                    tc::bulk_store_global(gs + SL_QW + kQWBlk + 8192, st + ST_W + 8192, 8192);
                     tc::bulk_commit();
                 }
             }
         }
         tc_fence_before();
         __syncthreads();
-        CMARK(mk + 7);
 
         // ------------------------------------------------ publish the image through L2
         // Every thread's generic stores into the slot (Qs, Kb, e^{g_C}) precede thread 0's
         // release through the CTA barrier above; the release is cumulative.
         if (tid == 0) {
-            CMARK(mk + 9);
-            tc::bulk_store_global(gs + SL_UP, st + SL_UP, 16384);                  // U'
-            tc::bulk_commit();
-            tc::bulk_wait_all();   // [P;T], W and U' have reached the slot
-            tc::fence_proxy_async_global();
-            if (!*reinterpret_cast<volatile int *>(ctl.abort)) tc::mbar_arrive_remote(c_ready + 8 * rb);
+            if (!aborted(ctl)) {
+                tc::bulk_store_global(gs + SL_UP, st + ST_UP, 16384);                  // U'
+                tc::bulk_commit();
+            }
+            tc::bulk_wait_read_all();   // W and U' have left the stage
         }
-        CMARK(mk + 8);
+        __syncthreads();   // the next image may now write g^L over the stage
+        // The "ready" of this image is sent once its stores have reached L2: during the next
+        // image's phase 1a (before that image issues stores of its own), or after the loop.
+        pending = rb;
+        pending_img = img;
         ++img;
     }
-    if (tid == 0) tc::bulk_wait_read_all();
-    CMARK_FLUSH(0, 10);
+    publish();
+    // drain: what this CTA issued and has not seen complete (all of it after a give-up)
+    if (tid == 0) {
+        if (pend_in) drain(bar_in, ph_in, ctl);
+        if (pend_mma) drain(bar_mma, ph_mma, ctl);
+        tc::bulk_wait_all();
+    }
+    asm volatile("cp.async.wait_all;" ::: "memory");
 }
-
 // ============================================================ consumer
 __device__ void consumer(uint8_t *sm, uint32_t tmem, const uint8_t *ring, const float *__restrict__ S0,
                          __nv_bfloat16 *__restrict__ out, float *__restrict__ S_T, int T, int H,
@@ -464,6 +754,8 @@ __device__ void consumer(uint8_t *sm, uint32_t tmem, const uint8_t *ring, const 
     uint64_t *ready = full + 5;  // [kRingSlots]: producer p, ring slot b at ready[kRingDepth p + b]
     uint32_t ph_full = 0;   // bit s: parity of slot s's next fill
     uint32_t ph_x = 0, ph_s = 0, ph_o = 0;
+    uint32_t pend_full = 0;   // thread 0: bit s = a pull into slot s is in flight
+    bool pend_x = false, pend_s = false, pend_o = false;   // thread 0: an MMA group in flight
 
     const uint64_t d_s16 = tc::smem_desc(sbase + C_S16, 16384, 1024, tc::kSwizzle128);
     const uint64_t d_u16 = tc::smem_desc(sbase + C_U16, kTokBlk, 1024, tc::kSwizzle128);
@@ -487,9 +779,10 @@ __device__ void consumer(uint8_t *sm, uint32_t tmem, const uint8_t *ring, const 
                 wait_cluster(ready + rs, par, ctl);
             else if (!tc::mbar_test_cluster(ready + rs, par))
                 return;
-            if (*reinterpret_cast<volatile int *>(ctl.abort)) return;
+            if (aborted(ctl)) return;
             tc::fence_proxy_async_global();
             const int sl = next_load & 1;
+            pend_full |= 1u << sl;
             tc::mbar_arrive_expect_tx(full + sl, kSlotBytes);
             tc::bulk_load_global(sm + C_SLOT + sl * kSlotStride, ring + rs * kSlotStride, kSlotBytes,
                                  full + sl);
@@ -527,36 +820,36 @@ __device__ void consumer(uint8_t *sm, uint32_t tmem, const uint8_t *ring, const 
     __syncthreads();
     if (tid == 0) pull(0, true);
     if (nchunks > 0) {
-        wait_local(full, ph_full & 1, ctl);
-        if (tid == 0) issue_x(0);
+        if (wait_local(full, ph_full & 1, ctl)) pend_full &= ~1u;
+        if (tid == 0 && !aborted(ctl)) {
+            issue_x(0);
+            pend_x = true;
+        }
     }
 
-    CMARK_INIT(C_BAR);
     for (int c = 0; c < nchunks; ++c) {
+        if (__syncthreads_or(aborted(ctl))) break;   // uniform: the cluster gave up
         const int s = c & 1;
         const int t0 = c * kC;
         const int valid = min(kC, T - t0);
         const uint8_t *slot = sm + C_SLOT + s * kSlotStride;
         const uint32_t xcol = CCOL_X + s * 128;
-        wait_local(full + s, (ph_full >> s) & 1, ctl);  // (already complete) makes the slot visible
-        ph_full ^= 1u << s;
-        if (tid == 0 && c + kRingSlots < nchunks) {  // the ring slot of chunk c is reusable
+        if (wait_local(full + s, (ph_full >> s) & 1, ctl)) {  // (already complete) makes the slot visible
+            ph_full ^= 1u << s;
+            pend_full &= ~(1u << s);
+        }
+        if (tid == 0 && c + kRingSlots < nchunks && !aborted(ctl)) {  // the ring slot of chunk c is reusable
             // relaxed: the slot's bulk load has completed (observed above); no writes of
             // this thread need to be ordered before the producer's reuse of the slot
             const uint32_t rb = tc::map_to_rank(p_loaded + 8 * ((c / kProducers) % kRingDepth), c % kProducers);
             asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(rb) : "memory");
         }
-        CMARK(16);
-#ifdef KDA_PHASE_TIMING
-        const unsigned long long w0_ = clock64();
-#endif
-        wait_local(bar_x, ph_x, ctl);
-        ph_x ^= 1;
+        if (wait_local(bar_x, ph_x, ctl)) {
+            ph_x ^= 1;
+            pend_x = false;
+        }
         tc_fence_after();
-#ifndef KDA_NO_EARLY_PULL
         if (tid == 0) pull(c + 1, false);
-#endif
-        CMARK(17);
 
         // U = U' - W S  (lanes 64..127 = tokens)
         if (quad >= 2) {
@@ -583,13 +876,8 @@ __device__ void consumer(uint8_t *sm, uint32_t tmem, const uint8_t *ring, const 
         }
         fence_proxy_async_smem();
         tc_fence_before();
-#ifdef KDA_PHASE_TIMING
-        if (blockIdx.x == kCluster - 1 && (threadIdx.x & 31) == 0)
-            atomicAdd(&g_cluster_cycles[24 + (threadIdx.x >> 5)], clock64() - w0_);
-#endif
         __syncthreads();
-        CMARK(18);
-        if (tid == 0) {
+        if (tid == 0 && !aborted(ctl)) {
             tc_fence_after();
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
@@ -599,13 +887,15 @@ __device__ void consumer(uint8_t *sm, uint32_t tmem, const uint8_t *ring, const 
             for (int kk = 0; kk < 4; ++kk)
                 mma_f16(tmem + xcol, d_pt0 + s * kSlotDesc + ((kk * 32) >> 4), d_u16 + ((kk * 2048) >> 4), IDESC_X, 1);
             tc::mma_commit(bar_o);
+            pend_s = pend_o = true;
             pull(c + 1, false);
         }
         // S <- Diag(e^{g_C}) S + Kb^T U
-        wait_local(bar_s, ph_s, ctl);
-        ph_s ^= 1;
+        if (wait_local(bar_s, ph_s, ctl)) {
+            ph_s ^= 1;
+            pend_s = false;
+        }
         tc_fence_after();
-        CMARK(19);
         {
             const float gm = reinterpret_cast<const float *>(slot + SL_GAM)[row];
             float sv[64];
@@ -620,18 +910,20 @@ __device__ void consumer(uint8_t *sm, uint32_t tmem, const uint8_t *ring, const 
         fence_proxy_async_smem();
         tc_fence_before();
         __syncthreads();
-        CMARK(20);
         if (c + 1 < nchunks) {
             if (tid == 0) pull(c + 1, true);
-            wait_local(full + (s ^ 1), (ph_full >> (s ^ 1)) & 1, ctl);
-            if (tid == 0) issue_x(c + 1);
+            if (wait_local(full + (s ^ 1), (ph_full >> (s ^ 1)) & 1, ctl)) pend_full &= ~(1u << (s ^ 1));
+            if (tid == 0 && !aborted(ctl)) {
+                issue_x(c + 1);
+                pend_x = true;
+            }
         }
-        CMARK(21);
         // O = Qs S + P U  (lanes 0..63 = tokens)
-        wait_local(bar_o, ph_o, ctl);
-        ph_o ^= 1;
+        if (wait_local(bar_o, ph_o, ctl)) {
+            ph_o ^= 1;
+            pend_o = false;
+        }
         tc_fence_after();
-        CMARK(22);
         if (quad < 2) {
             float o[64];
             const uint32_t ta = tc::tmem_addr(tmem, 32 * quad, xcol + half * 64);
@@ -654,23 +946,31 @@ __device__ void consumer(uint8_t *sm, uint32_t tmem, const uint8_t *ring, const 
         tc_fence_before();
         __syncthreads();
         if (tid == 0) pull(c + 2, false);  // the slot of chunk c is free
-        CMARK(23);
+    }
+    // drain: what this CTA issued and has not seen complete (all of it after a give-up)
+    if (tid == 0) {
+#pragma unroll
+        for (int sl = 0; sl < 2; ++sl)
+            if ((pend_full >> sl) & 1) drain(full + sl, (ph_full >> sl) & 1, ctl);
+        if (pend_x) drain(bar_x, ph_x, ctl);
+        if (pend_s) drain(bar_s, ph_s, ctl);
+        if (pend_o) drain(bar_o, ph_o, ctl);
     }
     if (S_T) {
 #pragma unroll
         for (int j = 0; j < 64; ++j) S_T[(bh * kD + row) * kD + half * 64 + j] = S[j];
     }
-    CMARK_FLUSH(16, 24);
 }
 
+template <bool kFused>
 __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 1)
 chunk_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_la, const __grid_constant__ CUtensorMap tm_v,
-                     const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
-                     const __nv_bfloat16 *__restrict__ v, const float *__restrict__ log_alpha,
-                     const float *__restrict__ beta, const float *__restrict__ S0,
-                     __nv_bfloat16 *__restrict__ out, float *__restrict__ S_T, uint8_t *__restrict__ ws,
-                     int T, int H, int *err) {
+                     const __grid_constant__ CUtensorMap tm_qs, const __grid_constant__ CUtensorMap tm_ks,
+                     const __grid_constant__ CUtensorMap tm_las, const float *__restrict__ beta,
+                     const float *__restrict__ S0, __nv_bfloat16 *__restrict__ out,
+                     float *__restrict__ S_T, uint8_t *__restrict__ ws, int T, int H, int *err,
+                     int test_timeout) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~static_cast<uintptr_t>(1023));
@@ -700,14 +1000,17 @@ chunk_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     tc_fence_after();
     tc::cluster_sync();  // every barrier of the cluster is initialised before any remote use
     const uint32_t tmem = *tmem_slot;
-    const Ctl ctl{abort, err};
+    Ctl ctl{abort, err, {0, 0, 0, 0}, test_timeout ? kTestWaitLimit : kWaitLimit};
+#pragma unroll
+    for (int r = 0; r < kCluster; ++r)   // every CTA's abort flag (a producer's or the consumer's offset)
+        ctl.peer_abort[r] = tc::map_to_rank(tc::smem_u32(sm) + (r == kCluster - 1 ? C_BAR : P_BAR) + 132, r);
 
     uint8_t *ring = ws + bh * kRingSlots * kSlotStride;  // this head's ring: kRingDepth slots per producer
     if (is_consumer)
         consumer(sm, tmem, ring, S0, out, S_T, T, H, h, bh, ztok, nchunks, ctl);
     else
-        producer(sm, tmem, rank, ring, &tm_q, &tm_k, &tm_la, &tm_v, q, k, v, log_alpha, beta, T, H, h,
-                 ztok, nchunks, ctl);
+        producer<kFused>(sm, tmem, rank, ring, &tm_q, &tm_k, &tm_la, &tm_v, &tm_qs, &tm_ks, &tm_las, beta, T,
+                 H, h, ztok, nchunks, ctl, test_timeout);
 
     tc_fence_before();
     __syncthreads();
@@ -736,33 +1039,30 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// 3-D map over a [B*T, H, 128] tensor with a (128, 1, 64) box, used for L2 prefetches.
-bool make_map(CUtensorMap *m, const void *ptr, CUtensorMapDataType dt, int esize, int H, long tokens) {
+// 3-D map over a [B*T, H, 128] tensor with a (box_x, 1, 64) box. box_x = 128 without
+// swizzle (plain 256/512-byte rows: v loads and L2 prefetches), or 128 bytes' worth of
+// channels with the 128-byte swizzle (q, k, log alpha for the prologue).
+bool make_map(CUtensorMap *m, const void *ptr, CUtensorMapDataType dt, int esize, int H, long tokens,
+              bool swizzled) {
     EncodeTiledFn enc = encode_fn();
     if (!enc) return false;
     const cuuint64_t dims[3] = {static_cast<cuuint64_t>(kD), static_cast<cuuint64_t>(H),
                                 static_cast<cuuint64_t>(tokens)};
     const cuuint64_t strides[2] = {static_cast<cuuint64_t>(kD) * esize,
                                    static_cast<cuuint64_t>(kD) * esize * H};
-    const cuuint32_t box[3] = {static_cast<cuuint32_t>(kD), 1, kC};
+    const cuuint32_t box[3] = {swizzled ? static_cast<cuuint32_t>(128 / esize) : static_cast<cuuint32_t>(kD),
+                               1, kC};
     const cuuint32_t estr[3] = {1, 1, 1};
     return enc(m, dt, 3, const_cast<void *>(ptr), dims, strides, box, estr,
-               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+               CU_TENSOR_MAP_INTERLEAVE_NONE,
+               swizzled ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 }  // namespace
 
-#ifdef KDA_PHASE_TIMING
-extern "C" int kda_debug_cluster_cycles(unsigned long long *out32, int reset) {
-    cudaError_t e = cudaMemcpyFromSymbol(out32, g_cluster_cycles, sizeof(unsigned long long) * 32);
-    if (reset) {
-        unsigned long long z[32] = {0};
-        cudaMemcpyToSymbol(g_cluster_cycles, z, sizeof z);
-    }
-    return e == cudaSuccess ? 0 : -1;
-}
-#endif
+// Test hook (kda_test_inject_wait_timeout): small wait limits and one withheld "ready".
+int g_test_timeout = 0;
 
 bool chunk_cluster_supported(int dk, int dv, int chunk, int dtype) {
     return dtype == KDA_BF16 && dk == kD && dv == kD && chunk == kC;
@@ -774,23 +1074,33 @@ size_t chunk_cluster_workspace_bytes(int B, int H) {
 
 cudaError_t launch_chunk_cluster(const ChunkArgs &a, cudaStream_t s) {
     const long tokens = static_cast<long>(a.B) * a.T;
-    CUtensorMap mq, mk, mla, mv;
-    if (!make_map(&mq, a.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.H, tokens) ||
-        !make_map(&mk, a.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.H, tokens) ||
-        !make_map(&mla, a.log_alpha, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, a.H, tokens) ||
-        !make_map(&mv, a.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.H, tokens))
-        return cudaErrorInvalidValue;
-    cudaError_t e = cudaFuncSetAttribute(chunk_cluster_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+    const CUtensorMapDataType kB16 = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, kF32 = CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+    const bool fused = a.gate != nullptr;   // the layer prologue: gate pre-activation instead of log alpha
+    CUtensorMap mq, mk, mla, mv, mqs, mks, mlas;
+    const bool ok =
+        make_map(&mq, a.q, kB16, 2, a.H, tokens, false) && make_map(&mk, a.k, kB16, 2, a.H, tokens, false) &&
+        make_map(&mv, a.v, kB16, 2, a.H, tokens, false) &&
+        make_map(&mqs, a.q, kB16, 2, a.H, tokens, true) && make_map(&mks, a.k, kB16, 2, a.H, tokens, true) &&
+        (fused ? make_map(&mla, a.gate, kB16, 2, a.H, tokens, false) &&
+                     make_map(&mlas, a.gate, kB16, 2, a.H, tokens, true)
+               : make_map(&mla, a.log_alpha, kF32, 4, a.H, tokens, false) &&
+                     make_map(&mlas, a.log_alpha, kF32, 4, a.H, tokens, true));
+    if (!ok) return cudaErrorInvalidValue;
+    auto kern = fused ? chunk_cluster_kernel<true> : chunk_cluster_kernel<false>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(kSmemBytes));
     if (e != cudaSuccess) return e;
     const dim3 grid(static_cast<unsigned>(a.B) * a.H * kCluster);
-    chunk_cluster_kernel<<<grid, kThreads, kSmemBytes, s>>>(
-        mq, mk, mla, mv, static_cast<const __nv_bfloat16 *>(a.q),
-        static_cast<const __nv_bfloat16 *>(a.k), static_cast<const __nv_bfloat16 *>(a.v),
-        a.log_alpha, a.beta, a.S0, static_cast<__nv_bfloat16 *>(a.out), a.S_T,
-        static_cast<uint8_t *>(a.workspace), a.T, a.H, a.device_error);
+    kern<<<grid, kThreads, kSmemBytes, s>>>(
+        mq, mk, mla, mv, mqs, mks, mlas, a.beta, a.S0, static_cast<__nv_bfloat16 *>(a.out), a.S_T,
+        static_cast<uint8_t *>(a.workspace), a.T, a.H, a.device_error, g_test_timeout);
     return cudaGetLastError();
+}
+
+int set_test_timeout(int on) {
+    const int old = g_test_timeout;
+    g_test_timeout = on ? 1 : 0;
+    return old;
 }
 
 }  // namespace kda

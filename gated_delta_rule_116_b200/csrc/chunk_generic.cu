@@ -6,20 +6,19 @@
 // Chunked form (Kimi Linear summary, es.news.hada.io/topic?id=31936, section
 // "Algoritmo paralelo por chunks"). For one chunk of C tokens starting from
 // state S (d_k x d_v), with g_t the in-chunk inclusive prefix sum of log alpha
-// (per channel) and an anchor g_a = g_C / 2:
-//   q~ = q * e^{g - g_a},  k~ = k * e^{g - g_a},  k^ = k * e^{g_a - g}
-//   A  = Diag(beta) * strict_lower(K~ K^^T)           (k.k^T product)
-//   P  = lower(Q~ K^^T)                               (q.k^T product)
+// (per channel):
+//   A  = Diag(beta) * strict_lower(a_ij),  a_ij = sum_c k_ic k_jc e^{g_ic - g_jc}
+//   P  = lower(p_ij),                      p_ij = sum_c q_ic k_jc e^{g_ic - g_jc}
 //   T  = (I + A)^{-1} Diag(beta)                      (forward substitution)
-//   W  = T (K~ * e^{g_a}),  U' = T V                  (WY / UT form)
+//   W  = T Ks,  U' = T V                              (WY / UT form, Ks = K e^{g})
 //   U  = U' - W S
-//   O  = (Q~ * e^{g_a}) S + P U
-//   S <- Diag(e^{g_C}) S + (K^ * e^{g_C - g_a})^T U
-// In exact arithmetic this equals the token-by-token recurrence; the entries
-// of A and P carry e^{g_i - g_j} <= 1, split into two factors that stay
-// within e^{|g_C|/2} thanks to the midpoint anchor (section "Menor cantidad
-// de operaciones que DPLR general" names the precision problem of
-// fine-grained decay inside a chunk).
+//   O  = Qs S + P U                                   (Qs = Q e^{g})
+//   S <- Diag(e^{g_C}) S + Kb^T U                     (Kb = K e^{g_C - g})
+// In exact arithmetic this equals the token-by-token recurrence. The entries
+// of A and P take e^{g_i - g_j} <= 1 per term, evaluated directly for every
+// pair j <= i: no factor is split, so no decay, however fine-grained (section
+// "Menor cantidad de operaciones que DPLR general"), leaves the fp32 range.
+// Every other factor (e^{g}, e^{g_C - g}, e^{g_C}) is <= 1 as well.
 //
 // Mapping: one CTA of 256 threads per (b, h, slice of NV <= 32 value
 // columns). State columns evolve independently, so slices never communicate;
@@ -37,7 +36,7 @@ struct Smem {
     __host__ __device__ Smem(int C_, int dk_, int NV_)
         : C(C_), dk(dk_), NV(NV_), LD(dk_ + 1), LC(C_ + 1) {}
     __host__ __device__ size_t floats() const {
-        return 4ull * C * LD + 3ull * C * LC + 2ull * C * NV + 1ull * dk * NV + 5ull * dk + C;
+        return 4ull * C * LD + 3ull * C * LC + 2ull * C * NV + 1ull * dk * NV + 2ull * dk + C;
     }
 };
 
@@ -51,9 +50,9 @@ chunk_generic_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
     extern __shared__ float sm[];
     const Smem L(C, dk, NV);
     const int LD = L.LD, LC = L.LC;
-    float *Qt = sm;                 // [C][LD]  q~, then q~ * e^{g_a}
-    float *Kt = Qt + C * LD;        // [C][LD]  k~, then k~ * e^{g_a}
-    float *Kh = Kt + C * LD;        // [C][LD]  k^, then k^ * e^{g_C - g_a}
+    float *Qt = sm;                 // [C][LD]  q, then Qs = q e^{g}
+    float *Kt = Qt + C * LD;        // [C][LD]  k, then Ks = k e^{g}
+    float *Kh = Kt + C * LD;        // [C][LD]  Kb = k e^{g_C - g}
     float *G = Kh + C * LD;         // [C][LD]  prefix sums g, then W
     float *A = G + C * LD;          // [C][LC]
     float *Tm = A + C * LC;         // [C][LC]
@@ -61,13 +60,9 @@ chunk_generic_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
     float *V = P + C * LC;          // [C][NV]
     float *U = V + C * NV;          // [C][NV]
     float *S = U + C * NV;          // [dk][NV]
-    float *ga = S + dk * NV;        // [dk] anchor g_C / 2
-    float *e_a = ga + dk;           // [dk] e^{g_a}
-    float *e_ca = e_a + dk;         // [dk] e^{g_C - g_a}
-    float *e_c = e_ca + dk;         // [dk] e^{g_C}
+    float *e_c = S + dk * NV;       // [dk] e^{g_C}
     float *gsum = e_c + dk;         // [dk] g_C
     float *bt = gsum + dk;          // [C]  beta of the chunk
-
     const int tid = threadIdx.x;
     const int bh = blockIdx.x;
     const int b = bh / H, h = bh - (bh / H) * H;
@@ -110,7 +105,7 @@ chunk_generic_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
         for (int t = tid; t < C; t += kThreads)
             bt[t] = t < valid ? beta[(static_cast<long>(b) * T + t0 + t) * H + h] : 0.f;
         __syncthreads();
-        // 2. in-chunk prefix sum of log alpha per channel; anchor at g_C / 2
+        // 2. in-chunk prefix sum of log alpha per channel
         for (int c = tid; c < dk; c += kThreads) {
             float acc = 0.f;
             for (int t = 0; t < C; ++t) {
@@ -118,37 +113,36 @@ chunk_generic_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
                 G[t * LD + c] = acc;
             }
             gsum[c] = acc;
-            ga[c] = 0.5f * acc;
-            e_a[c] = expf(0.5f * acc);
-            e_ca[c] = expf(acc - 0.5f * acc);
             e_c[c] = expf(acc);
         }
         __syncthreads();
-        // 3. anchored gate factors
-        for (int e = tid; e < C * dk; e += kThreads) {
-            const int t = e / dk, c = e - t * dk;
-            const float d = G[t * LD + c] - ga[c];
-            const float up = expf(d), down = expf(-d);
-            const float kv = Kt[t * LD + c];
-            Qt[t * LD + c] *= up;
-            Kt[t * LD + c] = kv * up;
-            Kh[t * LD + c] = kv * down;
-        }
-        __syncthreads();
-        // 4. A = Diag(beta) strict_lower(K~ K^^T), P = lower(Q~ K^^T)
+        // 3. A = Diag(beta) strict_lower(a), P = lower(p), every term with its own e^{g_i - g_j}
         for (int e = tid; e < C * C; e += kThreads) {
             const int i = e / C, j = e - i * C;
             float a = 0.f, p = 0.f;
             if (j <= i) {
-                const float *qi = Qt + i * LD, *ki = Kt + i * LD, *kj = Kh + j * LD;
+                const float *qi = Qt + i * LD, *ki = Kt + i * LD, *kj = Kt + j * LD;
+                const float *gi = G + i * LD, *gj = G + j * LD;
                 for (int c = 0; c < dk; ++c) {
-                    p = fmaf(qi[c], kj[c], p);
-                    a = fmaf(ki[c], kj[c], a);
+                    const float kd = kj[c] * expf(gi[c] - gj[c]);
+                    p = fmaf(qi[c], kd, p);
+                    a = fmaf(ki[c], kd, a);
                 }
                 a = j < i ? a * bt[i] : 0.f;
             }
             A[i * LC + j] = a;
             P[i * LC + j] = p;
+        }
+        __syncthreads();
+        // 4. Qs = q e^{g}, Ks = k e^{g}, Kb = k e^{g_C - g}
+        for (int e = tid; e < C * dk; e += kThreads) {
+            const int t = e / dk, c = e - t * dk;
+            const float gv = G[t * LD + c];
+            const float up = expf(gv), down = expf(gsum[c] - gv);
+            const float kv = Kt[t * LD + c];
+            Qt[t * LD + c] *= up;
+            Kt[t * LD + c] = kv * up;
+            Kh[t * LD + c] = kv * down;
         }
         __syncthreads();
         // 5. T = (I + A)^{-1} Diag(beta), one column per thread, forward substitution
@@ -161,15 +155,8 @@ chunk_generic_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
                 Tm[i * LC + j] = -s;
             }
         }
-        // 6. re-anchor: K~ e^{g_a}, Q~ e^{g_a} (chunk-start scale), K^ e^{g_C - g_a}
-        for (int e = tid; e < C * dk; e += kThreads) {
-            const int t = e / dk, c = e - t * dk;
-            Qt[t * LD + c] *= e_a[c];
-            Kt[t * LD + c] *= e_a[c];
-            Kh[t * LD + c] *= e_ca[c];
-        }
         __syncthreads();
-        // 7. W = T K_start (into G), U' = T V
+        // 6. W = T Ks (into G), U' = T V
         for (int e = tid; e < C * dk; e += kThreads) {
             const int i = e / dk, c = e - i * dk;
             float w = 0.f;
@@ -183,7 +170,7 @@ chunk_generic_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
             U[e] = u;
         }
         __syncthreads();
-        // 8. U = U' - W S
+        // 7. U = U' - W S
         for (int e = tid; e < C * NV; e += kThreads) {
             const int i = e / NV, n = e - i * NV;
             float u = U[e];
@@ -191,7 +178,7 @@ chunk_generic_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
             U[e] = u;
         }
         __syncthreads();
-        // 9. O = Q_start S + P U
+        // 8. O = Qs S + P U
         for (int e = tid; e < C * NV; e += kThreads) {
             const int i = e / NV, n = e - i * NV;
             if (i < valid && n < nv) {
@@ -202,7 +189,7 @@ chunk_generic_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
             }
         }
         __syncthreads();
-        // 10. S = Diag(e^{g_C}) S + K_bar^T U
+        // 9. S = Diag(e^{g_C}) S + Kb^T U
         for (int e = tid; e < dk * NV; e += kThreads) {
             const int c = e / NV, n = e - c * NV;
             float s = S[e] * e_c[c];

@@ -56,7 +56,7 @@ __device__ void varlen_body(float *sm, const Tin *q, const Tin *k, const Tin *v,
             const int i = e / NV, j = e - i * NV;
             if (i >= valid || j >= nv) continue;
             float acc = 0.f;
-            for (int c = 0; c < dk; ++c) acc = fmaf(s.Qt[i * LD + c] * s.e_a[c], s.S[c * NV + j], acc);
+            for (int c = 0; c < dk; ++c) acc = fmaf(s.Qs[i * LD + c], s.S[c * NV + j], acc);
             for (int m = 0; m <= i; ++m) acc = fmaf(s.P[i * LC + m], s.U[m * NV + j], acc);
             out[(static_cast<long>(t0 + i) * H + h) * dv + n0 + j] = from_f32<Tin>(acc);
         }
@@ -64,8 +64,7 @@ __device__ void varlen_body(float *sm, const Tin *q, const Tin *k, const Tin *v,
         for (int e = tid; e < dk * NV; e += kThreads) {   // S <- Diag(gamma) S + Kb^T U
             const int c = e / NV, j = e - c * NV;
             float acc = s.gam[c] * s.S[e];
-            const float eca = s.e_ca[c];
-            for (int t = 0; t < kC; ++t) acc = fmaf(s.Kh[t * LD + c] * eca, s.U[t * NV + j], acc);
+            for (int t = 0; t < kC; ++t) acc = fmaf(s.Kh[t * LD + c], s.U[t * NV + j], acc);
             s.S[e] = acc;
         }
     }

@@ -30,6 +30,7 @@ struct ChunkArgs {
     void *workspace;
     size_t workspace_bytes;
     int *device_error;  // set to a nonzero code by a kernel whose bounded wait gave up
+    const void *gate = nullptr;  // fused layer prologue: gate pre-activation (log_alpha unused)
 };
 
 struct DecodeArgs {
@@ -44,7 +45,6 @@ struct DecodeArgs {
 // Launchers return cudaSuccess or the launch error. They do no argument checks.
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t s);
 cudaError_t launch_chunk_generic(const ChunkArgs &a, cudaStream_t s);
-cudaError_t launch_chunk_tc(const ChunkArgs &a, cudaStream_t s);
 cudaError_t launch_chunk_cluster(const ChunkArgs &a, cudaStream_t s);
 
 // Records `fmt` as the calling thread's kda_last_error_detail() and returns code.
@@ -52,9 +52,9 @@ int set_error_detail(int code, const char *fmt, ...);
 // Device address of the word kernels set when a bounded wait gives up (nullptr on error).
 int *device_error_word();
 
-bool chunk_tc_supported(int dk, int dv, int chunk, int dtype);
 bool chunk_cluster_supported(int dk, int dv, int chunk, int dtype);
-size_t chunk_tc_workspace_bytes(int B, int T, int H);
+// Test hook of the cluster engine's give-up path (kda_test_inject_wait_timeout); returns the old value.
+int set_test_timeout(int on);
 size_t chunk_cluster_workspace_bytes(int B, int H);
 // Backward pass (chunk_bwd.cu).
 size_t chunk_bwd_workspace_bytes(int B, int T, int H, int dk, int dv);

@@ -24,11 +24,10 @@
  *    Argument errors are detected on the host before anything is enqueued;
  *    kda_last_error_detail() names the offending argument.
  *  - Preconditions that are documented but not checked (checking would cost a
- *    pass over the data): log_alpha <= 0, beta in [0,1], finite inputs, and
- *    within any chunk the per-channel total decay |sum log_alpha| <= 160
- *    (the gate factors of the chunked form are anchored at the chunk's
- *    midpoint and must stay inside the fp32/bf16 exponent range). L2
- *    normalisation of q and k is the caller's job.
+ *    pass over the data): log_alpha <= 0, beta in [0,1], finite inputs. Any
+ *    decay is supported: no gate factor of the chunked form leaves the
+ *    floating-point range, whatever log_alpha is (16-token sub-chunks, see
+ *    kda_chunk_fwd). L2 normalisation of q and k is the caller's job.
  */
 #ifndef KDA_H
 #define KDA_H
@@ -53,12 +52,10 @@ typedef enum {
 /* Element type of q, k, v and out. Gates, beta and states are always fp32. */
 typedef enum { KDA_BF16 = 0, KDA_F32 = 1 } kda_dtype;
 
-/* Which prefill engine kda_chunk_fwd_engine runs. */
+/* Which prefill engine kda_chunk_fwd_engine runs (the value 2 is not used). */
 typedef enum {
     KDA_ENGINE_AUTO = 0,     /* cluster tensor-core engine where supported, else the generic one */
     KDA_ENGINE_GENERIC = 1,  /* fp32 CUDA-core chunked engine: any d_k, d_v <= 128, chunk 16/32/64 */
-    KDA_ENGINE_TC = 2,       /* tcgen05/TMEM engine, one CTA per (b, h, 32 value columns):
-                                bf16, d_k = d_v = 128, chunk = 64 */
     KDA_ENGINE_TC_CLUSTER = 3 /* tcgen05/TMEM engine, one 4-CTA cluster per (b, h): three
                                 CTAs build chunk operands, one runs the state chain;
                                 bf16, d_k = d_v = 128, chunk = 64 */
@@ -96,6 +93,16 @@ size_t kda_workspace_bytes(int B, int T, int H, int dk, int dv, int chunk, int d
  * T = 0 copies S0 (or zeros) to S_T. B = 0 or H = 0 is a no-op.
  * Supported: dk, dv in [1,128] with dv % 4 == 0 (generic engine); the
  * tensor-core engine additionally needs bf16, dk = dv = 128, chunk = 64.
+ * Gate range: any log_alpha <= 0. The intra-chunk products carry the decay
+ * e^{g_i - g_j} between tokens of a chunk (section "Menor cantidad de
+ * operaciones que DPLR general" names the precision problem of fine-grained
+ * decay there). The generic engine evaluates every such factor directly. The
+ * tensor-core engine splits the chunk into 16-token sub-chunks: blocks between
+ * two sub-chunks use factors anchored at the sub-chunk boundary (both <= 1);
+ * a diagonal block anchors at its 8th token, and a channel that decays by more
+ * than e^-87 inside one sub-chunk takes its diagonal-block factors from
+ * log_alpha clamped at -10 per token there (every factor this changes is below
+ * e^-10 either way: a change smaller than the tf32 rounding of the factor).
  * Limits: B*T <= 2^31 - 1 tokens and B*H <= 2^29 - 1 heads; larger problems
  * return KDA_ERR_UNSUPPORTED (split the batch).
  */
@@ -104,6 +111,29 @@ int kda_chunk_fwd(const void *q, const void *k, const void *v,
                   void *out, float *S_T,
                   int B, int T, int H, int dk, int dv, int chunk, int dtype,
                   void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * Chunked prefill with the layer's prologue fused into it (Kimi Linear summary,
+ * section "Configuracion del modelo Kimi Linear": q and k are L2-normalised,
+ * and the per-channel decay comes from a data-dependent gate like GDN's and
+ * Mamba's). Computes exactly what kda_chunk_fwd computes on
+ *     q / ||q||, k / ||k|| (over the head dimension, per token; a zero row
+ *     stays zero) and log_alpha = -softplus(gate) = -log(1 + e^gate),
+ * without those tensors ever being written: the prefill reads raw q, k and
+ * the gate's pre-activation (bf16, 2 bytes per channel instead of 4 for
+ * log_alpha).
+ *   q, k       [B,T,H,dk]  bf16         un-normalised queries and keys
+ *   v          [B,T,H,dv]  bf16
+ *   gate       [B,T,H,dk]  bf16         the gate's pre-activation x
+ *   beta, S0, out, S_T, workspace, stream: as kda_chunk_fwd
+ * Supported: dtype KDA_BF16, dk = dv = 128, chunk = 64 (the tensor-core
+ * engine); anything else returns KDA_ERR_UNSUPPORTED. Limits and T = 0 as
+ * kda_chunk_fwd. The workspace is kda_workspace_bytes(...) bytes.
+ */
+int kda_chunk_fwd_fused(const void *q, const void *k, const void *v, const void *gate,
+                        const float *beta, const float *S0, void *out, float *S_T,
+                        int B, int T, int H, int dk, int dv, int chunk, int dtype,
+                        void *workspace, size_t workspace_bytes, void *stream);
 
 /*
  * 1 if `engine` (kda_engine) can run a prefill of this shape and dtype, else 0.
@@ -249,6 +279,20 @@ const char *kda_last_error_detail(void);
  * clearing the flag; KDA_ERR_CUDA if synchronisation failed; else KDA_OK.
  */
 int kda_device_status(void *stream);
+
+/*
+ * Test hook for the give-up path of the bounded device-side waits of the
+ * tensor-core prefill engine; no counterpart in the pages. Not for production
+ * use and not thread-safe: a process-wide setting read at every launch. With
+ * on != 0, later launches of that engine use a short wait limit and its first
+ * producer CTA withholds the signal that its first chunk's operands are ready,
+ * so the state-chain CTA's wait runs out. The launch then gives up without a
+ * fault or a trap: every CTA stops issuing copies and MMAs, waits for those in
+ * flight, and exits; kda_device_status reports KDA_ERR_DEVICE_TIMEOUT and the
+ * outputs of that launch are undefined. on = 0 restores normal launches.
+ * Returns the previous setting.
+ */
+int kda_test_inject_wait_timeout(int on);
 
 /* ABI version of this header: major * 10000 + minor * 100 + patch. */
 int kda_version(void);

@@ -16,6 +16,14 @@ Workloads (one dict per entry of ``WORKLOADS``):
 * ``prefill_128k`` B=1,  H=16, T=131072, d=128, chunk=64, bf16 q/k/v, half the
                    channels with log a = -1e-3, the other half -softplus(N(0,1))
 
+Edge-case gate recipe ``strong`` (parity tests only): channel c gets, for every
+token, log a = -4 if c % 8 == 0 (a chunk of 64 tokens decays by e^-256),
+0 if c % 8 == 1 (no forgetting), -12 if c % 8 == 2 (a ~ 6e-6: the channel keeps
+almost nothing from one token to the next), -1e-3 if c % 8 == 3, and
+-softplus(N(0,1)) otherwise. It stresses the range of the gate factors of the
+chunked form (the fine-grained decay that the Kimi Linear summary names as the
+precision problem inside a chunk).
+
 Recipe (all workloads): q, k ~ N(0,1), L2-normalised over the head dimension
 per (batch, token, head) in fp32 and then cast to the workload's dtype; v ~
 N(0,1); beta = sigmoid(N(0,1)); log a = -softplus(N(0,1)) per channel unless
@@ -42,7 +50,7 @@ class Prefill:
     dv: int
     chunk: int
     dtype: torch.dtype          # dtype of q, k, v and out
-    gate: str = "softplus01"    # softplus01 | slow | mixed
+    gate: str = "softplus01"    # softplus01 | slow | mixed | strong
     s0_std: float = 0.0         # 0 -> no initial state (S0 = None)
     seed: int = 0
 
@@ -97,6 +105,13 @@ def _gates(logits: torch.Tensor, mode: str) -> torch.Tensor:
         out = -torch.nn.functional.softplus(logits)
         out[..., : out.shape[-1] // 2] = -1e-3
         return out
+    if mode == "strong":                                 # per channel c % 8: -4, 0, -12, -1e-3
+        out = -torch.nn.functional.softplus(logits)
+        out[..., 0::8] = -4.0
+        out[..., 1::8] = 0.0
+        out[..., 2::8] = -12.0
+        out[..., 3::8] = -1e-3
+        return out
     raise ValueError(f"unknown gate recipe {mode!r}")
 
 
@@ -125,6 +140,51 @@ def prefill_inputs(w: Prefill | str, device="cpu", **override) -> dict:
         S0 = torch.randn(B, H, dk, dv, **f32) * w.s0_std
     return dict(q=q.contiguous(), k=k.contiguous(), v=v.contiguous(),
                 log_alpha=log_alpha.contiguous(), beta=beta.contiguous(), S0=S0, w=w)
+
+
+# Gate pre-activations x with -softplus(x) equal to the fixed log a values of the gate
+# recipes (log(e^{-log a} - 1)); "no forgetting" (log a = 0) has no finite x and takes
+# x = -30 (log a = -9e-14).
+_X_FOR_LOG_A = {-1e-3: -6.907255, -4.0: 3.9814331, -12.0: 11.999994, 0.0: -30.0}
+
+
+def prefill_layer_inputs(w: Prefill | str, device="cpu", **override) -> dict:
+    """Inputs of the fused layer prologue: raw (un-normalised) q and k, v, the gate's
+    pre-activation x, beta and S0, all in the workload's dtype except beta and S0 (fp32).
+
+    The same draws as ``prefill_inputs`` (same generator and order), with q and k
+    left un-normalised and the gate logits turned into the x for which -softplus(x)
+    is the workload's log a: x = logits (softplus01), logits - 2 (slow), or the
+    fixed values above for the recipe's fixed channels.
+    """
+    if isinstance(w, str):
+        w = WORKLOADS[w]
+    if override:
+        w = dataclasses.replace(w, **override)
+    g = _gen(w.seed, device)
+    B, T, H, dk, dv = w.B, w.T, w.H, w.dk, w.dv
+    f32 = dict(device=device, dtype=torch.float32, generator=g)
+    q = torch.randn(B, T, H, dk, **f32).to(w.dtype)
+    k = torch.randn(B, T, H, dk, **f32).to(w.dtype)
+    v = torch.randn(B, T, H, dv, **f32).to(w.dtype)
+    beta = torch.sigmoid(torch.randn(B, T, H, **f32))
+    x = torch.randn(B, T, H, dk, **f32)
+    if w.gate == "slow":
+        x = x - 2.0
+    elif w.gate == "mixed":
+        x[..., : dk // 2] = _X_FOR_LOG_A[-1e-3]
+    elif w.gate == "strong":
+        x[..., 0::8] = _X_FOR_LOG_A[-4.0]
+        x[..., 1::8] = _X_FOR_LOG_A[0.0]
+        x[..., 2::8] = _X_FOR_LOG_A[-12.0]
+        x[..., 3::8] = _X_FOR_LOG_A[-1e-3]
+    elif w.gate != "softplus01":
+        raise ValueError(f"unknown gate recipe {w.gate!r}")
+    S0 = None
+    if w.s0_std > 0:
+        S0 = torch.randn(B, H, dk, dv, **f32) * w.s0_std
+    return dict(q=q.contiguous(), k=k.contiguous(), v=v.contiguous(), gate=x.to(w.dtype).contiguous(),
+                beta=beta.contiguous(), S0=S0, w=w)
 
 
 def decode_state(w: Decode | str = "decode_256", device="cpu", **override) -> torch.Tensor:

@@ -92,7 +92,7 @@ def test_chunk_misaligned_pointer(lib, field):
     (dict(dtype=5), -1), (dict(B=-1), -1), (dict(T=-3), -1), (dict(dk=0), -1),
     (dict(dk=256), -2), (dict(dv=130), -2), (dict(dv=6), -2), (dict(C=48), -2),
     (dict(C=128), -2), (dict(engine=9), -1), (dict(engine=3, C=16), -2), (dict(engine=3, dtype=1), -2),
-    (dict(engine=2, dtype=1), -2), (dict(engine=2, dk=64), -2), (dict(engine=2, C=32), -2),
+    (dict(engine=2), -1), (dict(engine=3, dk=64), -2), (dict(engine=3, C=32), -2),
     (dict(B=2, T=2**30), -2), (dict(B=2**15, H=2**15), -2), (dict(engine=1, B=3, T=2**30), -2),
 ])
 def test_chunk_rejects(lib, kw, code):

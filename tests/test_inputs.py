@@ -94,3 +94,32 @@ def test_decode_state_and_steps():
     assert s0["q"].shape == (16, 4, 128) and s0["beta"].shape == (16, 4)
     assert torch.equal(s0["k"], s0b["k"]) and not torch.equal(s0["k"], s1["k"])
     assert torch.all(s0["log_alpha"] <= 0)
+
+
+def test_strong_gate_recipe():
+    """The edge-case recipe: fixed log a on channel classes c % 8 = 0..3, softplus elsewhere."""
+    x = I.prefill_inputs("prefill_4k", B=1, T=256, H=2, gate="strong")
+    la = x["log_alpha"]
+    assert torch.all(la[..., 0::8] == -4.0) and torch.all(la[..., 1::8] == 0.0)
+    assert torch.all(la[..., 2::8] == -12.0) and torch.all(la[..., 3::8] == np.float32(-1e-3))
+    rest = torch.cat([la[..., c::8] for c in range(4, 8)], dim=-1)
+    assert torch.all(rest < 0)
+    assert abs(rest.mean().item() + normal_expectation(softplus)) < 2e-2
+    # a 64-token chunk on a c % 8 == 0 channel decays by e^-256: beyond a chunk-midpoint anchor
+    assert float(la[0, :64, 0, 0].sum()) == -256.0
+
+
+def test_layer_inputs_recipe():
+    """Raw q/k (not unit rows) and gate pre-activations whose -softplus gives the recipe's log a."""
+    x = I.prefill_layer_inputs("prefill_128k", T=64, H=2)
+    assert x["q"].dtype == torch.bfloat16 and x["gate"].dtype == torch.bfloat16
+    assert not torch.allclose(x["q"].float().norm(dim=-1), torch.ones(1, 64, 2), atol=0.1)
+    la = -torch.nn.functional.softplus(x["gate"].double())
+    np.testing.assert_allclose(la[..., :64].numpy(), -1e-3, rtol=5e-3)   # bf16 of the fixed x
+    s = I.prefill_layer_inputs("prefill_4k", B=1, T=32, H=1, gate="strong")
+    las = -torch.nn.functional.softplus(s["gate"].double())
+    np.testing.assert_allclose(las[..., 0::8].numpy(), -4.0, rtol=2e-2)
+    assert float(las[..., 1::8].abs().max()) < 1e-12
+    np.testing.assert_allclose(las[..., 2::8].numpy(), -12.0, rtol=2e-2)
+    sl = I.prefill_layer_inputs("prefill_32k", T=2048, H=4)
+    assert abs(sl["gate"].float().mean().item() + 2.0) < 0.02     # x ~ N(-2, 1): the slow recipe

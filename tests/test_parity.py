@@ -21,7 +21,7 @@ DEV = "cuda"
 
 
 def engines(dtype, dk, dv, chunk):
-    return [e for e in ("generic", "tc", "tc_cluster") if kda.engine_supported(e, dk, dv, chunk, dtype)]
+    return [e for e in ("generic", "tc_cluster") if kda.engine_supported(e, dk, dv, chunk, dtype)]
 
 
 def run_gpu(inp, chunk, engine="auto", with_state=True):
@@ -135,6 +135,46 @@ def test_bf16_initial_state_in_place():
         compare(inp, out, st, ref_out, ref_st)
 
 
+# --- strong decay (the fine-grained decay inside a chunk that the pages single out) --------
+
+@pytest.mark.parametrize("B,T,H", [(2, 300, 3), (1, 64, 2), (1, 1000, 4)])
+def test_bf16_strong_decay_all_engines(B, T, H):
+    """Channels with log a = -4 (a chunk decays by e^-256), 0, -12 and -1e-3 next to
+    softplus gates, with an initial state: beyond any chunk-wide anchor's range."""
+    inp = I.prefill_inputs("prefill_4k", B=B, T=T, H=H, gate="strong", s0_std=0.05)
+    ref = run_oracle(inp)
+    for eng in engines(torch.bfloat16, 128, 128, 64):
+        out, st = run_gpu(inp, 64, eng)
+        compare(inp, out, st, *ref)
+
+
+@pytest.mark.parametrize("chunk", [16, 32, 64])
+def test_bf16_strong_decay_chunk_sizes(chunk):
+    inp = I.prefill_inputs("prefill_4k", B=1, T=200, H=2, gate="strong", s0_std=0.05)
+    ref = run_oracle(inp)
+    for eng in engines(torch.bfloat16, 128, 128, chunk):
+        out, st = run_gpu(inp, chunk, eng)
+        compare(inp, out, st, *ref)
+
+
+@pytest.mark.parametrize("chunk", [16, 32, 64])
+def test_fp32_strong_decay(chunk):
+    inp = I.prefill_inputs("fp32_small", gate="strong", s0_std=0.5, T=100)
+    ref = run_oracle(inp)
+    out, st = run_gpu(inp, chunk)
+    compare(inp, out, st, *ref)
+
+
+def test_bf16_uniform_extreme_decay():
+    """Every channel at log a = -30 (a ~ 1e-13): the state keeps only the last token."""
+    inp = I.prefill_inputs("prefill_4k", B=1, T=150, H=2, s0_std=0.05)
+    inp["log_alpha"] = torch.full_like(inp["log_alpha"], -30.0)
+    ref = run_oracle(inp)
+    for eng in engines(torch.bfloat16, 128, 128, 64):
+        out, st = run_gpu(inp, 64, eng)
+        compare(inp, out, st, *ref)
+
+
 def test_zero_length_copies_state():
     inp = I.prefill_inputs("fp32_small", T=0, s0_std=1.0)
     out, st = run_gpu(inp, 16)
@@ -179,21 +219,22 @@ def test_unsupported_engine_shape_is_rejected():
     inp = I.prefill_inputs("fp32_small", T=8)
     g = {k: (v.to(DEV) if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
     with pytest.raises(kda.KdaError, match="UNSUPPORTED"):
-        kda.chunk_fwd(g["q"], g["k"], g["v"], g["log_alpha"], g["beta"], chunk=16, engine="tc")
+        kda.chunk_fwd(g["q"], g["k"], g["v"], g["log_alpha"], g["beta"], chunk=16, engine="tc_cluster")
 
 
 # --- full-size workloads, sampled heads -----------------------------------------
 
 FULL = [
-    ("prefill_4k", [0, 37, 130, 255]),
-    ("prefill_32k", [0, 7, 19, 31]),
-    ("prefill_128k", [0, 15]),
+    ("prefill_4k", [0, 37, 130, 255], {}),
+    ("prefill_32k", [0, 7, 19, 31], {}),
+    ("prefill_128k", [0, 15], {}),
+    ("prefill_32k", [3, 30], {"gate": "strong"}),
 ]
 
 
-@pytest.mark.parametrize("name,heads", FULL)
-def test_full_workload_sampled_heads(name, heads):
-    inp = I.prefill_inputs(name, device=DEV)
+@pytest.mark.parametrize("name,heads,kw", FULL)
+def test_full_workload_sampled_heads(name, heads, kw):
+    inp = I.prefill_inputs(name, device=DEV, **kw)
     out, st = kda.chunk_fwd(inp["q"], inp["k"], inp["v"], inp["log_alpha"], inp["beta"],
                             inp["S0"], chunk=inp["w"].chunk)
     torch.cuda.synchronize()

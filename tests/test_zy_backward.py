@@ -100,3 +100,13 @@ def test_autograd_through_the_library():
     for n in NAMES:
         r = ref["d" + n]
         assert_close(t[n].grad, r, 1e-4 * max(1.0, float(np.abs(r).max())), 0.0, f"grad {n}")
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_strong_decay(dtype):
+    """Channels with log a = -4, 0, -12 and -1e-3 (the strong-decay gate recipe)."""
+    name = "fp32_small" if dtype == torch.float32 else "prefill_4k"
+    inp = I.prefill_inputs(name, B=1, T=45, H=2, gate="strong", s0_std=0.1)
+    B, T, H, dk = inp["q"].shape
+    dO, dST = cotangents(B, T, H, dk, inp["v"].shape[-1], dtype, seed=77)
+    check(inp, dO, dST)

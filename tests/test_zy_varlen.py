@@ -92,3 +92,8 @@ def test_paged_prefill_then_decode():
         assert_close(cache[r], ref_s[0], atol, rtol, f"cache row {r}")
     for r in (1, 2):
         assert torch.equal(cache[r], cache0[r])
+
+
+def test_bf16_strong_decay_mixed_lengths():
+    flat, S0, cu = packed("prefill_4k", [70, 1, 33, 130], H=2, seed=9, gate="strong")
+    check(flat, S0, cu)
