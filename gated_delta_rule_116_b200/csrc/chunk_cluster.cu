@@ -31,13 +31,15 @@
 // is sequential over chunks. One head runs on a cluster of 4 CTAs (4 SMs):
 //   * ranks 0..2 are producers: rank p computes the key-side part of chunks
 //     p, p+3, p+6, ... as an 82 KB image and writes it into one of its three
-//     slots of a small ring in the workspace (it stays in L2): Qs, Kb and
-//     e^{g_C} straight from registers; [P;T] (an operand of its own MMA), W and
-//     U' staged in shared memory and bulk-stored (cp.async.bulk shared ->
-//     global), [P;T] as soon as T is formed and W while U' is formed. Once the
-//     stores are complete, thread 0 arrives (release, cluster scope; the
-//     generic stores of all threads precede it through a CTA barrier) on the
-//     consumer's "ready" barrier of that slot;
+//     slots of a small ring in the workspace (it stays in L2). Each part (Qs,
+//     Kb, [P;T] -- also an operand of its own MMA --, W, U') is staged in
+//     shared memory in its image layout and bulk-stored (cp.async.bulk shared
+//     -> global) by one thread of a warp that has no share of the phase that
+//     follows, so that the copies (~27 B/cycle per SM, like any store path of
+//     an SM into L2) overlap the computation; e^{g_C} goes straight from
+//     registers. Once the stores are complete, the same thread arrives
+//     (release, cluster scope; the generic stores of all threads precede it
+//     through a CTA barrier) on the consumer's "ready" barrier of that slot;
 //   * rank 3 is the consumer: it keeps the 128x128 fp32 state in registers and
 //     runs the chain for every chunk, on all 128 value columns. Its thread 0
 //     pulls published images into two shared-memory slots (bulk global ->
@@ -69,6 +71,8 @@ using ut::kLD;
 constexpr int kC = 64;
 constexpr int kD = 128;
 constexpr int kThreads = 256;
+constexpr int kLoader = 32;     // producer thread that issues the TMA input loads (warp 1)
+constexpr int kStorer = 224;    // producer thread that issues the bulk stores and publishes (warp 7)
 constexpr int kProducers = 3;
 constexpr int kCluster = kProducers + 1;
 constexpr int kRingDepth = 3;   // ring slots per producer
@@ -78,6 +82,7 @@ constexpr uint32_t kTestWaitLimit = 1u << 12;   // polls of a bounded wait under
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRangeLog = -87.f;   // e^-87 ~ 1.6e-38: factors of a sub-chunk stay normal above it
 constexpr float kClampLog = -10.f;   // per-token clamp of log alpha for the fallback factors
+constexpr float kFastTot = 40.f;     // sub-chunk decay bound of the one-anchor path (chunk total <= 160)
 
 // ---- slot image: what a producer hands the consumer for one chunk
 constexpr uint32_t SL_QW = 0;          // [Qs ; W] fp16 K-major SW128, 2 K-blocks x 16 KB
@@ -111,21 +116,29 @@ constexpr uint32_t P_XF = 64 * kLD * 4;        // X = (I + A)^{-1} fp32 [64][kLD
 constexpr uint32_t P_DX = 2 * 64 * kLD * 4;    // diagonal-block partials of channels 64..127 (8 KB)
 constexpr uint32_t P_PX = P_DX + 8192;         // off-diagonal-block partials, both halves: 2 x 6 x 2 KB
 // K e^{G_{J+1} - g} (fp32), the column operand of the off-diagonal blocks, in the
-// swizzled layout of log alpha; then Kb staged for the ring (image layout)
+// swizzled layout of log alpha (phases 1b and 2); then W (2 K-blocks x 8 KB) and U'
+// (16 KB) staged for the ring, until their bulk stores have read them (before the next
+// image's phase 1b)
 constexpr uint32_t P_KSIG = 81920;
-constexpr uint32_t P_KBS = P_KSIG + 32768;
-constexpr uint32_t P_STAGE = 131072;   // [P;T] 16 KB, W 2 x 8 KB, U' 16 KB (bulk-stored to the ring)
-constexpr uint32_t ST_PT = 0;
-constexpr uint32_t ST_W = 16384;
-constexpr uint32_t ST_UP = 32768;
-constexpr uint32_t ST_GL = ST_W;       // before W and U' exist: g^L in the layout of log alpha (32 KB),
-constexpr uint32_t ST_QS = ST_W;       // then Qs staged for the ring: 2 K-blocks x 8 KB (image layout)
+// (one-anchor path: the tf32 operands of [A;P] over the same region, 0 .. 96 KB)
+constexpr uint32_t P_KQT = 0;          // [K e^{g - g_C/2} ; Q e^{g - g_C/2}], 4 K-blocks (32 channels) x 16 KB
+constexpr uint32_t kKQTBlk = 16384;
+constexpr uint32_t P_KHT = 65536;      // K e^{g_C/2 - g}, 4 K-blocks x 8 KB
+constexpr uint32_t kKHTBlk = 8192;
+constexpr uint32_t P_WS = P_KSIG;
+constexpr uint32_t P_US = P_KSIG + 16384;
+constexpr uint32_t P_KBS = P_KSIG + 32768;   // Kb staged for the ring (image layout)
+constexpr uint32_t P_STAGE = 131072;
+constexpr uint32_t ST_PT = 0;          // [P;T] 16 KB (A operand of [W | U'], bulk-stored to the ring)
+constexpr uint32_t ST_GL = 16384;      // g^L in the layout of log alpha (32 KB, phases 1a-1b), then
+constexpr uint32_t ST_QS = ST_GL;      // Qs staged for the ring, 2 K-blocks x 8 KB
 constexpr uint32_t P_KSV = 180224;     // [Ks | V] fp16 [token][col], 4 blocks x 8 KB
 // beta of two chunks [2][64] (the next one arrives by cp.async during this one); per
 // sub-chunk I and channel c ([4][128] each): tot = total log alpha of the sub-chunk,
 // e^{-g_m}, e^{g_m - tot} (g_m = g^L at its 8th token) and e^{tot}; a flag
 constexpr uint32_t P_VEC = 212992;
 constexpr uint32_t V_TOT = 128, V_EM = V_TOT + 512, V_EC = V_EM + 512, V_P = V_EC + 512, V_FLAG = V_P + 512;
+constexpr uint32_t V_SLOW = V_FLAG + 1;  // some sub-chunk decays by more than e^{-kFastTot}
 constexpr uint32_t V_INV = V_FLAG + 4;   // fused prologue: 1 / ||q_t||, 1 / ||k_t|| ([2][64])
 constexpr uint32_t P_BAR = P_VEC + (V_INV + 128) * 4;
 // ---- consumer shared memory
@@ -137,13 +150,16 @@ constexpr uint32_t kSmemBytes =
     (P_BAR > C_BAR ? P_BAR : C_BAR) + 192 + 1024;  // + barriers + alignment slack
 static_assert(P_PX + 2 * 6 * 2048 <= P_KSIG, "producer layout");
 static_assert(P_KBS + 16384 <= P_STAGE, "producer layout");
+static_assert(P_KHT + 4 * kKHTBlk <= P_KBS, "producer layout");
 
 // TMEM columns.
+constexpr uint32_t PCOL_AP = 0;        // producer, one-anchor path: [A;P] (64 cols)
 constexpr uint32_t PCOL_WU = 128;      // producer: [P;T][Ks|V], lanes 64-127 = [W | U'] (256)
 constexpr uint32_t CCOL_X = 0;         // consumer: 2 x 128 cols ([Qs;W]S (+ [P;T]U))
 constexpr uint32_t CCOL_S = 256;       // consumer: Kb^T U (128 cols)
 constexpr uint32_t kTmemCols = 512;
 
+constexpr uint32_t IDESC_AP = tc::idesc(tc::kFmtTF32, 128, 64, 0, 0);
 constexpr uint32_t IDESC_WU = tc::idesc(tc::kFmtF16, 128, 256, 0, 1);
 constexpr uint32_t IDESC_X = tc::idesc(tc::kFmtF16, 128, 128, 0, 1);   // A K-major, B MN-major
 constexpr uint32_t IDESC_S = tc::idesc(tc::kFmtF16, 128, 128, 1, 1);   // A MN-major, B MN-major
@@ -227,6 +243,19 @@ __device__ __forceinline__ float scan8(float x, int g) {
 // Index of the off-diagonal block (I, J), J < I, among the six: (1,0) (2,0) (2,1) (3,0) (3,1) (3,2).
 __device__ __forceinline__ int pair_index(int I, int J) { return I * (I - 1) / 2 + J; }
 
+// Receives the blocks of X = (I + A)^{-1} from the UT solve and writes T = X Diag(beta)
+// as fp16 into the K-major, 128-byte-swizzled T operand (rows 64..127 of [P;T]).
+struct TWriter {
+    uint8_t *t;
+    const float *beta;
+    __device__ __forceinline__ void one(int i, int j, float x) const {
+        *reinterpret_cast<__half *>(t + sw128k_off(i, j, 0)) = __float2half_rn(x * beta[j]);
+    }
+    __device__ __forceinline__ void pair(int i, int j, float x0, float x1) const {
+        *reinterpret_cast<uint32_t *>(t + sw128k_off(i, j, 0)) = pack_f16(x0 * beta[j], x1 * beta[j + 1]);
+    }
+};
+
 // ============================================================ producer
 // Thread mapping of the gate prologue: warp w handles sub-chunk I = w % 4 (16
 // tokens) and channel half w / 4 (64 channels); lane (g, t) = (lane / 4, lane % 4)
@@ -237,7 +266,6 @@ __device__ __forceinline__ int pair_index(int I, int J) { return I * (I - 1) / 2
 // products need no shared-memory round trip.
 template <bool kFused>
 __device__ void producer(uint8_t *sm, uint32_t tmem, int rank, uint8_t *ring,
-                         const CUtensorMap *tm_q, const CUtensorMap *tm_k, const CUtensorMap *tm_la,
                          const CUtensorMap *tm_v, const CUtensorMap *tm_qs, const CUtensorMap *tm_ks,
                          const CUtensorMap *tm_las, const float *__restrict__ beta, int T, int H,
                          int h, long ztok, int nchunks, const Ctl &ctl, int test_timeout) {
@@ -267,21 +295,30 @@ __device__ void producer(uint8_t *sm, uint32_t tmem, int rank, uint8_t *ring,
     uint64_t *bar_in = bar_mma + 1 + kRingDepth;
     uint8_t *st = sm + P_STAGE;
     uint32_t ph_mma = 0, ph_in = 0;
-    bool pend_in = false, pend_mma = false;   // thread 0: a TMA input batch / an MMA group in flight
+    bool pend_in = false, pend_mma = false;   // kLoader: a TMA input batch; thread 0: an MMA group in flight
+    // bulk stores of the staged parts (thread kStorer); a CTA barrier follows each wait
+    auto store_part = [&](uint8_t *dst, const uint8_t *src, uint32_t bytes) {
+        if (!aborted(ctl)) tc::bulk_store_global(dst, src, bytes);
+    };
     int img = 0;  // index of this producer's next image
 
     const uint64_t d_pt = tc::smem_desc(sbase + P_STAGE + ST_PT, 16, 1024, tc::kSwizzle128);
     const uint64_t d_ksv = tc::smem_desc(sbase + P_KSV, kTokBlk, 1024, tc::kSwizzle128);
+    const uint64_t d_kqt = tc::smem_desc(sbase + P_KQT, 16, 1024, tc::kSwizzle128);
+    const uint64_t d_kht = tc::smem_desc(sbase + P_KHT, 16, 1024, tc::kSwizzle128);
     // the consumer's "ready" barriers for this producer's ring slots
     const uint32_t c_ready = tc::map_to_rank(sbase + C_BAR + 40 + 8 * kRingDepth * rank, kCluster - 1);
 
-    // P's blocks above the diagonal are zero in every image; nothing else writes them
-    for (int e = tid; e < 64 * 32; e += kThreads) {
-        const int i = e >> 5, j = 2 * (e & 31);
+    // the blocks of P and T above the diagonal are zero in every image; nothing else writes them
+    for (int e = tid; e < 128 * 32; e += kThreads) {
+        const int i = (e >> 5) & 63, j = 2 * (e & 31);
         if (j >= 16 * ((i >> 4) + 1))
-            *reinterpret_cast<uint32_t *>(st + ST_PT + sw128k_off(i, j, 0)) = 0u;
+            *reinterpret_cast<uint32_t *>(st + ST_PT + (e >> 11) * 8192 + sw128k_off(i, j, 0)) = 0u;
     }
-    if (tid == 0) *reinterpret_cast<volatile int *>(vec + V_FLAG) = 0;
+    if (tid == 0) {
+        *reinterpret_cast<volatile int *>(vec + V_FLAG) = 0;
+        *reinterpret_cast<volatile int *>(vec + V_SLOW) = 0;
+    }
     __syncthreads();
 
     auto load_inputs = [&](int cc) {   // TMA: the 64-token chunk cc of head h (all channels)
@@ -304,14 +341,14 @@ __device__ void producer(uint8_t *sm, uint32_t tmem, int rank, uint8_t *ring,
             tc::tma_load_3d(sm + P_IN_V, tm_v, bar_in, 0, h, z);
         }
     };
-    // Publication of an image: thread 0 waits until all its bulk stores (Qs, Kb, [P;T], W,
-    // U' of that image) are complete, then arrives (release, cluster scope; the generic
-    // stores of other threads into the slot precede it through CTA barriers) on the
-    // consumer's "ready" barrier of the image's ring slot.
+    // Publication of an image: thread kStorer waits until its bulk stores of the image are
+    // complete, then arrives (release, cluster scope; the generic stores of all threads into
+    // the slot precede it through CTA barriers) on the consumer's "ready" barrier of the
+    // image's ring slot.
     // (A test hook withholds producer 0's first "ready", so that the consumer's wait runs out.)
     int pending = -1, pending_img = 0;
     auto publish = [&]() {
-        if (tid == 0 && pending >= 0) {
+        if (tid == kStorer && pending >= 0) {
             tc::bulk_wait_all();
             tc::fence_proxy_async_global();
             const bool withheld = test_timeout && rank == 0 && pending_img == 0;
@@ -319,21 +356,13 @@ __device__ void producer(uint8_t *sm, uint32_t tmem, int rank, uint8_t *ring,
         }
         pending = -1;
     };
-    if (tid == 0 && rank < nchunks) load_inputs(rank);
+    if (tid == kLoader && rank < nchunks) load_inputs(rank);
     load_beta(rank, 0);
     for (int c = rank; c < nchunks; c += kProducers) {
         if (__syncthreads_or(aborted(ctl))) break;   // uniform: the cluster gave up
         const float *beta_s = vec + 64 * (img & 1);
         const int t0 = c * kC;
         const int valid = min(kC, T - t0);
-        const long trow0 = ztok + t0;
-        if (tid == 0 && c + 2 * kProducers < nchunks) {
-            const int z = static_cast<int>(trow0 + 2 * kProducers * kC);
-            tc::tma_prefetch_l2_3d(tm_q, 0, h, z);
-            tc::tma_prefetch_l2_3d(tm_k, 0, h, z);
-            tc::tma_prefetch_l2_3d(tm_la, 0, h, z);
-            tc::tma_prefetch_l2_3d(tm_v, 0, h, z);
-        }
         if (wait_local(bar_in, ph_in, ctl)) {
             ph_in ^= 1;
             pend_in = false;
@@ -410,259 +439,361 @@ __device__ void producer(uint8_t *sm, uint32_t tmem, int rank, uint8_t *ring,
             *reinterpret_cast<float2 *>(vec + V_P + e) =
                 make_float2(tc::ex2(s0 * kLog2e), tc::ex2(s1 * kLog2e));
             if (s0 < kRangeLog || s1 < kRangeLog) *reinterpret_cast<volatile int *>(vec + V_FLAG) = 1;
+            if (s0 < -kFastTot || s1 < -kFastTot) *reinterpret_cast<volatile int *>(vec + V_SLOW) = 1;
         }
-        publish();   // the previous image (its stores have had phase 1a to land)
+        if (tid == kStorer) tc::bulk_wait_read_all();   // the previous W and U' have left P_KSIG
         __syncthreads();
-        const bool far_decay = *reinterpret_cast<volatile int *>(vec + V_FLAG) != 0;
-
-        // ------------------------------------------------ phase 1b: diagonal blocks (tf32
-        // mma.sync, fragments straight from registers), rows of the off-diagonal blocks
-        const bool va = ta < valid, vb = tb < valid;
-        // the fused prologue's L2 normalisation, applied where q and k are unpacked
-        const float nqa = kFused ? vec[V_INV + ta] : 1.f, nqb = kFused ? vec[V_INV + tb] : 1.f;
-        const float nka = kFused ? vec[V_INV + 64 + ta] : 1.f, nkb = kFused ? vec[V_INV + 64 + tb] : 1.f;
-        uint32_t qA[8], qB[8], kA[8], kB[8];
-        float rA[8][2], rB[8][2], sA[8][2], sB[8][2];   // e^{g^L}, e^{tot - g^L} of tokens a, b
-        float accA[2][4] = {}, accP[2][4] = {};
-        const uint32_t rowa = static_cast<uint32_t>(ta) * 128u, rowb = static_cast<uint32_t>(tb) * 128u;
-#pragma unroll
-        for (int s = 0; s < 8; ++s) {
-            const int c0 = 64 * half + 8 * s + 2 * t4;
-            const uint32_t qk_off = half * kBoxBytes + ((s ^ g) << 4) + 4 * t4;
-            const uint32_t la_off = (c0 >> 5) * kBoxBytes + (((((c0 & 31) >> 2) ^ g) & 7) << 4) + 8 * (t4 & 1);
-            qA[s] = va ? *reinterpret_cast<const uint32_t *>(sm + P_IN_Q + rowa + qk_off) : 0u;
-            qB[s] = vb ? *reinterpret_cast<const uint32_t *>(sm + P_IN_Q + rowb + qk_off) : 0u;
-            kA[s] = va ? *reinterpret_cast<const uint32_t *>(sm + P_IN_K + rowa + qk_off) : 0u;
-            kB[s] = vb ? *reinterpret_cast<const uint32_t *>(sm + P_IN_K + rowb + qk_off) : 0u;
-            const float2 xa = *reinterpret_cast<const float2 *>(st + ST_GL + rowa + la_off);
-            const float2 xb = *reinterpret_cast<const float2 *>(st + ST_GL + rowb + la_off);
-            const int e = I * 128 + c0;
-            const float2 tot = *reinterpret_cast<const float2 *>(vec + V_TOT + e);
-            const float2 em = *reinterpret_cast<const float2 *>(vec + V_EM + e);
-            const float2 ec = *reinterpret_cast<const float2 *>(vec + V_EC + e);
-            // factors anchored at the sub-chunk's start (rho) and end (sigma), both <= 1
-            rA[s][0] = tc::ex2(xa.x * kLog2e);
-            rA[s][1] = tc::ex2(xa.y * kLog2e);
-            rB[s][0] = tc::ex2(xb.x * kLog2e);
-            rB[s][1] = tc::ex2(xb.y * kLog2e);
-            sA[s][0] = tc::ex2((tot.x - xa.x) * kLog2e);
-            sA[s][1] = tc::ex2((tot.y - xa.y) * kLog2e);
-            sB[s][0] = tc::ex2((tot.x - xb.x) * kLog2e);
-            sB[s][1] = tc::ex2((tot.y - xb.y) * kLog2e);
-            // diagonal-block factors around token 7: rows e^{g_i - g_m} = rho_i e^{-g_m},
-            // columns e^{g_m - g_j} = sigma_j e^{g_m - tot}
-            float ra0 = rA[s][0] * em.x, ra1 = rA[s][1] * em.y, rb0 = rB[s][0] * em.x, rb1 = rB[s][1] * em.y;
-            float ca0 = sA[s][0] * ec.x, ca1 = sA[s][1] * ec.y, cb0 = sB[s][0] * ec.x, cb1 = sB[s][1] * ec.y;
-            if (far_decay) {
-                // some channel of the chunk decays by more than e^-87 inside one sub-chunk: such a
-                // channel takes its diagonal factors from log alpha clamped at -10 per token
-                const bool f0 = tot.x >= kRangeLog, f1 = tot.y >= kRangeLog;
-                float2 la = make_float2(0.f, 0.f), lb = make_float2(0.f, 0.f);
-                if (kFused) {
-                    const uint32_t xa2 = va ? *reinterpret_cast<const uint32_t *>(sm + P_IN_X + rowa + qk_off) : 0u;
-                    const uint32_t xb2 = vb ? *reinterpret_cast<const uint32_t *>(sm + P_IN_X + rowb + qk_off) : 0u;
-                    if (va) la = make_float2(neg_softplus(tc::bf16_lo(xa2)), neg_softplus(tc::bf16_hi(xa2)));
-                    if (vb) lb = make_float2(neg_softplus(tc::bf16_lo(xb2)), neg_softplus(tc::bf16_hi(xb2)));
-                } else {
-                    if (va) la = *reinterpret_cast<const float2 *>(sm + P_IN_LA + rowa + la_off);
-                    if (vb) lb = *reinterpret_cast<const float2 *>(sm + P_IN_LA + rowb + la_off);
-                }
-                float ya0 = scan8(fmaxf(la.x, kClampLog), g), ya1 = scan8(fmaxf(la.y, kClampLog), g);
-                float yb0 = scan8(fmaxf(lb.x, kClampLog), g), yb1 = scan8(fmaxf(lb.y, kClampLog), g);
-                const float ym0 = __shfl_sync(0xffffffffu, ya0, 28 + t4);   // at token 7
-                const float ym1 = __shfl_sync(0xffffffffu, ya1, 28 + t4);
-                yb0 += ym0;
-                yb1 += ym1;
-                if (!f0) {
-                    ra0 = tc::ex2((ya0 - ym0) * kLog2e);
-                    rb0 = tc::ex2((yb0 - ym0) * kLog2e);
-                    ca0 = tc::ex2((ym0 - ya0) * kLog2e);
-                    cb0 = tc::ex2((ym0 - yb0) * kLog2e);
-                }
-                if (!f1) {
-                    ra1 = tc::ex2((ya1 - ym1) * kLog2e);
-                    rb1 = tc::ex2((yb1 - ym1) * kLog2e);
-                    ca1 = tc::ex2((ym1 - ya1) * kLog2e);
-                    cb1 = tc::ex2((ym1 - yb1) * kLog2e);
-                }
-            }
-            const float qa0 = tc::bf16_lo(qA[s]) * nqa, qa1 = tc::bf16_hi(qA[s]) * nqa;
-            const float qb0 = tc::bf16_lo(qB[s]) * nqb, qb1 = tc::bf16_hi(qB[s]) * nqb;
-            const float ka0 = tc::bf16_lo(kA[s]) * nka, ka1 = tc::bf16_hi(kA[s]) * nka;
-            const float kb0 = tc::bf16_lo(kB[s]) * nkb, kb1 = tc::bf16_hi(kB[s]) * nkb;
-            {   // diagonal block: A^d += K~ K^^T, P^d += Q~ K^^T over this k-step's 8 channels
-                // (fp32 operands; the tensor cores read them as tf32)
-                const uint32_t ak[4] = {__float_as_uint(ka0 * ra0), __float_as_uint(kb0 * rb0),
-                                        __float_as_uint(ka1 * ra1), __float_as_uint(kb1 * rb1)};
-                const uint32_t aq[4] = {__float_as_uint(qa0 * ra0), __float_as_uint(qb0 * rb0),
-                                        __float_as_uint(qa1 * ra1), __float_as_uint(qb1 * rb1)};
-                const uint32_t b00 = __float_as_uint(ka0 * ca0), b01 = __float_as_uint(ka1 * ca1);  // column token g
-                const uint32_t b10 = __float_as_uint(kb0 * cb0), b11 = __float_as_uint(kb1 * cb1);  // column token g + 8
-                tc::mma_16x8x8_tf32(accA[0], ak, b00, b01);
-                tc::mma_16x8x8_tf32(accA[1], ak, b10, b11);
-                tc::mma_16x8x8_tf32(accP[0], aq, b00, b01);
-                tc::mma_16x8x8_tf32(accP[1], aq, b10, b11);
-            }
-            // column operand of the off-diagonal blocks: K e^{G_{J+1} - g_j} for this sub-chunk J = I
-            *reinterpret_cast<float2 *>(sm + P_KSIG + rowa + la_off) = make_float2(ka0 * sA[s][0], ka1 * sA[s][1]);
-            *reinterpret_cast<float2 *>(sm + P_KSIG + rowb + la_off) = make_float2(kb0 * sB[s][0], kb1 * sB[s][1]);
-        }
-
         const int rb = img % kRingDepth;  // ring slot of this image; image img-kRingDepth used it before
         uint8_t *gs = ring + (kRingDepth * rank + rb) * kSlotStride;
-        if (tid == 0) {
-            tc::bulk_wait_read_all();  // the previous image's staged parts have left shared memory
-            if (img >= kRingDepth) wait_cluster(bar_loaded + rb, ((img / kRingDepth) - 1) & 1, ctl);
-        }
-        cp_async_wait_prev();   // this image's beta (all but the group just issued)
-        __syncthreads();   // the inputs and g^L are dead; every thread has read the flag
-        if (tid == 0) *reinterpret_cast<volatile int *>(vec + V_FLAG) = 0;   // for the next image
-
-        // ------------------------------------------------ phase 2: chunk-level factors
-        // (products of the sub-chunks' e^{tot}: e^{G_I}, e^{g_C - G_{I+1}}) and the off-diagonal blocks
-        if (half == 1) {   // diagonal partials of channels 64..127 for the half-0 warp of sub-chunk I
-            float4 *dx = reinterpret_cast<float4 *>(sm + P_DX) + (I * 32 + lane) * 4;
-            dx[0] = make_float4(accA[0][0], accA[0][1], accA[0][2], accA[0][3]);
-            dx[1] = make_float4(accA[1][0], accA[1][1], accA[1][2], accA[1][3]);
-            dx[2] = make_float4(accP[0][0], accP[0][1], accP[0][2], accP[0][3]);
-            dx[3] = make_float4(accP[1][0], accP[1][1], accP[1][2], accP[1][3]);
-        }
-        const uint32_t row_a = half * 8192u + (ta >> 3) * 1024u + g * 128u + 4u * t4;   // token a, no swizzle term
+        if (*reinterpret_cast<volatile int *>(vec + V_SLOW) == 0) {   // uniform: read after a CTA barrier
+            // -------------------------------------------- one-anchor path: every sub-chunk decays by
+            // at most e^{-kFastTot}, so the chunk by at most e^{-160}, and the factors e^{g - g_C/2},
+            // e^{g_C/2 - g} stay within e^{80}: [A;P] = [K~ ; Q~] K^T is one tf32 tcgen05 MMA over
+            // all 128 channels (K~ = K e^{g - g_C/2}, Q~ likewise, K^ = K e^{g_C/2 - g}).
+            // Thread (p, I) = (tid % 64, tid / 64) owns channels 2p, 2p + 1 of sub-chunk I.
+            const int p = tid & 63, Ib = tid >> 6, cp = 2 * p;
+            uint32_t qv[16], kv[16];
+            float2 gl[16];
+            {
+                const uint32_t off = (cp >> 5) * kBoxBytes + (cp & 3) * 4, ch = (cp & 31) >> 2;
+                const uint32_t qk = (cp >> 6) * kBoxBytes + (cp & 7) * 2, ch16 = (cp & 63) >> 3;
 #pragma unroll
-        for (int s = 0; s < 8; ++s) {
-            const int c0 = 64 * half + 8 * s + 2 * t4;
-            float2 pj[4];   // e^{tot_J} of the four sub-chunks
-#pragma unroll
-            for (int J = 0; J < 4; ++J) pj[J] = *reinterpret_cast<const float2 *>(vec + V_P + J * 128 + c0);
-            float eG0 = 1.f, eG1 = 1.f, eK0 = 1.f, eK1 = 1.f;
+                for (int u = 0; u < 16; ++u) {
+                    const int t = 16 * Ib + u;
+                    const bool ok = t < valid;
+                    gl[u] = *reinterpret_cast<const float2 *>(st + ST_GL + off + t * 128u + (((ch ^ (t & 7)) & 7u) << 4));
+                    const uint32_t o = qk + t * 128u + (((ch16 ^ (t & 7)) & 7u) << 4);
+                    qv[u] = ok ? *reinterpret_cast<const uint32_t *>(sm + P_IN_Q + o) : 0u;
+                    kv[u] = ok ? *reinterpret_cast<const uint32_t *>(sm + P_IN_K + o) : 0u;
+                }
+            }
+            float G0 = 0.f, G1 = 0.f, C0 = 0.f, C1 = 0.f;   // g before sub-chunk Ib; g_C
 #pragma unroll
             for (int J = 0; J < 4; ++J) {
-                if (J < I) { eG0 *= pj[J].x; eG1 *= pj[J].y; }
-                if (J > I) { eK0 *= pj[J].x; eK1 *= pj[J].y; }
+                const float2 tj = *reinterpret_cast<const float2 *>(vec + V_TOT + J * 128 + cp);
+                if (J < Ib) { G0 += tj.x; G1 += tj.y; }
+                C0 += tj.x;
+                C1 += tj.y;
             }
-            const float qa0 = tc::bf16_lo(qA[s]) * nqa, qa1 = tc::bf16_hi(qA[s]) * nqa;
-            const float qb0 = tc::bf16_lo(qB[s]) * nqb, qb1 = tc::bf16_hi(qB[s]) * nqb;
-            const float ka0 = tc::bf16_lo(kA[s]) * nka, ka1 = tc::bf16_hi(kA[s]) * nka;
-            const float kb0 = tc::bf16_lo(kB[s]) * nkb, kb1 = tc::bf16_hi(kB[s]) * nkb;
-            const float fa0 = rA[s][0] * eG0, fa1 = rA[s][1] * eG1, fb0 = rB[s][0] * eG0, fb1 = rB[s][1] * eG1;
-            // Qs = Q e^{g} and Kb = K e^{g_C - g} (staged for the ring slot), Ks = K e^{g} into [Ks | V];
-            // all three are [token][channel] tiles with 64-channel blocks 8 KB apart
-            const uint32_t oa = row_a + (((s ^ g) & 7) << 4), ob = oa + 1024;
-            *reinterpret_cast<uint32_t *>(st + ST_QS + oa) = pack_f16(qa0 * fa0, qa1 * fa1);
-            *reinterpret_cast<uint32_t *>(st + ST_QS + ob) = pack_f16(qb0 * fb0, qb1 * fb1);
-            *reinterpret_cast<uint32_t *>(sm + P_KSV + oa) = pack_f16(ka0 * fa0, ka1 * fa1);
-            *reinterpret_cast<uint32_t *>(sm + P_KSV + ob) = pack_f16(kb0 * fb0, kb1 * fb1);
-            *reinterpret_cast<uint32_t *>(sm + P_KBS + oa) = pack_f16(ka0 * sA[s][0] * eK0, ka1 * sA[s][1] * eK1);
-            *reinterpret_cast<uint32_t *>(sm + P_KBS + ob) = pack_f16(kb0 * sB[s][0] * eK0, kb1 * sB[s][1] * eK1);
-            if (I == 0 && g == 0)
-                *reinterpret_cast<float2 *>(gs + SL_GAM + 4 * c0) =
-                    make_float2(pj[0].x * pj[1].x * pj[2].x * pj[3].x, pj[0].y * pj[1].y * pj[2].y * pj[3].y);
-        }
-        // Off-diagonal blocks (I, J), J < I, over this warp's 64 channels:
-        //   A^o += [K e^{g - G_I} Diag(e^{G_I - G_{J+1}})] (K e^{G_{J+1} - g})^T, P^o likewise with Q;
-        // partials of both channel halves go to shared memory, summed by the half-1 warp below.
-        for (int J = 0; J < I; ++J) {
-            float oA[2][4] = {}, oP[2][4] = {};
+            __syncthreads();   // all inputs are in registers: the operand tiles may overwrite them
+            if (tid == 0) {   // for the next image
+                *reinterpret_cast<volatile int *>(vec + V_FLAG) = 0;
+                *reinterpret_cast<volatile int *>(vec + V_SLOW) = 0;
+            }
+            const float ga0 = 0.5f * C0, ga1 = 0.5f * C1;
+            const float ea0 = tc::ex2(ga0 * kLog2e), ea1 = tc::ex2(ga1 * kLog2e);   // e^{g_C/2}
+            // tf32 tiles: 32-channel K-blocks; fp16 tiles: 64-channel K-blocks; 128-byte rows, swizzled
+            const uint32_t rowq = Ib * 2048u;
+            const uint32_t b32 = (cp & 3u) * 4u + rowq, ch32 = (cp & 31u) >> 2, kb32 = cp >> 5;
+            const uint32_t b16 = (cp & 7u) * 2u + rowq, ch16 = (cp & 63u) >> 3, kb16 = cp >> 6;
 #pragma unroll
+            for (int u = 0; u < 16; ++u) {
+                const int t = 16 * Ib + u;
+                const uint32_t r = (u >> 3) * 1024u + (u & 7) * 128u;
+                const uint32_t o32 = b32 + r + (((ch32 ^ (u & 7)) & 7u) << 4);
+                const uint32_t o16 = b16 + r + (((ch16 ^ (u & 7)) & 7u) << 4);
+                const float d0 = (G0 + gl[u].x - ga0) * kLog2e, d1 = (G1 + gl[u].y - ga1) * kLog2e;
+                const float nq = kFused ? vec[V_INV + t] : 1.f, nk = kFused ? vec[V_INV + 64 + t] : 1.f;
+                const float q0 = tc::bf16_lo(qv[u]) * nq, q1 = tc::bf16_hi(qv[u]) * nq;
+                const float k0 = tc::bf16_lo(kv[u]) * nk, k1 = tc::bf16_hi(kv[u]) * nk;
+                const float E0 = tc::ex2(d0), E1 = tc::ex2(d1), F0 = tc::ex2(-d0), F1 = tc::ex2(-d1);
+                const float ke0 = k0 * E0, ke1 = k1 * E1, qe0 = q0 * E0, qe1 = q1 * E1;
+                const float kf0 = k0 * F0, kf1 = k1 * F1;
+                *reinterpret_cast<float2 *>(sm + P_KQT + kb32 * kKQTBlk + o32) = make_float2(ke0, ke1);
+                *reinterpret_cast<float2 *>(sm + P_KQT + kb32 * kKQTBlk + 8192 + o32) = make_float2(qe0, qe1);
+                *reinterpret_cast<float2 *>(sm + P_KHT + kb32 * kKHTBlk + o32) = make_float2(kf0, kf1);
+                // Qs = Q e^{g}, Ks = K e^{g}, Kb = K e^{g_C - g}
+                *reinterpret_cast<uint32_t *>(st + ST_QS + kb16 * 8192 + o16) = pack_f16(qe0 * ea0, qe1 * ea1);
+                *reinterpret_cast<uint32_t *>(sm + P_KSV + kb16 * kTokBlk + o16) = pack_f16(ke0 * ea0, ke1 * ea1);
+                *reinterpret_cast<uint32_t *>(sm + P_KBS + kb16 * 8192 + o16) = pack_f16(kf0 * ea0, kf1 * ea1);
+            }
+            fence_proxy_async_smem();
+            publish();   // the previous image (its stores have had phase 1a to land)
+            if (tid == 0 && img >= kRingDepth) wait_cluster(bar_loaded + rb, ((img / kRingDepth) - 1) & 1, ctl);
+            cp_async_wait_prev();   // this image's beta (all but the group just issued)
+            __syncthreads();
+            if (tid == 0 && !aborted(ctl)) {
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < 16; ++kk)
+                    tc::mma_tf32(tmem + PCOL_AP, d_kqt + (((kk >> 2) * kKQTBlk + (kk & 3) * 32) >> 4),
+                                 d_kht + (((kk >> 2) * kKHTBlk + (kk & 3) * 32) >> 4), IDESC_AP, kk > 0);
+                tc::mma_commit(bar_mma);
+                pend_mma = true;
+            }
+            if (tid == kStorer) {
+                store_part(gs + SL_QW, st + ST_QS, 8192);                 // Qs, K-block 0
+                store_part(gs + SL_QW + kQWBlk, st + ST_QS + 8192, 8192); // Qs, K-block 1
+                store_part(gs + SL_KB, sm + P_KBS, 16384);                // Kb
+                tc::bulk_commit();
+            }
+            if (Ib == 0)
+                *reinterpret_cast<float2 *>(gs + SL_GAM + 4 * cp) =
+                    make_float2(tc::ex2(C0 * kLog2e), tc::ex2(C1 * kLog2e));   // e^{g_C}
+            if (wait_local(bar_mma, ph_mma, ctl)) {
+                ph_mma ^= 1;
+                pend_mma = false;
+            }
+            tc_fence_after();
+            {   // A = Diag(beta) strict_lower(K~ K^T) (fp32), P = lower(Q~ K^T) (fp16, into [P;T])
+                float vv[32];
+                tc::tmem_ld32(tc::tmem_addr(tmem, 32 * quad, PCOL_AP + half * 32), vv);
+                tc::tmem_wait_ld();
+                if (quad < 2) {
+                    const int i = row;
+                    const float bi = beta_s[i];
+#pragma unroll
+                    for (int u = 0; u < 32; ++u) {
+                        const int j = half * 32 + u;
+                        Af[i * kLD + j] = j < i ? bi * vv[u] : 0.f;
+                    }
+                } else {
+                    const int i = row - 64;
+#pragma unroll
+                    for (int u = 0; u < 32; u += 2) {
+                        const int j = half * 32 + u;
+                        const float lo = j <= i ? vv[u] : 0.f, hi = j + 1 <= i ? vv[u + 1] : 0.f;
+                        *reinterpret_cast<uint32_t *>(st + ST_PT + sw128k_off(i, j, 0)) = pack_f16(lo, hi);
+                    }
+                }
+            }
+            tc_fence_before();
+        } else {
+            // -------------------------------------------- sub-chunk path (any decay)
+            const bool far_decay = *reinterpret_cast<volatile int *>(vec + V_FLAG) != 0;
+
+            // ------------------------------------------------ phase 1b: diagonal blocks (tf32
+            // mma.sync, fragments straight from registers), rows of the off-diagonal blocks
+            const bool va = ta < valid, vb = tb < valid;
+            // the fused prologue's L2 normalisation, applied where q and k are unpacked
+            const float nqa = kFused ? vec[V_INV + ta] : 1.f, nqb = kFused ? vec[V_INV + tb] : 1.f;
+            const float nka = kFused ? vec[V_INV + 64 + ta] : 1.f, nkb = kFused ? vec[V_INV + 64 + tb] : 1.f;
+            uint32_t qA[8], qB[8], kA[8], kB[8];
+            float rA[8][2], rB[8][2], sA[8][2], sB[8][2];   // e^{g^L}, e^{tot - g^L} of tokens a, b
+            float accA[2][4] = {}, accP[2][4] = {};
+            const uint32_t rowa = static_cast<uint32_t>(ta) * 128u, rowb = static_cast<uint32_t>(tb) * 128u;
+    #pragma unroll
             for (int s = 0; s < 8; ++s) {
                 const int c0 = 64 * half + 8 * s + 2 * t4;
-                float D0 = 1.f, D1 = 1.f;   // e^{G_I - G_{J+1}}: the sub-chunks strictly between J and I
-#pragma unroll
-                for (int Jm = 1; Jm < 3; ++Jm)
-                    if (Jm > J && Jm < I) {
-                        const float2 pm = *reinterpret_cast<const float2 *>(vec + V_P + Jm * 128 + c0);
-                        D0 *= pm.x;
-                        D1 *= pm.y;
-                    }
-                const float ra0 = rA[s][0] * D0, ra1 = rA[s][1] * D1, rb0 = rB[s][0] * D0, rb1 = rB[s][1] * D1;
-                const uint32_t ak[4] = {__float_as_uint(tc::bf16_lo(kA[s]) * nka * ra0), __float_as_uint(tc::bf16_lo(kB[s]) * nkb * rb0),
-                                        __float_as_uint(tc::bf16_hi(kA[s]) * nka * ra1), __float_as_uint(tc::bf16_hi(kB[s]) * nkb * rb1)};
-                const uint32_t aq[4] = {__float_as_uint(tc::bf16_lo(qA[s]) * nqa * ra0), __float_as_uint(tc::bf16_lo(qB[s]) * nqb * rb0),
-                                        __float_as_uint(tc::bf16_hi(qA[s]) * nqa * ra1), __float_as_uint(tc::bf16_hi(qB[s]) * nqb * rb1)};
+                const uint32_t qk_off = half * kBoxBytes + ((s ^ g) << 4) + 4 * t4;
                 const uint32_t la_off = (c0 >> 5) * kBoxBytes + (((((c0 & 31) >> 2) ^ g) & 7) << 4) + 8 * (t4 & 1);
-                const uint32_t rj = static_cast<uint32_t>(16 * J + g) * 128u;   // column token g of sub-chunk J
-                const float2 y0 = *reinterpret_cast<const float2 *>(sm + P_KSIG + rj + la_off);
-                const float2 y1 = *reinterpret_cast<const float2 *>(sm + P_KSIG + rj + 1024 + la_off);  // token g + 8
-                tc::mma_16x8x8_tf32(oA[0], ak, __float_as_uint(y0.x), __float_as_uint(y0.y));
-                tc::mma_16x8x8_tf32(oA[1], ak, __float_as_uint(y1.x), __float_as_uint(y1.y));
-                tc::mma_16x8x8_tf32(oP[0], aq, __float_as_uint(y0.x), __float_as_uint(y0.y));
-                tc::mma_16x8x8_tf32(oP[1], aq, __float_as_uint(y1.x), __float_as_uint(y1.y));
+                qA[s] = va ? *reinterpret_cast<const uint32_t *>(sm + P_IN_Q + rowa + qk_off) : 0u;
+                qB[s] = vb ? *reinterpret_cast<const uint32_t *>(sm + P_IN_Q + rowb + qk_off) : 0u;
+                kA[s] = va ? *reinterpret_cast<const uint32_t *>(sm + P_IN_K + rowa + qk_off) : 0u;
+                kB[s] = vb ? *reinterpret_cast<const uint32_t *>(sm + P_IN_K + rowb + qk_off) : 0u;
+                const float2 xa = *reinterpret_cast<const float2 *>(st + ST_GL + rowa + la_off);
+                const float2 xb = *reinterpret_cast<const float2 *>(st + ST_GL + rowb + la_off);
+                const int e = I * 128 + c0;
+                const float2 tot = *reinterpret_cast<const float2 *>(vec + V_TOT + e);
+                const float2 em = *reinterpret_cast<const float2 *>(vec + V_EM + e);
+                const float2 ec = *reinterpret_cast<const float2 *>(vec + V_EC + e);
+                // factors anchored at the sub-chunk's start (rho) and end (sigma), both <= 1
+                rA[s][0] = tc::ex2(xa.x * kLog2e);
+                rA[s][1] = tc::ex2(xa.y * kLog2e);
+                rB[s][0] = tc::ex2(xb.x * kLog2e);
+                rB[s][1] = tc::ex2(xb.y * kLog2e);
+                sA[s][0] = tc::ex2((tot.x - xa.x) * kLog2e);
+                sA[s][1] = tc::ex2((tot.y - xa.y) * kLog2e);
+                sB[s][0] = tc::ex2((tot.x - xb.x) * kLog2e);
+                sB[s][1] = tc::ex2((tot.y - xb.y) * kLog2e);
+                // diagonal-block factors around token 7: rows e^{g_i - g_m} = rho_i e^{-g_m},
+                // columns e^{g_m - g_j} = sigma_j e^{g_m - tot}
+                float ra0 = rA[s][0] * em.x, ra1 = rA[s][1] * em.y, rb0 = rB[s][0] * em.x, rb1 = rB[s][1] * em.y;
+                float ca0 = sA[s][0] * ec.x, ca1 = sA[s][1] * ec.y, cb0 = sB[s][0] * ec.x, cb1 = sB[s][1] * ec.y;
+                if (far_decay) {
+                    // some channel of the chunk decays by more than e^-87 inside one sub-chunk: such a
+                    // channel takes its diagonal factors from log alpha clamped at -10 per token
+                    const bool f0 = tot.x >= kRangeLog, f1 = tot.y >= kRangeLog;
+                    float2 la = make_float2(0.f, 0.f), lb = make_float2(0.f, 0.f);
+                    if (kFused) {
+                        const uint32_t xa2 = va ? *reinterpret_cast<const uint32_t *>(sm + P_IN_X + rowa + qk_off) : 0u;
+                        const uint32_t xb2 = vb ? *reinterpret_cast<const uint32_t *>(sm + P_IN_X + rowb + qk_off) : 0u;
+                        if (va) la = make_float2(neg_softplus(tc::bf16_lo(xa2)), neg_softplus(tc::bf16_hi(xa2)));
+                        if (vb) lb = make_float2(neg_softplus(tc::bf16_lo(xb2)), neg_softplus(tc::bf16_hi(xb2)));
+                    } else {
+                        if (va) la = *reinterpret_cast<const float2 *>(sm + P_IN_LA + rowa + la_off);
+                        if (vb) lb = *reinterpret_cast<const float2 *>(sm + P_IN_LA + rowb + la_off);
+                    }
+                    float ya0 = scan8(fmaxf(la.x, kClampLog), g), ya1 = scan8(fmaxf(la.y, kClampLog), g);
+                    float yb0 = scan8(fmaxf(lb.x, kClampLog), g), yb1 = scan8(fmaxf(lb.y, kClampLog), g);
+                    const float ym0 = __shfl_sync(0xffffffffu, ya0, 28 + t4);   // at token 7
+                    const float ym1 = __shfl_sync(0xffffffffu, ya1, 28 + t4);
+                    yb0 += ym0;
+                    yb1 += ym1;
+                    if (!f0) {
+                        ra0 = tc::ex2((ya0 - ym0) * kLog2e);
+                        rb0 = tc::ex2((yb0 - ym0) * kLog2e);
+                        ca0 = tc::ex2((ym0 - ya0) * kLog2e);
+                        cb0 = tc::ex2((ym0 - yb0) * kLog2e);
+                    }
+                    if (!f1) {
+                        ra1 = tc::ex2((ya1 - ym1) * kLog2e);
+                        rb1 = tc::ex2((yb1 - ym1) * kLog2e);
+                        ca1 = tc::ex2((ym1 - ya1) * kLog2e);
+                        cb1 = tc::ex2((ym1 - yb1) * kLog2e);
+                    }
+                }
+                const float qa0 = tc::bf16_lo(qA[s]) * nqa, qa1 = tc::bf16_hi(qA[s]) * nqa;
+                const float qb0 = tc::bf16_lo(qB[s]) * nqb, qb1 = tc::bf16_hi(qB[s]) * nqb;
+                const float ka0 = tc::bf16_lo(kA[s]) * nka, ka1 = tc::bf16_hi(kA[s]) * nka;
+                const float kb0 = tc::bf16_lo(kB[s]) * nkb, kb1 = tc::bf16_hi(kB[s]) * nkb;
+                {   // diagonal block: A^d += K~ K^^T, P^d += Q~ K^^T over this k-step's 8 channels
+                    // (fp32 operands; the tensor cores read them as tf32)
+                    const uint32_t ak[4] = {__float_as_uint(ka0 * ra0), __float_as_uint(kb0 * rb0),
+                                            __float_as_uint(ka1 * ra1), __float_as_uint(kb1 * rb1)};
+                    const uint32_t aq[4] = {__float_as_uint(qa0 * ra0), __float_as_uint(qb0 * rb0),
+                                            __float_as_uint(qa1 * ra1), __float_as_uint(qb1 * rb1)};
+                    const uint32_t b00 = __float_as_uint(ka0 * ca0), b01 = __float_as_uint(ka1 * ca1);  // column token g
+                    const uint32_t b10 = __float_as_uint(kb0 * cb0), b11 = __float_as_uint(kb1 * cb1);  // column token g + 8
+                    tc::mma_16x8x8_tf32(accA[0], ak, b00, b01);
+                    tc::mma_16x8x8_tf32(accA[1], ak, b10, b11);
+                    tc::mma_16x8x8_tf32(accP[0], aq, b00, b01);
+                    tc::mma_16x8x8_tf32(accP[1], aq, b10, b11);
+                }
+                // column operand of the off-diagonal blocks: K e^{G_{J+1} - g_j} for this sub-chunk J = I
+                *reinterpret_cast<float2 *>(sm + P_KSIG + rowa + la_off) = make_float2(ka0 * sA[s][0], ka1 * sA[s][1]);
+                *reinterpret_cast<float2 *>(sm + P_KSIG + rowb + la_off) = make_float2(kb0 * sB[s][0], kb1 * sB[s][1]);
             }
-            float4 *px = reinterpret_cast<float4 *>(sm + P_PX) + ((half * 6 + pair_index(I, J)) * 32 + lane) * 4;
-            px[0] = make_float4(oA[0][0], oA[0][1], oA[0][2], oA[0][3]);
-            px[1] = make_float4(oA[1][0], oA[1][1], oA[1][2], oA[1][3]);
-            px[2] = make_float4(oP[0][0], oP[0][1], oP[0][2], oP[0][3]);
-            px[3] = make_float4(oP[1][0], oP[1][1], oP[1][2], oP[1][3]);
-        }
-        fence_proxy_async_smem();   // Ks and the staged Qs, Kb reach the async proxy
-        __syncthreads();
 
-        if (tid == 0 && !aborted(ctl)) {
-            tc::bulk_store_global(gs + SL_QW, st + ST_QS, 8192);                 // Qs, K-block 0
-            tc::bulk_store_global(gs + SL_QW + kQWBlk, st + ST_QS + 8192, 8192); // Qs, K-block 1
-            tc::bulk_store_global(gs + SL_KB, sm + P_KBS, 16384);                // Kb
-            tc::bulk_commit();
-        }
-        const float ba = beta_s[ta], bb = beta_s[tb];
-        if (half == 0) {
-            // diagonal blocks of A (times beta, strictly lower) and P (lower), both channel halves summed
-            const float4 *dx = reinterpret_cast<const float4 *>(sm + P_DX) + (I * 32 + lane) * 4;
-            const float4 x0 = dx[0], x1 = dx[1], x2 = dx[2], x3 = dx[3];
-            accA[0][0] += x0.x; accA[0][1] += x0.y; accA[0][2] += x0.z; accA[0][3] += x0.w;
-            accA[1][0] += x1.x; accA[1][1] += x1.y; accA[1][2] += x1.z; accA[1][3] += x1.w;
-            accP[0][0] += x2.x; accP[0][1] += x2.y; accP[0][2] += x2.z; accP[0][3] += x2.w;
-            accP[1][0] += x3.x; accP[1][1] += x3.y; accP[1][2] += x3.z; accP[1][3] += x3.w;
-#pragma unroll
-            for (int nt = 0; nt < 2; ++nt) {
-                const int jl = 8 * nt + 2 * t4, j = 16 * I + jl;
-                *reinterpret_cast<float2 *>(Af + ta * kLD + j) =
-                    make_float2(jl < g ? ba * accA[nt][0] : 0.f, jl + 1 < g ? ba * accA[nt][1] : 0.f);
-                *reinterpret_cast<float2 *>(Af + tb * kLD + j) =
-                    make_float2(jl < g + 8 ? bb * accA[nt][2] : 0.f, jl + 1 < g + 8 ? bb * accA[nt][3] : 0.f);
-                *reinterpret_cast<uint32_t *>(st + ST_PT + sw128k_off(ta, j, 0)) =
-                    pack_f16(jl <= g ? accP[nt][0] : 0.f, jl + 1 <= g ? accP[nt][1] : 0.f);
-                *reinterpret_cast<uint32_t *>(st + ST_PT + sw128k_off(tb, j, 0)) =
-                    pack_f16(jl <= g + 8 ? accP[nt][2] : 0.f, jl + 1 <= g + 8 ? accP[nt][3] : 0.f);
+            publish();   // the previous image (its stores have had phases 1a and 1b to land)
+            if (tid == 0 && img >= kRingDepth) wait_cluster(bar_loaded + rb, ((img / kRingDepth) - 1) & 1, ctl);
+            cp_async_wait_prev();   // this image's beta (all but the group just issued)
+            __syncthreads();   // the inputs and g^L are dead; every thread has read the flag
+            if (tid == 0) {   // for the next image
+                *reinterpret_cast<volatile int *>(vec + V_FLAG) = 0;
+                *reinterpret_cast<volatile int *>(vec + V_SLOW) = 0;
             }
-        } else {
-            // off-diagonal blocks (I, J) of A and P, both channel halves summed
+
+            // ------------------------------------------------ phase 2: chunk-level factors
+            // (products of the sub-chunks' e^{tot}: e^{G_I}, e^{g_C - G_{I+1}}) and the off-diagonal blocks
+            if (half == 1) {   // diagonal partials of channels 64..127 for the half-0 warp of sub-chunk I
+                float4 *dx = reinterpret_cast<float4 *>(sm + P_DX) + (I * 32 + lane) * 4;
+                dx[0] = make_float4(accA[0][0], accA[0][1], accA[0][2], accA[0][3]);
+                dx[1] = make_float4(accA[1][0], accA[1][1], accA[1][2], accA[1][3]);
+                dx[2] = make_float4(accP[0][0], accP[0][1], accP[0][2], accP[0][3]);
+                dx[3] = make_float4(accP[1][0], accP[1][1], accP[1][2], accP[1][3]);
+            }
+            const uint32_t row_a = half * 8192u + (ta >> 3) * 1024u + g * 128u + 4u * t4;   // token a, no swizzle term
+    #pragma unroll
+            for (int s = 0; s < 8; ++s) {
+                const int c0 = 64 * half + 8 * s + 2 * t4;
+                float2 pj[4];   // e^{tot_J} of the four sub-chunks
+    #pragma unroll
+                for (int J = 0; J < 4; ++J) pj[J] = *reinterpret_cast<const float2 *>(vec + V_P + J * 128 + c0);
+                float eG0 = 1.f, eG1 = 1.f, eK0 = 1.f, eK1 = 1.f;
+    #pragma unroll
+                for (int J = 0; J < 4; ++J) {
+                    if (J < I) { eG0 *= pj[J].x; eG1 *= pj[J].y; }
+                    if (J > I) { eK0 *= pj[J].x; eK1 *= pj[J].y; }
+                }
+                const float qa0 = tc::bf16_lo(qA[s]) * nqa, qa1 = tc::bf16_hi(qA[s]) * nqa;
+                const float qb0 = tc::bf16_lo(qB[s]) * nqb, qb1 = tc::bf16_hi(qB[s]) * nqb;
+                const float ka0 = tc::bf16_lo(kA[s]) * nka, ka1 = tc::bf16_hi(kA[s]) * nka;
+                const float kb0 = tc::bf16_lo(kB[s]) * nkb, kb1 = tc::bf16_hi(kB[s]) * nkb;
+                const float fa0 = rA[s][0] * eG0, fa1 = rA[s][1] * eG1, fb0 = rB[s][0] * eG0, fb1 = rB[s][1] * eG1;
+                // Qs = Q e^{g} and Kb = K e^{g_C - g} (staged for the ring slot), Ks = K e^{g} into
+                // [Ks | V]; all three are [token][channel] tiles of 64-channel K-blocks 8 KB apart in
+                // the 128-byte swizzle
+                const uint32_t oa = row_a + (((s ^ g) & 7) << 4), ob = oa + 1024;
+                *reinterpret_cast<uint32_t *>(st + ST_QS + oa) = pack_f16(qa0 * fa0, qa1 * fa1);
+                *reinterpret_cast<uint32_t *>(st + ST_QS + ob) = pack_f16(qb0 * fb0, qb1 * fb1);
+                *reinterpret_cast<uint32_t *>(sm + P_KSV + oa) = pack_f16(ka0 * fa0, ka1 * fa1);
+                *reinterpret_cast<uint32_t *>(sm + P_KSV + ob) = pack_f16(kb0 * fb0, kb1 * fb1);
+                *reinterpret_cast<uint32_t *>(sm + P_KBS + oa) = pack_f16(ka0 * sA[s][0] * eK0, ka1 * sA[s][1] * eK1);
+                *reinterpret_cast<uint32_t *>(sm + P_KBS + ob) = pack_f16(kb0 * sB[s][0] * eK0, kb1 * sB[s][1] * eK1);
+                if (I == 0 && g == 0)
+                    *reinterpret_cast<float2 *>(gs + SL_GAM + 4 * c0) =
+                        make_float2(pj[0].x * pj[1].x * pj[2].x * pj[3].x, pj[0].y * pj[1].y * pj[2].y * pj[3].y);
+            }
+            // Off-diagonal blocks (I, J), J < I, over this warp's 64 channels:
+            //   A^o += [K e^{g - G_I} Diag(e^{G_I - G_{J+1}})] (K e^{G_{J+1} - g})^T, P^o likewise with Q;
+            // partials of both channel halves go to shared memory, summed by the half-1 warp below.
             for (int J = 0; J < I; ++J) {
-                const float4 *p0 = reinterpret_cast<const float4 *>(sm + P_PX) + (pair_index(I, J) * 32 + lane) * 4;
-                const float4 *p1 = p0 + 6 * 32 * 4;
-#pragma unroll
+                float oA[2][4] = {}, oP[2][4] = {};
+    #pragma unroll
+                for (int s = 0; s < 8; ++s) {
+                    const int c0 = 64 * half + 8 * s + 2 * t4;
+                    float D0 = 1.f, D1 = 1.f;   // e^{G_I - G_{J+1}}: the sub-chunks strictly between J and I
+    #pragma unroll
+                    for (int Jm = 1; Jm < 3; ++Jm)
+                        if (Jm > J && Jm < I) {
+                            const float2 pm = *reinterpret_cast<const float2 *>(vec + V_P + Jm * 128 + c0);
+                            D0 *= pm.x;
+                            D1 *= pm.y;
+                        }
+                    const float ra0 = rA[s][0] * D0, ra1 = rA[s][1] * D1, rb0 = rB[s][0] * D0, rb1 = rB[s][1] * D1;
+                    const uint32_t ak[4] = {__float_as_uint(tc::bf16_lo(kA[s]) * nka * ra0), __float_as_uint(tc::bf16_lo(kB[s]) * nkb * rb0),
+                                            __float_as_uint(tc::bf16_hi(kA[s]) * nka * ra1), __float_as_uint(tc::bf16_hi(kB[s]) * nkb * rb1)};
+                    const uint32_t aq[4] = {__float_as_uint(tc::bf16_lo(qA[s]) * nqa * ra0), __float_as_uint(tc::bf16_lo(qB[s]) * nqb * rb0),
+                                            __float_as_uint(tc::bf16_hi(qA[s]) * nqa * ra1), __float_as_uint(tc::bf16_hi(qB[s]) * nqb * rb1)};
+                    const uint32_t la_off = (c0 >> 5) * kBoxBytes + (((((c0 & 31) >> 2) ^ g) & 7) << 4) + 8 * (t4 & 1);
+                    const uint32_t rj = static_cast<uint32_t>(16 * J + g) * 128u;   // column token g of sub-chunk J
+                    const float2 y0 = *reinterpret_cast<const float2 *>(sm + P_KSIG + rj + la_off);
+                    const float2 y1 = *reinterpret_cast<const float2 *>(sm + P_KSIG + rj + 1024 + la_off);  // token g + 8
+                    tc::mma_16x8x8_tf32(oA[0], ak, __float_as_uint(y0.x), __float_as_uint(y0.y));
+                    tc::mma_16x8x8_tf32(oA[1], ak, __float_as_uint(y1.x), __float_as_uint(y1.y));
+                    tc::mma_16x8x8_tf32(oP[0], aq, __float_as_uint(y0.x), __float_as_uint(y0.y));
+                    tc::mma_16x8x8_tf32(oP[1], aq, __float_as_uint(y1.x), __float_as_uint(y1.y));
+                }
+                float4 *px = reinterpret_cast<float4 *>(sm + P_PX) + ((half * 6 + pair_index(I, J)) * 32 + lane) * 4;
+                px[0] = make_float4(oA[0][0], oA[0][1], oA[0][2], oA[0][3]);
+                px[1] = make_float4(oA[1][0], oA[1][1], oA[1][2], oA[1][3]);
+                px[2] = make_float4(oP[0][0], oP[0][1], oP[0][2], oP[0][3]);
+                px[3] = make_float4(oP[1][0], oP[1][1], oP[1][2], oP[1][3]);
+            }
+            fence_proxy_async_smem();   // Ks, and the staged Qs and Kb, reach the async proxy
+            __syncthreads();
+            if (tid == kStorer) {   // warp 7 (sub-chunk 0, channel half 1) has no share of the combine
+                store_part(gs + SL_QW, st + ST_QS, 8192);                 // Qs, K-block 0
+                store_part(gs + SL_QW + kQWBlk, st + ST_QS + 8192, 8192); // Qs, K-block 1
+                store_part(gs + SL_KB, sm + P_KBS, 16384);                // Kb
+                tc::bulk_commit();
+            }
+            const float ba = beta_s[ta], bb = beta_s[tb];
+            if (half == 0) {
+                // diagonal blocks of A (times beta, strictly lower) and P (lower), both channel halves summed
+                const float4 *dx = reinterpret_cast<const float4 *>(sm + P_DX) + (I * 32 + lane) * 4;
+                const float4 x0 = dx[0], x1 = dx[1], x2 = dx[2], x3 = dx[3];
+                accA[0][0] += x0.x; accA[0][1] += x0.y; accA[0][2] += x0.z; accA[0][3] += x0.w;
+                accA[1][0] += x1.x; accA[1][1] += x1.y; accA[1][2] += x1.z; accA[1][3] += x1.w;
+                accP[0][0] += x2.x; accP[0][1] += x2.y; accP[0][2] += x2.z; accP[0][3] += x2.w;
+                accP[1][0] += x3.x; accP[1][1] += x3.y; accP[1][2] += x3.z; accP[1][3] += x3.w;
+    #pragma unroll
                 for (int nt = 0; nt < 2; ++nt) {
-                    const float4 a0 = p0[nt], a1 = p1[nt], q0 = p0[2 + nt], q1 = p1[2 + nt];
-                    const int j = 16 * J + 8 * nt + 2 * t4;
-                    *reinterpret_cast<float2 *>(Af + ta * kLD + j) = make_float2(ba * (a0.x + a1.x), ba * (a0.y + a1.y));
-                    *reinterpret_cast<float2 *>(Af + tb * kLD + j) = make_float2(bb * (a0.z + a1.z), bb * (a0.w + a1.w));
-                    *reinterpret_cast<uint32_t *>(st + ST_PT + sw128k_off(ta, j, 0)) = pack_f16(q0.x + q1.x, q0.y + q1.y);
-                    *reinterpret_cast<uint32_t *>(st + ST_PT + sw128k_off(tb, j, 0)) = pack_f16(q0.z + q1.z, q0.w + q1.w);
+                    const int jl = 8 * nt + 2 * t4, j = 16 * I + jl;
+                    *reinterpret_cast<float2 *>(Af + ta * kLD + j) =
+                        make_float2(jl < g ? ba * accA[nt][0] : 0.f, jl + 1 < g ? ba * accA[nt][1] : 0.f);
+                    *reinterpret_cast<float2 *>(Af + tb * kLD + j) =
+                        make_float2(jl < g + 8 ? bb * accA[nt][2] : 0.f, jl + 1 < g + 8 ? bb * accA[nt][3] : 0.f);
+                    *reinterpret_cast<uint32_t *>(st + ST_PT + sw128k_off(ta, j, 0)) =
+                        pack_f16(jl <= g ? accP[nt][0] : 0.f, jl + 1 <= g ? accP[nt][1] : 0.f);
+                    *reinterpret_cast<uint32_t *>(st + ST_PT + sw128k_off(tb, j, 0)) =
+                        pack_f16(jl <= g + 8 ? accP[nt][2] : 0.f, jl + 1 <= g + 8 ? accP[nt][3] : 0.f);
+                }
+            } else {
+                // off-diagonal blocks (I, J) of A and P, both channel halves summed
+                for (int J = 0; J < I; ++J) {
+                    const float4 *p0 = reinterpret_cast<const float4 *>(sm + P_PX) + (pair_index(I, J) * 32 + lane) * 4;
+                    const float4 *p1 = p0 + 6 * 32 * 4;
+    #pragma unroll
+                    for (int nt = 0; nt < 2; ++nt) {
+                        const float4 a0 = p0[nt], a1 = p1[nt], q0 = p0[2 + nt], q1 = p1[2 + nt];
+                        const int j = 16 * J + 8 * nt + 2 * t4;
+                        *reinterpret_cast<float2 *>(Af + ta * kLD + j) = make_float2(ba * (a0.x + a1.x), ba * (a0.y + a1.y));
+                        *reinterpret_cast<float2 *>(Af + tb * kLD + j) = make_float2(bb * (a0.z + a1.z), bb * (a0.w + a1.w));
+                        *reinterpret_cast<uint32_t *>(st + ST_PT + sw128k_off(ta, j, 0)) = pack_f16(q0.x + q1.x, q0.y + q1.y);
+                        *reinterpret_cast<uint32_t *>(st + ST_PT + sw128k_off(tb, j, 0)) = pack_f16(q0.z + q1.z, q0.w + q1.w);
+                    }
                 }
             }
         }
         __syncthreads();
 
-        // ------------------------------------------------ UT solve, T (fp16)
-        ut::unit_lower_inverse(Af, Xf, tid);
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-            const int e = tid + u * kThreads;
-            const int i = e >> 5, j = (e & 31) * 2;
-            const float lo = j <= i ? Xf[i * kLD + j] * beta_s[j] : 0.f;
-            const float hi = j + 1 <= i ? Xf[i * kLD + j + 1] * beta_s[j + 1] : 0.f;
-            *reinterpret_cast<uint32_t *>(st + ST_PT + 8192 + sw128k_off(i, j, 0)) = pack_f16(lo, hi);
-        }
+        // ------------------------------------------------ UT solve; T = X Diag(beta) (fp16)
+        // written block by block as the solve finishes it
+        ut::unit_lower_inverse(Af, Xf, tid, TWriter{st + ST_PT + 8192, beta_s});
         fence_proxy_async_smem();
         __syncthreads();
-        // the input region (A, X) is dead until the next chunk: stage its inputs there
-        if (tid == 0) {
-            tc::bulk_wait_read_all();   // the staged Qs and Kb have left the input region
-            if (c + kProducers < nchunks) load_inputs(c + kProducers);
-            if (!aborted(ctl)) {
-                tc::bulk_store_global(gs + SL_PT, st + ST_PT, 16384);   // [P;T] to the ring slot
-                tc::bulk_commit();
-            }
-        }
 
         // ------------------------------------------------ [W | U'] = T [Ks | V] (fp16, N = 256)
         if (tid == 0 && !aborted(ctl)) {
@@ -673,20 +804,27 @@ __device__ void producer(uint8_t *sm, uint32_t tmem, int rank, uint8_t *ring,
             tc::mma_commit(bar_mma);
             pend_mma = true;
         }
+        // the input region (A, X) is dead until the next chunk: stage its inputs there
+        if (tid == kLoader && c + kProducers < nchunks) load_inputs(c + kProducers);
+        if (tid == kStorer) {
+            store_part(gs + SL_PT, st + ST_PT, 16384);   // [P;T], while the MMA runs
+            tc::bulk_commit();
+        }
         if (wait_local(bar_mma, ph_mma, ctl)) {
             ph_mma ^= 1;
             pend_mma = false;
         }
         tc_fence_after();
+        if (quad >= 2) {   // W (rows 64..127 of [Qs ; W]) and U', staged in their image layout
+            const int i = row - 64;
 #pragma unroll
-        for (int part = 0; part < 2; ++part) {   // part 0: W, part 1: U'
-            if (quad >= 2) {
-                const int i = row - 64;
+            for (int part = 0; part < 2; ++part) {   // part 0: W, part 1: U'
                 float w[64];
                 const uint32_t taddr = tc::tmem_addr(tmem, 32 * quad, PCOL_WU + part * 128 + half * 64);
                 tc::tmem_ld32(taddr, *reinterpret_cast<float(*)[32]>(&w[0]));
                 tc::tmem_ld32(taddr + 32, *reinterpret_cast<float(*)[32]>(&w[32]));
                 tc::tmem_wait_ld();
+                uint8_t *dst = sm + (part == 0 ? P_WS : P_US) + half * 8192;
 #pragma unroll
                 for (int u = 0; u < 64; u += 8) {
                     uint4 x;
@@ -694,49 +832,32 @@ __device__ void producer(uint8_t *sm, uint32_t tmem, int rank, uint8_t *ring,
                     x.y = pack_f16(w[u + 2], w[u + 3]);
                     x.z = pack_f16(w[u + 4], w[u + 5]);
                     x.w = pack_f16(w[u + 6], w[u + 7]);
-                    const int col = half * 64 + u;
-                    const uint32_t off = part == 0 ? ST_W + sw128k_off(i, col, 8192)
-                                                   : ST_UP + sw128k_off(i, col, kTokBlk);
-                    *reinterpret_cast<uint4 *>(st + off) = x;
-                }
-            }
-            fence_proxy_async_smem();
-            if (part == 0) {   // W leaves while U' is formed
-                __syncthreads();
-                if (tid == 0 && !aborted(ctl)) {
-                    tc::bulk_store_global(gs + SL_QW + 8192, st + ST_W, 8192);   // W, K-block 0
-                    tc::bulk_store_global(gs + SL_QW + kQWBlk + 8192, st + ST_W + 8192, 8192);
-                    tc::bulk_commit();
+                    *reinterpret_cast<uint4 *>(dst + sw128k_off(i, u, 0)) = x;
                 }
             }
         }
+        fence_proxy_async_smem();
         tc_fence_before();
+        if (tid == kStorer) tc::bulk_wait_read_all();   // the staged Qs has left ST_QS (= g^L)
         __syncthreads();
-
-        // ------------------------------------------------ publish the image through L2
-        // Every thread's generic stores into the slot (Qs, Kb, e^{g_C}) precede thread 0's
-        // release through the CTA barrier above; the release is cumulative.
-        if (tid == 0) {
-            if (!aborted(ctl)) {
-                tc::bulk_store_global(gs + SL_UP, st + ST_UP, 16384);                  // U'
-                tc::bulk_commit();
-            }
-            tc::bulk_wait_read_all();   // W and U' have left the stage
+        if (tid == kStorer) {
+            store_part(gs + SL_QW + 8192, sm + P_WS, 8192);                // W, K-block 0
+            store_part(gs + SL_QW + kQWBlk + 8192, sm + P_WS + 8192, 8192);
+            store_part(gs + SL_UP, sm + P_US, 16384);                      // U'
+            tc::bulk_commit();
         }
-        __syncthreads();   // the next image may now write g^L over the stage
-        // The "ready" of this image is sent once its stores have reached L2: during the next
-        // image's phase 1a (before that image issues stores of its own), or after the loop.
+        // Every thread's generic stores into the slot precede the storer's release through the
+        // CTA barriers (the release is cumulative). The "ready" of this image is sent once its
+        // bulk stores are complete: after the next image's phase 1b, or after the loop.
         pending = rb;
         pending_img = img;
         ++img;
     }
     publish();
     // drain: what this CTA issued and has not seen complete (all of it after a give-up)
-    if (tid == 0) {
-        if (pend_in) drain(bar_in, ph_in, ctl);
-        if (pend_mma) drain(bar_mma, ph_mma, ctl);
-        tc::bulk_wait_all();
-    }
+    if (tid == kLoader && pend_in) drain(bar_in, ph_in, ctl);
+    if (tid == 0 && pend_mma) drain(bar_mma, ph_mma, ctl);
+    if (tid == kStorer) tc::bulk_wait_all();
     asm volatile("cp.async.wait_all;" ::: "memory");
 }
 // ============================================================ consumer
@@ -964,9 +1085,7 @@ __device__ void consumer(uint8_t *sm, uint32_t tmem, const uint8_t *ring, const 
 
 template <bool kFused>
 __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 1)
-chunk_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                     const __grid_constant__ CUtensorMap tm_la, const __grid_constant__ CUtensorMap tm_v,
-                     const __grid_constant__ CUtensorMap tm_qs, const __grid_constant__ CUtensorMap tm_ks,
+chunk_cluster_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_qs, const __grid_constant__ CUtensorMap tm_ks,
                      const __grid_constant__ CUtensorMap tm_las, const float *__restrict__ beta,
                      const float *__restrict__ S0, __nv_bfloat16 *__restrict__ out,
                      float *__restrict__ S_T, uint8_t *__restrict__ ws, int T, int H, int *err,
@@ -1009,8 +1128,8 @@ chunk_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     if (is_consumer)
         consumer(sm, tmem, ring, S0, out, S_T, T, H, h, bh, ztok, nchunks, ctl);
     else
-        producer<kFused>(sm, tmem, rank, ring, &tm_q, &tm_k, &tm_la, &tm_v, &tm_qs, &tm_ks, &tm_las, beta, T,
-                 H, h, ztok, nchunks, ctl, test_timeout);
+        producer<kFused>(sm, tmem, rank, ring, &tm_v, &tm_qs, &tm_ks, &tm_las, beta, T, H, h, ztok, nchunks,
+                         ctl, test_timeout);
 
     tc_fence_before();
     __syncthreads();
@@ -1076,15 +1195,12 @@ cudaError_t launch_chunk_cluster(const ChunkArgs &a, cudaStream_t s) {
     const long tokens = static_cast<long>(a.B) * a.T;
     const CUtensorMapDataType kB16 = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, kF32 = CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
     const bool fused = a.gate != nullptr;   // the layer prologue: gate pre-activation instead of log alpha
-    CUtensorMap mq, mk, mla, mv, mqs, mks, mlas;
+    CUtensorMap mv, mqs, mks, mlas;
     const bool ok =
-        make_map(&mq, a.q, kB16, 2, a.H, tokens, false) && make_map(&mk, a.k, kB16, 2, a.H, tokens, false) &&
         make_map(&mv, a.v, kB16, 2, a.H, tokens, false) &&
         make_map(&mqs, a.q, kB16, 2, a.H, tokens, true) && make_map(&mks, a.k, kB16, 2, a.H, tokens, true) &&
-        (fused ? make_map(&mla, a.gate, kB16, 2, a.H, tokens, false) &&
-                     make_map(&mlas, a.gate, kB16, 2, a.H, tokens, true)
-               : make_map(&mla, a.log_alpha, kF32, 4, a.H, tokens, false) &&
-                     make_map(&mlas, a.log_alpha, kF32, 4, a.H, tokens, true));
+        (fused ? make_map(&mlas, a.gate, kB16, 2, a.H, tokens, true)
+               : make_map(&mlas, a.log_alpha, kF32, 4, a.H, tokens, true));
     if (!ok) return cudaErrorInvalidValue;
     auto kern = fused ? chunk_cluster_kernel<true> : chunk_cluster_kernel<false>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1092,7 +1208,7 @@ cudaError_t launch_chunk_cluster(const ChunkArgs &a, cudaStream_t s) {
     if (e != cudaSuccess) return e;
     const dim3 grid(static_cast<unsigned>(a.B) * a.H * kCluster);
     kern<<<grid, kThreads, kSmemBytes, s>>>(
-        mq, mk, mla, mv, mqs, mks, mlas, a.beta, a.S0, static_cast<__nv_bfloat16 *>(a.out), a.S_T,
+        mv, mqs, mks, mlas, a.beta, a.S0, static_cast<__nv_bfloat16 *>(a.out), a.S_T,
         static_cast<uint8_t *>(a.workspace), a.T, a.H, a.device_error, g_test_timeout);
     return cudaGetLastError();
 }

@@ -13,13 +13,20 @@ namespace ut {
 constexpr int kLD = 68;  // row stride (floats) of A and X: conflict-free mma fragments
 
 // X = (I + A)^{-1} for the strictly lower-triangular 64x64 A (row stride kLD),
-// organised in 16x16 blocks:
+// organised in 16x16 blocks, and every finished block handed to `out` as well
+// (the caller forms T = X Diag(beta) from it):
 //   1) X_II = (I + A_II)^{-1} for the 4 diagonal blocks: forward substitution,
 //      one column per thread, fp32.
-//   2) R_IJ = A_IJ X_JJ for the 6 blocks below the diagonal (one warp each).
-//   3) block column J, one warp each, top to bottom:
-//      X_IJ = -X_II (R_IJ + sum_{J<K<I} A_IK X_KJ).
+//   2) R_IJ = A_IJ X_JJ for the 6 blocks below the diagonal (one warp each); the
+//      three next to the diagonal finish at once: X_{I,I-1} = -X_II R_{I,I-1}.
+//   3) X_20 = -X_22 (R_20 + A_21 X_10), X_31 = -X_33 (R_31 + A_32 X_21), and the
+//      first two terms of X_30's sum, R_30 + A_31 X_10.
+//   4) X_30 = -X_33 (R_30 + A_31 X_10 + A_32 X_20).
+// Three dependent levels of two block products each after the diagonal blocks.
 // Block products use warp-level tf32 mma.sync (m16n8k8, fp32 accumulate).
+// `out.one(i, j, x)` receives single elements of the diagonal blocks (all of
+// them, zeros above the diagonal included); `out.pair(i, j, x0, x1)` receives
+// elements (i, j), (i, j + 1) of the blocks below the diagonal, j even.
 
 __device__ __forceinline__ uint32_t to_tf32(float x) {
     uint32_t r;
@@ -77,7 +84,31 @@ __device__ __forceinline__ const float *blk(const float *M, int I, int J) {
 }
 __device__ __forceinline__ float *blk(float *M, int I, int J) { return M + 16 * I * kLD + 16 * J; }
 
-__device__ inline void unit_lower_inverse(const float *A, float *X, int tid) {
+template <class Out>
+__device__ __forceinline__ void acc_emit16(const float (&acc)[2][4], int I, int J, int lane, const Out &out) {
+    const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+    for (int ns = 0; ns < 2; ++ns) {
+        out.pair(16 * I + g, 16 * J + 8 * ns + 2 * t, acc[ns][0], acc[ns][1]);
+        out.pair(16 * I + g + 8, 16 * J + 8 * ns + 2 * t, acc[ns][2], acc[ns][3]);
+    }
+}
+// X_IJ = -X_II Y with Y = X's (I, J) block on entry; the result replaces Y (one warp).
+template <class Out>
+__device__ __forceinline__ void finish_block(float *X, int I, int J, int lane, const Out &out) {
+    float r[2][4] = {};
+    warp_mm16(r, blk(X, I, I), blk(X, I, J), lane);
+#pragma unroll
+    for (int ns = 0; ns < 2; ++ns)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) r[ns][e] = -r[ns][e];
+    __syncwarp();
+    acc_store16(r, blk(X, I, J), 1.f, lane);
+    acc_emit16(r, I, J, lane, out);
+}
+
+template <class Out>
+__device__ inline void unit_lower_inverse(const float *A, float *X, int tid, const Out &out) {
     const int warp = tid >> 5, lane = tid & 31;
     // 1) diagonal blocks, one column per thread
     if (tid < 64) {
@@ -94,36 +125,51 @@ __device__ inline void unit_lower_inverse(const float *A, float *X, int tid) {
             x[i] = i < jj ? 0.f : (i == jj ? 1.f : -(s0 + s1));
         }
 #pragma unroll
-        for (int i = 0; i < 16; ++i) X[(base + i) * kLD + base + jj] = x[i];
-    }
-    __syncthreads();
-    // 2) R_IJ = A_IJ X_JJ, stored in X's (I,J) block; warps 0..5
-    if (warp < 6) {
-        const int I = warp < 3 ? warp + 1 : (warp < 5 ? warp - 1 : 3);  // 1,2,3,2,3,3
-        const int J = warp < 3 ? 0 : (warp < 5 ? 1 : 2);                // 0,0,0,1,1,2
-        float acc[2][4] = {};
-        warp_mm16(acc, blk(A, I, J), blk(X, J, J), lane);
-        acc_store16(acc, blk(X, I, J), 1.f, lane);
-    }
-    __syncthreads();
-    // 3) block column J = warp (0..2), top to bottom
-    if (warp < 3) {
-        const int J = warp;
-        for (int I = J + 1; I < 4; ++I) {
-            float acc[2][4];
-            acc_load16(acc, blk(X, I, J), lane);  // R_IJ
-            for (int K = J + 1; K < I; ++K) warp_mm16(acc, blk(A, I, K), blk(X, K, J), lane);
-            __syncwarp();
-            acc_store16(acc, blk(X, I, J), 1.f, lane);  // Y
-            __syncwarp();
-            float out[2][4] = {};
-            warp_mm16(out, blk(X, I, I), blk(X, I, J), lane);
-            __syncwarp();
-            acc_store16(out, blk(X, I, J), -1.f, lane);
-            __syncwarp();
+        for (int i = 0; i < 16; ++i) {
+            X[(base + i) * kLD + base + jj] = x[i];
+            out.one(base + i, base + jj, x[i]);
         }
     }
     __syncthreads();
+    // 2) warps 0..2: blocks (1,0), (2,1), (3,2), finished; warps 3..5: R_20, R_31, R_30
+    if (warp < 6) {
+        const int I = warp < 3 ? warp + 1 : (warp == 5 ? 3 : warp - 1);   // 1,2,3,2,3,3
+        const int J = warp < 3 ? warp : (warp == 5 ? 0 : warp - 3);        // 0,1,2,0,1,0
+        float acc[2][4] = {};
+        warp_mm16(acc, blk(A, I, J), blk(X, J, J), lane);
+        acc_store16(acc, blk(X, I, J), 1.f, lane);
+        if (warp < 3) {
+            __syncwarp();
+            finish_block(X, I, J, lane, out);
+        }
+    }
+    __syncthreads();
+    // 3) warp 0: X_20; warp 1: X_31; warp 2: R_30 + A_31 X_10
+    if (warp < 3) {
+        const int I = warp == 1 ? 3 : (warp == 0 ? 2 : 3);
+        const int J = warp == 1 ? 1 : 0;
+        const int K = warp == 1 ? 2 : 1;   // the finished block X_KJ this step adds: A_IK X_KJ
+        float acc[2][4];
+        acc_load16(acc, blk(X, I, J), lane);
+        warp_mm16(acc, blk(A, I, K), blk(X, K, J), lane);
+        __syncwarp();
+        acc_store16(acc, blk(X, I, J), 1.f, lane);
+        if (warp < 2) {
+            __syncwarp();
+            finish_block(X, I, J, lane, out);
+        }
+    }
+    __syncthreads();
+    // 4) warp 0: X_30
+    if (warp == 0) {
+        float acc[2][4];
+        acc_load16(acc, blk(X, 3, 0), lane);
+        warp_mm16(acc, blk(A, 3, 2), blk(X, 2, 0), lane);
+        __syncwarp();
+        acc_store16(acc, blk(X, 3, 0), 1.f, lane);
+        __syncwarp();
+        finish_block(X, 3, 0, lane, out);
+    }
 }
 
 }  // namespace ut

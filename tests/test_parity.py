@@ -165,6 +165,33 @@ def test_fp32_strong_decay(chunk):
     compare(inp, out, st, *ref)
 
 
+@pytest.mark.parametrize("T", [64 * 7 + 5, 64 * 12])
+def test_bf16_decay_changes_from_chunk_to_chunk(T):
+    """The gate's range changes from one 64-token chunk to the next, so that an engine
+    that picks its factorisation per chunk switches inside one head: softplus gates;
+    log a = -2.49 on every channel (a 16-token sub-chunk decays by e^-39.8 and the chunk by
+    e^-159); the strong recipe; log a = -2.6 on every other channel (sub-chunks just past
+    e^-40); uniform -30."""
+    inp = I.prefill_inputs("prefill_4k", B=2, T=T, H=3, s0_std=0.05)
+    strong = I.prefill_inputs("prefill_4k", B=2, T=T, H=3, gate="strong")["log_alpha"]
+    la = inp["log_alpha"]
+    for c in range((T + 63) // 64):
+        sl = slice(64 * c, 64 * (c + 1))
+        kind = c % 5
+        if kind == 1:
+            la[:, sl] = -2.49
+        elif kind == 2:
+            la[:, sl] = strong[:, sl]
+        elif kind == 3:
+            la[:, sl, :, 0::2] = -2.6
+        elif kind == 4:
+            la[:, sl] = -30.0
+    ref = run_oracle(inp)
+    for eng in engines(torch.bfloat16, 128, 128, 64):
+        out, st = run_gpu(inp, 64, eng)
+        compare(inp, out, st, *ref)
+
+
 def test_bf16_uniform_extreme_decay():
     """Every channel at log a = -30 (a ~ 1e-13): the state keeps only the last token."""
     inp = I.prefill_inputs("prefill_4k", B=1, T=150, H=2, s0_std=0.05)
