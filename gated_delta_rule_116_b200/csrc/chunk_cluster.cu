@@ -369,19 +369,19 @@ __device__ void producer(uint8_t *sm, uint32_t tmem, int rank, uint8_t *ring,
         }
 
         load_beta(c + kProducers, (img + 1) & 1);   // the next image's beta, one image ahead
-        {   // V -> fp16 columns 128..255 of the [Ks | V] operand (read by [W | U'] only)
-            const int t = tid >> 2, piece = tid & 3;
-            const uint4 *src = reinterpret_cast<const uint4 *>(sm + (kFused ? P_IN_VF : P_IN_V) + t * 256 + 64 * piece);
+        {   // V -> fp16 columns 128..255 of the [Ks | V] operand (read by [W | U'] only); 16-byte
+            // piece e = tid + 256 m of the [64][128] bf16 tile, so a warp reads 512 contiguous bytes
+            const uint4 *src = reinterpret_cast<const uint4 *>(sm + (kFused ? P_IN_VF : P_IN_V));
 #pragma unroll
             for (int m = 0; m < 4; ++m) {
-                const uint4 vin = t < valid ? src[m] : make_uint4(0, 0, 0, 0);
+                const int e = tid + m * kThreads, t = e >> 4;
+                const uint4 vin = t < valid ? src[e] : make_uint4(0, 0, 0, 0);
                 uint4 w;
                 w.x = pack_f16(tc::bf16_lo(vin.x), tc::bf16_hi(vin.x));
                 w.y = pack_f16(tc::bf16_lo(vin.y), tc::bf16_hi(vin.y));
                 w.z = pack_f16(tc::bf16_lo(vin.z), tc::bf16_hi(vin.z));
                 w.w = pack_f16(tc::bf16_lo(vin.w), tc::bf16_hi(vin.w));
-                *reinterpret_cast<uint4 *>(sm + P_KSV + 2 * kTokBlk +
-                                           sw128k_off(t, 32 * piece + 8 * m, kTokBlk)) = w;
+                *reinterpret_cast<uint4 *>(sm + P_KSV + 2 * kTokBlk + sw128k_off(t, (e & 15) * 8, kTokBlk)) = w;
             }
         }
 

@@ -14,16 +14,19 @@ constexpr int kLD = 68;  // row stride (floats) of A and X: conflict-free mma fr
 
 // X = (I + A)^{-1} for the strictly lower-triangular 64x64 A (row stride kLD),
 // organised in 16x16 blocks, and every finished block handed to `out` as well
-// (the caller forms T = X Diag(beta) from it):
-//   1) X_II = (I + A_II)^{-1} for the 4 diagonal blocks: forward substitution,
-//      one column per thread, fp32.
-//   2) R_IJ = A_IJ X_JJ for the 6 blocks below the diagonal (one warp each); the
-//      three next to the diagonal finish at once: X_{I,I-1} = -X_II R_{I,I-1}.
-//   3) X_20 = -X_22 (R_20 + A_21 X_10), X_31 = -X_33 (R_31 + A_32 X_21), and the
-//      first two terms of X_30's sum, R_30 + A_31 X_10.
-//   4) X_30 = -X_33 (R_30 + A_31 X_10 + A_32 X_20).
-// Three dependent levels of two block products each after the diagonal blocks.
-// Block products use warp-level tf32 mma.sync (m16n8k8, fp32 accumulate).
+// (the caller forms T = X Diag(beta) from it). With N_IJ = X_II A_IJ, block
+// forward substitution reads X_IJ = -sum_{J<=K<I} N_IK X_KJ:
+//   1) X_II = (I + A_II)^{-1} for the 4 diagonal blocks, one column per thread,
+//      fp32, in 8x8 halves (forward substitution inside each half, then the
+//      lower-left half as -X_11 A_10 X_00).
+//   2) one warp per block below the diagonal: N_IJ (kept in A's (I,J) block),
+//      then -N_IJ X_JJ, which is X_IJ itself next to the diagonal (J = I-1)
+//      and the first term of X_20, X_31, X_30 otherwise.
+//   3) X_20 -= N_21 X_10, X_31 -= N_32 X_21, X_30 -= N_31 X_10.
+//   4) X_30 -= N_32 X_20.
+// Four dependent block products after the diagonal blocks. Block products use
+// warp-level tf32 mma.sync (m16n8k8, fp32 accumulate). The solve overwrites
+// A's blocks below the diagonal.
 // `out.one(i, j, x)` receives single elements of the diagonal blocks (all of
 // them, zeros above the diagonal included); `out.pair(i, j, x0, x1)` receives
 // elements (i, j), (i, j + 1) of the blocks below the diagonal, j even.
@@ -93,82 +96,110 @@ __device__ __forceinline__ void acc_emit16(const float (&acc)[2][4], int I, int 
         out.pair(16 * I + g + 8, 16 * J + 8 * ns + 2 * t, acc[ns][2], acc[ns][3]);
     }
 }
-// X_IJ = -X_II Y with Y = X's (I, J) block on entry; the result replaces Y (one warp).
 template <class Out>
-__device__ __forceinline__ void finish_block(float *X, int I, int J, int lane, const Out &out) {
-    float r[2][4] = {};
-    warp_mm16(r, blk(X, I, I), blk(X, I, J), lane);
-#pragma unroll
-    for (int ns = 0; ns < 2; ++ns)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) r[ns][e] = -r[ns][e];
-    __syncwarp();
-    acc_store16(r, blk(X, I, J), 1.f, lane);
-    acc_emit16(r, I, J, lane, out);
-}
-
-template <class Out>
-__device__ inline void unit_lower_inverse(const float *A, float *X, int tid, const Out &out) {
+__device__ inline void unit_lower_inverse(float *A, float *X, int tid, const Out &out) {
     const int warp = tid >> 5, lane = tid & 31;
-    // 1) diagonal blocks, one column per thread
+    // 1) diagonal blocks, one column per thread, each in 8x8 halves: the column's own
+    //    8x8 diagonal sub-block by forward substitution, then (columns 0..7) the rows
+    //    below it as -X_11 (A_10 x) with the neighbour columns' X_11 from shared memory
     if (tid < 64) {
-        const int I = tid >> 4, jj = tid & 15, base = 16 * I;
-        float x[16];
+        const int I = tid >> 4, jj = tid & 15, base = 16 * I, lo = jj & 8;
+        const float *Ab = A + base * kLD + base;
+        float *Xb = X + base * kLD + base;
+        float xa[8];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
+        for (int r = 0; r < 8; ++r) {
+            const int i = lo + r;
             float s0 = 0.f, s1 = 0.f;
 #pragma unroll
-            for (int m = 0; m < i; ++m) {
-                if (m & 1) s1 = fmaf(A[(base + i) * kLD + base + m], x[m], s1);
-                else s0 = fmaf(A[(base + i) * kLD + base + m], x[m], s0);
+            for (int m = 0; m < r; ++m) {
+                const float a = Ab[i * kLD + lo + m];
+                if (m & 1) s1 = fmaf(a, xa[m], s1);
+                else s0 = fmaf(a, xa[m], s0);
             }
-            x[i] = i < jj ? 0.f : (i == jj ? 1.f : -(s0 + s1));
+            xa[r] = i < jj ? 0.f : (i == jj ? 1.f : -(s0 + s1));
         }
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            X[(base + i) * kLD + base + jj] = x[i];
-            out.one(base + i, base + jj, x[i]);
+        for (int r = 0; r < 8; ++r) {
+            Xb[(lo + r) * kLD + jj] = xa[r];
+            out.one(base + lo + r, base + jj, xa[r]);
+        }
+        __syncwarp();
+        if (jj < 8) {
+            float y[8];
+#pragma unroll
+            for (int r = 0; r < 8; ++r) {
+                float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+                for (int m = 0; m < 8; m += 2) {
+                    s0 = fmaf(Ab[(8 + r) * kLD + m], xa[m], s0);
+                    s1 = fmaf(Ab[(8 + r) * kLD + m + 1], xa[m + 1], s1);
+                }
+                y[r] = s0 + s1;
+            }
+#pragma unroll
+            for (int r = 0; r < 8; ++r) {
+                float z = 0.f;
+#pragma unroll
+                for (int m = 0; m <= r; ++m) z = fmaf(Xb[(8 + r) * kLD + 8 + m], y[m], z);
+                Xb[(8 + r) * kLD + jj] = -z;
+                out.one(base + 8 + r, base + jj, -z);
+            }
+        } else {
+#pragma unroll
+            for (int r = 0; r < 8; ++r) {   // rows 0..7 of columns 8..15
+                Xb[r * kLD + jj] = 0.f;
+                out.one(base + r, base + jj, 0.f);
+            }
         }
     }
     __syncthreads();
-    // 2) warps 0..2: blocks (1,0), (2,1), (3,2), finished; warps 3..5: R_20, R_31, R_30
+    // 2) warps 0..5 take blocks (1,0), (2,1), (3,2), (2,0), (3,1), (3,0)
     if (warp < 6) {
-        const int I = warp < 3 ? warp + 1 : (warp == 5 ? 3 : warp - 1);   // 1,2,3,2,3,3
-        const int J = warp < 3 ? warp : (warp == 5 ? 0 : warp - 3);        // 0,1,2,0,1,0
-        float acc[2][4] = {};
-        warp_mm16(acc, blk(A, I, J), blk(X, J, J), lane);
-        acc_store16(acc, blk(X, I, J), 1.f, lane);
+        const int I = warp < 3 ? warp + 1 : (warp == 5 ? 3 : warp - 1);
+        const int J = warp < 3 ? warp : (warp == 5 ? 0 : warp - 3);
+        float n[2][4] = {};
+        warp_mm16(n, blk(X, I, I), blk(A, I, J), lane);   // N_IJ = X_II A_IJ
+        __syncwarp();
+        acc_store16(n, blk(A, I, J), 1.f, lane);
+        __syncwarp();
+        float y[2][4] = {};
+        warp_mm16(y, blk(A, I, J), blk(X, J, J), lane);   // N_IJ X_JJ
+        acc_store16(y, blk(X, I, J), -1.f, lane);
         if (warp < 3) {
-            __syncwarp();
-            finish_block(X, I, J, lane, out);
+#pragma unroll
+            for (int ns = 0; ns < 2; ++ns)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) y[ns][e] = -y[ns][e];
+            acc_emit16(y, I, J, lane, out);
         }
     }
     __syncthreads();
-    // 3) warp 0: X_20; warp 1: X_31; warp 2: R_30 + A_31 X_10
+    // 3) warp 0: X_20 -= N_21 X_10; warp 1: X_31 -= N_32 X_21; warp 2: X_30 -= N_31 X_10
     if (warp < 3) {
-        const int I = warp == 1 ? 3 : (warp == 0 ? 2 : 3);
-        const int J = warp == 1 ? 1 : 0;
-        const int K = warp == 1 ? 2 : 1;   // the finished block X_KJ this step adds: A_IK X_KJ
-        float acc[2][4];
+        const int I = warp == 0 ? 2 : 3, J = warp == 1 ? 1 : 0, K = warp == 1 ? 2 : 1;
+        float acc[2][4], t[2][4] = {};
         acc_load16(acc, blk(X, I, J), lane);
-        warp_mm16(acc, blk(A, I, K), blk(X, K, J), lane);
-        __syncwarp();
+        warp_mm16(t, blk(A, I, K), blk(X, K, J), lane);
+#pragma unroll
+        for (int ns = 0; ns < 2; ++ns)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) acc[ns][e] -= t[ns][e];
         acc_store16(acc, blk(X, I, J), 1.f, lane);
-        if (warp < 2) {
-            __syncwarp();
-            finish_block(X, I, J, lane, out);
-        }
+        if (warp < 2) acc_emit16(acc, I, J, lane, out);
     }
     __syncthreads();
-    // 4) warp 0: X_30
+    // 4) warp 0: X_30 -= N_32 X_20
     if (warp == 0) {
-        float acc[2][4];
+        float acc[2][4], t[2][4] = {};
         acc_load16(acc, blk(X, 3, 0), lane);
-        warp_mm16(acc, blk(A, 3, 2), blk(X, 2, 0), lane);
-        __syncwarp();
+        warp_mm16(t, blk(A, 3, 2), blk(X, 2, 0), lane);
+#pragma unroll
+        for (int ns = 0; ns < 2; ++ns)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) acc[ns][e] -= t[ns][e];
         acc_store16(acc, blk(X, 3, 0), 1.f, lane);
-        __syncwarp();
-        finish_block(X, 3, 0, lane, out);
+        acc_emit16(acc, 3, 0, lane, out);
     }
 }
 
