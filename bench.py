@@ -8,7 +8,11 @@ H=32, T=32768, d=128, chunk 64, bf16 q/k/v, fp32 gates and state), i.e. every
 prefill row of the hot path over one batch; ``value`` is prefill tokens/s
 over all ranks. The decode row is timed in the same run on the ``decode_256``
 workload (256 sequences x 32 heads, 128x128 fp32 states, 1000 consecutive
-steps) and reported under ``"decode"`` as state GB/s.
+steps) and reported under ``"decode"`` as state GB/s. Outside the timed region
+the same run also times, each with its own roofline fraction: the prefill with
+the layer prologue fused in (``"fused_prologue"``), the backward pass on
+prefill_4k's shape (``"backward"``) and the packed variable-length prefill into
+a state cache (``"varlen"``).
 
 Heads and batches are independent, so with N GPUs every rank runs its own copy
 of the workload (weak scaling, no collective on the data path); the timed
@@ -22,6 +26,7 @@ from __future__ import annotations
 
 import argparse
 import hashlib
+import itertools
 import json
 import os
 import statistics
@@ -218,6 +223,8 @@ def run_ours(args, rank, world, device):
                 "tensor_tflops_achieved": round(prefill_flops(w) / (ms_kernel / 1e3) / 1e12, 2)}
 
     fused = run_fused(kda, w, ws, args, device, stream) if engine == "tc_cluster" else None
+    backward = run_backward(kda, args, device, stream) if not args.skip_extra_legs else None
+    varlen = run_varlen(kda, args, device, stream) if not args.skip_extra_legs else None
     e2e = run_e2e(kda, w, inp, engine, ws, args, device, stream, world)
     decode = run_decode(kda, args, device, stream, world)
     clocks = clk.summary()
@@ -239,7 +246,8 @@ def run_ours(args, rank, world, device):
                        "engine": engine, "per_rank": "one full workload per GPU",
                        "l2": f"inputs larger than L2 ({bytes_alg / 1e9:.2f} GB moved per step)"},
             "roofline": roofline, "e2e": e2e, "gpu_launches": launches + decode.pop("launches"),
-            "clocks": clocks, "decode": decode, "fused_prologue": fused, "cpu_baseline": cpu,
+            "clocks": clocks, "decode": decode, "fused_prologue": fused, "backward": backward,
+            "varlen": varlen, "cpu_baseline": cpu,
         }
         print(json.dumps(line), flush=True)
 
@@ -269,6 +277,76 @@ def run_fused(kda, w, ws, args, device, stream):
     gbs = bytes_alg / (ms / 1e3) / 1e9
     return {"entry": "kda_chunk_fwd_fused", "kernel_ms": round(ms, 4),
             "tokens_per_s": round(w.tokens / (ms / 1e3), 1), "bytes_per_launch": bytes_alg,
+            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm, "unit": "GB/s",
+                         "frac": round(gbs / hbm, 4), "peak_source": src}}
+
+
+def run_backward(kda, args, device, stream):
+    """The backward pass (kda_chunk_bwd) on prefill_4k's shape: gradients of q, k, v, log
+    alpha, beta and S0 from dL/d(out) (bf16, seeded N(0,1)) and dL/d(S_T) (fp32). Its
+    algorithmic bytes per token-head are 2824 at d = 128 with bf16 inputs (the forward's
+    inputs and dL/d(out) read, six gradients written), plus S0, dL/d(S_T) and dL/d(S0) per
+    head; the states it stores for the reverse chain are extra traffic, not counted."""
+    w = I.WORKLOADS["prefill_4k"]
+    inp = I.prefill_inputs(w, device=device, s0_std=0.05)
+    g = torch.Generator(device=device).manual_seed(11)
+    gout = torch.randn(w.B, w.T, w.H, w.dv, device=device, generator=g).to(w.dtype)
+    gst = torch.randn(w.B, w.H, w.dk, w.dv, device=device, generator=g)
+    ws = torch.empty(max(1, kda.bwd_workspace_bytes(w.B, w.T, w.H, w.dk, w.dv, w.dtype)),
+                     device=device, dtype=torch.uint8)
+
+    def step():
+        kda.chunk_bwd(inp["q"], inp["k"], inp["v"], inp["log_alpha"], inp["beta"], gout, inp["S0"],
+                      gst, workspace=ws, stream=stream)
+
+    step()
+    torch.cuda.synchronize(device)
+    evs = time_events(step, max(1, min(args.steps, 3)), stream)
+    torch.cuda.synchronize(device)
+    ms = statistics.mean(s.elapsed_time(e) for s, e in evs)
+    bytes_alg = w.tokens * w.H * 2824 + w.B * w.H * 3 * w.dk * w.dv * 4
+    hbm, src = peaks()
+    gbs = bytes_alg / (ms / 1e3) / 1e9
+    return {"entry": "kda_chunk_bwd", "workload": "prefill_4k (B=8, H=32, T=4096, d=128, bf16, S0 ~ N(0,0.05))",
+            "kernel_ms": round(ms, 3), "tokens_per_s": round(w.tokens / (ms / 1e3), 1),
+            "bytes_per_launch": bytes_alg, "kernels": "bwd_states_kernel + bwd_chunk_kernel (fp32 CUDA cores, 16-token chunks)",
+            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm, "unit": "GB/s",
+                         "frac": round(gbs / hbm, 4), "peak_source": src}}
+
+
+def run_varlen(kda, args, device, stream):
+    """Packed variable-length prefill (kda_chunk_fwd_varlen) into a state cache through a
+    slot map: 32 sequences of 256..4096 tokens (kda_inputs.packed_lengths), H = 32,
+    d = 128, bf16, prefill_4k's distributions; a 64-slot fp32 cache ~ N(0, 0.05), the
+    sequences on every other slot, updated in place. Algorithmic bytes: 1540 per
+    token-head plus each sequence's state read and written."""
+    H, d = 32, 128
+    lens = I.packed_lengths(32, 256, 4096)
+    total = sum(lens)
+    x = I.prefill_inputs("prefill_4k", device=device, B=1, T=total)
+    flat = {n: x[n][0] for n in ("q", "k", "v", "log_alpha", "beta")}
+    cu = torch.tensor([0] + list(itertools.accumulate(lens)), device=device, dtype=torch.int32)
+    g = torch.Generator(device=device).manual_seed(12)
+    cache = 0.05 * torch.randn(64, H, d, d, device=device, generator=g)
+    slot = torch.arange(0, 64, 2, device=device, dtype=torch.int32)
+    out = torch.empty(total, H, d, device=device, dtype=torch.bfloat16)
+
+    def step():
+        kda.chunk_fwd_varlen(flat["q"], flat["k"], flat["v"], flat["log_alpha"], flat["beta"], cu,
+                             cache, slot=slot, out=out, stream=stream)
+
+    step()
+    torch.cuda.synchronize(device)
+    evs = time_events(step, max(1, min(args.steps, 5)), stream)
+    torch.cuda.synchronize(device)
+    ms = statistics.mean(s.elapsed_time(e) for s, e in evs)
+    bytes_alg = total * H * (3 * 2 * d + 4 * d + 4 + 2 * d) + len(lens) * H * 2 * d * d * 4
+    hbm, src = peaks()
+    gbs = bytes_alg / (ms / 1e3) / 1e9
+    return {"entry": "kda_chunk_fwd_varlen", "sequences": len(lens), "tokens": total,
+            "lengths": "uniform 256..4096, seed 5", "slots": 64,
+            "kernel_ms": round(ms, 3), "tokens_per_s": round(total / (ms / 1e3), 1),
+            "bytes_per_launch": bytes_alg, "kernel": "chunk_varlen_kernel (fp32 CUDA cores, 16-token chunks)",
             "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm, "unit": "GB/s",
                          "frac": round(gbs / hbm, 4), "peak_source": src}}
 
@@ -516,6 +594,8 @@ def main(argv=None):
                     help="tokens per head per step of the reference arm")
     ap.add_argument("--cpu-threads", type=int, default=0)
     ap.add_argument("--skip-cpu-baseline", action="store_true")
+    ap.add_argument("--skip-extra-legs", action="store_true",
+                    help="skip the backward and variable-length legs")
     ap.add_argument("--only", choices=["prefill", "decode"],
                     help="profiling mode: run just this kernel's workload (warm-up + steps), "
                          "print its time, no JSON line")

@@ -109,6 +109,11 @@ def workspace_bytes(B, T, H, dk, dv, chunk=64, dtype=torch.bfloat16) -> int:
     return int(load().kda_workspace_bytes(B, T, H, dk, dv, chunk, _DTYPES[dtype]))
 
 
+def bwd_workspace_bytes(B, T, H, dk, dv, dtype=torch.bfloat16) -> int:
+    """Device scratch that ``chunk_bwd`` needs (``kda_bwd_workspace_bytes``)."""
+    return int(load().kda_bwd_workspace_bytes(B, T, H, dk, dv, _DTYPES[dtype]))
+
+
 def chunk_fwd(q, k, v, log_alpha, beta, S0=None, chunk: int = 64, *, out=None, S_T=None,
               output_final_state: bool = True, engine: str = "auto", workspace=None, stream=None):
     """Chunked KDA prefill (``kda_chunk_fwd``).

@@ -187,6 +187,13 @@ def prefill_layer_inputs(w: Prefill | str, device="cpu", **override) -> dict:
                 beta=beta.contiguous(), S0=S0, w=w)
 
 
+def packed_lengths(n: int, lo: int, hi: int, seed: int = 5) -> list[int]:
+    """Lengths of n packed sequences for the variable-length prefill: uniform integers
+    in [lo, hi] from a generator seeded with `seed` (a mix of short and long prompts)."""
+    g = torch.Generator().manual_seed(int(seed))
+    return [int(x) for x in torch.randint(lo, hi + 1, (n,), generator=g)]
+
+
 def decode_state(w: Decode | str = "decode_256", device="cpu", **override) -> torch.Tensor:
     """The initial fp32 state cache ``[N, H, dk, dv]`` ~ N(0, state_std)."""
     if isinstance(w, str):
