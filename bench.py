@@ -315,7 +315,7 @@ def run_backward(kda, args, device, stream):
 
 
 def run_varlen(kda, args, device, stream):
-    """Packed variable-length prefill (kda_chunk_fwd_varlen) into a state cache through a
+    """Packed variable-length prefill (kda_chunk_fwd_varlen_engine) into a state cache through a
     slot map: 32 sequences of 256..4096 tokens (kda_inputs.packed_lengths), H = 32,
     d = 128, bf16, prefill_4k's distributions; a 64-slot fp32 cache ~ N(0, 0.05), the
     sequences on every other slot, updated in place. Algorithmic bytes: 1540 per
@@ -330,10 +330,12 @@ def run_varlen(kda, args, device, stream):
     cache = 0.05 * torch.randn(64, H, d, d, device=device, generator=g)
     slot = torch.arange(0, 64, 2, device=device, dtype=torch.int32)
     out = torch.empty(total, H, d, device=device, dtype=torch.bfloat16)
+    engine = "tc_cluster" if kda.engine_supported("tc_cluster", d, d, 64, torch.bfloat16) else "generic"
+    ws = torch.empty(max(1, kda.varlen_workspace_bytes(len(lens), H, d, d)), device=device, dtype=torch.uint8)
 
     def step():
         kda.chunk_fwd_varlen(flat["q"], flat["k"], flat["v"], flat["log_alpha"], flat["beta"], cu,
-                             cache, slot=slot, out=out, stream=stream)
+                             cache, slot=slot, out=out, engine=engine, workspace=ws, stream=stream)
 
     step()
     torch.cuda.synchronize(device)
@@ -346,7 +348,9 @@ def run_varlen(kda, args, device, stream):
     return {"entry": "kda_chunk_fwd_varlen", "sequences": len(lens), "tokens": total,
             "lengths": "uniform 256..4096, seed 5", "slots": 64,
             "kernel_ms": round(ms, 3), "tokens_per_s": round(total / (ms / 1e3), 1),
-            "bytes_per_launch": bytes_alg, "kernel": "chunk_varlen_kernel (fp32 CUDA cores, 16-token chunks)",
+            "bytes_per_launch": bytes_alg, "engine": engine,
+            "kernel": ("chunk_cluster_kernel (tensor cores, one 4-CTA cluster per sequence and head)"
+                       if engine == "tc_cluster" else "varlen_kernel (fp32 CUDA cores, 16-token chunks)"),
             "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm, "unit": "GB/s",
                          "frac": round(gbs / hbm, 4), "peak_source": src}}
 

@@ -12,8 +12,8 @@ The compute runs in ``libkda.so`` (hand-written CUDA, C ABI in
 """
 from .binding import (ENGINES, KDA_BF16, KDA_F32, LIB_PATH, KdaError, bwd_workspace_bytes, chunk_bwd,
                       chunk_fwd, chunk_fwd_fused, chunk_fwd_varlen, device_status, engine_supported,
-                      load, recurrent_step, workspace_bytes)
+                      load, recurrent_step, varlen_workspace_bytes, workspace_bytes)
 from .autograd import kda_prefill
 
-__all__ = ["chunk_fwd", "chunk_fwd_fused", "chunk_fwd_varlen", "chunk_bwd", "kda_prefill", "recurrent_step", "workspace_bytes", "bwd_workspace_bytes", "device_status",
+__all__ = ["chunk_fwd", "chunk_fwd_fused", "chunk_fwd_varlen", "chunk_bwd", "kda_prefill", "recurrent_step", "workspace_bytes", "bwd_workspace_bytes", "varlen_workspace_bytes", "device_status",
            "engine_supported", "load", "KdaError", "ENGINES", "KDA_BF16", "KDA_F32", "LIB_PATH"]

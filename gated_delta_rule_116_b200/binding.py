@@ -51,6 +51,10 @@ def load():
     lib.kda_engine_supported.restype = i
     lib.kda_chunk_fwd_varlen.argtypes = [p] * 10 + [i, i, i, i, i, i, p]
     lib.kda_chunk_fwd_varlen.restype = i
+    lib.kda_chunk_fwd_varlen_engine.argtypes = [i] + [p] * 10 + [i, i, i, i, i, i, p, sz, p]
+    lib.kda_chunk_fwd_varlen_engine.restype = i
+    lib.kda_varlen_workspace_bytes.argtypes = [i, i, i, i, i]
+    lib.kda_varlen_workspace_bytes.restype = sz
     lib.kda_chunk_bwd.argtypes = [p] * 14 + [i, i, i, i, i, i, p, sz, p]
     lib.kda_chunk_bwd.restype = i
     lib.kda_bwd_workspace_bytes.argtypes = [i, i, i, i, i, i]
@@ -197,16 +201,25 @@ def chunk_fwd_fused(q, k, v, gate, beta, S0=None, chunk: int = 64, *, out=None, 
     return out, S_T
 
 
+def varlen_workspace_bytes(N, H, dk, dv, dtype=torch.bfloat16) -> int:
+    """Device scratch of the tensor-core engine of ``chunk_fwd_varlen`` (``kda_varlen_workspace_bytes``)."""
+    return int(load().kda_varlen_workspace_bytes(N, H, dk, dv, _DTYPES[dtype]))
+
+
 def chunk_fwd_varlen(q, k, v, log_alpha, beta, cu_seqlens, S0=None, *, slot=None, out=None,
-                     S_T=None, output_final_state: bool = True, stream=None):
-    """Chunked prefill of packed variable-length sequences (``kda_chunk_fwd_varlen``).
+                     S_T=None, output_final_state: bool = True, engine: str = "auto",
+                     workspace=None, stream=None):
+    """Chunked prefill of packed variable-length sequences (``kda_chunk_fwd_varlen_engine``).
 
     q, k ``[total_T,H,dk]``, v ``[total_T,H,dv]`` (bf16 or fp32), log_alpha
     ``[total_T,H,dk]`` and beta ``[total_T,H]`` fp32, cu_seqlens ``[N+1]`` int32
     token offsets on the device. Without ``slot``, S0 and S_T are ``[N,H,dk,dv]``.
     With ``slot`` (``[N]`` int32), they are a state cache ``[slots,H,dk,dv]``
     (the decode step's) and sequence n uses row ``slot[n]``; S_T then defaults
-    to S0, updated in place. Returns ``(out, S_T)``.
+    to S0, updated in place. ``engine`` is "auto" (the tensor-core engine where it
+    supports the shape: bf16, dk = dv = 128), "tc_cluster" or "generic" (fp32 CUDA
+    cores); the tensor-core engine's ``workspace`` is allocated when not given.
+    Returns ``(out, S_T)``.
     """
     lib = load()
     device = q.device
@@ -244,11 +257,21 @@ def chunk_fwd_varlen(q, k, v, log_alpha, beta, cu_seqlens, S0=None, *, slot=None
     if out is None:
         out = torch.empty(TT, H, dv, device=device, dtype=q.dtype)
     _require(out, "out", device, q.dtype, (TT, H, dv))
+    if engine not in ENGINES:
+        raise ValueError(f"unknown engine {engine!r}")
+    ws_bytes = 0
+    if engine != "generic" and TT > 0:
+        need = int(lib.kda_varlen_workspace_bytes(N, H, dk, dv, _DTYPES[q.dtype]))
+        if need > 0 and workspace is None:
+            workspace = torch.empty(need, device=device, dtype=torch.uint8)
+    if workspace is not None:
+        _require(workspace, "workspace", device, torch.uint8)
+        ws_bytes = workspace.numel()
     with torch.cuda.device(device):
-        rc = lib.kda_chunk_fwd_varlen(
-            _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(cu_seqlens), _ptr(slot),
-            _ptr(S0), _ptr(out), _ptr(S_T), N, TT, H, dk, dv, _DTYPES[q.dtype],
-            _stream(device, stream))
+        rc = lib.kda_chunk_fwd_varlen_engine(
+            ENGINES[engine], _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(cu_seqlens),
+            _ptr(slot), _ptr(S0), _ptr(out), _ptr(S_T), N, TT, H, dk, dv, _DTYPES[q.dtype],
+            _ptr(workspace), ws_bytes, _stream(device, stream))
     _check(rc)
     return out, S_T
 

@@ -313,11 +313,28 @@ int kda_chunk_bwd(const void *q, const void *k, const void *v, const float *log_
     return e == cudaSuccess ? KDA_OK : cuda_fail(e, "launching the backward kernels");
 }
 
+size_t kda_varlen_workspace_bytes(int N, int H, int dk, int dv, int dtype) {
+    if (N <= 0 || H <= 0) return 0;
+    if (kda::chunk_cluster_supported(dk, dv, 64, dtype)) return kda::chunk_cluster_workspace_bytes(N, H);
+    return 0;
+}
+
 int kda_chunk_fwd_varlen(const void *q, const void *k, const void *v, const float *log_alpha,
                          const float *beta, const int32_t *cu_seqlens, const int32_t *slot,
                          const float *S0, void *out, float *S_T, int N, int total_T, int H, int dk,
                          int dv, int dtype, void *stream) {
+    return kda_chunk_fwd_varlen_engine(KDA_ENGINE_GENERIC, q, k, v, log_alpha, beta, cu_seqlens, slot, S0,
+                                       out, S_T, N, total_T, H, dk, dv, dtype, nullptr, 0, stream);
+}
+
+int kda_chunk_fwd_varlen_engine(int engine, const void *q, const void *k, const void *v,
+                                const float *log_alpha, const float *beta, const int32_t *cu_seqlens,
+                                const int32_t *slot, const float *S0, void *out, float *S_T, int N,
+                                int total_T, int H, int dk, int dv, int dtype, void *workspace,
+                                size_t workspace_bytes, void *stream) {
     g_detail[0] = '\0';
+    if (engine != KDA_ENGINE_AUTO && engine != KDA_ENGINE_GENERIC && engine != KDA_ENGINE_TC_CLUSTER)
+        return fail(KDA_ERR_INVALID_ARG, "engine %d is not a kda_engine", engine);
     if (dtype != KDA_BF16 && dtype != KDA_F32)
         return fail(KDA_ERR_INVALID_ARG, "dtype %d is neither KDA_BF16 nor KDA_F32", dtype);
     if (N < 0 || total_T < 0 || H < 0)
@@ -337,12 +354,38 @@ int kda_chunk_fwd_varlen(const void *q, const void *k, const void *v, const floa
     const bool tokens = total_T > 0;
     const Ptr ps[] = {{q, "q", tokens}, {k, "k", tokens}, {v, "v", tokens},
                       {log_alpha, "log_alpha", tokens}, {beta, "beta", tokens}, {out, "out", tokens},
-                      {S0, "S0", false}, {S_T, "S_T", false}};
+                      {S0, "S0", false}, {S_T, "S_T", false}, {workspace, "workspace", false}};
     int rc = check_pointers(ps, sizeof ps / sizeof ps[0]);
     if (rc != KDA_OK) return rc;
-    cudaError_t e = kda::launch_chunk_varlen(q, k, v, log_alpha, beta, cu_seqlens, slot, S0, out,
-                                             S_T, N, total_T, H, dk, dv, dtype,
-                                             static_cast<cudaStream_t>(stream));
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    // the tensor-core engine: bf16, dk = dv = 128, with its operand ring in the workspace
+    const bool cl_ok = kda::chunk_cluster_supported(dk, dv, 64, dtype);
+    const size_t need = kda::chunk_cluster_workspace_bytes(N, H);
+    bool use_cluster = false;
+    if (engine == KDA_ENGINE_TC_CLUSTER) {
+        if (!cl_ok)
+            return fail(KDA_ERR_UNSUPPORTED,
+                        "the tensor-core engine needs bf16 and dk = dv = 128 (got dtype %d, dk %d, dv %d)",
+                        dtype, dk, dv);
+        if (!workspace || workspace_bytes < need)
+            return fail(KDA_ERR_WORKSPACE, "workspace of %zu bytes given, %zu needed",
+                        workspace ? workspace_bytes : static_cast<size_t>(0), need);
+        use_cluster = true;
+    } else if (engine == KDA_ENGINE_AUTO) {
+        use_cluster = cl_ok && workspace && workspace_bytes >= need;
+    }
+    cudaError_t e;
+    if (use_cluster && tokens) {
+        kda::ChunkArgs a{q, k, v, log_alpha, beta, S0, out, S_T, N, total_T, H, dk, dv, 64, dtype,
+                         workspace, workspace_bytes, device_error_ptr()};
+        if (!a.device_error) return fail(KDA_ERR_CUDA, "device error word not addressable");
+        a.cu_seqlens = cu_seqlens;
+        a.slot = slot;
+        e = kda::launch_chunk_cluster(a, s);
+    } else {   // the CUDA-core kernel (also every call without tokens: it only moves the states)
+        e = kda::launch_chunk_varlen(q, k, v, log_alpha, beta, cu_seqlens, slot, S0, out, S_T, N, total_T,
+                                     H, dk, dv, dtype, s);
+    }
     return e == cudaSuccess ? KDA_OK : cuda_fail(e, "launching the variable-length prefill");
 }
 

@@ -861,9 +861,11 @@ __device__ void producer(uint8_t *sm, uint32_t tmem, int rank, uint8_t *ring,
     asm volatile("cp.async.wait_all;" ::: "memory");
 }
 // ============================================================ consumer
-__device__ void consumer(uint8_t *sm, uint32_t tmem, const uint8_t *ring, const float *__restrict__ S0,
-                         __nv_bfloat16 *__restrict__ out, float *__restrict__ S_T, int T, int H,
-                         int h, long bh, long ztok, int nchunks, const Ctl &ctl) {
+// S0 and S_T may be the same array (a state cache updated in place): each CTA reads its
+// row of S0 before the chunk loop and writes the same row of S_T after it.
+__device__ void consumer(uint8_t *sm, uint32_t tmem, const uint8_t *ring, const float *S0,
+                         __nv_bfloat16 *__restrict__ out, float *S_T, int T, int H,
+                         int h, long srow, long ztok, int nchunks, const Ctl &ctl) {
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int quad = warp & 3, half = warp >> 2;
     const int row = 32 * quad + lane;   // TMEM lane; state row (key channel)
@@ -915,7 +917,7 @@ __device__ void consumer(uint8_t *sm, uint32_t tmem, const uint8_t *ring, const 
     float S[64];
 #pragma unroll
     for (int j = 0; j < 64; ++j)
-        S[j] = S0 ? S0[(bh * kD + row) * kD + half * 64 + j] : 0.f;
+        S[j] = S0 ? S0[(srow * kD + row) * kD + half * 64 + j] : 0.f;
     auto write_s16 = [&]() {
 #pragma unroll
         for (int u = 0; u < 64; u += 8) {
@@ -1079,7 +1081,7 @@ __device__ void consumer(uint8_t *sm, uint32_t tmem, const uint8_t *ring, const 
     }
     if (S_T) {
 #pragma unroll
-        for (int j = 0; j < 64; ++j) S_T[(bh * kD + row) * kD + half * 64 + j] = S[j];
+        for (int j = 0; j < 64; ++j) S_T[(srow * kD + row) * kD + half * 64 + j] = S[j];
     }
 }
 
@@ -1087,17 +1089,27 @@ template <bool kFused>
 __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 1)
 chunk_cluster_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_qs, const __grid_constant__ CUtensorMap tm_ks,
                      const __grid_constant__ CUtensorMap tm_las, const float *__restrict__ beta,
-                     const float *__restrict__ S0, __nv_bfloat16 *__restrict__ out,
-                     float *__restrict__ S_T, uint8_t *__restrict__ ws, int T, int H, int *err,
-                     int test_timeout) {
+                     const float *S0, __nv_bfloat16 *__restrict__ out,
+                     float *S_T, uint8_t *__restrict__ ws, int T, int H, int *err,
+                     int test_timeout, const int32_t *__restrict__ cu_seqlens,
+                     const int32_t *__restrict__ slot) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~static_cast<uintptr_t>(1023));
     const int rank = static_cast<int>(tc::cluster_rank());
     const long bh = blockIdx.x / kCluster;
     const int b = static_cast<int>(bh / H), h = static_cast<int>(bh - static_cast<long>(b) * H);
-    const long ztok = static_cast<long>(b) * T;
-    const int nchunks = (T + kC - 1) / kC;
+    // this cluster's tokens and state row: batch b of a dense [B, T] batch, or packed sequence
+    // b (T is then the packed total; offsets clamped to [0, T]) with an optional slot map
+    long ztok = static_cast<long>(b) * T, srow = bh;
+    int len = T;
+    if (cu_seqlens) {
+        const int a0 = min(max(cu_seqlens[b], 0), T), a1 = min(max(cu_seqlens[b + 1], a0), T);
+        ztok = a0;
+        len = a1 - a0;
+        if (slot) srow = static_cast<long>(slot[b]) * H + h;
+    }
+    const int nchunks = (len + kC - 1) / kC;
     const bool is_consumer = rank == kCluster - 1;
     const uint32_t bar_off = is_consumer ? C_BAR : P_BAR;
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + bar_off);
@@ -1126,9 +1138,9 @@ chunk_cluster_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_cons
 
     uint8_t *ring = ws + bh * kRingSlots * kSlotStride;  // this head's ring: kRingDepth slots per producer
     if (is_consumer)
-        consumer(sm, tmem, ring, S0, out, S_T, T, H, h, bh, ztok, nchunks, ctl);
+        consumer(sm, tmem, ring, S0, out, S_T, len, H, h, srow, ztok, nchunks, ctl);
     else
-        producer<kFused>(sm, tmem, rank, ring, &tm_v, &tm_qs, &tm_ks, &tm_las, beta, T, H, h, ztok, nchunks,
+        producer<kFused>(sm, tmem, rank, ring, &tm_v, &tm_qs, &tm_ks, &tm_las, beta, len, H, h, ztok, nchunks,
                          ctl, test_timeout);
 
     tc_fence_before();
@@ -1192,7 +1204,7 @@ size_t chunk_cluster_workspace_bytes(int B, int H) {
 }
 
 cudaError_t launch_chunk_cluster(const ChunkArgs &a, cudaStream_t s) {
-    const long tokens = static_cast<long>(a.B) * a.T;
+    const long tokens = a.cu_seqlens ? static_cast<long>(a.T) : static_cast<long>(a.B) * a.T;
     const CUtensorMapDataType kB16 = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, kF32 = CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
     const bool fused = a.gate != nullptr;   // the layer prologue: gate pre-activation instead of log alpha
     CUtensorMap mv, mqs, mks, mlas;
@@ -1209,7 +1221,7 @@ cudaError_t launch_chunk_cluster(const ChunkArgs &a, cudaStream_t s) {
     const dim3 grid(static_cast<unsigned>(a.B) * a.H * kCluster);
     kern<<<grid, kThreads, kSmemBytes, s>>>(
         mv, mqs, mks, mlas, a.beta, a.S0, static_cast<__nv_bfloat16 *>(a.out), a.S_T,
-        static_cast<uint8_t *>(a.workspace), a.T, a.H, a.device_error, g_test_timeout);
+        static_cast<uint8_t *>(a.workspace), a.T, a.H, a.device_error, g_test_timeout, a.cu_seqlens, a.slot);
     return cudaGetLastError();
 }
 

@@ -31,6 +31,10 @@ struct ChunkArgs {
     size_t workspace_bytes;
     int *device_error;  // set to a nonzero code by a kernel whose bounded wait gave up
     const void *gate = nullptr;  // fused layer prologue: gate pre-activation (log_alpha unused)
+    // packed sequences: B = N sequences, T = the packed total; sequence n is tokens
+    // cu_seqlens[n] .. cu_seqlens[n+1]-1 and uses state row slot[n] (n without a slot map)
+    const int32_t *cu_seqlens = nullptr;
+    const int32_t *slot = nullptr;
 };
 
 struct DecodeArgs {

@@ -177,8 +177,12 @@ int kda_recurrent_step(const void *q, const void *k, const void *v,
  * tensors and starts from its own initial state (or zeros); no state crosses a
  * sequence boundary. With a slot map the states live in a state cache of the
  * decode step's layout: a prefill reads and writes row slot[n], and
- * kda_recurrent_step continues from the same rows. Computes in fp32 on CUDA
- * cores with 16-token chunks.
+ * kda_recurrent_step continues from the same rows (the serving path: packed
+ * prompts prefill the decode step's cache "without modifying the cache or
+ * scheduling interfaces", Kimi Linear summary, section "Uso de NoPE y
+ * resultados de evaluacion"). This entry computes in fp32 on CUDA cores with
+ * 16-token chunks; kda_chunk_fwd_varlen_engine below also runs the tensor-core
+ * engine.
  *
  *   q, k       [total_T,H,dk]  dtype     (packed over sequences)
  *   v          [total_T,H,dv]  dtype
@@ -208,6 +212,39 @@ int kda_chunk_fwd_varlen(const void *q, const void *k, const void *v,
                          const float *S0, void *out, float *S_T,
                          int N, int total_T, int H, int dk, int dv, int dtype,
                          void *stream);
+
+/*
+ * Device scratch of kda_chunk_fwd_varlen_engine's tensor-core engine for N
+ * packed sequences of H heads: the operand ring of one 4-CTA cluster per
+ * (sequence, head), N*H*9*82944 bytes, independent of the lengths. 0 when the
+ * engine does not support (dk, dv, dtype).
+ */
+size_t kda_varlen_workspace_bytes(int N, int H, int dk, int dv, int dtype);
+
+/*
+ * kda_chunk_fwd_varlen with a choice of engine. Arguments, layouts, results
+ * and limits as kda_chunk_fwd_varlen, plus:
+ *   engine     KDA_ENGINE_GENERIC: the fp32 CUDA-core kernel (16-token chunks);
+ *              KDA_ENGINE_TC_CLUSTER: the tensor-core engine of kda_chunk_fwd
+ *              (bf16, dk = dv = 128, chunk 64), one 4-CTA cluster per
+ *              (sequence, head) over the same packed tensors; anything else
+ *              returns KDA_ERR_UNSUPPORTED, a missing or small workspace
+ *              KDA_ERR_WORKSPACE;
+ *              KDA_ENGINE_AUTO: the tensor-core engine when it supports the
+ *              shape and the workspace is large enough, else the CUDA-core one.
+ *   workspace  device scratch, 16-byte aligned, kda_varlen_workspace_bytes(...)
+ *              bytes (the caller owns it; not kept after the call; one call at
+ *              a time per workspace). May be NULL for KDA_ENGINE_GENERIC.
+ * Calls with total_T = 0 only move the states and run the CUDA-core kernel.
+ * A bounded device wait that gives up on the tensor-core engine is reported by
+ * kda_device_status as KDA_ERR_DEVICE_TIMEOUT, as for kda_chunk_fwd.
+ */
+int kda_chunk_fwd_varlen_engine(int engine, const void *q, const void *k, const void *v,
+                                const float *log_alpha, const float *beta,
+                                const int32_t *cu_seqlens, const int32_t *slot,
+                                const float *S0, void *out, float *S_T,
+                                int N, int total_T, int H, int dk, int dv, int dtype,
+                                void *workspace, size_t workspace_bytes, void *stream);
 
 /*
  * Backward pass of kda_chunk_fwd: the gradients of a scalar loss L with respect

@@ -29,11 +29,11 @@ def packed(name, lens, H, seed, **kw):
     return flat, S0, cu
 
 
-def check(flat, S0, cu, with_state=True):
+def check(flat, S0, cu, with_state=True, engine="auto"):
     dev = {n: t.to(DEV) for n, t in flat.items()}
     out, ST = kda.chunk_fwd_varlen(dev["q"], dev["k"], dev["v"], dev["log_alpha"], dev["beta"],
                                    cu.to(DEV), None if S0 is None else S0.to(DEV),
-                                   output_final_state=with_state)
+                                   output_final_state=with_state, engine=engine)
     torch.cuda.synchronize()
     out = out.cpu()
     atol, rtol = tol_for(flat["q"].dtype)
@@ -57,9 +57,22 @@ def test_fp32_other_sizes_no_state():
     check(flat, None, cu, with_state=False)
 
 
-def test_bf16_head_size_128():
+BF16_ENGINES = ["generic", "tc_cluster"]
+
+
+@pytest.mark.parametrize("engine", BF16_ENGINES)
+def test_bf16_head_size_128(engine):
     flat, S0, cu = packed("prefill_4k", [50, 0, 70], H=2, seed=3)
-    check(flat, S0, cu)
+    check(flat, S0, cu, engine=engine)
+
+
+@pytest.mark.parametrize("lens", [[0, 1, 63, 64, 65, 200, 129], [300], [5, 0, 0, 190, 64 * 5 + 7]])
+def test_bf16_tensor_core_engine_lengths(lens):
+    """The tensor-core engine over packed sequences: empty and one-token sequences,
+    lengths at and around the 64-token chunk, several chunks and a ragged tail."""
+    flat, S0, cu = packed("prefill_4k", lens, H=3, seed=4)
+    check(flat, S0, cu, engine="tc_cluster")
+    check(flat, None, cu, with_state=False, engine="tc_cluster")
 
 
 def test_paged_prefill_then_decode():
@@ -94,6 +107,47 @@ def test_paged_prefill_then_decode():
         assert torch.equal(cache[r], cache0[r])
 
 
-def test_bf16_strong_decay_mixed_lengths():
+@pytest.mark.parametrize("engine", BF16_ENGINES)
+def test_bf16_strong_decay_mixed_lengths(engine):
     flat, S0, cu = packed("prefill_4k", [70, 1, 33, 130], H=2, seed=9, gate="strong")
-    check(flat, S0, cu)
+    check(flat, S0, cu, engine=engine)
+
+
+def test_bf16_tensor_core_paged_prefill_then_decode():
+    """The serving handoff on the tensor-core engine: bf16 prompts prefilled into rows
+    of a state cache through a slot map (in place), then one decode step from the same
+    rows; rows outside the map are untouched."""
+    lens, slots, H = [130, 0, 64, 7], [5, 1, 0, 3], 2
+    flat, _, cu = packed("prefill_4k", lens, H=H, seed=10)
+    g = torch.Generator().manual_seed(11)
+    cache0 = 0.05 * torch.randn(7, H, 128, 128, generator=g)
+    nxt = I.prefill_inputs("prefill_4k", B=1, T=len(lens), H=H, seed=12)
+    step = {n: nxt[n][0].contiguous() for n in ("q", "k", "v", "log_alpha", "beta")}
+    cache = cache0.to(DEV)
+    slot = torch.tensor(slots, dtype=torch.int32, device=DEV)
+    dev = {n: t.to(DEV) for n, t in flat.items()}
+    out, ST = kda.chunk_fwd_varlen(dev["q"], dev["k"], dev["v"], dev["log_alpha"], dev["beta"],
+                                   cu.to(DEV), cache, slot=slot, engine="tc_cluster")
+    assert ST.data_ptr() == cache.data_ptr()
+    kda.device_status()
+    o1 = kda.recurrent_step(*(step[n].to(DEV) for n in ("q", "k", "v", "log_alpha", "beta")), cache, slot)
+    torch.cuda.synchronize()
+    out, o1, cache = out.cpu(), o1.cpu(), cache.cpu()
+    atol, rtol = tol_for(torch.bfloat16)
+    for n, r in enumerate(slots):
+        a, b = int(cu[n]), int(cu[n + 1])
+        cat = lambda name: torch.cat([flat[name][a:b], step[name][n:n + 1]])[None]
+        ref_o, ref_s = oracle.forward(cat("q"), cat("k"), cat("v"), cat("log_alpha"), cat("beta"), cache0[r][None])
+        assert_close(out[a:b], ref_o[0, :-1], atol, rtol, f"prefill out of sequence {n}")
+        assert_close(o1[n], ref_o[0, -1], atol, rtol, f"decode out of sequence {n}")
+        assert_close(cache[r], ref_s[0], atol, rtol, f"cache row {r}")
+    for r in (2, 4, 6):
+        assert torch.equal(cache[r], cache0[r])
+
+
+def test_engine_choice_errors():
+    flat, S0, cu = packed("fp32_small", [10, 20], H=2, seed=13)
+    dev = {n: t.to(DEV) for n, t in flat.items()}
+    with pytest.raises(kda.KdaError):   # fp32, d = 16: not the tensor-core engine's shape
+        kda.chunk_fwd_varlen(dev["q"], dev["k"], dev["v"], dev["log_alpha"], dev["beta"], cu.to(DEV),
+                             S0.to(DEV), engine="tc_cluster")
