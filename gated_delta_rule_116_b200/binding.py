@@ -53,6 +53,10 @@ def load():
     lib.kda_chunk_fwd_varlen.restype = i
     lib.kda_chunk_fwd_varlen_engine.argtypes = [i] + [p] * 10 + [i, i, i, i, i, i, p, sz, p]
     lib.kda_chunk_fwd_varlen_engine.restype = i
+    lib.kda_layer_fwd.argtypes = [p, p, p, p, p, p, p, ctypes.c_float, p, p, p, i, i, i, i, i, i, i, p, sz, p]
+    lib.kda_layer_fwd.restype = i
+    lib.kda_short_conv_swish.argtypes = [p, p, p, p, i, i, i, i, i, i, p]
+    lib.kda_short_conv_swish.restype = i
     lib.kda_varlen_workspace_bytes.argtypes = [i, i, i, i, i]
     lib.kda_varlen_workspace_bytes.restype = sz
     lib.kda_chunk_bwd.argtypes = [p] * 14 + [i, i, i, i, i, i, p, sz, p]
@@ -201,6 +205,47 @@ def chunk_fwd_fused(q, k, v, gate, beta, S0=None, chunk: int = 64, *, out=None, 
     return out, S_T
 
 
+def layer_fwd(q, k, v, gate, beta, out_gate, norm_weight, S0=None, eps: float = 1e-6, chunk: int = 64, *,
+              out=None, S_T=None, output_final_state: bool = True, workspace=None, stream=None):
+    """The KDA layer between its projections (``kda_layer_fwd``): ``chunk_fwd_fused`` followed
+    by the per-head RMSNorm and the sigmoid output gate on every output row, in one kernel.
+
+    q, k, v, gate as ``chunk_fwd_fused``; out_gate ``[B,T,H,128]`` bf16 (the output gate's
+    pre-activation); norm_weight ``[128]`` fp32. Returns ``(out, S_T)``.
+    """
+    lib = load()
+    device = q.device
+    _require(q, "q", device, torch.bfloat16)
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    _require(k, "k", device, torch.bfloat16, (B, T, H, dk))
+    _require(v, "v", device, torch.bfloat16, (B, T, H, dv))
+    _require(gate, "gate", device, torch.bfloat16, (B, T, H, dk))
+    _require(beta, "beta", device, torch.float32, (B, T, H))
+    _require(out_gate, "out_gate", device, torch.bfloat16, (B, T, H, dv))
+    _require(norm_weight, "norm_weight", device, torch.float32, (dv,))
+    if S0 is not None:
+        _require(S0, "S0", device, torch.float32, (B, H, dk, dv))
+    if out is None:
+        out = torch.empty(B, T, H, dv, device=device, dtype=torch.bfloat16)
+    _require(out, "out", device, torch.bfloat16, (B, T, H, dv))
+    if S_T is None and output_final_state:
+        S_T = torch.empty(B, H, dk, dv, device=device, dtype=torch.float32)
+    if S_T is not None:
+        _require(S_T, "S_T", device, torch.float32, (B, H, dk, dv))
+    need = int(lib.kda_workspace_bytes(B, T, H, dk, dv, chunk, KDA_BF16))
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, device=device, dtype=torch.uint8)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    with torch.cuda.device(device):
+        rc = lib.kda_layer_fwd(
+            _ptr(q), _ptr(k), _ptr(v), _ptr(gate), _ptr(beta), _ptr(out_gate), _ptr(norm_weight),
+            float(eps), _ptr(S0), _ptr(out), _ptr(S_T), B, T, H, dk, dv, chunk, KDA_BF16,
+            _ptr(workspace), ws_bytes, _stream(device, stream))
+    _check(rc)
+    return out, S_T
+
+
 def varlen_workspace_bytes(N, H, dk, dv, dtype=torch.bfloat16) -> int:
     """Device scratch of the tensor-core engine of ``chunk_fwd_varlen`` (``kda_varlen_workspace_bytes``)."""
     return int(load().kda_varlen_workspace_bytes(N, H, dk, dv, _DTYPES[dtype]))
@@ -274,6 +319,34 @@ def chunk_fwd_varlen(q, k, v, log_alpha, beta, cu_seqlens, S0=None, *, slot=None
             _ptr(workspace), ws_bytes, _stream(device, stream))
     _check(rc)
     return out, S_T
+
+
+def short_conv_swish(x, weight, cu_seqlens=None, *, out=None, stream=None):
+    """ShortConv + Swish (``kda_short_conv_swish``): y_t = swish(sum_j weight[h,c,j] x_{t-j}),
+    causal per sequence. x ``[B,T,H,d]`` (or packed ``[T,H,d]`` with ``cu_seqlens``
+    ``[N+1]`` int32), bf16 or fp32; weight ``[H,d,W]`` fp32 with W <= 4. Returns y."""
+    lib = load()
+    device = x.device
+    _require(x, "x", device)
+    if x.dtype not in _DTYPES:
+        raise TypeError(f"x must be bf16 or fp32 (got {x.dtype})")
+    if cu_seqlens is None:
+        B, T, H, d = x.shape
+    else:
+        T, H, d = x.shape
+        _require(cu_seqlens, "cu_seqlens", device, torch.int32)
+        B = cu_seqlens.numel() - 1
+    if weight.dim() != 3 or tuple(weight.shape[:2]) != (H, d):
+        raise ValueError(f"weight must be [{H},{d},W] (got {tuple(weight.shape)})")
+    _require(weight, "weight", device, torch.float32)
+    if out is None:
+        out = torch.empty_like(x)
+    _require(out, "out", device, x.dtype, tuple(x.shape))
+    with torch.cuda.device(device):
+        rc = lib.kda_short_conv_swish(_ptr(x), _ptr(weight), _ptr(cu_seqlens), _ptr(out), B, T, H, d,
+                                      weight.shape[2], _DTYPES[x.dtype], _stream(device, stream))
+    _check(rc)
+    return out
 
 
 def chunk_bwd(q, k, v, log_alpha, beta, grad_out, S0=None, grad_S_T=None, *, workspace=None,

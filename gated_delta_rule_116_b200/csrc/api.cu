@@ -181,10 +181,13 @@ int kda_chunk_fwd_engine(int engine, const void *q, const void *k, const void *v
     return e == cudaSuccess ? KDA_OK : cuda_fail(e, "launching the prefill kernel");
 }
 
-int kda_chunk_fwd_fused(const void *q, const void *k, const void *v, const void *gate,
-                        const float *beta, const float *S0, void *out, float *S_T, int B, int T,
-                        int H, int dk, int dv, int chunk, int dtype, void *workspace,
-                        size_t workspace_bytes, void *stream) {
+namespace {
+// kda_chunk_fwd_fused and kda_layer_fwd: the prefill on the tensor-core engine with the
+// layer prologue, and (out_gate != NULL) the layer epilogue.
+int fused_impl(const void *q, const void *k, const void *v, const void *gate, const float *beta,
+               bool gated, const void *out_gate, const float *norm_weight, float eps, const float *S0, void *out,
+               float *S_T, int B, int T, int H, int dk, int dv, int chunk, int dtype, void *workspace,
+               size_t workspace_bytes, void *stream) {
     g_detail[0] = '\0';
     if (B < 0 || T < 0 || H < 0)
         return fail(KDA_ERR_INVALID_ARG, "B=%d T=%d H=%d must be >= 0", B, T, H);
@@ -202,9 +205,12 @@ int kda_chunk_fwd_fused(const void *q, const void *k, const void *v, const void 
                     static_cast<long long>(B) * H);
     if (B == 0 || H == 0) return KDA_OK;
     const bool tokens = T > 0;
+    if (gated && !(eps >= 0.f && eps < 1e30f))
+        return fail(KDA_ERR_INVALID_ARG, "eps = %g is not a finite value >= 0", static_cast<double>(eps));
     const Ptr ps[] = {{q, "q", tokens},       {k, "k", tokens},   {v, "v", tokens},
                       {gate, "gate", tokens}, {beta, "beta", tokens}, {out, "out", tokens},
-                      {S0, "S0", false},      {S_T, "S_T", false}, {workspace, "workspace", false}};
+                      {S0, "S0", false},      {S_T, "S_T", false}, {workspace, "workspace", false},
+                      {out_gate, "out_gate", gated && tokens}, {norm_weight, "norm_weight", gated && tokens}};
     rc = check_pointers(ps, sizeof ps / sizeof ps[0]);
     if (rc != KDA_OK) return rc;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -223,9 +229,32 @@ int kda_chunk_fwd_fused(const void *q, const void *k, const void *v, const void 
     kda::ChunkArgs a{q, k, v, nullptr, beta, S0, out, S_T, B, T, H, dk, dv, chunk, dtype,
                      workspace, workspace_bytes, device_error_ptr(), gate};
     if (!a.device_error) return fail(KDA_ERR_CUDA, "device error word not addressable");
+    if (gated) {
+        a.out_gate = out_gate;
+        a.norm_weight = norm_weight;
+        a.norm_eps = eps;
+    }
     const cudaError_t e = kda::launch_chunk_cluster(a, s);
     return e == cudaSuccess ? KDA_OK : cuda_fail(e, "launching the prefill kernel");
 }
+}  // namespace
+
+int kda_chunk_fwd_fused(const void *q, const void *k, const void *v, const void *gate,
+                        const float *beta, const float *S0, void *out, float *S_T, int B, int T,
+                        int H, int dk, int dv, int chunk, int dtype, void *workspace,
+                        size_t workspace_bytes, void *stream) {
+    return fused_impl(q, k, v, gate, beta, false, nullptr, nullptr, 0.f, S0, out, S_T, B, T, H, dk, dv, chunk,
+                      dtype, workspace, workspace_bytes, stream);
+}
+
+int kda_layer_fwd(const void *q, const void *k, const void *v, const void *gate, const float *beta,
+                  const void *out_gate, const float *norm_weight, float eps, const float *S0, void *out,
+                  float *S_T, int B, int T, int H, int dk, int dv, int chunk, int dtype, void *workspace,
+                  size_t workspace_bytes, void *stream) {
+    return fused_impl(q, k, v, gate, beta, true, out_gate, norm_weight, eps, S0, out, S_T, B, T, H, dk, dv,
+                      chunk, dtype, workspace, workspace_bytes, stream);
+}
+
 
 int kda_chunk_fwd(const void *q, const void *k, const void *v, const float *log_alpha,
                   const float *beta, const float *S0, void *out, float *S_T, int B, int T, int H,
@@ -387,6 +416,30 @@ int kda_chunk_fwd_varlen_engine(int engine, const void *q, const void *k, const 
                                      H, dk, dv, dtype, s);
     }
     return e == cudaSuccess ? KDA_OK : cuda_fail(e, "launching the variable-length prefill");
+}
+
+int kda_short_conv_swish(const void *x, const float *weight, const int32_t *cu_seqlens, void *y, int B,
+                         int T, int H, int d, int W, int dtype, void *stream) {
+    g_detail[0] = '\0';
+    if (dtype != KDA_BF16 && dtype != KDA_F32)
+        return fail(KDA_ERR_INVALID_ARG, "dtype %d is neither KDA_BF16 nor KDA_F32", dtype);
+    if (B < 0 || T < 0 || H < 0 || d < 0)
+        return fail(KDA_ERR_INVALID_ARG, "B=%d T=%d H=%d d=%d must be >= 0", B, T, H, d);
+    if (W < 1 || W > 4) return fail(KDA_ERR_UNSUPPORTED, "W=%d: filters of 1..4 taps", W);
+    if (d % 8 != 0) return fail(KDA_ERR_UNSUPPORTED, "d=%d is not a multiple of 8", d);
+    const long long tokens = cu_seqlens ? static_cast<long long>(T) : static_cast<long long>(B) * T;
+    if (tokens * H * d > (1ll << 40))
+        return fail(KDA_ERR_UNSUPPORTED, "%lld x %d x %d elements: too many for one call", tokens, H, d);
+    if (B == 0 || T == 0 || H == 0 || d == 0) return KDA_OK;
+    if ((reinterpret_cast<uintptr_t>(cu_seqlens) & 3u) != 0)
+        return fail(KDA_ERR_ALIGNMENT, "cu_seqlens is not 4-byte aligned");
+    const Ptr ps[] = {{x, "x", true}, {weight, "weight", true}, {y, "y", true}};
+    int rc = check_pointers(ps, sizeof ps / sizeof ps[0]);
+    if (rc != KDA_OK) return rc;
+    if (x == y) return fail(KDA_ERR_INVALID_ARG, "y must not alias x");
+    cudaError_t e = kda::launch_short_conv_swish(x, weight, y, cu_seqlens, B, T, H, d, W, dtype,
+                                                 static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? KDA_OK : cuda_fail(e, "launching the short convolution");
 }
 
 int kda_device_status(void *stream) {

@@ -146,9 +146,14 @@ constexpr uint32_t C_SLOT = 0;         // 2 slots
 constexpr uint32_t C_S16 = 2 * kSlotStride;        // S fp16, MN-major SW128: 2 blocks x 16 KB
 constexpr uint32_t C_U16 = C_S16 + 32768;          // U fp16, MN-major SW128: 2 blocks x 8 KB
 constexpr uint32_t C_BAR = C_U16 + 16384;
+// layer epilogue (RMSNorm + output gate): per-row partial sums of squares [128][2] and the
+// norm weight [128], after the barriers
+constexpr uint32_t C_RED = C_BAR + 256;
+constexpr uint32_t C_NW = C_RED + 1024;
 constexpr uint32_t kSmemBytes =
     (P_BAR > C_BAR ? P_BAR : C_BAR) + 192 + 1024;  // + barriers + alignment slack
 static_assert(P_PX + 2 * 6 * 2048 <= P_KSIG, "producer layout");
+static_assert(C_NW + 512 <= (P_BAR > C_BAR ? P_BAR : C_BAR) + 192, "consumer layout");
 static_assert(P_KBS + 16384 <= P_STAGE, "producer layout");
 static_assert(P_KHT + 4 * kKHTBlk <= P_KBS, "producer layout");
 
@@ -863,9 +868,16 @@ __device__ void producer(uint8_t *sm, uint32_t tmem, int rank, uint8_t *ring,
 // ============================================================ consumer
 // S0 and S_T may be the same array (a state cache updated in place): each CTA reads its
 // row of S0 before the chunk loop and writes the same row of S_T after it.
+// kGated: the layer's epilogue on each output row (Kimi Linear summary, section
+// "Configuracion del modelo Kimi Linear": per-head RMSNorm and a data-dependent output
+// gate before the output projection), out = o / sqrt(mean(o^2) + eps) * norm_w *
+// sigmoid(z), z the gate's pre-activation (bf16, the layout of out).
+template <bool kGated>
 __device__ void consumer(uint8_t *sm, uint32_t tmem, const uint8_t *ring, const float *S0,
                          __nv_bfloat16 *__restrict__ out, float *S_T, int T, int H,
-                         int h, long srow, long ztok, int nchunks, const Ctl &ctl) {
+                         int h, long srow, long ztok, int nchunks, const Ctl &ctl,
+                         const __nv_bfloat16 *__restrict__ out_gate, const float *__restrict__ norm_w,
+                         float eps) {
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int quad = warp & 3, half = warp >> 2;
     const int row = 32 * quad + lane;   // TMEM lane; state row (key channel)
@@ -937,6 +949,9 @@ __device__ void consumer(uint8_t *sm, uint32_t tmem, const uint8_t *ring, const 
                     d_s16 + ((kk * 2048) >> 4), IDESC_X, kk > 0);
         tc::mma_commit(bar_x);
     };
+    float *red = reinterpret_cast<float *>(sm + C_RED);
+    float *nw = reinterpret_cast<float *>(sm + C_NW);
+    if (kGated && tid < kD) nw[tid] = norm_w[tid];
     write_s16();
     fence_proxy_async_smem();
     tc_fence_before();
@@ -1047,23 +1062,50 @@ __device__ void consumer(uint8_t *sm, uint32_t tmem, const uint8_t *ring, const 
             pend_o = false;
         }
         tc_fence_after();
+        float o[64];
         if (quad < 2) {
-            float o[64];
             const uint32_t ta = tc::tmem_addr(tmem, 32 * quad, xcol + half * 64);
             tc::tmem_ld32(ta, *reinterpret_cast<float(*)[32]>(&o[0]));
             tc::tmem_ld32(ta + 32, *reinterpret_cast<float(*)[32]>(&o[32]));
             tc::tmem_wait_ld();
-            if (row < valid) {
-                uint4 *dst = reinterpret_cast<uint4 *>(out + ((ztok + t0 + row) * H + h) * kD + half * 64);
+            if (kGated) {   // this thread's half of the row's sum of squares
+                float ss0 = 0.f, ss1 = 0.f;
+#pragma unroll
+                for (int j = 0; j < 64; j += 2) {
+                    ss0 = fmaf(o[j], o[j], ss0);
+                    ss1 = fmaf(o[j + 1], o[j + 1], ss1);
+                }
+                red[2 * row + half] = ss0 + ss1;
+            }
+        }
+        if (kGated) __syncthreads();
+        if (quad < 2 && row < valid) {
+            const long orow = ((ztok + t0 + row) * H + h) * kD + half * 64;
+            if (kGated) {
+                const float r = rsqrtf((red[2 * row] + red[2 * row + 1]) * (1.f / kD) + eps);
+                const uint4 *zp = reinterpret_cast<const uint4 *>(out_gate + orow);
 #pragma unroll
                 for (int u = 0; u < 64; u += 8) {
-                    uint4 x;
-                    x.x = pack_bf16(o[u], o[u + 1]);
-                    x.y = pack_bf16(o[u + 2], o[u + 3]);
-                    x.z = pack_bf16(o[u + 4], o[u + 5]);
-                    x.w = pack_bf16(o[u + 6], o[u + 7]);
-                    dst[u / 8] = x;
+                    const uint4 z4 = zp[u / 8];
+                    const uint32_t zw[4] = {z4.x, z4.y, z4.z, z4.w};
+#pragma unroll
+                    for (int m = 0; m < 4; ++m) {
+                        const float z0 = tc::bf16_lo(zw[m]), z1 = tc::bf16_hi(zw[m]);
+                        const int j = u + 2 * m;
+                        o[j] *= r * nw[half * 64 + j] / (1.f + tc::ex2(-z0 * kLog2e));
+                        o[j + 1] *= r * nw[half * 64 + j + 1] / (1.f + tc::ex2(-z1 * kLog2e));
+                    }
                 }
+            }
+            uint4 *dst = reinterpret_cast<uint4 *>(out + orow);
+#pragma unroll
+            for (int u = 0; u < 64; u += 8) {
+                uint4 x;
+                x.x = pack_bf16(o[u], o[u + 1]);
+                x.y = pack_bf16(o[u + 2], o[u + 3]);
+                x.z = pack_bf16(o[u + 4], o[u + 5]);
+                x.w = pack_bf16(o[u + 6], o[u + 7]);
+                dst[u / 8] = x;
             }
         }
         tc_fence_before();
@@ -1085,14 +1127,15 @@ __device__ void consumer(uint8_t *sm, uint32_t tmem, const uint8_t *ring, const 
     }
 }
 
-template <bool kFused>
+template <bool kFused, bool kGated>
 __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 1)
 chunk_cluster_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_qs, const __grid_constant__ CUtensorMap tm_ks,
                      const __grid_constant__ CUtensorMap tm_las, const float *__restrict__ beta,
                      const float *S0, __nv_bfloat16 *__restrict__ out,
                      float *S_T, uint8_t *__restrict__ ws, int T, int H, int *err,
                      int test_timeout, const int32_t *__restrict__ cu_seqlens,
-                     const int32_t *__restrict__ slot) {
+                     const int32_t *__restrict__ slot, const __nv_bfloat16 *__restrict__ out_gate,
+                     const float *__restrict__ norm_w, float norm_eps) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~static_cast<uintptr_t>(1023));
@@ -1138,7 +1181,8 @@ chunk_cluster_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_cons
 
     uint8_t *ring = ws + bh * kRingSlots * kSlotStride;  // this head's ring: kRingDepth slots per producer
     if (is_consumer)
-        consumer(sm, tmem, ring, S0, out, S_T, len, H, h, srow, ztok, nchunks, ctl);
+        consumer<kGated>(sm, tmem, ring, S0, out, S_T, len, H, h, srow, ztok, nchunks, ctl, out_gate,
+                         norm_w, norm_eps);
     else
         producer<kFused>(sm, tmem, rank, ring, &tm_v, &tm_qs, &tm_ks, &tm_las, beta, len, H, h, ztok, nchunks,
                          ctl, test_timeout);
@@ -1214,14 +1258,18 @@ cudaError_t launch_chunk_cluster(const ChunkArgs &a, cudaStream_t s) {
         (fused ? make_map(&mlas, a.gate, kB16, 2, a.H, tokens, true)
                : make_map(&mlas, a.log_alpha, kF32, 4, a.H, tokens, true));
     if (!ok) return cudaErrorInvalidValue;
-    auto kern = fused ? chunk_cluster_kernel<true> : chunk_cluster_kernel<false>;
+    // the layer epilogue comes with the layer prologue only (kda_layer_fwd)
+    const bool gated = fused && a.out_gate != nullptr;
+    auto kern = gated ? chunk_cluster_kernel<true, true>
+                      : (fused ? chunk_cluster_kernel<true, false> : chunk_cluster_kernel<false, false>);
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(kSmemBytes));
     if (e != cudaSuccess) return e;
     const dim3 grid(static_cast<unsigned>(a.B) * a.H * kCluster);
     kern<<<grid, kThreads, kSmemBytes, s>>>(
         mv, mqs, mks, mlas, a.beta, a.S0, static_cast<__nv_bfloat16 *>(a.out), a.S_T,
-        static_cast<uint8_t *>(a.workspace), a.T, a.H, a.device_error, g_test_timeout, a.cu_seqlens, a.slot);
+        static_cast<uint8_t *>(a.workspace), a.T, a.H, a.device_error, g_test_timeout, a.cu_seqlens, a.slot,
+        static_cast<const __nv_bfloat16 *>(a.out_gate), a.norm_weight, a.norm_eps);
     return cudaGetLastError();
 }
 

@@ -35,6 +35,10 @@ struct ChunkArgs {
     // cu_seqlens[n] .. cu_seqlens[n+1]-1 and uses state row slot[n] (n without a slot map)
     const int32_t *cu_seqlens = nullptr;
     const int32_t *slot = nullptr;
+    // layer epilogue (with the fused prologue): out = RMSNorm(o) * norm_weight * sigmoid(out_gate)
+    const void *out_gate = nullptr;
+    const float *norm_weight = nullptr;
+    float norm_eps = 1e-6f;
 };
 
 struct DecodeArgs {
@@ -71,6 +75,9 @@ cudaError_t launch_chunk_varlen(const void *q, const void *k, const void *v, con
                                 const float *beta, const int32_t *cu_seqlens, const int32_t *slot,
                                 const float *S0, void *out, float *S_T, int N, int total_T, int H,
                                 int dk, int dv, int dtype, cudaStream_t s);
+// ShortConv + Swish (short_conv.cu): dense [B,T,H,d], or B packed sequences over T tokens.
+cudaError_t launch_short_conv_swish(const void *x, const float *w, void *y, const int32_t *cu_seqlens,
+                                    int B, int T, int H, int d, int W, int dtype, cudaStream_t s);
 // Ring of operand images of the cluster engine: 3 producers x 3 slots of 81 KB per head.
 constexpr size_t kClusterRingBytesPerHead = 9ull * 82944;
 

@@ -247,6 +247,53 @@ int kda_chunk_fwd_varlen_engine(int engine, const void *q, const void *k, const 
                                 void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * The KDA layer between its projections, on the tensor-core engine: the fused
+ * prologue of kda_chunk_fwd_fused, the recurrence, and the layer's epilogue on
+ * every output row (Kimi Linear summary, section "Configuracion del modelo
+ * Kimi Linear": per-head RMSNorm and a data-dependent output gate before the
+ * output projection; the page gives no formulas). With o the output that
+ * kda_chunk_fwd_fused would write, this entry writes instead
+ *     out[t][h][c] = o[t][h][c] / sqrt(mean_c'(o[t][h][c']^2) + eps)
+ *                    * norm_weight[c] * sigmoid(out_gate[t][h][c]),
+ * the mean over the head's dv channels; o itself is never written.
+ *   out_gate     [B,T,H,dv] bf16  the output gate's pre-activation
+ *   norm_weight  [dv]       fp32  the RMSNorm weight (shared by the heads)
+ *   eps          finite, >= 0 (1e-6 is usual)
+ *   everything else as kda_chunk_fwd_fused (same support, limits, workspace);
+ *   out_gate and norm_weight may be NULL only when T = 0.
+ */
+int kda_layer_fwd(const void *q, const void *k, const void *v, const void *gate,
+                  const float *beta, const void *out_gate, const float *norm_weight, float eps,
+                  const float *S0, void *out, float *S_T, int B, int T, int H, int dk, int dv,
+                  int chunk, int dtype, void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * The layer's q/k/v prologue ahead of the prefill: ShortConv followed by Swish
+ * (Kimi Linear summary, es.news.hada.io/topic?id=31936, section "Configuracion
+ * del modelo Kimi Linear": each head's queries, keys and values pass through
+ * ShortConv and Swish; the page gives no formula). Read as a causal depthwise
+ * convolution along each sequence's tokens with one W-tap filter per (head,
+ * channel), no bias:
+ *     y[t][h][c] = swish(sum_{j<W} weight[h][c][j] * x[t-j][h][c]),
+ *     swish(u) = u / (1 + e^{-u}),
+ * where x before a sequence's first token is zero (no value crosses a
+ * sequence boundary). Apply it to each of q, k and v (separate filters), then
+ * pass q and k un-normalised to kda_chunk_fwd_fused or kda_layer_fwd, which
+ * L2-normalise them.
+ *   x          [B,T,H,d] dtype, or packed [T,H,d] with cu_seqlens
+ *   weight     [H,d,W]   fp32   the filter taps (caller-owned)
+ *   cu_seqlens [B+1] int32 (device) or NULL: with it, B sequences packed over
+ *              T tokens in all (offsets clamped to [0, T], not checked;
+ *              tokens outside every sequence keep their y values); without
+ *              it, B rows of T tokens
+ *   y          same shape and dtype as x (written), must not alias x
+ * Supported: dtype KDA_BF16 or KDA_F32, W in [1,4], d % 8 == 0. All tensors
+ * 16-byte aligned (cu_seqlens 4-byte). B, T, H or d = 0 is a no-op.
+ */
+int kda_short_conv_swish(const void *x, const float *weight, const int32_t *cu_seqlens, void *y,
+                         int B, int T, int H, int d, int W, int dtype, void *stream);
+
+/*
  * Backward pass of kda_chunk_fwd: the gradients of a scalar loss L with respect
  * to q, k, v, log_alpha, beta and S0, given dL/d(out) and dL/d(S_T). The pages
  * print no backward pass; this is the derivative of the same recurrence, in

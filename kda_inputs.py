@@ -187,6 +187,30 @@ def prefill_layer_inputs(w: Prefill | str, device="cpu", **override) -> dict:
                 beta=beta.contiguous(), S0=S0, w=w)
 
 
+def layer_extras(w: Prefill | str, device="cpu", conv_width: int = 4, **override) -> dict:
+    """Seeded synthetic weights and data of the layer steps around the recurrence (the
+    pages give no trained weights): the output gate's pre-activation z ~ N(0,1)
+    ``[B,T,H,dv]`` (workload dtype), the RMSNorm weight 1 + 0.1 N(0,1) ``[dv]`` fp32,
+    ShortConv filters for q, k and v ~ N(0, 0.5^2) ``[H,d,conv_width]`` fp32, and
+    pre-convolution inputs x_q, x_k, x_v ~ N(0,1) ``[B,T,H,d]`` (workload dtype).
+    Drawn from the workload's seed + 1000, in that order."""
+    if isinstance(w, str):
+        w = WORKLOADS[w]
+    if override:
+        w = dataclasses.replace(w, **override)
+    g = _gen(w.seed + 1000, device)
+    B, T, H, dk, dv = w.B, w.T, w.H, w.dk, w.dv
+    f32 = dict(device=device, dtype=torch.float32, generator=g)
+    z = torch.randn(B, T, H, dv, **f32).to(w.dtype).contiguous()
+    norm_w = (1.0 + 0.1 * torch.randn(dv, **f32)).contiguous()
+    conv = {n: (0.5 * torch.randn(H, d, conv_width, **f32)).contiguous()
+            for n, d in (("q", dk), ("k", dk), ("v", dv))}
+    pre = {n: torch.randn(B, T, H, d, **f32).to(w.dtype).contiguous()
+           for n, d in (("q", dk), ("k", dk), ("v", dv))}
+    return dict(out_gate=z, norm_weight=norm_w, conv_q=conv["q"], conv_k=conv["k"], conv_v=conv["v"],
+                x_q=pre["q"], x_k=pre["k"], x_v=pre["v"], w=w)
+
+
 def packed_lengths(n: int, lo: int, hi: int, seed: int = 5) -> list[int]:
     """Lengths of n packed sequences for the variable-length prefill: uniform integers
     in [lo, hi] from a generator seeded with `seed` (a mix of short and long prompts)."""

@@ -123,3 +123,14 @@ def test_layer_inputs_recipe():
     np.testing.assert_allclose(las[..., 2::8].numpy(), -12.0, rtol=2e-2)
     sl = I.prefill_layer_inputs("prefill_32k", T=2048, H=4)
     assert abs(sl["gate"].float().mean().item() + 2.0) < 0.02     # x ~ N(-2, 1): the slow recipe
+
+
+def test_layer_extras_shapes_and_determinism():
+    a = I.layer_extras("prefill_4k", B=1, T=5, H=2, conv_width=3)
+    b = I.layer_extras("prefill_4k", B=1, T=5, H=2, conv_width=3)
+    assert a["out_gate"].shape == (1, 5, 2, 128) and a["out_gate"].dtype == torch.bfloat16
+    assert a["norm_weight"].shape == (128,) and a["norm_weight"].dtype == torch.float32
+    assert a["conv_q"].shape == (2, 128, 3) and a["x_v"].shape == (1, 5, 2, 128)
+    for key in ("out_gate", "norm_weight", "conv_q", "conv_k", "conv_v", "x_q", "x_k", "x_v"):
+        assert torch.equal(a[key], b[key])
+    assert abs(float(a["norm_weight"].mean()) - 1.0) < 0.05
