@@ -211,6 +211,29 @@ def layer_extras(w: Prefill | str, device="cpu", conv_width: int = 4, **override
                 x_q=pre["q"], x_k=pre["k"], x_v=pre["v"], w=w)
 
 
+def dplr_inputs(w: Prefill | str, device="cpu", **override) -> dict:
+    """Inputs of the general DPLR recurrence S_t = (Diag(alpha_t) + a_t b_t^T) S_{t-1} + k_t v_t^T
+    (the comparator of KDA's operator efficiency): q, k, v, log alpha and S0 as
+    ``prefill_inputs`` (same draws), and two low-rank vectors drawn from the workload's
+    seed + 2000: a = -gamma * unit(r1) with gamma = sigmoid(N(0,1)) per token, and
+    b = e^{log alpha} * unit(r1 + 0.5 r2) (r1, r2 ~ N(0,1) per channel), so that a and b
+    differ but the transition stays contracting, as KDA's does. a and b in the
+    workload's dtype."""
+    base = prefill_inputs(w, device=device, **override)
+    w = base["w"]
+    g = _gen(w.seed + 2000, device)
+    f32 = dict(device=device, dtype=torch.float32, generator=g)
+    B, T, H, dk = w.B, w.T, w.H, w.dk
+    r1 = torch.randn(B, T, H, dk, **f32)
+    r2 = torch.randn(B, T, H, dk, **f32)
+    gamma = torch.sigmoid(torch.randn(B, T, H, **f32))
+    a = -gamma[..., None] * _unit_rows(r1)
+    b = torch.exp(base["log_alpha"]) * _unit_rows(r1 + 0.5 * r2)
+    base["a"] = a.to(w.dtype).contiguous()
+    base["b"] = b.to(w.dtype).contiguous()
+    return base
+
+
 def packed_lengths(n: int, lo: int, hi: int, seed: int = 5) -> list[int]:
     """Lengths of n packed sequences for the variable-length prefill: uniform integers
     in [lo, hi] from a generator seeded with `seed` (a mix of short and long prompts)."""
