@@ -10,9 +10,11 @@ over all ranks. The decode row is timed in the same run on the ``decode_256``
 workload (256 sequences x 32 heads, 128x128 fp32 states, 1000 consecutive
 steps) and reported under ``"decode"`` as state GB/s. Outside the timed region
 the same run also times, each with its own roofline fraction: the prefill with
-the layer prologue fused in (``"fused_prologue"``), the backward pass on
-prefill_4k's shape (``"backward"``) and the packed variable-length prefill into
-a state cache (``"varlen"``).
+the layer prologue fused in (``"fused_prologue"``), the whole layer between
+its projections with seeded synthetic weights (``"layer"``), the backward pass on
+prefill_4k's shape (``"backward"``), the packed variable-length prefill into
+a state cache (``"varlen"``) and KDA against the general DPLR recurrence on the
+same CUDA-core engine design (``"dplr_comparator"``).
 
 Heads and batches are independent, so with N GPUs every rank runs its own copy
 of the workload (weak scaling, no collective on the data path); the timed
@@ -223,7 +225,9 @@ def run_ours(args, rank, world, device):
                 "tensor_tflops_achieved": round(prefill_flops(w) / (ms_kernel / 1e3) / 1e12, 2)}
 
     fused = run_fused(kda, w, ws, args, device, stream) if engine == "tc_cluster" else None
+    layer = run_layer(kda, w, ws, args, device, stream) if engine == "tc_cluster" else None
     backward = run_backward(kda, args, device, stream) if not args.skip_extra_legs else None
+    dplr = run_dplr(kda, args, device, stream) if not args.skip_extra_legs else None
     varlen = run_varlen(kda, args, device, stream) if not args.skip_extra_legs else None
     e2e = run_e2e(kda, w, inp, engine, ws, args, device, stream, world)
     decode = run_decode(kda, args, device, stream, world)
@@ -246,8 +250,8 @@ def run_ours(args, rank, world, device):
                        "engine": engine, "per_rank": "one full workload per GPU",
                        "l2": f"inputs larger than L2 ({bytes_alg / 1e9:.2f} GB moved per step)"},
             "roofline": roofline, "e2e": e2e, "gpu_launches": launches + decode.pop("launches"),
-            "clocks": clocks, "decode": decode, "fused_prologue": fused, "backward": backward,
-            "varlen": varlen, "cpu_baseline": cpu,
+            "clocks": clocks, "decode": decode, "fused_prologue": fused, "layer": layer, "backward": backward,
+            "varlen": varlen, "dplr_comparator": dplr, "cpu_baseline": cpu,
         }
         print(json.dumps(line), flush=True)
 
@@ -279,6 +283,85 @@ def run_fused(kda, w, ws, args, device, stream):
             "tokens_per_s": round(w.tokens / (ms / 1e3), 1), "bytes_per_launch": bytes_alg,
             "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm, "unit": "GB/s",
                          "frac": round(gbs / hbm, 4), "peak_source": src}}
+
+
+def run_layer(kda, w, ws, args, device, stream):
+    """The layer between its projections on the bench workload's shape, with seeded
+    synthetic weights (kda_inputs.layer_extras): ShortConv + Swish on the projected q,
+    k and v (three kda_short_conv_swish launches, W = 4), then kda_layer_fwd (L2 norm,
+    gate, recurrence, per-head RMSNorm, sigmoid output gate). Algorithmic bytes per
+    token-head at d = 128, bf16: ShortConv 3 x (256 read + 256 written) = 1536; the
+    layer kernel 3 x 256 (q, k, v) + 256 (gate) + 4 (beta) + 256 (output gate) + 256
+    (out) = 1540, plus S0 read and S_T written per head."""
+    lw = I.prefill_layer_inputs(w, device=device)
+    ex = I.layer_extras(w, device=device)
+    conv = {n: torch.empty_like(ex[f"x_{n}"]) for n in ("q", "k", "v")}
+    out = torch.empty(w.B, w.T, w.H, w.dv, device=device, dtype=w.dtype)
+    S_T = torch.empty(w.B, w.H, w.dk, w.dv, device=device, dtype=torch.float32)
+
+    def convs():
+        for n in ("q", "k", "v"):
+            kda.short_conv_swish(ex[f"x_{n}"], ex[f"conv_{n}"], out=conv[n], stream=stream)
+
+    def core():
+        kda.layer_fwd(conv["q"], conv["k"], conv["v"], lw["gate"], lw["beta"], ex["out_gate"],
+                      ex["norm_weight"], lw["S0"], out=out, S_T=S_T, workspace=ws, stream=stream)
+
+    for _ in range(max(1, args.warmup)):
+        convs()
+        core()
+    torch.cuda.synchronize(device)
+    n = max(1, min(args.steps, 5))
+    ev_c = time_events(convs, n, stream)
+    ev_l = time_events(core, n, stream)
+    torch.cuda.synchronize(device)
+    ms_c = statistics.mean(a.elapsed_time(b) for a, b in ev_c)
+    ms_l = statistics.mean(a.elapsed_time(b) for a, b in ev_l)
+    th = w.tokens * w.H
+    heads_state = w.B * w.H * 4 * w.dk * w.dv * (2 if w.s0_std > 0 else 1)
+    b_conv, b_core = th * 1536, th * 1540 + heads_state
+    hbm, src = peaks()
+
+    def roof(b, ms):
+        gbs = b / (ms / 1e3) / 1e9
+        return {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm, "unit": "GB/s",
+                "frac": round(gbs / hbm, 4), "peak_source": src}
+    return {"entries": "3 x kda_short_conv_swish + kda_layer_fwd", "weights": "seeded synthetic (kda_inputs.layer_extras)",
+            "ms": round(ms_c + ms_l, 4), "tokens_per_s": round(w.tokens / ((ms_c + ms_l) / 1e3), 1),
+            "short_conv": {"kernel_ms": round(ms_c, 4), "bytes": b_conv, "roofline": roof(b_conv, ms_c)},
+            "layer_fwd": {"kernel_ms": round(ms_l, 4), "bytes": b_core, "roofline": roof(b_core, ms_l)}}
+
+
+def run_dplr(kda, args, device, stream):
+    """KDA against the general DPLR recurrence on the same CUDA-core engine design
+    (kda_chunk_fwd_engine with KDA_ENGINE_GENERIC vs kda_dplr_chunk_fwd; chunk 32, the
+    largest both fit in shared memory at d = 128), per input length: B x T = 16384
+    tokens of H = 32 heads, bf16 inputs, T = 2048 and 8192. The ratio DPLR time / KDA
+    time re-measures the operator-efficiency comparison of the pages on B200."""
+    res = []
+    for T in (2048, 8192):
+        inp = I.dplr_inputs("prefill_4k", device=device, B=16384 // T, T=T)
+        w = inp["w"]
+        out = torch.empty(w.B, w.T, w.H, w.dv, device=device, dtype=w.dtype)
+
+        def kda_step():
+            kda.chunk_fwd(inp["q"], inp["k"], inp["v"], inp["log_alpha"], inp["beta"], None, 32,
+                          out=out, engine="generic", output_final_state=False, stream=stream)
+
+        def dplr_step():
+            kda.dplr_chunk_fwd(inp["q"], inp["k"], inp["v"], inp["a"], inp["b"], inp["log_alpha"], None,
+                               32, out=out, output_final_state=False, stream=stream)
+
+        ms = {}
+        for name, fn in (("kda", kda_step), ("dplr", dplr_step)):
+            fn()
+            torch.cuda.synchronize(device)
+            evs = time_events(fn, max(1, min(args.steps, 3)), stream)
+            torch.cuda.synchronize(device)
+            ms[name] = statistics.mean(a.elapsed_time(b) for a, b in evs)
+        res.append({"T": T, "B": w.B, "kda_generic_ms": round(ms["kda"], 3), "dplr_ms": round(ms["dplr"], 3),
+                    "dplr_over_kda": round(ms["dplr"] / ms["kda"], 3)})
+    return {"engines": "fp32 CUDA cores, chunk 32, H=32, d=128, bf16 inputs", "by_length": res}
 
 
 def run_backward(kda, args, device, stream):

@@ -11,10 +11,11 @@ The compute runs in ``libkda.so`` (hand-written CUDA, C ABI in
     out = recurrent_step(q, k, v, log_alpha, beta, state, slot)
 """
 from .binding import (ENGINES, KDA_BF16, KDA_F32, LIB_PATH, KdaError, bwd_workspace_bytes, chunk_bwd,
-                      chunk_fwd, chunk_fwd_fused, chunk_fwd_varlen, device_status, engine_supported, layer_fwd,
+                      chunk_fwd, chunk_fwd_fused, chunk_fwd_varlen, device_status, dplr_chunk_fwd, engine_supported,
+                      layer_fwd,
                       load, recurrent_step, short_conv_swish, varlen_workspace_bytes,
                       workspace_bytes)
 from .autograd import kda_prefill
 
-__all__ = ["chunk_fwd", "chunk_fwd_fused", "chunk_fwd_varlen", "chunk_bwd", "kda_prefill", "recurrent_step", "workspace_bytes", "bwd_workspace_bytes", "varlen_workspace_bytes", "short_conv_swish", "layer_fwd", "device_status",
+__all__ = ["chunk_fwd", "chunk_fwd_fused", "chunk_fwd_varlen", "chunk_bwd", "kda_prefill", "recurrent_step", "workspace_bytes", "bwd_workspace_bytes", "varlen_workspace_bytes", "short_conv_swish", "layer_fwd", "dplr_chunk_fwd", "device_status",
            "engine_supported", "load", "KdaError", "ENGINES", "KDA_BF16", "KDA_F32", "LIB_PATH"]

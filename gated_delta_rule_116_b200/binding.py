@@ -55,6 +55,8 @@ def load():
     lib.kda_chunk_fwd_varlen_engine.restype = i
     lib.kda_layer_fwd.argtypes = [p, p, p, p, p, p, p, ctypes.c_float, p, p, p, i, i, i, i, i, i, i, p, sz, p]
     lib.kda_layer_fwd.restype = i
+    lib.kda_dplr_chunk_fwd.argtypes = [p] * 9 + [i] * 7 + [p]
+    lib.kda_dplr_chunk_fwd.restype = i
     lib.kda_short_conv_swish.argtypes = [p, p, p, p, i, i, i, i, i, i, p]
     lib.kda_short_conv_swish.restype = i
     lib.kda_varlen_workspace_bytes.argtypes = [i, i, i, i, i]
@@ -317,6 +319,36 @@ def chunk_fwd_varlen(q, k, v, log_alpha, beta, cu_seqlens, S0=None, *, slot=None
             ENGINES[engine], _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(cu_seqlens),
             _ptr(slot), _ptr(S0), _ptr(out), _ptr(S_T), N, TT, H, dk, dv, _DTYPES[q.dtype],
             _ptr(workspace), ws_bytes, _stream(device, stream))
+    _check(rc)
+    return out, S_T
+
+
+def dplr_chunk_fwd(q, k, v, a, b, log_alpha, S0=None, chunk: int = 32, *, out=None, S_T=None,
+                   output_final_state: bool = True, stream=None):
+    """The general DPLR comparator (``kda_dplr_chunk_fwd``): S_t = (Diag(alpha_t) + a_t b_t^T)
+    S_{t-1} + k_t v_t^T, o_t = S_t^T q_t, fp32 CUDA cores. q, k, a, b ``[B,T,H,dk]`` and v in
+    one dtype (bf16 or fp32), log_alpha fp32. Returns ``(out, S_T)``."""
+    lib = load()
+    device = q.device
+    _require(q, "q", device)
+    if q.dtype not in _DTYPES:
+        raise TypeError(f"q must be bf16 or fp32 (got {q.dtype})")
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    for t, name in ((k, "k"), (a, "a"), (b, "b")):
+        _require(t, name, device, q.dtype, (B, T, H, dk))
+    _require(v, "v", device, q.dtype, (B, T, H, dv))
+    _require(log_alpha, "log_alpha", device, torch.float32, (B, T, H, dk))
+    if S0 is not None:
+        _require(S0, "S0", device, torch.float32, (B, H, dk, dv))
+    if out is None:
+        out = torch.empty(B, T, H, dv, device=device, dtype=q.dtype)
+    if S_T is None and output_final_state:
+        S_T = torch.empty(B, H, dk, dv, device=device, dtype=torch.float32)
+    with torch.cuda.device(device):
+        rc = lib.kda_dplr_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(a), _ptr(b), _ptr(log_alpha), _ptr(S0),
+                                    _ptr(out), _ptr(S_T), B, T, H, dk, dv, chunk, _DTYPES[q.dtype],
+                                    _stream(device, stream))
     _check(rc)
     return out, S_T
 

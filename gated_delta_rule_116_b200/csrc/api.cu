@@ -442,6 +442,32 @@ int kda_short_conv_swish(const void *x, const float *weight, const int32_t *cu_s
     return e == cudaSuccess ? KDA_OK : cuda_fail(e, "launching the short convolution");
 }
 
+int kda_dplr_chunk_fwd(const void *q, const void *k, const void *v, const void *a, const void *b,
+                       const float *log_alpha, const float *S0, void *out, float *S_T, int B, int T, int H,
+                       int dk, int dv, int chunk, int dtype, void *stream) {
+    g_detail[0] = '\0';
+    if (B < 0 || T < 0 || H < 0)
+        return fail(KDA_ERR_INVALID_ARG, "B=%d T=%d H=%d must be >= 0", B, T, H);
+    int rc = check_common(dk, dv, dtype);
+    if (rc != KDA_OK) return rc;
+    if (chunk != 16 && chunk != 32) return fail(KDA_ERR_UNSUPPORTED, "chunk=%d is not 16 or 32", chunk);
+    if (kda::chunk_dplr_smem_bytes(chunk, dk, dv) > 227u * 1024u)
+        return fail(KDA_ERR_UNSUPPORTED, "chunk=%d with dk=%d: shared memory beyond 227 KB", chunk, dk);
+    if (static_cast<long long>(B) * T > INT_MAX || static_cast<long long>(B) * H > INT_MAX / 4)
+        return fail(KDA_ERR_UNSUPPORTED, "B*T = %lld, B*H = %lld: split the batch",
+                    static_cast<long long>(B) * T, static_cast<long long>(B) * H);
+    if (B == 0 || H == 0) return KDA_OK;
+    const bool tokens = T > 0;
+    const Ptr ps[] = {{q, "q", tokens}, {k, "k", tokens}, {v, "v", tokens}, {a, "a", tokens},
+                      {b, "b", tokens}, {log_alpha, "log_alpha", tokens}, {out, "out", tokens},
+                      {S0, "S0", false}, {S_T, "S_T", false}};
+    rc = check_pointers(ps, sizeof ps / sizeof ps[0]);
+    if (rc != KDA_OK) return rc;
+    cudaError_t e = kda::launch_chunk_dplr(q, k, v, a, b, log_alpha, S0, out, S_T, B, T, H, dk, dv, chunk,
+                                           dtype, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? KDA_OK : cuda_fail(e, "launching the DPLR comparator");
+}
+
 int kda_device_status(void *stream) {
     g_detail[0] = '\0';
     cudaStream_t s = static_cast<cudaStream_t>(stream);

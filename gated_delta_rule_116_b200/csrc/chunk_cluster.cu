@@ -234,6 +234,14 @@ __device__ __forceinline__ float neg_softplus(float x) {
     return -(fmaxf(x, 0.f) + l);
 }
 
+// tanh by the hardware approximation (relative error about 2^-11, below the bf16
+// rounding of the outputs it scales).
+__device__ __forceinline__ float tanh_fast(float x) {
+    float y;
+    asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 // Inclusive prefix sum over the 8 lanes 4g + t (g = 0..7) that share t.
 __device__ __forceinline__ float scan8(float x, int g) {
     float y = __shfl_up_sync(0xffffffffu, x, 4);
@@ -877,7 +885,7 @@ __device__ void consumer(uint8_t *sm, uint32_t tmem, const uint8_t *ring, const 
                          __nv_bfloat16 *__restrict__ out, float *S_T, int T, int H,
                          int h, long srow, long ztok, int nchunks, const Ctl &ctl,
                          const __nv_bfloat16 *__restrict__ out_gate, const float *__restrict__ norm_w,
-                         float eps) {
+                         float eps, const CUtensorMap *tm_z) {
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int quad = warp & 3, half = warp >> 2;
     const int row = 32 * quad + lane;   // TMEM lane; state row (key channel)
@@ -965,11 +973,17 @@ __device__ void consumer(uint8_t *sm, uint32_t tmem, const uint8_t *ring, const 
         }
     }
 
+    if (kGated && tid == 32)   // the output gate's rows of the first two chunks, into L2
+        for (int c2 = 0; c2 < 2 && c2 < nchunks; ++c2)
+            tc::tma_prefetch_l2_3d(tm_z, 0, h, static_cast<int>(ztok + c2 * kC));
     for (int c = 0; c < nchunks; ++c) {
         if (__syncthreads_or(aborted(ctl))) break;   // uniform: the cluster gave up
         const int s = c & 1;
         const int t0 = c * kC;
         const int valid = min(kC, T - t0);
+        // the epilogue reads the output gate's rows from L2, two chunks after their prefetch
+        if (kGated && tid == 32 && c + 2 < nchunks)
+            tc::tma_prefetch_l2_3d(tm_z, 0, h, static_cast<int>(ztok + (c + 2) * kC));
         const uint8_t *slot = sm + C_SLOT + s * kSlotStride;
         const uint32_t xcol = CCOL_X + s * 128;
         if (wait_local(full + s, (ph_full >> s) & 1, ctl)) {  // (already complete) makes the slot visible
@@ -1062,14 +1076,34 @@ __device__ void consumer(uint8_t *sm, uint32_t tmem, const uint8_t *ring, const 
             pend_o = false;
         }
         tc_fence_after();
-        float o[64];
-        if (quad < 2) {
-            const uint32_t ta = tc::tmem_addr(tmem, 32 * quad, xcol + half * 64);
-            tc::tmem_ld32(ta, *reinterpret_cast<float(*)[32]>(&o[0]));
-            tc::tmem_ld32(ta + 32, *reinterpret_cast<float(*)[32]>(&o[32]));
-            tc::tmem_wait_ld();
-            if (kGated) {   // this thread's half of the row's sum of squares
-                float ss0 = 0.f, ss1 = 0.f;
+        if constexpr (!kGated) {
+            if (quad < 2) {
+                float o[64];
+                const uint32_t ta = tc::tmem_addr(tmem, 32 * quad, xcol + half * 64);
+                tc::tmem_ld32(ta, *reinterpret_cast<float(*)[32]>(&o[0]));
+                tc::tmem_ld32(ta + 32, *reinterpret_cast<float(*)[32]>(&o[32]));
+                tc::tmem_wait_ld();
+                if (row < valid) {
+                    uint4 *dst = reinterpret_cast<uint4 *>(out + ((ztok + t0 + row) * H + h) * kD + half * 64);
+#pragma unroll
+                    for (int u = 0; u < 64; u += 8) {
+                        uint4 x;
+                        x.x = pack_bf16(o[u], o[u + 1]);
+                        x.y = pack_bf16(o[u + 2], o[u + 3]);
+                        x.z = pack_bf16(o[u + 4], o[u + 5]);
+                        x.w = pack_bf16(o[u + 6], o[u + 7]);
+                        dst[u / 8] = x;
+                    }
+                }
+            }
+        } else {   // the layer epilogue: RMSNorm over the row's 128 channels, then the output gate
+            float o[64];
+            if (quad < 2) {
+                const uint32_t ta = tc::tmem_addr(tmem, 32 * quad, xcol + half * 64);
+                tc::tmem_ld32(ta, *reinterpret_cast<float(*)[32]>(&o[0]));
+                tc::tmem_ld32(ta + 32, *reinterpret_cast<float(*)[32]>(&o[32]));
+                tc::tmem_wait_ld();
+                float ss0 = 0.f, ss1 = 0.f;   // this thread's half of the row's sum of squares
 #pragma unroll
                 for (int j = 0; j < 64; j += 2) {
                     ss0 = fmaf(o[j], o[j], ss0);
@@ -1077,11 +1111,9 @@ __device__ void consumer(uint8_t *sm, uint32_t tmem, const uint8_t *ring, const 
                 }
                 red[2 * row + half] = ss0 + ss1;
             }
-        }
-        if (kGated) __syncthreads();
-        if (quad < 2 && row < valid) {
-            const long orow = ((ztok + t0 + row) * H + h) * kD + half * 64;
-            if (kGated) {
+            __syncthreads();
+            if (quad < 2 && row < valid) {
+                const long orow = ((ztok + t0 + row) * H + h) * kD + half * 64;
                 const float r = rsqrtf((red[2 * row] + red[2 * row + 1]) * (1.f / kD) + eps);
                 const uint4 *zp = reinterpret_cast<const uint4 *>(out_gate + orow);
 #pragma unroll
@@ -1092,20 +1124,21 @@ __device__ void consumer(uint8_t *sm, uint32_t tmem, const uint8_t *ring, const 
                     for (int m = 0; m < 4; ++m) {
                         const float z0 = tc::bf16_lo(zw[m]), z1 = tc::bf16_hi(zw[m]);
                         const int j = u + 2 * m;
-                        o[j] *= r * nw[half * 64 + j] / (1.f + tc::ex2(-z0 * kLog2e));
-                        o[j + 1] *= r * nw[half * 64 + j + 1] / (1.f + tc::ex2(-z1 * kLog2e));
+                        // sigmoid(z) = (1 + tanh(z / 2)) / 2: one MUFU operation per element
+                        o[j] *= r * nw[half * 64 + j] * fmaf(0.5f, tanh_fast(0.5f * z0), 0.5f);
+                        o[j + 1] *= r * nw[half * 64 + j + 1] * fmaf(0.5f, tanh_fast(0.5f * z1), 0.5f);
                     }
                 }
-            }
-            uint4 *dst = reinterpret_cast<uint4 *>(out + orow);
+                uint4 *dst = reinterpret_cast<uint4 *>(out + orow);
 #pragma unroll
-            for (int u = 0; u < 64; u += 8) {
-                uint4 x;
-                x.x = pack_bf16(o[u], o[u + 1]);
-                x.y = pack_bf16(o[u + 2], o[u + 3]);
-                x.z = pack_bf16(o[u + 4], o[u + 5]);
-                x.w = pack_bf16(o[u + 6], o[u + 7]);
-                dst[u / 8] = x;
+                for (int u = 0; u < 64; u += 8) {
+                    uint4 x;
+                    x.x = pack_bf16(o[u], o[u + 1]);
+                    x.y = pack_bf16(o[u + 2], o[u + 3]);
+                    x.z = pack_bf16(o[u + 4], o[u + 5]);
+                    x.w = pack_bf16(o[u + 6], o[u + 7]);
+                    dst[u / 8] = x;
+                }
             }
         }
         tc_fence_before();
@@ -1135,7 +1168,8 @@ chunk_cluster_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_cons
                      float *S_T, uint8_t *__restrict__ ws, int T, int H, int *err,
                      int test_timeout, const int32_t *__restrict__ cu_seqlens,
                      const int32_t *__restrict__ slot, const __nv_bfloat16 *__restrict__ out_gate,
-                     const float *__restrict__ norm_w, float norm_eps) {
+                     const float *__restrict__ norm_w, float norm_eps,
+                     const __grid_constant__ CUtensorMap tm_z) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~static_cast<uintptr_t>(1023));
@@ -1182,7 +1216,7 @@ chunk_cluster_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_cons
     uint8_t *ring = ws + bh * kRingSlots * kSlotStride;  // this head's ring: kRingDepth slots per producer
     if (is_consumer)
         consumer<kGated>(sm, tmem, ring, S0, out, S_T, len, H, h, srow, ztok, nchunks, ctl, out_gate,
-                         norm_w, norm_eps);
+                         norm_w, norm_eps, &tm_z);
     else
         producer<kFused>(sm, tmem, rank, ring, &tm_v, &tm_qs, &tm_ks, &tm_las, beta, len, H, h, ztok, nchunks,
                          ctl, test_timeout);
@@ -1258,8 +1292,11 @@ cudaError_t launch_chunk_cluster(const ChunkArgs &a, cudaStream_t s) {
         (fused ? make_map(&mlas, a.gate, kB16, 2, a.H, tokens, true)
                : make_map(&mlas, a.log_alpha, kF32, 4, a.H, tokens, true));
     if (!ok) return cudaErrorInvalidValue;
-    // the layer epilogue comes with the layer prologue only (kda_layer_fwd)
+    // the layer epilogue comes with the layer prologue only (kda_layer_fwd); its output gate
+    // is prefetched into L2 through a map over [tokens, H, 128] bf16 (unused otherwise)
     const bool gated = fused && a.out_gate != nullptr;
+    CUtensorMap mz{};
+    if (gated && !make_map(&mz, a.out_gate, kB16, 2, a.H, tokens, false)) return cudaErrorInvalidValue;
     auto kern = gated ? chunk_cluster_kernel<true, true>
                       : (fused ? chunk_cluster_kernel<true, false> : chunk_cluster_kernel<false, false>);
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1269,7 +1306,7 @@ cudaError_t launch_chunk_cluster(const ChunkArgs &a, cudaStream_t s) {
     kern<<<grid, kThreads, kSmemBytes, s>>>(
         mv, mqs, mks, mlas, a.beta, a.S0, static_cast<__nv_bfloat16 *>(a.out), a.S_T,
         static_cast<uint8_t *>(a.workspace), a.T, a.H, a.device_error, g_test_timeout, a.cu_seqlens, a.slot,
-        static_cast<const __nv_bfloat16 *>(a.out_gate), a.norm_weight, a.norm_eps);
+        static_cast<const __nv_bfloat16 *>(a.out_gate), a.norm_weight, a.norm_eps, mz);
     return cudaGetLastError();
 }
 

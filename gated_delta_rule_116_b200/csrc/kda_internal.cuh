@@ -78,6 +78,11 @@ cudaError_t launch_chunk_varlen(const void *q, const void *k, const void *v, con
 // ShortConv + Swish (short_conv.cu): dense [B,T,H,d], or B packed sequences over T tokens.
 cudaError_t launch_short_conv_swish(const void *x, const float *w, void *y, const int32_t *cu_seqlens,
                                     int B, int T, int H, int d, int W, int dtype, cudaStream_t s);
+// General DPLR comparator (chunk_dplr.cu).
+size_t chunk_dplr_smem_bytes(int chunk, int dk, int dv);
+cudaError_t launch_chunk_dplr(const void *q, const void *k, const void *v, const void *a, const void *b,
+                              const float *la, const float *S0, void *out, float *S_T, int B, int T, int H,
+                              int dk, int dv, int chunk, int dtype, cudaStream_t s);
 // Ring of operand images of the cluster engine: 3 producers x 3 slots of 81 KB per head.
 constexpr size_t kClusterRingBytesPerHead = 9ull * 82944;
 

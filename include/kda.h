@@ -268,6 +268,27 @@ int kda_layer_fwd(const void *q, const void *k, const void *v, const void *gate,
                   int chunk, int dtype, void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * The comparator of KDA's operator efficiency: the chunked forward of the general
+ * diagonal-plus-low-rank delta recurrence (Kimi Linear summary, section "Menor
+ * cantidad de operaciones que DPLR general": KDA ties both low-rank vectors of the
+ * DPLR transition to the key, halving the secondary-chunk products and removing
+ * three matrix products, for about twice the operator efficiency; the page gives
+ * the claim, not the formula). Per head, with a d_k x d_v fp32 state,
+ *     S_t = (Diag(e^{log_alpha_t}) + a_t b_t^T) S_{t-1} + k_t v_t^T,  o_t = S_t^T q_t;
+ * KDA is a_t = -beta_t k_t, b_t = e^{log_alpha_t} * k_t with write vector
+ * beta_t k_t. Computes in fp32 on CUDA cores with the structure of the fp32 KDA
+ * engine (KDA_ENGINE_GENERIC), so that timing both measures the two algorithms.
+ *   q, k, a, b [B,T,H,dk] dtype;  v [B,T,H,dv] dtype;  log_alpha [B,T,H,dk] fp32
+ *   S0, S_T    [B,H,dk,dv] fp32 (NULL: zeros / skipped);  out [B,T,H,dv] dtype
+ * Supported: dtype KDA_BF16 or KDA_F32, dk, dv in [1,128], dv % 4 == 0, chunk 16
+ * or 32 (shared memory). Limits as kda_chunk_fwd. Not a product path.
+ */
+int kda_dplr_chunk_fwd(const void *q, const void *k, const void *v, const void *a,
+                       const void *b, const float *log_alpha, const float *S0, void *out,
+                       float *S_T, int B, int T, int H, int dk, int dv, int chunk,
+                       int dtype, void *stream);
+
+/*
  * The layer's q/k/v prologue ahead of the prefill: ShortConv followed by Swish
  * (Kimi Linear summary, es.news.hada.io/topic?id=31936, section "Configuracion
  * del modelo Kimi Linear": each head's queries, keys and values pass through
