@@ -1,3 +1,4 @@
+import json
 import os
 import sys
 
@@ -41,3 +42,7 @@ def pytest_terminal_summary(terminalreporter):
     for what, ma, mr, ratio in rows[:40]:
         tr.write_line(f"{what[:60]:60s} {ma:10.3e} {mr:10.3e} {ratio:9.3f}")
     tr.write_line(f"{len(rows)} comparisons; worst error/bound {rows[0][3]:.3f} ({rows[0][0]})")
+    path = os.environ.get("KDA_MARGINS_FILE")
+    if path:   # every record, for the run's evidence
+        with open(path, "w") as f:
+            json.dump([{"what": w, "max_abs": a, "max_rel": r, "err_over_bound": q} for w, a, r, q in rows], f, indent=0)

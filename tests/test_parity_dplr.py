@@ -8,7 +8,7 @@ import torch
 
 import kda_inputs as I
 import oracle
-from kda_check import assert_close, tol_for
+from kda_check import assert_close, state_max_abs, tol_for
 from oracle import dplr
 
 kda = pytest.importorskip("gated_delta_rule_116_b200")
@@ -38,7 +38,7 @@ def test_dplr_matches_oracle(name, kw, chunk):
     ref_o, ref_s = dplr.forward(inp["q"], inp["k"], inp["v"], inp["a"], inp["b"], inp["log_alpha"], inp["S0"])
     atol, rtol = tol_for(inp["q"].dtype)
     assert_close(out, ref_o, atol, rtol, f"dplr out {name} C={chunk}")
-    assert_close(st, ref_s, atol, rtol, f"dplr S_T {name} C={chunk}")
+    assert_close(st, ref_s, atol, rtol, f"dplr S_T {name} C={chunk}", max_abs=state_max_abs(inp["q"].dtype))
 
 
 def test_dplr_kernel_reproduces_kda():

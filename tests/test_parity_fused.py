@@ -12,7 +12,7 @@ import pytest
 import torch
 
 import kda_inputs as I
-from kda_check import assert_close, tol_for
+from kda_check import BF16_STATE_MAX_ABS, assert_close, tol_for
 from oracle import layer
 
 kda = pytest.importorskip("gated_delta_rule_116_b200")
@@ -31,7 +31,7 @@ def check(inp, heads=None):
     atol, rtol = tol_for(torch.bfloat16)
     ref_o, ref_s = layer.fused_forward(inp["q"], inp["k"], inp["v"], inp["gate"], inp["beta"], inp["S0"])
     assert_close(out, ref_o, atol, rtol, "fused out")
-    assert_close(st, ref_s, atol, rtol, "fused S_T")
+    assert_close(st, ref_s, atol, rtol, "fused S_T", max_abs=BF16_STATE_MAX_ABS)
 
 
 @pytest.mark.parametrize("name,kw", [

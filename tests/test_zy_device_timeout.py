@@ -14,7 +14,7 @@ import torch
 
 import kda_inputs as I
 import oracle
-from kda_check import assert_close, tol_for
+from kda_check import assert_close, state_max_abs, tol_for
 
 kda = pytest.importorskip("gated_delta_rule_116_b200")
 from gated_delta_rule_116_b200 import binding  # noqa: E402
@@ -51,4 +51,4 @@ def test_bounded_wait_gives_up_and_the_next_launch_is_correct():
                                      inp["S0"])
     atol, rtol = tol_for(torch.bfloat16)
     assert_close(out, ref_out, atol, rtol, "out after a give-up")
-    assert_close(st, ref_st, atol, rtol, "S_T after a give-up")
+    assert_close(st, ref_st, atol, rtol, "S_T after a give-up", max_abs=state_max_abs(torch.bfloat16))

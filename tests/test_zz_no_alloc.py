@@ -22,7 +22,7 @@ import torch
 
 import kda_inputs as I
 import oracle
-from kda_check import BF16_ATOL, BF16_RTOL, assert_close
+from kda_check import BF16_ATOL, BF16_RTOL, BF16_STATE_MAX_ABS, assert_close
 from gated_delta_rule_116_b200 import binding
 
 KDA_BF16 = 0
@@ -122,4 +122,4 @@ def test_static_matches_workspace_entry_point_on_two_calls_in_a_row():
     cpu = {k: (v.cpu() if isinstance(v, torch.Tensor) else v) for k, v in second.items()}
     o_ref, s_ref = oracle.forward(cpu["q"], cpu["k"], cpu["v"], cpu["la"], cpu["beta"], None)
     assert_close(second["out"], o_ref, BF16_ATOL, BF16_RTOL, "second out vs oracle")
-    assert_close(second["S_T"], s_ref, BF16_ATOL, BF16_RTOL, "second S_T vs oracle")
+    assert_close(second["S_T"], s_ref, BF16_ATOL, BF16_RTOL, "second S_T vs oracle", max_abs=BF16_STATE_MAX_ABS)
