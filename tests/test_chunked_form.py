@@ -181,3 +181,120 @@ def test_sequence_split_with_output_correction(T, split, C, seed):
                                   torch.from_numpy(S0[None, None]))
     np.testing.assert_allclose(out, ref_o[0, :, 0], rtol=1e-9, atol=1e-10)
     np.testing.assert_allclose(ST, ref_s[0, 0], rtol=1e-9, atol=1e-10)
+
+
+# --- the anchored factorisations of the intra-chunk products -----------------------------
+# The tensor-core engine never forms e^{g_i - g_j} per term; it splits the factor so that
+# every piece stays in floating-point range (the summary's secondary chunking, section
+# "Menor cantidad de operaciones que DPLR general"). These checks write both of its
+# factorisations out in NumPy and compare them with the direct products above.
+
+def direct_products(qc, kc, lc):
+    g = np.cumsum(lc, axis=0)
+    D = np.exp(np.minimum(g[:, None, :] - g[None, :, :], 0.0))   # j > i is masked below
+    n = qc.shape[0]
+    return (np.einsum("ic,jc,ijc->ij", kc, kc, D) * np.tril(np.ones((n, n)), -1),
+            np.einsum("ic,jc,ijc->ij", qc, kc, D) * np.tril(np.ones((n, n))))
+
+
+def one_anchor_products(qc, kc, lc):
+    """Factors anchored at the chunk midpoint: rows e^{g - g_C/2}, columns e^{g_C/2 - g}."""
+    g = np.cumsum(lc, axis=0)
+    ga = 0.5 * g[-1]
+    E, F = np.exp(g - ga), np.exp(ga - g)
+    n = qc.shape[0]
+    return (((kc * E) @ (kc * F).T) * np.tril(np.ones((n, n)), -1),
+            ((qc * E) @ (kc * F).T) * np.tril(np.ones((n, n))))
+
+
+def subchunk_products(qc, kc, lc, S=16, range_log=-87.0, clamp_log=-10.0):
+    """16-token sub-chunks: a block (I, J < I) as e^{g_i - G_I} e^{G_I - G_{J+1}} e^{G_{J+1} - g_j}
+    (G_I = g at the end of sub-chunk I-1; every factor <= 1); a diagonal block anchored at
+    the sub-chunk's 8th token m, e^{g_i - g_m} e^{g_m - g_j}, with the factors of a channel
+    whose sub-chunk decays below e^{range_log} taken from log alpha clamped at clamp_log."""
+    n, d = qc.shape
+    g = np.cumsum(lc, axis=0)
+    nb = n // S
+    G = np.zeros((nb + 1, d))
+    for I in range(nb):
+        G[I + 1] = g[S * I + S - 1]
+    A, P = np.zeros((n, n)), np.zeros((n, n))
+    for I in range(nb):
+        ri = slice(S * I, S * I + S)
+        for J in range(I):
+            rj = slice(S * J, S * J + S)
+            row = np.exp(g[ri] - G[I])               # e^{g_i - G_I}
+            mid = np.exp(G[I] - G[J + 1])            # e^{G_I - G_{J+1}}, per channel
+            col = np.exp(G[J + 1] - g[rj])           # e^{G_{J+1} - g_j}
+            A[ri, rj] = (kc[ri] * row * mid) @ (kc[rj] * col).T
+            P[ri, rj] = (qc[ri] * row * mid) @ (kc[rj] * col).T
+        gl = g[ri] - G[I]                            # prefix inside the sub-chunk
+        tot = gl[-1]
+        far = tot < range_log
+        glc = np.cumsum(np.maximum(lc[ri], clamp_log), axis=0)
+        gl_use = np.where(far[None, :], glc, gl)
+        m = gl_use[7]
+        rowf, colf = np.exp(gl_use - m), np.exp(m - gl_use)
+        A[ri, ri] = np.tril((kc[ri] * rowf) @ (kc[ri] * colf).T, -1)
+        P[ri, ri] = np.tril((qc[ri] * rowf) @ (kc[ri] * colf).T)
+    return A, P
+
+
+def _chunk_inputs(seed, gate):
+    rng = np.random.default_rng(seed)
+    n, d = 64, 24
+    q, k = rng.standard_normal((n, d)), rng.standard_normal((n, d))
+    q /= np.linalg.norm(q, axis=1, keepdims=True)
+    k /= np.linalg.norm(k, axis=1, keepdims=True)
+    la = -np.log1p(np.exp(rng.standard_normal((n, d))))
+    if gate == "steep":           # -5 per token: sub-chunks at e^-80, inside the anchors' range
+        la[:, 0::6], la[:, 1::6] = -5.0, 0.0
+    elif gate == "strong":        # -12 per token on some channels: sub-chunks at e^-192
+        la[:, 0::6], la[:, 1::6], la[:, 2::6] = -4.0, 0.0, -12.0
+    elif gate == "edge":          # every sub-chunk at e^-39.8: the one-anchor path's limit
+        la[:] = -2.49
+    elif gate == "far":           # sub-chunks below e^-87 on some channels: the clamped fallback
+        la[:, 0::3] = -30.0
+    return q, k, la
+
+
+@pytest.mark.parametrize("gate,seed", [("softplus", 0), ("steep", 1), ("edge", 2)])
+def test_subchunk_factorisation_is_exact(gate, seed):
+    q, k, la = _chunk_inputs(seed, gate)
+    A0, P0 = direct_products(q, k, la)
+    A1, P1 = subchunk_products(q, k, la)
+    np.testing.assert_allclose(A1, A0, rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(P1, P0, rtol=1e-10, atol=1e-12)
+
+
+@pytest.mark.parametrize("gate,seed", [("softplus", 3), ("edge", 4)])
+def test_one_anchor_factorisation_is_exact_in_range(gate, seed):
+    q, k, la = _chunk_inputs(seed, gate)
+    assert (np.cumsum(la, 0)[15::16] - np.vstack([np.zeros((1, la.shape[1])), np.cumsum(la, 0)[15::16][:-1]])).min() >= -40
+    A0, P0 = direct_products(q, k, la)
+    A1, P1 = one_anchor_products(q, k, la)
+    np.testing.assert_allclose(A1, A0, rtol=1e-9, atol=1e-12)
+    np.testing.assert_allclose(P1, P0, rtol=1e-9, atol=1e-12)
+
+
+@pytest.mark.parametrize("gate,seed", [("far", 5), ("strong", 6)])
+def test_clamped_fallback_changes_only_tiny_products(gate, seed):
+    """With log alpha = -30 or -12 on some channels (sub-chunks far below e^-87), the clamped
+    factors change only products that are below e^-10 before and after: the difference is
+    at most e^-10 times the sum of |k_i k_j| over the channels that take the fallback."""
+    q, k, la = _chunk_inputs(seed, gate)
+    A0, P0 = direct_products(q, k, la)
+    A1, P1 = subchunk_products(q, k, la)
+    g = np.cumsum(la, axis=0)
+    far = np.zeros(la.shape[1], dtype=bool)
+    for I in range(4):
+        far |= (g[16 * I + 15] - (g[16 * I - 1] if I else 0.0)) < -87.0
+    assert far.any()
+    bound_a = 2 * np.exp(-10.0) * (np.abs(k[:, far]) @ np.abs(k[:, far]).T)
+    bound_p = 2 * np.exp(-10.0) * (np.abs(q[:, far]) @ np.abs(k[:, far]).T)
+    assert np.all(np.abs(A1 - A0) <= bound_a + 1e-15)
+    assert np.all(np.abs(P1 - P0) <= bound_p + 1e-15)
+    # and the one-anchor form is out of range there: its factors overflow
+    with np.errstate(over="ignore", invalid="ignore"):
+        A2, _ = one_anchor_products(q, k, la)
+    assert not np.all(np.isfinite(A2)) or np.abs(A2 - A0).max() > 1e-6
