@@ -4,11 +4,14 @@
 // through ShortConv and Swish). ShortConv is read as a causal depthwise convolution
 // along the tokens of each sequence, one filter of W <= 4 taps per (head, channel):
 //   y_t = swish(sum_{j<W} w[h][c][j] x_{t-j}),  swish(u) = u / (1 + e^{-u}),
-// with x before a sequence's first token taken as zero.
+// with x before a sequence's first token taken as zero. Computed in fp32, rounded once
+// to the output type.
 //
-// Bandwidth-bound: each thread owns 8 channels of one head-row and walks kTile
+// Bandwidth-bound: each thread owns 8 channels of one head-row and walks kRun
 // consecutive tokens, keeping the W-1 previous inputs in registers, so every input
-// is read once (plus a W-1 token halo per tile) and every output written once. The
+// is read once (plus a W-1 token halo per run) and every output written once; its
+// loads run kAhead tokens ahead of the arithmetic, so a thread keeps that many
+// 16-byte loads in flight, and the grid is about one wave. The
 // 32 lanes of a warp cover 256 consecutive channels of one token: 512 contiguous
 // bytes per access for bf16.
 #include "kda_internal.cuh"
@@ -16,7 +19,9 @@
 namespace kda {
 namespace {
 
-constexpr int kTile = 16;
+constexpr int kRun = 128;     // consecutive tokens per thread
+// tokens loaded ahead of the arithmetic, a ring of packed registers (4 per token for bf16, 8 for fp32)
+template <typename Tin> constexpr int ahead_of() { return sizeof(Tin) == 2 ? 8 : 4; }
 constexpr int kThreadsSC = 256;
 constexpr float kLog2eSC = 1.4426950408889634f;
 
@@ -49,21 +54,54 @@ __device__ __forceinline__ void store8(float *p, const float (&x)[8]) {
     reinterpret_cast<float4 *>(p)[1] = make_float4(x[4], x[5], x[6], x[7]);
 }
 
+__device__ __forceinline__ float ex2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// A token's 8 channels as loaded (bf16: one 16-byte piece; fp32: two), widened when used.
+template <typename Tin> struct Raw8;
+template <> struct Raw8<__nv_bfloat16> {
+    uint4 v;
+    __device__ __forceinline__ void load(const __nv_bfloat16 *p) { v = *reinterpret_cast<const uint4 *>(p); }
+    __device__ __forceinline__ float at(int m) const {
+        const uint32_t word = (m >> 1) == 0 ? v.x : ((m >> 1) == 1 ? v.y : ((m >> 1) == 2 ? v.z : v.w));
+        return (m & 1) ? __uint_as_float(word & 0xffff0000u) : __uint_as_float(word << 16);
+    }
+};
+template <> struct Raw8<float> {
+    float4 a, b;
+    __device__ __forceinline__ void load(const float *p) {
+        a = reinterpret_cast<const float4 *>(p)[0];
+        b = reinterpret_cast<const float4 *>(p)[1];
+    }
+    __device__ __forceinline__ float at(int m) const {
+        const float4 &h = m < 4 ? a : b;
+        const int r = m & 3;
+        return r == 0 ? h.x : (r == 1 ? h.y : (r == 2 ? h.z : h.w));
+    }
+};
+
 // Token range [s, e) of packed sequence n, offsets clamped to [0, total].
 __device__ __forceinline__ void seq_range(const int32_t *cu, int n, long total, long &s, long &e) {
     s = min(max(static_cast<long>(cu[n]), 0L), total);
     e = min(max(static_cast<long>(cu[n + 1]), s), total);
 }
 
+// One thread: 8 channels (group g) of a run of kRun consecutive tokens starting at t0,
+// loads kept kAhead tokens ahead of the arithmetic in a register ring.
 template <typename Tin, int W>
-__global__ void __launch_bounds__(kThreadsSC)
+__global__ void __launch_bounds__(kThreadsSC, 2)
 short_conv_swish_kernel(const Tin *__restrict__ x, const float *__restrict__ w, Tin *__restrict__ y,
                         const int32_t *__restrict__ cu, int nseq, long total, int T, int H, int d) {
+    constexpr int kAhead = ahead_of<Tin>();
     const int groups = H * d / 8;   // 8-channel groups of one token's [H][d] row
     const long gid = static_cast<long>(blockIdx.x) * kThreadsSC + threadIdx.x;
     const int g = static_cast<int>(gid % groups);
-    const long t0 = (gid / groups) * kTile;
+    const long t0 = (gid / groups) * kRun;
     if (t0 >= total) return;
+    const long t1 = min(t0 + kRun, total);
     const int h = (8 * g) / d, c0 = (8 * g) % d;
     const long row = static_cast<long>(H) * d;   // elements per token
     float tap[W][8];
@@ -96,46 +134,58 @@ short_conv_swish_kernel(const Tin *__restrict__ x, const float *__restrict__ w, 
 #pragma unroll
             for (int m = 0; m < 8; ++m) prev[j - 1][m] = 0.f;
     }
-    for (int u = 0; u < kTile; ++u) {
-        const long t = t0 + u;
-        if (t >= total) break;
-        if (t >= e || t < s) {   // into the next sequence: its first tokens see zeros before them
-            if (cu) {
-                while (n + 1 < nseq && t >= e) {
-                    ++n;
-                    seq_range(cu, n, total, s, e);
+    Raw8<Tin> ring[kAhead];
+#pragma unroll
+    for (int u = 0; u < kAhead; ++u)
+        if (t0 + u < t1) ring[u].load(x + (t0 + u) * row + 8 * g);
+    for (long tb = t0; tb < t1; tb += kAhead) {
+#pragma unroll
+        for (int u = 0; u < kAhead; ++u) {
+            const long t = tb + u;
+            if (t >= t1) continue;
+            float cur[8];
+#pragma unroll
+            for (int m = 0; m < 8; ++m) cur[m] = ring[u].at(m);
+            if (t + kAhead < t1) ring[u].load(x + (t + kAhead) * row + 8 * g);   // refill the slot
+            if (t >= e || t < s) {   // into the next sequence: its first tokens see zeros before them
+                if (cu) {
+                    while (n + 1 < nseq && t >= e) {
+                        ++n;
+                        seq_range(cu, n, total, s, e);
+                    }
+                } else {
+                    s = (t / T) * T;
+                    e = s + T;
                 }
-            } else {
-                s = (t / T) * T;
-                e = s + T;
+#pragma unroll
+                for (int j = 1; j < W; ++j)
+#pragma unroll
+                    for (int m = 0; m < 8; ++m) prev[j - 1][m] = 0.f;
             }
-#pragma unroll
-            for (int j = 1; j < W; ++j)
-#pragma unroll
-                for (int m = 0; m < 8; ++m) prev[j - 1][m] = 0.f;
             if (t < s || t >= e) continue;   // outside every sequence
+            float out[8];
+#pragma unroll
+            for (int m = 0; m < 8; ++m) {
+                float a = tap[0][m] * cur[m];
+#pragma unroll
+                for (int j = 1; j < W; ++j) a = fmaf(tap[j][m], prev[j - 1][m], a);
+                // swish(a) = a / (1 + e^{-a}): hardware exp2 and a fast divide (relative error
+                // about 2^-21, far below the output's rounding; e^{-a} = inf for a << 0 gives 0)
+                out[m] = __fdividef(a, 1.f + ex2_approx(-a * kLog2eSC));
+            }
+            store8(y + t * row + 8 * g, out);
+#pragma unroll
+            for (int j = W - 1; j >= 1; --j)
+#pragma unroll
+                for (int m = 0; m < 8; ++m) prev[j - 1][m] = j == 1 ? cur[m] : prev[j - 2][m];
         }
-        float cur[8], out[8];
-        load8(x + t * row + 8 * g, cur);
-#pragma unroll
-        for (int m = 0; m < 8; ++m) {
-            float a = tap[0][m] * cur[m];
-#pragma unroll
-            for (int j = 1; j < W; ++j) a = fmaf(tap[j][m], prev[j - 1][m], a);
-            out[m] = a / (1.f + exp2f(-a * kLog2eSC));
-        }
-        store8(y + t * row + 8 * g, out);
-#pragma unroll
-        for (int j = W - 1; j >= 1; --j)
-#pragma unroll
-            for (int m = 0; m < 8; ++m) prev[j - 1][m] = j == 1 ? cur[m] : prev[j - 2][m];
     }
 }
 
 template <typename Tin>
 cudaError_t launch_typed(const void *x, const float *w, void *y, const int32_t *cu, int nseq, long total,
                          int T, int H, int d, int W, cudaStream_t s) {
-    const long threads = static_cast<long>(H) * d / 8 * ((total + kTile - 1) / kTile);
+    const long threads = static_cast<long>(H) * d / 8 * ((total + kRun - 1) / kRun);
     const unsigned blocks = static_cast<unsigned>((threads + kThreadsSC - 1) / kThreadsSC);
     const Tin *xi = static_cast<const Tin *>(x);
     Tin *yo = static_cast<Tin *>(y);
