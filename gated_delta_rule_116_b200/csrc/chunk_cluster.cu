@@ -95,6 +95,7 @@ constexpr uint32_t kSlotBytes = 82432;
 constexpr uint32_t kSlotStride = 82944;
 constexpr uint32_t kTokBlk = 8192;
 static_assert(kRingSlots * kSlotStride == kClusterRingBytesPerHead, "ring size");
+static_assert(kClusterMaxRings <= 8 * static_cast<int>(kClusterPoolHeader), "pool bitmap");
 
 // ---- producer shared memory
 // Inputs of a chunk (TMA). q, k and log alpha come as 128-byte rows in the
@@ -251,6 +252,37 @@ __device__ __forceinline__ float scan8(float x, int g) {
     y = __shfl_up_sync(0xffffffffu, x, 16);
     if (g >= 4) x += y;
     return x;
+}
+
+// Claims a free ring of the workspace's pool (bit r of the in-use bitmap), waiting
+// (bounded) while all are taken; -1 if the wait runs out. The returned ring is this
+// cluster's until release_ring: the acquire below orders the cluster's use of it after
+// the previous holder's release.
+__device__ int claim_ring(uint32_t *pool, int nrings, uint32_t limit) {
+    const int words = (nrings + 31) >> 5;
+    for (uint32_t it = 0; it < limit; ++it) {
+        for (int w = 0; w < words; ++w) {
+            const uint32_t valid = 32 * (w + 1) <= nrings ? 0xffffffffu : (1u << (nrings - 32 * w)) - 1u;
+            uint32_t free_bits = ~*reinterpret_cast<volatile uint32_t *>(pool + w) & valid;
+            while (free_bits) {
+                const int b = __ffs(free_bits) - 1;
+                const uint32_t old = atomicOr(pool + w, 1u << b);
+                if (!(old & (1u << b))) {
+                    __threadfence();
+                    tc::fence_proxy_async_global();
+                    return 32 * w + b;
+                }
+                free_bits &= ~old & ~(1u << b);
+            }
+        }
+        __nanosleep(256);
+    }
+    return -1;
+}
+// Releases ring r after every access of the cluster to it (the final cluster barrier).
+__device__ void release_ring(uint32_t *pool, int r) {
+    __threadfence();
+    atomicAnd(pool + (r >> 5), ~(1u << (r & 31)));
 }
 
 // Index of the off-diagonal block (I, J), J < I, among the six: (1,0) (2,0) (2,1) (3,0) (3,1) (3,2).
@@ -1169,7 +1201,7 @@ chunk_cluster_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_cons
                      int test_timeout, const int32_t *__restrict__ cu_seqlens,
                      const int32_t *__restrict__ slot, const __nv_bfloat16 *__restrict__ out_gate,
                      const float *__restrict__ norm_w, float norm_eps,
-                     const __grid_constant__ CUtensorMap tm_z) {
+                     const __grid_constant__ CUtensorMap tm_z, int nrings) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~static_cast<uintptr_t>(1023));
@@ -1194,10 +1226,13 @@ chunk_cluster_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_cons
     int *abort = reinterpret_cast<int *>(sm + bar_off + 132);
     const int tid = threadIdx.x;
 
+    int *ring_slot = reinterpret_cast<int *>(sm + bar_off + 136);
+    uint32_t *pool = reinterpret_cast<uint32_t *>(ws);
     if (tid == 0) {
         for (int i = 0; i < 14; ++i) tc::mbar_init(bars + i, 1);
         *abort = 0;
         tc::fence_mbar_init();
+        if (rank == 0) *ring_slot = claim_ring(pool, nrings, kWaitLimit);   // this cluster's ring
     }
     if ((tid >> 5) == 0) {
         tc::tmem_alloc(tmem_slot, kTmemCols);
@@ -1213,8 +1248,14 @@ chunk_cluster_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_cons
     for (int r = 0; r < kCluster; ++r)   // every CTA's abort flag (a producer's or the consumer's offset)
         ctl.peer_abort[r] = tc::map_to_rank(tc::smem_u32(sm) + (r == kCluster - 1 ? C_BAR : P_BAR) + 132, r);
 
-    uint8_t *ring = ws + bh * kRingSlots * kSlotStride;  // this head's ring: kRingDepth slots per producer
-    if (is_consumer)
+    // the ring rank 0 claimed (read from its shared memory after the cluster barrier above)
+    int ring_id;
+    asm volatile("ld.shared::cluster.u32 %0, [%1];"
+                 : "=r"(ring_id) : "r"(tc::map_to_rank(tc::smem_u32(sm) + P_BAR + 136, 0)) : "memory");
+    uint8_t *ring = ws + kClusterPoolHeader + static_cast<size_t>(ring_id < 0 ? 0 : ring_id) * kRingSlots * kSlotStride;
+    if (ring_id < 0) {   // no ring became free within the wait: report it and do nothing
+        if (rank == 0 && tid == 0) atomicExch(err, 2);
+    } else if (is_consumer)
         consumer<kGated>(sm, tmem, ring, S0, out, S_T, len, H, h, srow, ztok, nchunks, ctl, out_gate,
                          norm_w, norm_eps, &tm_z);
     else
@@ -1224,6 +1265,7 @@ chunk_cluster_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_cons
     tc_fence_before();
     __syncthreads();
     tc::cluster_sync();  // no CTA leaves while a peer may still touch its shared memory
+    if (rank == 0 && tid == 0 && ring_id >= 0) release_ring(pool, ring_id);   // every access to it is done
     if ((tid >> 5) == 0) {
         tc_fence_after();
         tc::tmem_dealloc(tmem, kTmemCols);
@@ -1278,7 +1320,9 @@ bool chunk_cluster_supported(int dk, int dv, int chunk, int dtype) {
 }
 
 size_t chunk_cluster_workspace_bytes(int B, int H) {
-    return static_cast<size_t>(B) * H * kRingSlots * kSlotStride;
+    const long heads = static_cast<long>(B) * H;
+    return kClusterPoolHeader + static_cast<size_t>(heads < kClusterMaxRings ? heads : kClusterMaxRings) *
+                                    kRingSlots * kSlotStride;
 }
 
 cudaError_t launch_chunk_cluster(const ChunkArgs &a, cudaStream_t s) {
@@ -1302,11 +1346,16 @@ cudaError_t launch_chunk_cluster(const ChunkArgs &a, cudaStream_t s) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(kSmemBytes));
     if (e != cudaSuccess) return e;
+    // the ring pool: as many rings as the workspace was sized for; a caller's workspace has its
+    // in-use bitmap cleared here (the library's fixed pool keeps its own clear between calls)
+    const long heads = static_cast<long>(a.B) * a.H;
+    const int nrings = static_cast<int>(heads < kClusterMaxRings ? heads : kClusterMaxRings);
+    if (!a.fixed_pool && (e = cudaMemsetAsync(a.workspace, 0, kClusterPoolHeader, s)) != cudaSuccess) return e;
     const dim3 grid(static_cast<unsigned>(a.B) * a.H * kCluster);
     kern<<<grid, kThreads, kSmemBytes, s>>>(
         mv, mqs, mks, mlas, a.beta, a.S0, static_cast<__nv_bfloat16 *>(a.out), a.S_T,
         static_cast<uint8_t *>(a.workspace), a.T, a.H, a.device_error, g_test_timeout, a.cu_seqlens, a.slot,
-        static_cast<const __nv_bfloat16 *>(a.out_gate), a.norm_weight, a.norm_eps, mz);
+        static_cast<const __nv_bfloat16 *>(a.out_gate), a.norm_weight, a.norm_eps, mz, nrings);
     return cudaGetLastError();
 }
 

@@ -7,21 +7,23 @@
 // then fails or fragments that pool); a plug-in running inside a host
 // framework that owns every allocation; code on a path where an allocation
 // would synchronise the device or is simply not allowed. Such callers pass
-// only inputs and outputs here. The scratch the engine needs -- the ring of
-// per-chunk operand images its producer CTAs hand to the state-chain CTA --
-// lives in g_static_ring below, sized for at most kMaxHeads heads (B*H).
+// only inputs and outputs here. The scratch the engine needs -- the pool of
+// rings of per-chunk operand images its producer CTAs hand to the state-chain
+// CTA -- lives in g_static_ring below: kClusterMaxRings rings behind an in-use
+// bitmap, which every cluster (one sequence and head) claims a ring from when it
+// starts and returns it to when it ends, so any number of heads fits.
 //
 // Properties a caller has to know:
-//  * every GPU that loads this library holds kStaticBytes (22.8 MiB) of device
+//  * every GPU that loads this library holds kStaticBytes (29.9 MiB) of device
 //    memory for the array until the process exits;
 //  * the first call on each device looks up the array's device address
 //    (cudaGetSymbolAddress, with that device current); make that first call
 //    before any stream capture;
-//  * all calls share the one array and it keeps the last call's contents. No
-//    part of it needs to start at zero: each chunk's image is written before
-//    it is read in the same call. Calls that overlap on the GPU (on different
-//    streams, or from different threads) race on the array and give wrong
-//    results; serialise them;
+//  * the bitmap starts clear (the array is zero when the module loads) and every
+//    call leaves it clear; the rings keep the last call's contents, and no ring
+//    needs to start at zero (each chunk's image is written before it is read).
+//    Calls that overlap on the GPU (other streams, other threads) claim
+//    different rings, so they may overlap;
 //  * nothing here allocates: no cudaMalloc, no cudaFree, no library routine
 //    that allocates.
 #include <cuda.h>
@@ -36,8 +38,7 @@
 namespace kda {
 namespace {
 
-constexpr int kMaxHeads = 32;                       // limit on B * H
-constexpr size_t kStaticBytes = kMaxHeads * kClusterRingBytesPerHead;
+constexpr size_t kStaticBytes = kClusterPoolHeader + kClusterMaxRings * kClusterRingBytesPerHead;
 constexpr int kMaxDevices = 64;
 
 static __device__ __align__(256) uint8_t g_static_ring[kStaticBytes];
@@ -111,11 +112,9 @@ extern "C" int kda_chunk_fwd_static(const void *q, const void *k, const void *v,
         return set_error_detail(KDA_ERR_UNSUPPORTED,
                                 "B*T = %lld tokens: more than 2^31 - 1; split the batch",
                                 static_cast<long long>(B) * T);
-    if (static_cast<long>(B) * H > kMaxHeads)
-        return set_error_detail(KDA_ERR_UNSUPPORTED,
-                                "B*H = %ld heads exceed the %d heads kda_chunk_fwd_static's fixed "
-                                "scratch holds; use kda_chunk_fwd with a workspace",
-                                static_cast<long>(B) * H, kMaxHeads);
+    if (static_cast<long long>(B) * H > INT_MAX / 4)
+        return set_error_detail(KDA_ERR_UNSUPPORTED, "B*H = %lld heads: more than 2^29 - 1; split the batch",
+                                static_cast<long long>(B) * H);
     if (chunk_cluster_workspace_bytes(B, H) > kStaticBytes)
         return set_error_detail(KDA_ERR_UNSUPPORTED, "fixed scratch too small for this problem");
     if (B == 0 || H == 0) return set_error_detail(KDA_OK, "");
@@ -148,6 +147,7 @@ extern "C" int kda_chunk_fwd_static(const void *q, const void *k, const void *v,
     if (!err_word) return set_error_detail(KDA_ERR_CUDA, "device error word not addressable");
     ChunkArgs a{q, k, v, log_alpha, beta, S0, out, S_T, B, T, H, dk, dv, chunk, dtype,
                 ring, kStaticBytes, err_word};
+    a.fixed_pool = true;
     e = launch_chunk_cluster(a, s);
     return e == cudaSuccess ? set_error_detail(KDA_OK, "")
                             : set_error_detail(KDA_ERR_CUDA, "launching the prefill kernel: %s",

@@ -39,6 +39,9 @@ struct ChunkArgs {
     const void *out_gate = nullptr;
     const float *norm_weight = nullptr;
     float norm_eps = 1e-6f;
+    // the workspace's ring pool is this library's fixed array: its in-use bitmap is kept
+    // clear between calls rather than cleared by each launch
+    bool fixed_pool = false;
 };
 
 struct DecodeArgs {
@@ -83,7 +86,12 @@ size_t chunk_dplr_smem_bytes(int chunk, int dk, int dv);
 cudaError_t launch_chunk_dplr(const void *q, const void *k, const void *v, const void *a, const void *b,
                               const float *la, const float *S0, void *out, float *S_T, int B, int T, int H,
                               int dk, int dv, int chunk, int dtype, cudaStream_t s);
-// Ring of operand images of the cluster engine: 3 producers x 3 slots of 81 KB per head.
+// Ring of operand images of the cluster engine: 3 producers x 3 slots of 81 KB. A workspace
+// holds a pool of rings behind a 256-byte in-use bitmap; each 4-CTA cluster (one sequence
+// and head) claims a ring when it starts and releases it when it ends, so the pool needs
+// only as many rings as clusters can be resident at once (148 SMs / 4 = 37 on B200).
 constexpr size_t kClusterRingBytesPerHead = 9ull * 82944;
+constexpr int kClusterMaxRings = 40;
+constexpr size_t kClusterPoolHeader = 256;
 
 }  // namespace kda

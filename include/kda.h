@@ -64,7 +64,12 @@ typedef enum {
 /*
  * Bytes of device workspace kda_chunk_fwd needs for this problem (0 when the
  * chosen engine needs none). Returns 0 for unsupported shapes as well; the
- * forward call reports those.
+ * forward call reports those. The tensor-core engine's workspace is a pool of
+ * operand rings behind a 256-byte in-use bitmap, min(B*H, 40) rings of
+ * 746,496 bytes (at most 29.9 MiB whatever the batch): each cluster claims a
+ * ring when it starts and returns it when it ends, and 40 is more than the
+ * clusters a B200 holds at once. The call clears the bitmap itself, so the
+ * workspace needs no initialisation.
  */
 size_t kda_workspace_bytes(int B, int T, int H, int dk, int dv, int chunk, int dtype);
 
@@ -215,9 +220,9 @@ int kda_chunk_fwd_varlen(const void *q, const void *k, const void *v,
 
 /*
  * Device scratch of kda_chunk_fwd_varlen_engine's tensor-core engine for N
- * packed sequences of H heads: the operand ring of one 4-CTA cluster per
- * (sequence, head), N*H*9*82944 bytes, independent of the lengths. 0 when the
- * engine does not support (dk, dv, dtype).
+ * packed sequences of H heads: the pool of operand rings of kda_workspace_bytes
+ * for N*H clusters (one per sequence and head), at most 29.9 MiB, independent of
+ * the lengths. 0 when the engine does not support (dk, dv, dtype).
  */
 size_t kda_varlen_workspace_bytes(int N, int H, int dk, int dv, int dtype);
 
@@ -357,14 +362,17 @@ size_t kda_bwd_workspace_bytes(int B, int T, int H, int dk, int dv, int dtype);
  * process whose pool allocator owns all free memory, or a plug-in inside a
  * framework that owns every allocation.
  *   Arguments as kda_chunk_fwd without the workspace; supported: bf16,
- *   dk = dv = 128, chunk = 64, B * H <= 32 heads and B * T <= 2^31 - 1 tokens
- *   (larger problems return KDA_ERR_UNSUPPORTED; they must use kda_chunk_fwd).
- *   Every GPU that loads the library holds the array (22.8 MiB) until exit.
- *   The first call on a device looks up the array's address with that device
- *   current (again after a device reset re-creates the context); make it
- *   before any stream capture. All calls share the array:
- *   calls that overlap on the GPU race and must be serialised by the caller.
- *   No cudaMalloc, cudaFree or allocating library routine is called.
+ *   dk = dv = 128, chunk = 64, B * T <= 2^31 - 1 tokens and B * H <= 2^29 - 1
+ *   heads (larger problems return KDA_ERR_UNSUPPORTED).
+ *   Every GPU that loads the library holds the array (29.9 MiB: a pool of 40
+ *   operand rings behind an in-use bitmap) until exit. Each 4-CTA cluster (one
+ *   sequence and head) claims a ring from the pool when it starts and returns
+ *   it when it ends, so any number of heads fits, and calls that overlap on
+ *   the GPU (other streams, other threads) claim different rings. The first
+ *   call on a device looks up the array's address with that device current
+ *   (again after a device reset re-creates the context); make it before any
+ *   stream capture. No cudaMalloc, cudaFree or allocating library routine is
+ *   called.
  */
 int kda_chunk_fwd_static(const void *q, const void *k, const void *v,
                          const float *log_alpha, const float *beta, const float *S0,
