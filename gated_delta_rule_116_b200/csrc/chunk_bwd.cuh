@@ -30,12 +30,14 @@ constexpr int kThreads = 256;
 constexpr int kC = 16;
 constexpr int kNV = 32;
 
+// Row strides are one float longer than the rows (LD = dk + 1, LC = C + 1, NP = NV + 1), so
+// that a warp reading a column (one row per lane) hits 32 different banks.
 struct Layout {
-    int dk, NV, LD, LC;
-    __host__ __device__ Layout(int dk_, int NV_) : dk(dk_), NV(NV_), LD(dk_ + 1), LC(kC + 1) {}
-    // 12 [C][LD] tiles, 7 [C][LC], 5 [C][NV], 3 [dk][NV], vectors
+    int dk, NV, NP, LD, LC;
+    __host__ __device__ Layout(int dk_, int NV_) : dk(dk_), NV(NV_), NP(NV_ + 1), LD(dk_ + 1), LC(kC + 1) {}
+    // 12 [C][LD] tiles, 7 [C][LC], 5 [C][NP], 3 [dk][NP], vectors
     __host__ __device__ size_t floats() const {
-        return 12ull * kC * LD + 7ull * kC * LC + 5ull * kC * NV + 3ull * dk * NV + 3ull * dk + 3ull * kC;
+        return 12ull * kC * LD + 7ull * kC * LC + 5ull * kC * NP + 3ull * dk * NP + 3ull * dk + 3ull * kC;
     }
 };
 
@@ -43,12 +45,12 @@ struct Tiles {
     // Qt, Kt: q and k; Qs = q e^{g}, Ks = k e^{g}, Kh = Kb = k e^{g_C - g}; G: prefix sums g
     float *Qt, *Kt, *Kh, *G, *W, *dQs, *dKb, *dW, *dKs, *dQt, *Qs, *Ks;   // [C][LD]
     float *At, *P, *X, *Tm, *dT, *dA, *dP;                      // [C][LC]
-    float *V, *Up, *U, *dO, *dU;                                 // [C][NV]
-    float *S, *dS, *dSn;                                         // [dk][NV]
+    float *V, *Up, *U, *dO, *dU;                                 // [C][NP]
+    float *S, *dS, *dSn;                                         // [dk][NP]
     float *gam, *dgam, *gsum;                                    // [dk]
     float *bt, *dbt, *pad;                                       // [C]
     __device__ Tiles(float *sm, const Layout &L) {
-        const int CD = kC * L.LD, CC = kC * L.LC, CN = kC * L.NV, DN = L.dk * L.NV;
+        const int CD = kC * L.LD, CC = kC * L.LC, CN = kC * L.NP, DN = L.dk * L.NP;
         float *p = sm;
         Qt = p; p += CD; Kt = p; p += CD; Kh = p; p += CD; G = p; p += CD; W = p; p += CD;
         dQs = p; p += CD; dKb = p; p += CD; dW = p; p += CD; dKs = p; p += CD; dQt = p; p += CD;
@@ -69,7 +71,7 @@ template <typename Tin>
 __device__ void chunk_terms(Tiles &s, const Layout &L, const Tin *q, const Tin *k, const Tin *v,
                             const float *log_alpha, const float *beta, int b, int h, int T, int H,
                             int dv, int t0, int valid, int n0, int nv, bool need_p) {
-    const int tid = threadIdx.x, dk = L.dk, LD = L.LD, LC = L.LC, NV = L.NV;
+    const int tid = threadIdx.x, dk = L.dk, LD = L.LD, LC = L.LC, NV = L.NV, NP = L.NP;
     for (int e = tid; e < kC * dk; e += kThreads) {
         const int t = e / dk, c = e - t * dk;
         float qv = 0.f, kv = 0.f, gv = 0.f;
@@ -87,7 +89,7 @@ __device__ void chunk_terms(Tiles &s, const Layout &L, const Tin *q, const Tin *
         const int t = e / NV, n = e - t * NV;
         float vv = 0.f;
         if (t < valid && n < nv) vv = to_f32(v[((static_cast<long>(b) * T + t0 + t) * H + h) * dv + n0 + n]);
-        s.V[e] = vv;
+        s.V[t * NP + n] = vv;
     }
     for (int t = tid; t < kC; t += kThreads)
         s.bt[t] = t < valid ? beta[(static_cast<long>(b) * T + t0 + t) * H + h] : 0.f;
@@ -147,8 +149,8 @@ __device__ void chunk_terms(Tiles &s, const Layout &L, const Tin *q, const Tin *
         } else {
             const int r = e - kC * dk, i = r / NV, n = r - i * NV;
             float acc = 0.f;
-            for (int j = 0; j <= i; ++j) acc = fmaf(s.Tm[i * LC + j], s.V[j * NV + n], acc);
-            s.Up[r] = acc;
+            for (int j = 0; j <= i; ++j) acc = fmaf(s.Tm[i * LC + j], s.V[j * NP + n], acc);
+            s.Up[i * NP + n] = acc;
         }
     }
     __syncthreads();
@@ -161,13 +163,13 @@ __device__ void states_body(float *sm, const Tin *q, const Tin *k, const Tin *v,
                             int dv) {
     const Layout L(dk, kNV);
     Tiles s(sm, L);
-    const int tid = threadIdx.x, LD = L.LD, NV = L.NV;
+    const int tid = threadIdx.x, LD = L.LD, NV = L.NV, NP = L.NP;
     const int bh = blockIdx.x, b = bh / H, h = bh - b * H;
     const int n0 = blockIdx.y * NV, nv = min(NV, dv - n0);
     const int nchunks = (T + kC - 1) / kC;
     for (int e = tid; e < dk * NV; e += kThreads) {
         const int c = e / NV, n = e - c * NV;
-        s.S[e] = (S0 && n < nv) ? S0[(static_cast<long>(bh) * dk + c) * dv + n0 + n] : 0.f;
+        s.S[c * NP + n] = (S0 && n < nv) ? S0[(static_cast<long>(bh) * dk + c) * dv + n0 + n] : 0.f;
     }
     for (int ch = 0; ch < nchunks; ++ch) {
         const int t0 = ch * kC, valid = min(kC, T - t0);
@@ -175,21 +177,21 @@ __device__ void states_body(float *sm, const Tin *q, const Tin *k, const Tin *v,
         float *dst = states + (static_cast<long>(bh) * nchunks + ch) * dk * dv;
         for (int e = tid; e < dk * NV; e += kThreads) {
             const int c = e / NV, n = e - c * NV;
-            if (n < nv) dst[static_cast<long>(c) * dv + n0 + n] = s.S[e];
+            if (n < nv) dst[static_cast<long>(c) * dv + n0 + n] = s.S[c * NP + n];
         }
         chunk_terms(s, L, q, k, v, log_alpha, beta, b, h, T, H, dv, t0, valid, n0, nv, false);
         for (int e = tid; e < kC * NV; e += kThreads) {   // U = U' - W S
             const int i = e / NV, n = e - i * NV;
-            float acc = s.Up[e];
-            for (int c = 0; c < dk; ++c) acc = fmaf(-s.W[i * LD + c], s.S[c * NV + n], acc);
-            s.U[e] = acc;
+            float acc = s.Up[i * NP + n];
+            for (int c = 0; c < dk; ++c) acc = fmaf(-s.W[i * LD + c], s.S[c * NP + n], acc);
+            s.U[i * NP + n] = acc;
         }
         __syncthreads();
         for (int e = tid; e < dk * NV; e += kThreads) {   // S <- Diag(gamma) S + Kb^T U
             const int c = e / NV, n = e - c * NV;
-            float acc = s.gam[c] * s.S[e];
-            for (int t = 0; t < kC; ++t) acc = fmaf(s.Kh[t * LD + c], s.U[t * NV + n], acc);
-            s.S[e] = acc;
+            float acc = s.gam[c] * s.S[c * NP + n];
+            for (int t = 0; t < kC; ++t) acc = fmaf(s.Kh[t * LD + c], s.U[t * NP + n], acc);
+            s.S[c * NP + n] = acc;
         }
     }
 }
@@ -204,13 +206,13 @@ __device__ void bwd_body(float *sm, const Tin *q, const Tin *k, const Tin *v, co
                          float *dS0, int T, int H, int dk, int dv) {
     const Layout L(dk, kNV);
     Tiles s(sm, L);
-    const int tid = threadIdx.x, LD = L.LD, LC = L.LC, NV = L.NV;
+    const int tid = threadIdx.x, LD = L.LD, LC = L.LC, NV = L.NV, NP = L.NP;
     const int bh = blockIdx.x, b = bh / H, h = bh - b * H;
     const int n0 = blockIdx.y * NV, nv = min(NV, dv - n0);
     const int nchunks = (T + kC - 1) / kC;
     for (int e = tid; e < dk * NV; e += kThreads) {
         const int c = e / NV, n = e - c * NV;
-        s.dS[e] = (dS_T && n < nv) ? dS_T[(static_cast<long>(bh) * dk + c) * dv + n0 + n] : 0.f;
+        s.dS[c * NP + n] = (dS_T && n < nv) ? dS_T[(static_cast<long>(bh) * dk + c) * dv + n0 + n] : 0.f;
     }
     for (int ch = nchunks - 1; ch >= 0; --ch) {
         const int t0 = ch * kC, valid = min(kC, T - t0);
@@ -218,11 +220,11 @@ __device__ void bwd_body(float *sm, const Tin *q, const Tin *k, const Tin *v, co
         const float *src = states + (static_cast<long>(bh) * nchunks + ch) * dk * dv;
         for (int e = tid; e < dk * NV; e += kThreads) {
             const int c = e / NV, n = e - c * NV;
-            s.S[e] = n < nv ? src[static_cast<long>(c) * dv + n0 + n] : 0.f;
+            s.S[c * NP + n] = n < nv ? src[static_cast<long>(c) * dv + n0 + n] : 0.f;
         }
         for (int e = tid; e < kC * NV; e += kThreads) {
             const int t = e / NV, n = e - t * NV;
-            s.dO[e] = (t < valid && n < nv)
+            s.dO[t * NP + n] = (t < valid && n < nv)
                           ? to_f32(dout[((static_cast<long>(b) * T + t0 + t) * H + h) * dv + n0 + n])
                           : 0.f;
         }
@@ -230,33 +232,33 @@ __device__ void bwd_body(float *sm, const Tin *q, const Tin *k, const Tin *v, co
         // U = U' - W S
         for (int e = tid; e < kC * NV; e += kThreads) {
             const int i = e / NV, n = e - i * NV;
-            float acc = s.Up[e];
-            for (int c = 0; c < dk; ++c) acc = fmaf(-s.W[i * LD + c], s.S[c * NV + n], acc);
-            s.U[e] = acc;
+            float acc = s.Up[i * NP + n];
+            for (int c = 0; c < dk; ++c) acc = fmaf(-s.W[i * LD + c], s.S[c * NP + n], acc);
+            s.U[i * NP + n] = acc;
         }
         __syncthreads();
         // dU = P^T dO + Kb dS
         for (int e = tid; e < kC * NV; e += kThreads) {
             const int j = e / NV, n = e - j * NV;
             float acc = 0.f;
-            for (int i = j; i < kC; ++i) acc = fmaf(s.P[i * LC + j], s.dO[i * NV + n], acc);
-            for (int c = 0; c < dk; ++c) acc = fmaf(s.Kh[j * LD + c], s.dS[c * NV + n], acc);
-            s.dU[e] = acc;
+            for (int i = j; i < kC; ++i) acc = fmaf(s.P[i * LC + j], s.dO[i * NP + n], acc);
+            for (int c = 0; c < dk; ++c) acc = fmaf(s.Kh[j * LD + c], s.dS[c * NP + n], acc);
+            s.dU[j * NP + n] = acc;
         }
         __syncthreads();
         // the new state gradient, and the slice's partial key-side terms
         for (int e = tid; e < dk * NV; e += kThreads) {   // dSn = Qs^T dO + Diag(gamma) dS - W^T dU
             const int c = e / NV, n = e - c * NV;
-            float acc = s.gam[c] * s.dS[e];
+            float acc = s.gam[c] * s.dS[c * NP + n];
             for (int i = 0; i < kC; ++i) {
-                acc = fmaf(s.Qs[i * LD + c], s.dO[i * NV + n], acc);
-                acc = fmaf(-s.W[i * LD + c], s.dU[i * NV + n], acc);
+                acc = fmaf(s.Qs[i * LD + c], s.dO[i * NP + n], acc);
+                acc = fmaf(-s.W[i * LD + c], s.dU[i * NP + n], acc);
             }
-            s.dSn[e] = acc;
+            s.dSn[c * NP + n] = acc;
         }
         for (int c = tid; c < dk; c += kThreads) {   // gamma's gradient (through the state decay)
             float acc = 0.f;
-            for (int n = 0; n < NV; ++n) acc = fmaf(s.dS[c * NV + n], s.S[c * NV + n], acc);
+            for (int n = 0; n < NV; ++n) acc = fmaf(s.dS[c * NP + n], s.S[c * NP + n], acc);
             s.dgam[c] = acc * s.gam[c];
         }
         for (int e = tid; e < 3 * kC * dk; e += kThreads) {   // dQs = dO S^T, dKb = U dS^T, dW = -dU S^T
@@ -265,7 +267,7 @@ __device__ void bwd_body(float *sm, const Tin *q, const Tin *k, const Tin *v, co
             const float *a = which == 0 ? s.dO : (which == 1 ? s.U : s.dU);
             const float *m = which == 1 ? s.dS : s.S;
             float acc = 0.f;
-            for (int n = 0; n < NV; ++n) acc = fmaf(a[i * NV + n], m[c * NV + n], acc);
+            for (int n = 0; n < NV; ++n) acc = fmaf(a[i * NP + n], m[c * NP + n], acc);
             (which == 0 ? s.dQs : (which == 1 ? s.dKb : s.dW))[i * LD + c] = which == 2 ? -acc : acc;
         }
         for (int e = tid; e < kC * kC + kC * NV; e += kThreads) {   // dP = lower(dO U^T), dV = T^T dU
@@ -273,12 +275,12 @@ __device__ void bwd_body(float *sm, const Tin *q, const Tin *k, const Tin *v, co
                 const int i = e / kC, j = e - i * kC;
                 float acc = 0.f;
                 if (j <= i)
-                    for (int n = 0; n < NV; ++n) acc = fmaf(s.dO[i * NV + n], s.U[j * NV + n], acc);
+                    for (int n = 0; n < NV; ++n) acc = fmaf(s.dO[i * NP + n], s.U[j * NP + n], acc);
                 s.dP[i * LC + j] = acc;
             } else {
                 const int r = e - kC * kC, j = r / NV, n = r - j * NV;
                 float acc = 0.f;
-                for (int i = j; i < kC; ++i) acc = fmaf(s.Tm[i * LC + j], s.dU[i * NV + n], acc);
+                for (int i = j; i < kC; ++i) acc = fmaf(s.Tm[i * LC + j], s.dU[i * NP + n], acc);
                 if (j < valid && n < nv)
                     dv_out[((static_cast<long>(b) * T + t0 + j) * H + h) * dv + n0 + n] = from_f32<Tin>(acc);
             }
@@ -296,7 +298,7 @@ __device__ void bwd_body(float *sm, const Tin *q, const Tin *k, const Tin *v, co
                 float acc = 0.f;
                 if (j <= i) {
                     for (int c = 0; c < dk; ++c) acc = fmaf(s.dW[i * LD + c], s.Ks[j * LD + c], acc);
-                    for (int n = 0; n < NV; ++n) acc = fmaf(s.dU[i * NV + n], s.V[j * NV + n], acc);
+                    for (int n = 0; n < NV; ++n) acc = fmaf(s.dU[i * NP + n], s.V[j * NP + n], acc);
                 }
                 s.dT[i * LC + j] = acc;
             } else {
@@ -405,7 +407,7 @@ __device__ void bwd_body(float *sm, const Tin *q, const Tin *k, const Tin *v, co
     if (dS0)
         for (int e = tid; e < dk * NV; e += kThreads) {
             const int c = e / NV, n = e - c * NV;
-            if (n < nv) dS0[(static_cast<long>(bh) * dk + c) * dv + n0 + n] = s.dS[e];
+            if (n < nv) dS0[(static_cast<long>(bh) * dk + c) * dv + n0 + n] = s.dS[c * NP + n];
         }
 }
 

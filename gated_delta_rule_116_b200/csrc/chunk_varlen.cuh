@@ -28,7 +28,7 @@ __device__ void varlen_body(float *sm, const Tin *q, const Tin *k, const Tin *v,
                             int dv) {
     const kbwd::Layout L(dk, kNV);
     kbwd::Tiles s(sm, L);
-    const int tid = threadIdx.x, LD = L.LD, LC = L.LC, NV = L.NV;
+    const int tid = threadIdx.x, LD = L.LD, LC = L.LC, NV = L.NV, NP = L.NP;
     const int nh = blockIdx.x, n = nh / H, h = nh - n * H;
     const int n0 = blockIdx.y * NV, nv = min(NV, dv - n0);
     // the offsets are device data: clamp them so that every access stays in [0, total_T)
@@ -38,7 +38,7 @@ __device__ void varlen_body(float *sm, const Tin *q, const Tin *k, const Tin *v,
     const long row = (slot ? static_cast<long>(slot[n]) : static_cast<long>(n)) * H + h;   // state row
     for (int e = tid; e < dk * NV; e += kThreads) {
         const int c = e / NV, j = e - c * NV;
-        s.S[e] = (S0 && j < nv) ? S0[(row * dk + c) * dv + n0 + j] : 0.f;
+        s.S[c * NP + j] = (S0 && j < nv) ? S0[(row * dk + c) * dv + n0 + j] : 0.f;
     }
     const int nchunks = (len + kC - 1) / kC;
     for (int ch = 0; ch < nchunks; ++ch) {
@@ -47,32 +47,32 @@ __device__ void varlen_body(float *sm, const Tin *q, const Tin *k, const Tin *v,
         kbwd::chunk_terms(s, L, q, k, v, log_alpha, beta, 0, h, total_T, H, dv, t0, valid, n0, nv, true);
         for (int e = tid; e < kC * NV; e += kThreads) {   // U = U' - W S
             const int i = e / NV, j = e - i * NV;
-            float acc = s.Up[e];
-            for (int c = 0; c < dk; ++c) acc = fmaf(-s.W[i * LD + c], s.S[c * NV + j], acc);
-            s.U[e] = acc;
+            float acc = s.Up[i * NP + j];
+            for (int c = 0; c < dk; ++c) acc = fmaf(-s.W[i * LD + c], s.S[c * NP + j], acc);
+            s.U[i * NP + j] = acc;
         }
         __syncthreads();
         for (int e = tid; e < kC * NV; e += kThreads) {   // O = Qs S + P U
             const int i = e / NV, j = e - i * NV;
             if (i >= valid || j >= nv) continue;
             float acc = 0.f;
-            for (int c = 0; c < dk; ++c) acc = fmaf(s.Qs[i * LD + c], s.S[c * NV + j], acc);
-            for (int m = 0; m <= i; ++m) acc = fmaf(s.P[i * LC + m], s.U[m * NV + j], acc);
+            for (int c = 0; c < dk; ++c) acc = fmaf(s.Qs[i * LD + c], s.S[c * NP + j], acc);
+            for (int m = 0; m <= i; ++m) acc = fmaf(s.P[i * LC + m], s.U[m * NP + j], acc);
             out[(static_cast<long>(t0 + i) * H + h) * dv + n0 + j] = from_f32<Tin>(acc);
         }
         __syncthreads();
         for (int e = tid; e < dk * NV; e += kThreads) {   // S <- Diag(gamma) S + Kb^T U
             const int c = e / NV, j = e - c * NV;
-            float acc = s.gam[c] * s.S[e];
-            for (int t = 0; t < kC; ++t) acc = fmaf(s.Kh[t * LD + c], s.U[t * NV + j], acc);
-            s.S[e] = acc;
+            float acc = s.gam[c] * s.S[c * NP + j];
+            for (int t = 0; t < kC; ++t) acc = fmaf(s.Kh[t * LD + c], s.U[t * NP + j], acc);
+            s.S[c * NP + j] = acc;
         }
     }
     __syncthreads();
     if (S_T)
         for (int e = tid; e < dk * NV; e += kThreads) {
             const int c = e / NV, j = e - c * NV;
-            if (j < nv) S_T[(row * dk + c) * dv + n0 + j] = s.S[e];
+            if (j < nv) S_T[(row * dk + c) * dv + n0 + j] = s.S[c * NP + j];
         }
 }
 
