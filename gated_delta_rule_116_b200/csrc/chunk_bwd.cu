@@ -3,6 +3,7 @@
 // [B,H,chunks,dk,dv]) and fp32 accumulators for dq and dk, cast to the input
 // dtype at the end.
 #include "kda_internal.cuh"
+#include "tc_sm100.cuh"
 
 namespace kda {
 #include "chunk_bwd.cuh"

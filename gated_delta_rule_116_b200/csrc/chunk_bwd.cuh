@@ -19,38 +19,48 @@
 // linear in a slice's partial terms and are summed over slices with atomics.
 // Two kernels: a forward pass that stores every chunk's entry state, then the
 // reverse pass. Chunk length 16 (the chunk length is free in exact
-// arithmetic; 16 keeps a CTA's tiles within shared memory at d = 128).
-// The bodies use only plain CUDA-core code; the kernels, their launch and the
-// fp32 -> dtype casts are in chunk_bwd.cu.
+// arithmetic; 16 keeps a CTA's tiles within shared memory at d = 128). The
+// dense products run on the tensor cores as warp-level tf32 tiles; the terms
+// with a pairwise decay e^{g_i - g_j} (At, P and their gradients) and the 16 x 16
+// triangular algebra stay on the CUDA cores, so no decay factor is ever split
+// into a growing and a shrinking part. The kernels, their launch and the fp32 ->
+// dtype casts are in chunk_bwd.cu.
 #pragma once
 
 namespace kbwd {
 
-constexpr int kThreads = 256;
+constexpr int kThreads = 512;
+constexpr int kWarps = kThreads / 32;
 constexpr int kC = 16;
 constexpr int kNV = 32;
+static_assert(kC * kNV % kThreads == 0 && kC * 128 % kThreads == 0, "whole loads per thread");
+constexpr float kLog2e = 1.4426950408889634f;
 
-// Row strides are one float longer than the rows (LD = dk + 1, LC = C + 1, NP = NV + 1), so
-// that a warp reading a column (one row per lane) hits 32 different banks.
+// Key-side rows are padded to dkp = dk rounded up to 16 (zeros past dk), so every
+// product tiles into 16 x 8 blocks. Row strides are 4 floats longer than the rows
+// (LD = dkp + 4, LC = C + 4, NP = NV + 4): the eight rows a warp's tensor-core
+// fragment reads then start in eight different bank quads.
 struct Layout {
-    int dk, NV, NP, LD, LC;
-    __host__ __device__ Layout(int dk_, int NV_) : dk(dk_), NV(NV_), NP(NV_ + 1), LD(dk_ + 1), LC(kC + 1) {}
-    // 12 [C][LD] tiles, 7 [C][LC], 5 [C][NP], 3 [dk][NP], vectors
+    int dk, dkp, NV, NP, LD, LC;
+    __host__ __device__ Layout(int dk_, int NV_)
+        : dk(dk_), dkp((dk_ + 15) & ~15), NV(NV_), NP(NV_ + 4), LD(((dk_ + 15) & ~15) + 4), LC(kC + 4) {}
+    // 12 [C][LD] tiles, 7 [C][LC], 5 [C][NP], 3 [dkp][NP], vectors
     __host__ __device__ size_t floats() const {
-        return 12ull * kC * LD + 7ull * kC * LC + 5ull * kC * NP + 3ull * dk * NP + 3ull * dk + 3ull * kC;
+        return 12ull * kC * LD + 7ull * kC * LC + 5ull * kC * NP + 3ull * dkp * NP + 3ull * dkp + 3ull * kC;
     }
 };
 
 struct Tiles {
-    // Qt, Kt: q and k; Qs = q e^{g}, Ks = k e^{g}, Kh = Kb = k e^{g_C - g}; G: prefix sums g
+    // Qt, Kt: q and k; Qs = q e^{g}, Ks = k e^{g}, Kh = Kb = k e^{g_C - g};
+    // G: prefix sums g, in log2 units (g log2 e)
     float *Qt, *Kt, *Kh, *G, *W, *dQs, *dKb, *dW, *dKs, *dQt, *Qs, *Ks;   // [C][LD]
     float *At, *P, *X, *Tm, *dT, *dA, *dP;                      // [C][LC]
     float *V, *Up, *U, *dO, *dU;                                 // [C][NP]
-    float *S, *dS, *dSn;                                         // [dk][NP]
-    float *gam, *dgam, *gsum;                                    // [dk]
+    float *S, *dS, *dSn;                                         // [dkp][NP]
+    float *gam, *dgam, *gsum;                                    // [dkp]; gsum in log2 units
     float *bt, *dbt, *pad;                                       // [C]
     __device__ Tiles(float *sm, const Layout &L) {
-        const int CD = kC * L.LD, CC = kC * L.LC, CN = kC * L.NP, DN = L.dk * L.NP;
+        const int CD = kC * L.LD, CC = kC * L.LC, CN = kC * L.NP, DN = L.dkp * L.NP;
         float *p = sm;
         Qt = p; p += CD; Kt = p; p += CD; Kh = p; p += CD; G = p; p += CD; W = p; p += CD;
         dQs = p; p += CD; dKb = p; p += CD; dW = p; p += CD; dKs = p; p += CD; dQt = p; p += CD;
@@ -59,11 +69,109 @@ struct Tiles {
         dA = p; p += CC; dP = p; p += CC;
         V = p; p += CN; Up = p; p += CN; U = p; p += CN; dO = p; p += CN; dU = p; p += CN;
         S = p; p += DN; dS = p; p += DN; dSn = p; p += DN;
-        gam = p; p += L.dk;
-        dgam = p; p += L.dk; gsum = p; p += L.dk;
+        gam = p; p += L.dkp;
+        dgam = p; p += L.dkp; gsum = p; p += L.dkp;
         bt = p; p += kC; dbt = p; p += kC; pad = p;
     }
 };
+
+// ------------------------------------------------------------------ warp-level tensor-core tiles
+// Products of shared-memory tiles on the tensor cores, one warp per 16 x 8 output
+// block (mma.sync m16n8k8, tf32 operands, fp32 accumulation). With kSplit each
+// operand x is split into tf32 parts hi(x) + lo(x) and three products are summed
+// (hi hi + hi lo + lo hi), which keeps about 22 significant bits. Every product
+// here takes that form, for bf16 inputs too: the gradients are differences of
+// terms much larger than themselves (the gradient of k sums four such terms), and
+// single tf32 products (11 bits) left errors of 6 % of a gradient element.
+constexpr bool kSplitProducts = true;
+
+__device__ __forceinline__ uint32_t tf32_bits(float x) { return tc::to_tf32(x) & 0xFFFFE000u; }
+
+// d += A B for one 8-deep step; the low-part products go to e (a separate chain).
+template <bool kSplit>
+__device__ __forceinline__ void mma_step(float (&d)[4], float (&e)[4], const float (&a)[4],
+                                         const float (&b)[2]) {
+    uint32_t ah[4], bh[2];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) ah[i] = tf32_bits(a[i]);
+    bh[0] = tf32_bits(b[0]);
+    bh[1] = tf32_bits(b[1]);
+    if constexpr (kSplit) {
+        uint32_t al[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) al[i] = tf32_bits(a[i] - __uint_as_float(ah[i]));
+        const uint32_t bl0 = tf32_bits(b[0] - __uint_as_float(bh[0]));
+        const uint32_t bl1 = tf32_bits(b[1] - __uint_as_float(bh[1]));
+        tc::mma_16x8x8_tf32(e, al, bh[0], bh[1]);
+        tc::mma_16x8x8_tf32(e, ah, bl0, bl1);
+    }
+    tc::mma_16x8x8_tf32(d, ah, bh[0], bh[1]);
+}
+
+// d += sum_{k0 <= k < k1} A(m, k) B(k, n) over the block at rows m0..m0+15, columns
+// n0..n0+7; k1 - k0 is a multiple of 8. A and B read shared memory. Even and odd
+// 8-deep steps, and the high and low parts, accumulate in separate chains.
+template <bool kSplit, class FA, class FB>
+__device__ __forceinline__ void tile_mma(float (&d)[4], const FA &A, const FB &B, int m0, int n0, int k0,
+                                         int k1) {
+    const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+    float d1[4] = {0.f, 0.f, 0.f, 0.f}, e0[4] = {0.f, 0.f, 0.f, 0.f}, e1[4] = {0.f, 0.f, 0.f, 0.f};
+    int k = k0;
+    for (; k + 16 <= k1; k += 16) {
+        const float a0[4] = {A(m0 + g, k + t), A(m0 + g + 8, k + t), A(m0 + g, k + t + 4),
+                             A(m0 + g + 8, k + t + 4)};
+        const float b0[2] = {B(k + t, n0 + g), B(k + t + 4, n0 + g)};
+        const float a1[4] = {A(m0 + g, k + 8 + t), A(m0 + g + 8, k + 8 + t), A(m0 + g, k + 12 + t),
+                             A(m0 + g + 8, k + 12 + t)};
+        const float b1[2] = {B(k + 8 + t, n0 + g), B(k + 12 + t, n0 + g)};
+        mma_step<kSplit>(d, e0, a0, b0);
+        mma_step<kSplit>(d1, e1, a1, b1);
+    }
+    if (k < k1) {
+        const float a0[4] = {A(m0 + g, k + t), A(m0 + g + 8, k + t), A(m0 + g, k + t + 4),
+                             A(m0 + g + 8, k + t + 4)};
+        const float b0[2] = {B(k + t, n0 + g), B(k + t + 4, n0 + g)};
+        mma_step<kSplit>(d, e0, a0, b0);
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) d[i] += d1[i] + (e0[i] + e1[i]);
+}
+
+// Visits the lane's four accumulator entries with their (row, column).
+template <class F>
+__device__ __forceinline__ void tile_each(float (&d)[4], int m0, int n0, const F &f) {
+    const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+    f(m0 + g, n0 + 2 * t, d[0]);
+    f(m0 + g, n0 + 2 * t + 1, d[1]);
+    f(m0 + g + 8, n0 + 2 * t, d[2]);
+    f(m0 + g + 8, n0 + 2 * t + 1, d[3]);
+}
+
+// Brings the rows of chunk [t0, t0 + C) of q, k, log alpha, v (value slice) and, when
+// given, dL/dO (value slice) and a stored state slice into L2 ahead of their loads.
+template <typename Tin>
+__device__ __forceinline__ void prefetch_chunk(const Tin *q, const Tin *k, const Tin *v, const float *log_alpha,
+                                               const Tin *dout, const float *state, int b, int h, int T,
+                                               int H, int dk, int dv, int t0, int n0) {
+    const int tid = threadIdx.x;
+    if (t0 < 0 || t0 >= T) return;
+    const int valid = min(kC, T - t0);
+    const auto pf = [](const void *p) { asm volatile("prefetch.global.L2 [%0];" ::"l"(p)); };
+    // 128-byte lines: per token, q and k rows (dk elements), log alpha (dk floats), v and dO slices
+    const int qlines = (dk * static_cast<int>(sizeof(Tin)) + 127) / 128, glines = (dk * 4 + 127) / 128;
+    const int per_tok = 2 * qlines + glines + (dout ? 2 : 1);
+    for (int e = tid; e < valid * per_tok; e += kThreads) {
+        const int t = e / per_tok, r = e - t * per_tok;
+        const long row = (static_cast<long>(b) * T + t0 + t) * H + h;
+        if (r < qlines) pf(reinterpret_cast<const char *>(q + row * dk) + 128 * r);
+        else if (r < 2 * qlines) pf(reinterpret_cast<const char *>(k + row * dk) + 128 * (r - qlines));
+        else if (r < 2 * qlines + glines) pf(reinterpret_cast<const char *>(log_alpha + row * dk) + 128 * (r - 2 * qlines));
+        else if (r == 2 * qlines + glines) pf(v + row * dv + n0);
+        else pf(dout + row * dv + n0);
+    }
+    if (state)
+        for (int c = tid; c < dk; c += kThreads) pf(state + static_cast<long>(c) * dv + n0);
+}
 
 // The state-independent terms of one chunk: g, Qs, Ks, Kb, At, P,
 // X = (I + A)^{-1}, T, W = T Ks, U' = T V. Loads q, k, log alpha, v (slice), beta.
@@ -71,89 +179,149 @@ template <typename Tin>
 __device__ void chunk_terms(Tiles &s, const Layout &L, const Tin *q, const Tin *k, const Tin *v,
                             const float *log_alpha, const float *beta, int b, int h, int T, int H,
                             int dv, int t0, int valid, int n0, int nv, bool need_p) {
-    const int tid = threadIdx.x, dk = L.dk, LD = L.LD, LC = L.LC, NV = L.NV, NP = L.NP;
-    for (int e = tid; e < kC * dk; e += kThreads) {
-        const int t = e / dk, c = e - t * dk;
-        float qv = 0.f, kv = 0.f, gv = 0.f;
-        if (t < valid) {
+    constexpr bool kSplit = kSplitProducts;
+    const int tid = threadIdx.x, warp = tid >> 5, dk = L.dk, dkp = L.dkp, LD = L.LD, LC = L.LC,
+              NV = L.NV, NP = L.NP;
+    // every global load of the chunk is issued before the first shared-memory store
+    constexpr int kPerK = kC * 128 / kThreads, kPerV = kC * kNV / kThreads;
+    float qr[kPerK], kr[kPerK], gr[kPerK], vr[kPerV], br = 0.f;
+#pragma unroll
+    for (int u = 0; u < kPerK; ++u) {
+        const int e = tid + u * kThreads, t = e / dkp, c = e - t * dkp;
+        qr[u] = kr[u] = gr[u] = 0.f;
+        if (e < kC * dkp && t < valid && c < dk) {
             const long o = ((static_cast<long>(b) * T + t0 + t) * H + h) * dk + c;
-            qv = to_f32(q[o]);
-            kv = to_f32(k[o]);
-            gv = log_alpha[o];
+            qr[u] = to_f32(q[o]);
+            kr[u] = to_f32(k[o]);
+            gr[u] = log_alpha[o];
         }
-        s.Qt[t * LD + c] = qv;
-        s.Kt[t * LD + c] = kv;
-        s.G[t * LD + c] = gv;
     }
-    for (int e = tid; e < kC * NV; e += kThreads) {
-        const int t = e / NV, n = e - t * NV;
-        float vv = 0.f;
-        if (t < valid && n < nv) vv = to_f32(v[((static_cast<long>(b) * T + t0 + t) * H + h) * dv + n0 + n]);
-        s.V[t * NP + n] = vv;
+#pragma unroll
+    for (int u = 0; u < kPerV; ++u) {
+        const int e = tid + u * kThreads, t = e / NV, n = e - t * NV;
+        vr[u] = 0.f;
+        if (t < valid && n < nv) vr[u] = to_f32(v[((static_cast<long>(b) * T + t0 + t) * H + h) * dv + n0 + n]);
     }
-    for (int t = tid; t < kC; t += kThreads)
-        s.bt[t] = t < valid ? beta[(static_cast<long>(b) * T + t0 + t) * H + h] : 0.f;
+    if (tid < valid) br = beta[(static_cast<long>(b) * T + t0 + tid) * H + h];
+#pragma unroll
+    for (int u = 0; u < kPerK; ++u) {
+        const int e = tid + u * kThreads, t = e / dkp, c = e - t * dkp;
+        if (e < kC * dkp) {
+            s.Qt[t * LD + c] = qr[u];
+            s.Kt[t * LD + c] = kr[u];
+            s.G[t * LD + c] = gr[u];
+        }
+    }
+#pragma unroll
+    for (int u = 0; u < kPerV; ++u) {
+        const int e = tid + u * kThreads, t = e / NV, n = e - t * NV;
+        s.V[t * NP + n] = vr[u];
+    }
+    if (tid < kC) s.bt[tid] = br;
     __syncthreads();
-    for (int c = tid; c < dk; c += kThreads) {   // prefix sums
+    for (int c = tid; c < dkp; c += kThreads) {   // prefix sums (natural log), kept in log2 units
         float acc = 0.f;
         for (int t = 0; t < kC; ++t) {
             acc += s.G[t * LD + c];
-            s.G[t * LD + c] = acc;
+            s.G[t * LD + c] = acc * kLog2e;
         }
-        s.gsum[c] = acc;
-        s.gam[c] = expf(acc);
+        s.gsum[c] = acc * kLog2e;
+        s.gam[c] = tc::ex2(acc * kLog2e);
     }
     __syncthreads();
-    for (int e = tid; e < kC * dk; e += kThreads) {   // Qs = q e^{g}, Ks = k e^{g}, Kb = k e^{g_C - g}
-        const int t = e / dk, c = e - t * dk;
+    for (int e = tid; e < kC * dkp; e += kThreads) {   // Qs = q e^{g}, Ks = k e^{g}, Kb = k e^{g_C - g}
+        const int t = e / dkp, c = e - t * dkp;
         const float gv = s.G[t * LD + c];
-        const float up = expf(gv), down = expf(s.gsum[c] - gv);
+        const float up = tc::ex2(gv), down = tc::ex2(s.gsum[c] - gv);
         const float kv = s.Kt[t * LD + c];
         s.Qs[t * LD + c] = s.Qt[t * LD + c] * up;
         s.Ks[t * LD + c] = kv * up;
         s.Kh[t * LD + c] = kv * down;
     }
-    for (int e = tid; e < 2 * kC * kC; e += kThreads) {   // At (strict lower), P (lower)
-        const int which = e / (kC * kC), r = e - which * kC * kC;
-        const int i = r / kC, j = r - i * kC;
-        float acc = 0.f;
-        if (which == 0 ? j < i : (need_p && j <= i)) {
-            const float *x = (which == 0 ? s.Kt : s.Qt) + i * LD;
-            const float *y = s.Kt + j * LD;
-            const float *gi = s.G + i * LD, *gj = s.G + j * LD;
-            for (int c = 0; c < dk; ++c) acc = fmaf(x[c], y[c] * expf(gi[c] - gj[c]), acc);
+    // At (strict lower) and P (lower), one thread per pair i >= j, both from the same
+    // pairwise decays e^{g_i - g_j} <= 1; entries above the diagonal are zero
+    for (int e = tid; e < kC * kC; e += kThreads) {
+        const int i = e / kC, j = e - i * kC;
+        if (j > i) {
+            s.At[i * LC + j] = 0.f;
+            s.P[i * LC + j] = 0.f;
+            continue;
         }
-        (which == 0 ? s.At : s.P)[i * LC + j] = acc;
+        const float4 *ki = reinterpret_cast<const float4 *>(s.Kt + i * LD);
+        const float4 *kj = reinterpret_cast<const float4 *>(s.Kt + j * LD);
+        const float4 *qi = reinterpret_cast<const float4 *>(s.Qt + i * LD);
+        const float4 *gi = reinterpret_cast<const float4 *>(s.G + i * LD);
+        const float4 *gj = reinterpret_cast<const float4 *>(s.G + j * LD);
+        float at[4] = {0.f, 0.f, 0.f, 0.f}, pp[4] = {0.f, 0.f, 0.f, 0.f};
+        for (int c4 = 0; c4 < dkp / 4; ++c4) {
+            const float4 a = ki[c4], bj = kj[c4], q4 = qi[c4], x = gi[c4], y = gj[c4];
+            const float w0 = bj.x * tc::ex2(x.x - y.x), w1 = bj.y * tc::ex2(x.y - y.y);
+            const float w2 = bj.z * tc::ex2(x.z - y.z), w3 = bj.w * tc::ex2(x.w - y.w);
+            at[0] = fmaf(a.x, w0, at[0]); at[1] = fmaf(a.y, w1, at[1]);
+            at[2] = fmaf(a.z, w2, at[2]); at[3] = fmaf(a.w, w3, at[3]);
+            pp[0] = fmaf(q4.x, w0, pp[0]); pp[1] = fmaf(q4.y, w1, pp[1]);
+            pp[2] = fmaf(q4.z, w2, pp[2]); pp[3] = fmaf(q4.w, w3, pp[3]);
+        }
+        s.At[i * LC + j] = j < i ? (at[0] + at[1]) + (at[2] + at[3]) : 0.f;
+        s.P[i * LC + j] = need_p ? (pp[0] + pp[1]) + (pp[2] + pp[3]) : 0.f;
     }
     __syncthreads();
     if (tid < kC) {   // X = (I + A)^{-1}, A = Diag(beta) At: column j by forward substitution
         const int j = tid;
+        float xc[kC];   // column j of X, in registers
+#pragma unroll
         for (int i = 0; i < kC; ++i) {
-            float x = i == j ? 1.f : 0.f;
-            if (i > j) {
-                float acc = 0.f;
-                for (int m = j; m < i; ++m) acc = fmaf(s.At[i * LC + m], s.X[m * LC + j], acc);
-                x = -s.bt[i] * acc;
+            float acc = 0.f;
+#pragma unroll
+            for (int m = 0; m < i; ++m) acc = fmaf(s.At[i * LC + m], xc[m], acc);   // xc[m] = 0 for m < j
+            xc[i] = i == j ? 1.f : (i > j ? -s.bt[i] * acc : 0.f);
+            s.X[i * LC + j] = xc[i];
+            s.Tm[i * LC + j] = xc[i] * s.bt[j];
+        }
+    }
+    __syncthreads();
+    {   // W = T Ks (dkp / 8 blocks), U' = T V (NV / 8 blocks); T is lower triangular
+        const int nW = dkp / 8, nU = NV / 8;
+        for (int tl = warp; tl < nW + nU; tl += kWarps) {
+            float d[4] = {0.f, 0.f, 0.f, 0.f};
+            const auto A = [&](int m, int kk) { return s.Tm[m * LC + kk]; };
+            if (tl < nW) {
+                const int c0 = tl * 8;
+                tile_mma<kSplit>(d, A, [&](int kk, int n) { return s.Ks[kk * LD + n]; }, 0, c0, 0, kC);
+                tile_each(d, 0, c0, [&](int r, int c, float &x) { s.W[r * LD + c] = x; });
+            } else {
+                const int j0 = (tl - nW) * 8;
+                tile_mma<kSplit>(d, A, [&](int kk, int n) { return s.V[kk * NP + n]; }, 0, j0, 0, kC);
+                tile_each(d, 0, j0, [&](int r, int c, float &x) { s.Up[r * NP + c] = x; });
             }
-            s.X[i * LC + j] = x;
-            s.Tm[i * LC + j] = x * s.bt[j];
         }
     }
     __syncthreads();
-    for (int e = tid; e < kC * dk + kC * NV; e += kThreads) {   // W = T Ks, U' = T V
-        if (e < kC * dk) {
-            const int i = e / dk, c = e - i * dk;
-            float acc = 0.f;
-            for (int j = 0; j <= i; ++j) acc = fmaf(s.Tm[i * LC + j], s.Ks[j * LD + c], acc);
-            s.W[i * LD + c] = acc;
-        } else {
-            const int r = e - kC * dk, i = r / NV, n = r - i * NV;
-            float acc = 0.f;
-            for (int j = 0; j <= i; ++j) acc = fmaf(s.Tm[i * LC + j], s.V[j * NP + n], acc);
-            s.Up[i * NP + n] = acc;
-        }
+}
+
+// U = U' - W S, one warp per 8 value columns (warps NV/8 and up idle).
+template <bool kSplit>
+__device__ __forceinline__ void u_block(Tiles &s, const Layout &L, int j0) {
+    const int LD = L.LD, NP = L.NP;
+    float d[4];
+    tile_each(d, 0, j0, [&](int r, int c, float &x) { x = s.Up[r * NP + c]; });
+    tile_mma<kSplit>(d, [&](int m, int kk) { return -s.W[m * LD + kk]; },
+                     [&](int kk, int n) { return s.S[kk * NP + n]; }, 0, j0, 0, L.dkp);
+    tile_each(d, 0, j0, [&](int r, int c, float &x) { s.U[r * NP + c] = x; });
+}
+
+// S <- Diag(gamma) S + Kb^T U over all dkp x NV blocks.
+template <bool kSplit>
+__device__ __forceinline__ void state_update(Tiles &s, const Layout &L) {
+    const int warp = threadIdx.x >> 5, LD = L.LD, NP = L.NP, nN = L.NV / 8;
+    for (int tl = warp; tl < (L.dkp / 16) * nN; tl += kWarps) {
+        const int m0 = (tl / nN) * 16, j0 = (tl - (tl / nN) * nN) * 8;
+        float d[4];
+        tile_each(d, m0, j0, [&](int r, int c, float &x) { x = s.gam[r] * s.S[r * NP + c]; });
+        tile_mma<kSplit>(d, [&](int m, int kk) { return s.Kh[kk * LD + m]; },
+                         [&](int kk, int n) { return s.U[kk * NP + n]; }, m0, j0, 0, kC);
+        tile_each(d, m0, j0, [&](int r, int c, float &x) { s.S[r * NP + c] = x; });
     }
-    __syncthreads();
 }
 
 // Forward chain storing the entry state of every chunk: states[bh][chunk][dk][dv].
@@ -161,38 +329,30 @@ template <typename Tin>
 __device__ void states_body(float *sm, const Tin *q, const Tin *k, const Tin *v, const float *log_alpha,
                             const float *beta, const float *S0, float *states, int T, int H, int dk,
                             int dv) {
+    constexpr bool kSplit = kSplitProducts;
     const Layout L(dk, kNV);
     Tiles s(sm, L);
-    const int tid = threadIdx.x, LD = L.LD, NV = L.NV, NP = L.NP;
+    const int tid = threadIdx.x, warp = tid >> 5, dkp = L.dkp, NV = L.NV, NP = L.NP;
     const int bh = blockIdx.x, b = bh / H, h = bh - b * H;
     const int n0 = blockIdx.y * NV, nv = min(NV, dv - n0);
     const int nchunks = (T + kC - 1) / kC;
-    for (int e = tid; e < dk * NV; e += kThreads) {
+    for (int e = tid; e < dkp * NV; e += kThreads) {
         const int c = e / NV, n = e - c * NV;
-        s.S[c * NP + n] = (S0 && n < nv) ? S0[(static_cast<long>(bh) * dk + c) * dv + n0 + n] : 0.f;
+        s.S[c * NP + n] = (S0 && c < dk && n < nv) ? S0[(static_cast<long>(bh) * dk + c) * dv + n0 + n] : 0.f;
     }
     for (int ch = 0; ch < nchunks; ++ch) {
         const int t0 = ch * kC, valid = min(kC, T - t0);
         __syncthreads();
         float *dst = states + (static_cast<long>(bh) * nchunks + ch) * dk * dv;
+        prefetch_chunk<Tin>(q, k, v, log_alpha, nullptr, nullptr, b, h, T, H, dk, dv, t0 + kC, n0);
         for (int e = tid; e < dk * NV; e += kThreads) {
             const int c = e / NV, n = e - c * NV;
             if (n < nv) dst[static_cast<long>(c) * dv + n0 + n] = s.S[c * NP + n];
         }
         chunk_terms(s, L, q, k, v, log_alpha, beta, b, h, T, H, dv, t0, valid, n0, nv, false);
-        for (int e = tid; e < kC * NV; e += kThreads) {   // U = U' - W S
-            const int i = e / NV, n = e - i * NV;
-            float acc = s.Up[i * NP + n];
-            for (int c = 0; c < dk; ++c) acc = fmaf(-s.W[i * LD + c], s.S[c * NP + n], acc);
-            s.U[i * NP + n] = acc;
-        }
+        for (int tl = warp; tl < NV / 8; tl += kWarps) u_block<kSplit>(s, L, tl * 8);   // U = U' - W S
         __syncthreads();
-        for (int e = tid; e < dk * NV; e += kThreads) {   // S <- Diag(gamma) S + Kb^T U
-            const int c = e / NV, n = e - c * NV;
-            float acc = s.gam[c] * s.S[c * NP + n];
-            for (int t = 0; t < kC; ++t) acc = fmaf(s.Kh[t * LD + c], s.U[t * NP + n], acc);
-            s.S[c * NP + n] = acc;
-        }
+        state_update<kSplit>(s, L);   // S <- Diag(gamma) S + Kb^T U
     }
 }
 
@@ -204,85 +364,125 @@ __device__ void bwd_body(float *sm, const Tin *q, const Tin *k, const Tin *v, co
                          const float *beta, const Tin *dout, const float *dS_T, const float *states,
                          float *dq_acc, float *dk_acc, Tin *dv_out, float *dlog_alpha, float *dbeta,
                          float *dS0, int T, int H, int dk, int dv) {
+    constexpr bool kSplit = kSplitProducts;
     const Layout L(dk, kNV);
     Tiles s(sm, L);
-    const int tid = threadIdx.x, LD = L.LD, LC = L.LC, NV = L.NV, NP = L.NP;
+    const int tid = threadIdx.x, warp = tid >> 5, dkp = L.dkp, LD = L.LD, LC = L.LC, NV = L.NV,
+              NP = L.NP;
     const int bh = blockIdx.x, b = bh / H, h = bh - b * H;
     const int n0 = blockIdx.y * NV, nv = min(NV, dv - n0);
     const int nchunks = (T + kC - 1) / kC;
-    for (int e = tid; e < dk * NV; e += kThreads) {
+    const int nU = NV / 8, nQ = dkp / 8, nS = (dkp / 16) * nU;   // block counts
+    for (int e = tid; e < dkp * NV; e += kThreads) {
         const int c = e / NV, n = e - c * NV;
-        s.dS[c * NP + n] = (dS_T && n < nv) ? dS_T[(static_cast<long>(bh) * dk + c) * dv + n0 + n] : 0.f;
+        s.dS[c * NP + n] =
+            (dS_T && c < dk && n < nv) ? dS_T[(static_cast<long>(bh) * dk + c) * dv + n0 + n] : 0.f;
     }
     for (int ch = nchunks - 1; ch >= 0; --ch) {
         const int t0 = ch * kC, valid = min(kC, T - t0);
         __syncthreads();
-        const float *src = states + (static_cast<long>(bh) * nchunks + ch) * dk * dv;
-        for (int e = tid; e < dk * NV; e += kThreads) {
-            const int c = e / NV, n = e - c * NV;
-            s.S[c * NP + n] = n < nv ? src[static_cast<long>(c) * dv + n0 + n] : 0.f;
-        }
-        for (int e = tid; e < kC * NV; e += kThreads) {
-            const int t = e / NV, n = e - t * NV;
-            s.dO[t * NP + n] = (t < valid && n < nv)
-                          ? to_f32(dout[((static_cast<long>(b) * T + t0 + t) * H + h) * dv + n0 + n])
-                          : 0.f;
+        if (ch > 0)
+            prefetch_chunk<Tin>(q, k, v, log_alpha, dout,
+                                states + (static_cast<long>(bh) * nchunks + ch - 1) * dk * dv, b, h, T, H,
+                                dk, dv, t0 - kC, n0);
+        {   // the chunk's entry state and dL/dO, all loads issued before the stores
+            const float *src = states + (static_cast<long>(bh) * nchunks + ch) * dk * dv;
+            constexpr int kPerS = 128 * kNV / kThreads, kPerO = kC * kNV / kThreads;
+            float sr[kPerS], orr[kPerO];
+#pragma unroll
+            for (int u = 0; u < kPerS; ++u) {
+                const int e = tid + u * kThreads, c = e / NV, n = e - c * NV;
+                sr[u] = (c < dk && n < nv) ? src[static_cast<long>(c) * dv + n0 + n] : 0.f;
+            }
+#pragma unroll
+            for (int u = 0; u < kPerO; ++u) {
+                const int e = tid + u * kThreads, t = e / NV, n = e - t * NV;
+                orr[u] = (t < valid && n < nv)
+                             ? to_f32(dout[((static_cast<long>(b) * T + t0 + t) * H + h) * dv + n0 + n])
+                             : 0.f;
+            }
+#pragma unroll
+            for (int u = 0; u < kPerS; ++u) {
+                const int e = tid + u * kThreads, c = e / NV, n = e - c * NV;
+                if (c < dkp) s.S[c * NP + n] = sr[u];
+            }
+#pragma unroll
+            for (int u = 0; u < kPerO; ++u) {
+                const int e = tid + u * kThreads, t = e / NV, n = e - t * NV;
+                s.dO[t * NP + n] = orr[u];
+            }
         }
         chunk_terms(s, L, q, k, v, log_alpha, beta, b, h, T, H, dv, t0, valid, n0, nv, true);
-        // U = U' - W S
-        for (int e = tid; e < kC * NV; e += kThreads) {
-            const int i = e / NV, n = e - i * NV;
-            float acc = s.Up[i * NP + n];
-            for (int c = 0; c < dk; ++c) acc = fmaf(-s.W[i * LD + c], s.S[c * NP + n], acc);
-            s.U[i * NP + n] = acc;
-        }
-        __syncthreads();
-        // dU = P^T dO + Kb dS
-        for (int e = tid; e < kC * NV; e += kThreads) {
-            const int j = e / NV, n = e - j * NV;
-            float acc = 0.f;
-            for (int i = j; i < kC; ++i) acc = fmaf(s.P[i * LC + j], s.dO[i * NP + n], acc);
-            for (int c = 0; c < dk; ++c) acc = fmaf(s.Kh[j * LD + c], s.dS[c * NP + n], acc);
-            s.dU[j * NP + n] = acc;
-        }
-        __syncthreads();
-        // the new state gradient, and the slice's partial key-side terms
-        for (int e = tid; e < dk * NV; e += kThreads) {   // dSn = Qs^T dO + Diag(gamma) dS - W^T dU
-            const int c = e / NV, n = e - c * NV;
-            float acc = s.gam[c] * s.dS[c * NP + n];
-            for (int i = 0; i < kC; ++i) {
-                acc = fmaf(s.Qs[i * LD + c], s.dO[i * NP + n], acc);
-                acc = fmaf(-s.W[i * LD + c], s.dU[i * NP + n], acc);
-            }
-            s.dSn[c * NP + n] = acc;
-        }
-        for (int c = tid; c < dk; c += kThreads) {   // gamma's gradient (through the state decay)
-            float acc = 0.f;
-            for (int n = 0; n < NV; ++n) acc = fmaf(s.dS[c * NP + n], s.S[c * NP + n], acc);
-            s.dgam[c] = acc * s.gam[c];
-        }
-        for (int e = tid; e < 3 * kC * dk; e += kThreads) {   // dQs = dO S^T, dKb = U dS^T, dW = -dU S^T
-            const int which = e / (kC * dk), r = e - which * kC * dk;
-            const int i = r / dk, c = r - i * dk;
-            const float *a = which == 0 ? s.dO : (which == 1 ? s.U : s.dU);
-            const float *m = which == 1 ? s.dS : s.S;
-            float acc = 0.f;
-            for (int n = 0; n < NV; ++n) acc = fmaf(a[i * NP + n], m[c * NP + n], acc);
-            (which == 0 ? s.dQs : (which == 1 ? s.dKb : s.dW))[i * LD + c] = which == 2 ? -acc : acc;
-        }
-        for (int e = tid; e < kC * kC + kC * NV; e += kThreads) {   // dP = lower(dO U^T), dV = T^T dU
-            if (e < kC * kC) {
-                const int i = e / kC, j = e - i * kC;
-                float acc = 0.f;
-                if (j <= i)
-                    for (int n = 0; n < NV; ++n) acc = fmaf(s.dO[i * NP + n], s.U[j * NP + n], acc);
-                s.dP[i * LC + j] = acc;
+        // U = U' - W S; dQs = dO S^T
+        for (int tl = warp; tl < nU + nQ; tl += kWarps) {
+            if (tl < nU) {
+                u_block<kSplit>(s, L, tl * 8);
             } else {
-                const int r = e - kC * kC, j = r / NV, n = r - j * NV;
-                float acc = 0.f;
-                for (int i = j; i < kC; ++i) acc = fmaf(s.Tm[i * LC + j], s.dU[i * NP + n], acc);
-                if (j < valid && n < nv)
-                    dv_out[((static_cast<long>(b) * T + t0 + j) * H + h) * dv + n0 + n] = from_f32<Tin>(acc);
+                const int c0 = (tl - nU) * 8;
+                float d[4] = {0.f, 0.f, 0.f, 0.f};
+                tile_mma<kSplit>(d, [&](int m, int kk) { return s.dO[m * NP + kk]; },
+                                 [&](int kk, int c) { return s.S[c * NP + kk]; }, 0, c0, 0, NV);
+                tile_each(d, 0, c0, [&](int r, int c, float &x) { s.dQs[r * LD + c] = x; });
+            }
+        }
+        __syncthreads();
+        // dU = P^T dO + Kb dS; dKb = U dS^T; dP = lower(dO U^T); gamma's gradient
+        for (int tl = warp; tl < nU + nQ + 2; tl += kWarps) {
+            float d[4] = {0.f, 0.f, 0.f, 0.f};
+            if (tl < nU) {
+                const int j0 = tl * 8;
+                tile_mma<kSplit>(d, [&](int m, int kk) { return s.P[kk * LC + m]; },
+                                 [&](int kk, int n) { return s.dO[kk * NP + n]; }, 0, j0, 0, kC);
+                tile_mma<kSplit>(d, [&](int m, int kk) { return s.Kh[m * LD + kk]; },
+                                 [&](int kk, int n) { return s.dS[kk * NP + n]; }, 0, j0, 0, dkp);
+                tile_each(d, 0, j0, [&](int r, int c, float &x) { s.dU[r * NP + c] = x; });
+            } else if (tl < nU + nQ) {
+                const int c0 = (tl - nU) * 8;
+                tile_mma<kSplit>(d, [&](int m, int kk) { return s.U[m * NP + kk]; },
+                                 [&](int kk, int c) { return s.dS[c * NP + kk]; }, 0, c0, 0, NV);
+                tile_each(d, 0, c0, [&](int r, int c, float &x) { s.dKb[r * LD + c] = x; });
+            } else {
+                const int j0 = (tl - nU - nQ) * 8;
+                tile_mma<kSplit>(d, [&](int m, int kk) { return s.dO[m * NP + kk]; },
+                                 [&](int kk, int j) { return s.U[j * NP + kk]; }, 0, j0, 0, NV);
+                tile_each(d, 0, j0, [&](int r, int c, float &x) { s.dP[r * LC + c] = c <= r ? x : 0.f; });
+            }
+        }
+        static_assert(kThreads >= 4 * 128, "four threads per state row");
+        {   // gamma's gradient (through the state decay): four threads per row
+            const int c = tid >> 2, part = tid & 3;
+            float acc = 0.f;
+            if (c < dkp)
+                for (int n = part; n < NV; n += 4) acc = fmaf(s.dS[c * NP + n], s.S[c * NP + n], acc);
+            acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+            acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+            if (c < dkp && part == 0) s.dgam[c] = acc * s.gam[c];
+        }
+        __syncthreads();
+        // dSn = Diag(gamma) dS + Qs^T dO - W^T dU; dW = -dU S^T; dV = T^T dU
+        for (int tl = warp; tl < nS + nQ + nU; tl += kWarps) {
+            float d[4] = {0.f, 0.f, 0.f, 0.f};
+            if (tl < nS) {
+                const int m0 = (tl / nU) * 16, j0 = (tl - (tl / nU) * nU) * 8;
+                tile_each(d, m0, j0, [&](int r, int c, float &x) { x = s.gam[r] * s.dS[r * NP + c]; });
+                tile_mma<kSplit>(d, [&](int m, int kk) { return s.Qs[kk * LD + m]; },
+                                 [&](int kk, int n) { return s.dO[kk * NP + n]; }, m0, j0, 0, kC);
+                tile_mma<kSplit>(d, [&](int m, int kk) { return -s.W[kk * LD + m]; },
+                                 [&](int kk, int n) { return s.dU[kk * NP + n]; }, m0, j0, 0, kC);
+                tile_each(d, m0, j0, [&](int r, int c, float &x) { s.dSn[r * NP + c] = x; });
+            } else if (tl < nS + nQ) {
+                const int c0 = (tl - nS) * 8;
+                tile_mma<kSplit>(d, [&](int m, int kk) { return -s.dU[m * NP + kk]; },
+                                 [&](int kk, int c) { return s.S[c * NP + kk]; }, 0, c0, 0, NV);
+                tile_each(d, 0, c0, [&](int r, int c, float &x) { s.dW[r * LD + c] = x; });
+            } else {
+                const int j0 = (tl - nS - nQ) * 8;
+                tile_mma<kSplit>(d, [&](int m, int kk) { return s.Tm[kk * LC + m]; },
+                                 [&](int kk, int n) { return s.dU[kk * NP + n]; }, 0, j0, 0, kC);
+                tile_each(d, 0, j0, [&](int r, int c, float &x) {
+                    if (r < valid && c < nv)
+                        dv_out[((static_cast<long>(b) * T + t0 + r) * H + h) * dv + n0 + c] = from_f32<Tin>(x);
+                });
             }
         }
         __syncthreads();
@@ -292,20 +492,20 @@ __device__ void bwd_body(float *sm, const Tin *q, const Tin *k, const Tin *v, co
             s.dSn = t;
         }
         // dT = dW Ks^T + dU V^T (lower incl. diagonal), dKs = T^T dW
-        for (int e = tid; e < kC * kC + kC * dk; e += kThreads) {
-            if (e < kC * kC) {
-                const int i = e / kC, j = e - i * kC;
-                float acc = 0.f;
-                if (j <= i) {
-                    for (int c = 0; c < dk; ++c) acc = fmaf(s.dW[i * LD + c], s.Ks[j * LD + c], acc);
-                    for (int n = 0; n < NV; ++n) acc = fmaf(s.dU[i * NP + n], s.V[j * NP + n], acc);
-                }
-                s.dT[i * LC + j] = acc;
+        for (int tl = warp; tl < 2 + nQ; tl += kWarps) {
+            float d[4] = {0.f, 0.f, 0.f, 0.f};
+            if (tl < 2) {
+                const int j0 = tl * 8;
+                tile_mma<kSplit>(d, [&](int m, int kk) { return s.dW[m * LD + kk]; },
+                                 [&](int kk, int j) { return s.Ks[j * LD + kk]; }, 0, j0, 0, dkp);
+                tile_mma<kSplit>(d, [&](int m, int kk) { return s.dU[m * NP + kk]; },
+                                 [&](int kk, int j) { return s.V[j * NP + kk]; }, 0, j0, 0, NV);
+                tile_each(d, 0, j0, [&](int r, int c, float &x) { s.dT[r * LC + c] = c <= r ? x : 0.f; });
             } else {
-                const int r = e - kC * kC, j = r / dk, c = r - j * dk;
-                float acc = 0.f;
-                for (int i = j; i < kC; ++i) acc = fmaf(s.Tm[i * LC + j], s.dW[i * LD + c], acc);
-                s.dKs[j * LD + c] = acc;
+                const int c0 = (tl - 2) * 8;
+                tile_mma<kSplit>(d, [&](int m, int kk) { return s.Tm[kk * LC + m]; },
+                                 [&](int kk, int c) { return s.dW[kk * LD + c]; }, 0, c0, 0, kC);
+                tile_each(d, 0, c0, [&](int r, int c, float &x) { s.dKs[r * LD + c] = x; });
             }
         }
         __syncthreads();
@@ -350,31 +550,44 @@ __device__ void bwd_body(float *sm, const Tin *q, const Tin *k, const Tin *v, co
         //   Cc_j = sum_{i>j}  dAt_ij k_i E_ij
         //        + sum_{i>=j} dP_ij  q_i E_ij             (column side,     into W)
         //   Rq_i = sum_{j<=i} dP_ij  k_j E_ij             (row side of P,   into dQt)
-        for (int e = tid; e < 3 * kC * dk; e += kThreads) {
-            const int which = e / (kC * dk), r = e - which * kC * dk;
-            const int i = r / dk, c = r - i * dk;
-            const float gi = s.G[i * LD + c];
-            float acc = 0.f;
-            if (which == 0) {
-                for (int j = 0; j < i; ++j)
-                    acc = fmaf(s.dT[i * LC + j], s.Kt[j * LD + c] * expf(gi - s.G[j * LD + c]), acc);
-            } else if (which == 1) {
-                for (int a = i + 1; a < kC; ++a)
-                    acc = fmaf(s.dT[a * LC + i], s.Kt[a * LD + c] * expf(s.G[a * LD + c] - gi), acc);
-                for (int a = i; a < kC; ++a)
-                    acc = fmaf(s.dP[a * LC + i], s.Qt[a * LD + c] * expf(s.G[a * LD + c] - gi), acc);
-            } else {
-                for (int j = 0; j <= i; ++j)
-                    acc = fmaf(s.dP[i * LC + j], s.Kt[j * LD + c] * expf(gi - s.G[j * LD + c]), acc);
+        // One thread per channel walks every pair j < i once, so each decay is computed
+        // once for the three sums; the diagonal (E = 1) starts Cc and Rq.
+        for (int c = tid; c < dkp; c += kThreads) {
+            float g[kC], kk[kC], qq[kC], R[kC], Cc[kC], Rq[kC];
+#pragma unroll
+            for (int i = 0; i < kC; ++i) {
+                g[i] = s.G[i * LD + c];
+                kk[i] = s.Kt[i * LD + c];
+                qq[i] = s.Qt[i * LD + c];
+                const float pd = s.dP[i * LC + i];
+                R[i] = 0.f;
+                Cc[i] = pd * qq[i];
+                Rq[i] = pd * kk[i];
             }
-            (which == 0 ? s.dW : (which == 1 ? s.W : s.dQt))[i * LD + c] = acc;
+#pragma unroll
+            for (int i = 1; i < kC; ++i) {
+#pragma unroll
+                for (int j = 0; j < i; ++j) {
+                    const float E = tc::ex2(g[i] - g[j]);
+                    const float a = s.dT[i * LC + j], p = s.dP[i * LC + j];
+                    R[i] = fmaf(a * kk[j], E, R[i]);
+                    Rq[i] = fmaf(p * kk[j], E, Rq[i]);
+                    Cc[j] = fmaf(fmaf(a, kk[i], p * qq[i]), E, Cc[j]);
+                }
+            }
+#pragma unroll
+            for (int i = 0; i < kC; ++i) {
+                s.dW[i * LD + c] = R[i];
+                s.W[i * LD + c] = Cc[i];
+                s.dQt[i * LD + c] = Rq[i];
+            }
         }
         __syncthreads();
         // dk, dq; dg per token and channel (into dKs, after its use)
-        for (int e = tid; e < kC * dk; e += kThreads) {
-            const int t = e / dk, c = e - t * dk;
+        for (int e = tid; e < kC * dkp; e += kThreads) {
+            const int t = e / dkp, c = e - t * dkp;
             const float gv = s.G[t * LD + c];
-            const float up = expf(gv), down = expf(s.gsum[c] - gv);
+            const float up = tc::ex2(gv), down = tc::ex2(s.gsum[c] - gv);
             const float kv = s.Kt[t * LD + c], qv = s.Qt[t * LD + c];
             const float rk = s.dW[t * LD + c], cc = s.W[t * LD + c], rq = s.dQt[t * LD + c];
             const float dks = s.dKs[t * LD + c], dkb = s.dKb[t * LD + c], dqs = s.dQs[t * LD + c];
@@ -383,7 +596,7 @@ __device__ void bwd_body(float *sm, const Tin *q, const Tin *k, const Tin *v, co
             const float dg = kv * (rk - cc) + qv * rq + dks * s.Ks[t * LD + c] + dqs * s.Qs[t * LD + c] -
                              dkb * s.Kh[t * LD + c];
             s.dKs[t * LD + c] = dg;
-            if (t < valid) {
+            if (t < valid && c < dk) {
                 const long o = ((static_cast<long>(b) * T + t0 + t) * H + h) * dk + c;
                 atomicAdd(dk_acc + o, dk_v);
                 atomicAdd(dq_acc + o, dq_v);

@@ -1,6 +1,7 @@
 // chunk_varlen.cu -- kernel and launch of the variable-length prefill (body in
 // chunk_varlen.cuh, chunk terms shared with the backward pass in chunk_bwd.cuh).
 #include "kda_internal.cuh"
+#include "tc_sm100.cuh"
 
 namespace kda {
 #include "chunk_bwd.cuh"

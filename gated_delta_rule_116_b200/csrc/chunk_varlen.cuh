@@ -1,5 +1,6 @@
 // chunk_varlen.cuh -- chunked KDA prefill over a packed batch of variable-length
-// sequences, fp32 on CUDA cores (bodies; kernels and launch in chunk_varlen.cu).
+// sequences, fp32 state, products on the tensor cores through warp-level tf32 tiles (bodies;
+// kernels and launch in chunk_varlen.cu).
 //
 // Sequence n occupies tokens cu_seqlens[n] .. cu_seqlens[n+1]-1 of packed
 // [total_T, H, d] tensors and starts from its own state (or zeros); the
@@ -26,9 +27,11 @@ __device__ void varlen_body(float *sm, const Tin *q, const Tin *k, const Tin *v,
                             const float *beta, const int32_t *cu_seqlens, const int32_t *slot,
                             const float *S0, Tin *out, float *S_T, int total_T, int H, int dk,
                             int dv) {
+    constexpr bool kSplit = kbwd::kSplitProducts;
     const kbwd::Layout L(dk, kNV);
     kbwd::Tiles s(sm, L);
-    const int tid = threadIdx.x, LD = L.LD, LC = L.LC, NV = L.NV, NP = L.NP;
+    const int tid = threadIdx.x, warp = tid >> 5, dkp = L.dkp, LD = L.LD, LC = L.LC, NV = L.NV,
+              NP = L.NP;
     const int nh = blockIdx.x, n = nh / H, h = nh - n * H;
     const int n0 = blockIdx.y * NV, nv = min(NV, dv - n0);
     // the offsets are device data: clamp them so that every access stays in [0, total_T)
@@ -36,37 +39,35 @@ __device__ void varlen_body(float *sm, const Tin *q, const Tin *k, const Tin *v,
     const int end = min(max(cu_seqlens[n + 1], start), total_T);
     const int len = end - start;
     const long row = (slot ? static_cast<long>(slot[n]) : static_cast<long>(n)) * H + h;   // state row
-    for (int e = tid; e < dk * NV; e += kThreads) {
+    const int nU = NV / 8;
+    static_assert(2 * (kNV / 8) <= kbwd::kWarps, "one output block per warp");
+    for (int e = tid; e < dkp * NV; e += kThreads) {
         const int c = e / NV, j = e - c * NV;
-        s.S[c * NP + j] = (S0 && j < nv) ? S0[(row * dk + c) * dv + n0 + j] : 0.f;
+        s.S[c * NP + j] = (S0 && c < dk && j < nv) ? S0[(row * dk + c) * dv + n0 + j] : 0.f;
     }
     const int nchunks = (len + kC - 1) / kC;
     for (int ch = 0; ch < nchunks; ++ch) {
         const int t0 = start + ch * kC, valid = min(kC, end - t0);
         __syncthreads();
         kbwd::chunk_terms(s, L, q, k, v, log_alpha, beta, 0, h, total_T, H, dv, t0, valid, n0, nv, true);
-        for (int e = tid; e < kC * NV; e += kThreads) {   // U = U' - W S
-            const int i = e / NV, j = e - i * NV;
-            float acc = s.Up[i * NP + j];
-            for (int c = 0; c < dk; ++c) acc = fmaf(-s.W[i * LD + c], s.S[c * NP + j], acc);
-            s.U[i * NP + j] = acc;
+        // U = U' - W S (warps 0 .. nU-1); the inter-chunk part of O, Qs S (warps nU .. 2nU-1)
+        float od[4] = {0.f, 0.f, 0.f, 0.f};
+        const int oj0 = (warp - nU) * 8;
+        if (warp < nU) {
+            kbwd::u_block<kSplit>(s, L, warp * 8);
+        } else if (warp < 2 * nU) {
+            kbwd::tile_mma<kSplit>(od, [&](int m, int kk) { return s.Qs[m * LD + kk]; },
+                                   [&](int kk, int j) { return s.S[kk * NP + j]; }, 0, oj0, 0, dkp);
         }
         __syncthreads();
-        for (int e = tid; e < kC * NV; e += kThreads) {   // O = Qs S + P U
-            const int i = e / NV, j = e - i * NV;
-            if (i >= valid || j >= nv) continue;
-            float acc = 0.f;
-            for (int c = 0; c < dk; ++c) acc = fmaf(s.Qs[i * LD + c], s.S[c * NP + j], acc);
-            for (int m = 0; m <= i; ++m) acc = fmaf(s.P[i * LC + m], s.U[m * NP + j], acc);
-            out[(static_cast<long>(t0 + i) * H + h) * dv + n0 + j] = from_f32<Tin>(acc);
+        if (warp >= nU && warp < 2 * nU) {   // O += P U, written out
+            kbwd::tile_mma<kSplit>(od, [&](int m, int kk) { return s.P[m * LC + kk]; },
+                                   [&](int kk, int j) { return s.U[kk * NP + j]; }, 0, oj0, 0, kC);
+            kbwd::tile_each(od, 0, oj0, [&](int i, int j, float &x) {
+                if (i < valid && j < nv) out[(static_cast<long>(t0 + i) * H + h) * dv + n0 + j] = from_f32<Tin>(x);
+            });
         }
-        __syncthreads();
-        for (int e = tid; e < dk * NV; e += kThreads) {   // S <- Diag(gamma) S + Kb^T U
-            const int c = e / NV, j = e - c * NV;
-            float acc = s.gam[c] * s.S[c * NP + j];
-            for (int t = 0; t < kC; ++t) acc = fmaf(s.Kh[t * LD + c], s.U[t * NP + j], acc);
-            s.S[c * NP + j] = acc;
-        }
+        kbwd::state_update<kSplit>(s, L);   // S <- Diag(gamma) S + Kb^T U
     }
     __syncthreads();
     if (S_T)
