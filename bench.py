@@ -392,7 +392,7 @@ def run_backward(kda, args, device, stream):
     gbs = bytes_alg / (ms / 1e3) / 1e9
     return {"entry": "kda_chunk_bwd", "workload": "prefill_4k (B=8, H=32, T=4096, d=128, bf16, S0 ~ N(0,0.05))",
             "kernel_ms": round(ms, 3), "tokens_per_s": round(w.tokens / (ms / 1e3), 1),
-            "bytes_per_launch": bytes_alg, "kernels": "bwd_states_kernel + bwd_chunk_kernel (fp32 CUDA cores, 16-token chunks)",
+            "bytes_per_launch": bytes_alg, "kernels": "bwd_states_kernel + bwd_chunk_kernel (16-token chunks, dense products as warp-level 3xTF32 tensor-core tiles, pairwise decays on CUDA cores)",
             "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm, "unit": "GB/s",
                          "frac": round(gbs / hbm, 4), "peak_source": src}}
 

@@ -44,9 +44,9 @@ struct Layout {
     int dk, dkp, NV, NP, LD, LC;
     __host__ __device__ Layout(int dk_, int NV_)
         : dk(dk_), dkp((dk_ + 15) & ~15), NV(NV_), NP(NV_ + 4), LD(((dk_ + 15) & ~15) + 4), LC(kC + 4) {}
-    // 12 [C][LD] tiles, 7 [C][LC], 5 [C][NP], 3 [dkp][NP], vectors
+    // 12 [C][LD] tiles, 7 [C][LC], 5 [C][NP], 2 [dkp][NP], vectors
     __host__ __device__ size_t floats() const {
-        return 12ull * kC * LD + 7ull * kC * LC + 5ull * kC * NP + 3ull * dkp * NP + 3ull * dkp + 3ull * kC;
+        return 12ull * kC * LD + 7ull * kC * LC + 5ull * kC * NP + 2ull * dkp * NP + 3ull * dkp + 3ull * kC;
     }
 };
 
@@ -56,7 +56,7 @@ struct Tiles {
     float *Qt, *Kt, *Kh, *G, *W, *dQs, *dKb, *dW, *dKs, *dQt, *Qs, *Ks;   // [C][LD]
     float *At, *P, *X, *Tm, *dT, *dA, *dP;                      // [C][LC]
     float *V, *Up, *U, *dO, *dU;                                 // [C][NP]
-    float *S, *dS, *dSn;                                         // [dkp][NP]
+    float *S, *dS;                                               // [dkp][NP]
     float *gam, *dgam, *gsum;                                    // [dkp]; gsum in log2 units
     float *bt, *dbt, *pad;                                       // [C]
     __device__ Tiles(float *sm, const Layout &L) {
@@ -68,7 +68,7 @@ struct Tiles {
         At = p; p += CC; P = p; p += CC; X = p; p += CC; Tm = p; p += CC; dT = p; p += CC;
         dA = p; p += CC; dP = p; p += CC;
         V = p; p += CN; Up = p; p += CN; U = p; p += CN; dO = p; p += CN; dU = p; p += CN;
-        S = p; p += DN; dS = p; p += DN; dSn = p; p += DN;
+        S = p; p += DN; dS = p; p += DN;
         gam = p; p += L.dkp;
         dgam = p; p += L.dkp; gsum = p; p += L.dkp;
         bt = p; p += kC; dbt = p; p += kC; pad = p;
@@ -174,11 +174,18 @@ __device__ __forceinline__ void prefetch_chunk(const Tin *q, const Tin *k, const
 }
 
 // The state-independent terms of one chunk: g, Qs, Ks, Kb, At, P,
-// X = (I + A)^{-1}, T, W = T Ks, U' = T V. Loads q, k, log alpha, v (slice), beta.
-template <typename Tin>
+// X = (I + A)^{-1}, T, W = T Ks, U' = T V. Loads q, k, log alpha, v (slice), beta,
+// and zeroes U, At and P (which split sums accumulate into). While warp 0
+// solves for X, warps 1 and up run other(warp - 1): work of the caller's that needs
+// none of these terms.
+struct NoWork {
+    __device__ void operator()(int) const {}
+};
+template <typename Tin, class Other = NoWork>
 __device__ void chunk_terms(Tiles &s, const Layout &L, const Tin *q, const Tin *k, const Tin *v,
                             const float *log_alpha, const float *beta, int b, int h, int T, int H,
-                            int dv, int t0, int valid, int n0, int nv, bool need_p) {
+                            int dv, int t0, int valid, int n0, int nv, bool need_p,
+                            const Other &other = Other()) {
     constexpr bool kSplit = kSplitProducts;
     const int tid = threadIdx.x, warp = tid >> 5, dk = L.dk, dkp = L.dkp, LD = L.LD, LC = L.LC,
               NV = L.NV, NP = L.NP;
@@ -218,6 +225,11 @@ __device__ void chunk_terms(Tiles &s, const Layout &L, const Tin *q, const Tin *
         s.V[t * NP + n] = vr[u];
     }
     if (tid < kC) s.bt[tid] = br;
+    for (int e = tid; e < kC * NP; e += kThreads) s.U[e] = 0.f;
+    for (int e = tid; e < kC * LC; e += kThreads) {
+        s.At[e] = 0.f;
+        s.P[e] = 0.f;
+    }
     __syncthreads();
     for (int c = tid; c < dkp; c += kThreads) {   // prefix sums (natural log), kept in log2 units
         float acc = 0.f;
@@ -238,35 +250,42 @@ __device__ void chunk_terms(Tiles &s, const Layout &L, const Tin *q, const Tin *
         s.Ks[t * LD + c] = kv * up;
         s.Kh[t * LD + c] = kv * down;
     }
-    // At (strict lower) and P (lower), one thread per pair i >= j, both from the same
-    // pairwise decays e^{g_i - g_j} <= 1; entries above the diagonal are zero
-    for (int e = tid; e < kC * kC; e += kThreads) {
-        const int i = e / kC, j = e - i * kC;
-        if (j > i) {
-            s.At[i * LC + j] = 0.f;
-            s.P[i * LC + j] = 0.f;
-            continue;
+    // At (strict lower) and P (lower): one thread per (pair i >= j, third of the
+    // channels), summed into the zeroed tiles with shared-memory atomics; both sums use
+    // the same pairwise decays e^{g_i - g_j} <= 1
+    {
+        constexpr int kPairs = kC * (kC + 1) / 2;
+        static_assert(3 * kPairs <= kThreads, "one pass over the items");
+        const int n4 = dkp / 4;
+        if (tid < 3 * kPairs) {
+            const int part = tid / kPairs, p = tid - part * kPairs;
+            int i = static_cast<int>((sqrtf(8.f * p + 1.f) - 1.f) * 0.5f);   // p = i (i + 1) / 2 + j
+            if ((i + 1) * (i + 2) / 2 <= p) ++i;
+            if (i * (i + 1) / 2 > p) --i;
+            const int j = p - i * (i + 1) / 2;
+            const float4 *ki = reinterpret_cast<const float4 *>(s.Kt + i * LD);
+            const float4 *kj = reinterpret_cast<const float4 *>(s.Kt + j * LD);
+            const float4 *qi = reinterpret_cast<const float4 *>(s.Qt + i * LD);
+            const float4 *gi = reinterpret_cast<const float4 *>(s.G + i * LD);
+            const float4 *gj = reinterpret_cast<const float4 *>(s.G + j * LD);
+            float at[4] = {0.f, 0.f, 0.f, 0.f}, pp[4] = {0.f, 0.f, 0.f, 0.f};
+            for (int c4 = part * n4 / 3; c4 < (part + 1) * n4 / 3; ++c4) {
+                const float4 a = ki[c4], bj = kj[c4], q4 = qi[c4], x = gi[c4], y = gj[c4];
+                const float w0 = bj.x * tc::ex2(x.x - y.x), w1 = bj.y * tc::ex2(x.y - y.y);
+                const float w2 = bj.z * tc::ex2(x.z - y.z), w3 = bj.w * tc::ex2(x.w - y.w);
+                at[0] = fmaf(a.x, w0, at[0]); at[1] = fmaf(a.y, w1, at[1]);
+                at[2] = fmaf(a.z, w2, at[2]); at[3] = fmaf(a.w, w3, at[3]);
+                pp[0] = fmaf(q4.x, w0, pp[0]); pp[1] = fmaf(q4.y, w1, pp[1]);
+                pp[2] = fmaf(q4.z, w2, pp[2]); pp[3] = fmaf(q4.w, w3, pp[3]);
+            }
+            if (j < i) atomicAdd(&s.At[i * LC + j], (at[0] + at[1]) + (at[2] + at[3]));
+            if (need_p) atomicAdd(&s.P[i * LC + j], (pp[0] + pp[1]) + (pp[2] + pp[3]));
         }
-        const float4 *ki = reinterpret_cast<const float4 *>(s.Kt + i * LD);
-        const float4 *kj = reinterpret_cast<const float4 *>(s.Kt + j * LD);
-        const float4 *qi = reinterpret_cast<const float4 *>(s.Qt + i * LD);
-        const float4 *gi = reinterpret_cast<const float4 *>(s.G + i * LD);
-        const float4 *gj = reinterpret_cast<const float4 *>(s.G + j * LD);
-        float at[4] = {0.f, 0.f, 0.f, 0.f}, pp[4] = {0.f, 0.f, 0.f, 0.f};
-        for (int c4 = 0; c4 < dkp / 4; ++c4) {
-            const float4 a = ki[c4], bj = kj[c4], q4 = qi[c4], x = gi[c4], y = gj[c4];
-            const float w0 = bj.x * tc::ex2(x.x - y.x), w1 = bj.y * tc::ex2(x.y - y.y);
-            const float w2 = bj.z * tc::ex2(x.z - y.z), w3 = bj.w * tc::ex2(x.w - y.w);
-            at[0] = fmaf(a.x, w0, at[0]); at[1] = fmaf(a.y, w1, at[1]);
-            at[2] = fmaf(a.z, w2, at[2]); at[3] = fmaf(a.w, w3, at[3]);
-            pp[0] = fmaf(q4.x, w0, pp[0]); pp[1] = fmaf(q4.y, w1, pp[1]);
-            pp[2] = fmaf(q4.z, w2, pp[2]); pp[3] = fmaf(q4.w, w3, pp[3]);
-        }
-        s.At[i * LC + j] = j < i ? (at[0] + at[1]) + (at[2] + at[3]) : 0.f;
-        s.P[i * LC + j] = need_p ? (pp[0] + pp[1]) + (pp[2] + pp[3]) : 0.f;
     }
     __syncthreads();
-    if (tid < kC) {   // X = (I + A)^{-1}, A = Diag(beta) At: column j by forward substitution
+    if (warp > 0) {
+        other(warp - 1);
+    } else if (tid < kC) {   // X = (I + A)^{-1}, A = Diag(beta) At: column j by forward substitution
         const int j = tid;
         float xc[kC];   // column j of X, in registers
 #pragma unroll
@@ -297,6 +316,25 @@ __device__ void chunk_terms(Tiles &s, const Layout &L, const Tin *q, const Tin *
         }
     }
     __syncthreads();
+}
+
+// Bounds of part p of 4 of a depth of k8 8-deep steps (some parts empty when k8 < 4).
+__device__ __forceinline__ int depth_lo(int p, int k8) { return (p * k8) / 4 * 8; }
+
+// U += U' - W S over all blocks, the depth (dkp) split in four parts on separate
+// warps and summed with shared-memory atomics; U must be zero on entry.
+template <bool kSplit>
+__device__ __forceinline__ void u_split(Tiles &s, const Layout &L) {
+    const int warp = threadIdx.x >> 5, LD = L.LD, NP = L.NP, nU = L.NV / 8, k8 = L.dkp / 8;
+    for (int tl = warp; tl < 4 * nU; tl += kWarps) {
+        const int part = tl / nU, j0 = (tl - part * nU) * 8;
+        float d[4];
+        tile_each(d, 0, j0, [&](int r, int c, float &x) { x = part == 0 ? s.Up[r * NP + c] : 0.f; });
+        tile_mma<kSplit>(d, [&](int m, int kk) { return -s.W[m * LD + kk]; },
+                         [&](int kk, int n) { return s.S[kk * NP + n]; }, 0, j0, depth_lo(part, k8),
+                         depth_lo(part + 1, k8));
+        tile_each(d, 0, j0, [&](int r, int c, float &x) { atomicAdd(&s.U[r * NP + c], x); });
+    }
 }
 
 // U = U' - W S, one warp per 8 value columns (warps NV/8 and up idle).
@@ -332,7 +370,7 @@ __device__ void states_body(float *sm, const Tin *q, const Tin *k, const Tin *v,
     constexpr bool kSplit = kSplitProducts;
     const Layout L(dk, kNV);
     Tiles s(sm, L);
-    const int tid = threadIdx.x, warp = tid >> 5, dkp = L.dkp, NV = L.NV, NP = L.NP;
+    const int tid = threadIdx.x, dkp = L.dkp, NV = L.NV, NP = L.NP;
     const int bh = blockIdx.x, b = bh / H, h = bh - b * H;
     const int n0 = blockIdx.y * NV, nv = min(NV, dv - n0);
     const int nchunks = (T + kC - 1) / kC;
@@ -345,12 +383,14 @@ __device__ void states_body(float *sm, const Tin *q, const Tin *k, const Tin *v,
         __syncthreads();
         float *dst = states + (static_cast<long>(bh) * nchunks + ch) * dk * dv;
         prefetch_chunk<Tin>(q, k, v, log_alpha, nullptr, nullptr, b, h, T, H, dk, dv, t0 + kC, n0);
-        for (int e = tid; e < dk * NV; e += kThreads) {
-            const int c = e / NV, n = e - c * NV;
-            if (n < nv) dst[static_cast<long>(c) * dv + n0 + n] = s.S[c * NP + n];
-        }
-        chunk_terms(s, L, q, k, v, log_alpha, beta, b, h, T, H, dv, t0, valid, n0, nv, false);
-        for (int tl = warp; tl < NV / 8; tl += kWarps) u_block<kSplit>(s, L, tl * 8);   // U = U' - W S
+        // the chunk's entry state goes out while warp 0 solves for X
+        chunk_terms(s, L, q, k, v, log_alpha, beta, b, h, T, H, dv, t0, valid, n0, nv, false, [&](int w) {
+            for (int e = w * 32 + (tid & 31); e < dk * NV; e += kThreads - 32) {
+                const int c = e / NV, n = e - c * NV;
+                if (n < nv) dst[static_cast<long>(c) * dv + n0 + n] = s.S[c * NP + n];
+            }
+        });
+        u_split<kSplit>(s, L);   // U = U' - W S
         __syncthreads();
         state_update<kSplit>(s, L);   // S <- Diag(gamma) S + Kb^T U
     }
@@ -412,54 +452,62 @@ __device__ void bwd_body(float *sm, const Tin *q, const Tin *k, const Tin *v, co
                 s.dO[t * NP + n] = orr[u];
             }
         }
-        chunk_terms(s, L, q, k, v, log_alpha, beta, b, h, T, H, dv, t0, valid, n0, nv, true);
-        // U = U' - W S; dQs = dO S^T
-        for (int tl = warp; tl < nU + nQ; tl += kWarps) {
-            if (tl < nU) {
-                u_block<kSplit>(s, L, tl * 8);
+        for (int e = tid; e < kC * NP; e += kThreads) s.dU[e] = 0.f;   // split-depth sums
+        for (int e = tid; e < kC * LC; e += kThreads) s.dT[e] = 0.f;
+        // While warp 0 solves for X: gamma's gradient (through the state decay, warps 1-4,
+        // one state row per thread) and dQs = dO S^T (warps 5 and up)
+        chunk_terms(s, L, q, k, v, log_alpha, beta, b, h, T, H, dv, t0, valid, n0, nv, true, [&](int w) {
+            if (w < 4) {
+                const int c = w * 32 + (tid & 31);
+                if (c < dkp) {
+                    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+                    for (int n = 0; n < NV; n += 4) {
+                        a0 = fmaf(s.dS[c * NP + n], s.S[c * NP + n], a0);
+                        a1 = fmaf(s.dS[c * NP + n + 1], s.S[c * NP + n + 1], a1);
+                        a2 = fmaf(s.dS[c * NP + n + 2], s.S[c * NP + n + 2], a2);
+                        a3 = fmaf(s.dS[c * NP + n + 3], s.S[c * NP + n + 3], a3);
+                    }
+                    s.dgam[c] = ((a0 + a1) + (a2 + a3)) * s.gam[c];
+                }
             } else {
-                const int c0 = (tl - nU) * 8;
-                float d[4] = {0.f, 0.f, 0.f, 0.f};
-                tile_mma<kSplit>(d, [&](int m, int kk) { return s.dO[m * NP + kk]; },
-                                 [&](int kk, int c) { return s.S[c * NP + kk]; }, 0, c0, 0, NV);
-                tile_each(d, 0, c0, [&](int r, int c, float &x) { s.dQs[r * LD + c] = x; });
+                for (int tl = w - 4; tl < nQ; tl += kWarps - 5) {
+                    const int c0 = tl * 8;
+                    float d[4] = {0.f, 0.f, 0.f, 0.f};
+                    tile_mma<kSplit>(d, [&](int m, int kk) { return s.dO[m * NP + kk]; },
+                                     [&](int kk, int c) { return s.S[c * NP + kk]; }, 0, c0, 0, NV);
+                    tile_each(d, 0, c0, [&](int r, int c, float &x) { s.dQs[r * LD + c] = x; });
+                }
             }
-        }
+        });
+        u_split<kSplit>(s, L);   // U = U' - W S
         __syncthreads();
-        // dU = P^T dO + Kb dS; dKb = U dS^T; dP = lower(dO U^T); gamma's gradient
-        for (int tl = warp; tl < nU + nQ + 2; tl += kWarps) {
+        // dU = P^T dO + Kb dS (depth split in four); dKb = U dS^T; dP = lower(dO U^T)
+        for (int tl = warp; tl < 4 * nU + nQ + 2; tl += kWarps) {
             float d[4] = {0.f, 0.f, 0.f, 0.f};
-            if (tl < nU) {
-                const int j0 = tl * 8;
-                tile_mma<kSplit>(d, [&](int m, int kk) { return s.P[kk * LC + m]; },
-                                 [&](int kk, int n) { return s.dO[kk * NP + n]; }, 0, j0, 0, kC);
+            if (tl < 4 * nU) {
+                const int part = tl / nU, j0 = (tl - part * nU) * 8;
+                if (part == 0)
+                    tile_mma<kSplit>(d, [&](int m, int kk) { return s.P[kk * LC + m]; },
+                                     [&](int kk, int n) { return s.dO[kk * NP + n]; }, 0, j0, 0, kC);
                 tile_mma<kSplit>(d, [&](int m, int kk) { return s.Kh[m * LD + kk]; },
-                                 [&](int kk, int n) { return s.dS[kk * NP + n]; }, 0, j0, 0, dkp);
-                tile_each(d, 0, j0, [&](int r, int c, float &x) { s.dU[r * NP + c] = x; });
-            } else if (tl < nU + nQ) {
-                const int c0 = (tl - nU) * 8;
+                                 [&](int kk, int n) { return s.dS[kk * NP + n]; }, 0, j0,
+                                 depth_lo(part, dkp / 8), depth_lo(part + 1, dkp / 8));
+                tile_each(d, 0, j0, [&](int r, int c, float &x) { atomicAdd(&s.dU[r * NP + c], x); });
+            } else if (tl < 4 * nU + nQ) {
+                const int c0 = (tl - 4 * nU) * 8;
                 tile_mma<kSplit>(d, [&](int m, int kk) { return s.U[m * NP + kk]; },
                                  [&](int kk, int c) { return s.dS[c * NP + kk]; }, 0, c0, 0, NV);
                 tile_each(d, 0, c0, [&](int r, int c, float &x) { s.dKb[r * LD + c] = x; });
             } else {
-                const int j0 = (tl - nU - nQ) * 8;
+                const int j0 = (tl - 4 * nU - nQ) * 8;
                 tile_mma<kSplit>(d, [&](int m, int kk) { return s.dO[m * NP + kk]; },
                                  [&](int kk, int j) { return s.U[j * NP + kk]; }, 0, j0, 0, NV);
                 tile_each(d, 0, j0, [&](int r, int c, float &x) { s.dP[r * LC + c] = c <= r ? x : 0.f; });
             }
         }
-        static_assert(kThreads >= 4 * 128, "four threads per state row");
-        {   // gamma's gradient (through the state decay): four threads per row
-            const int c = tid >> 2, part = tid & 3;
-            float acc = 0.f;
-            if (c < dkp)
-                for (int n = part; n < NV; n += 4) acc = fmaf(s.dS[c * NP + n], s.S[c * NP + n], acc);
-            acc += __shfl_xor_sync(0xffffffffu, acc, 1);
-            acc += __shfl_xor_sync(0xffffffffu, acc, 2);
-            if (c < dkp && part == 0) s.dgam[c] = acc * s.gam[c];
-        }
         __syncthreads();
-        // dSn = Diag(gamma) dS + Qs^T dO - W^T dU; dW = -dU S^T; dV = T^T dU
+        // dS <- Diag(gamma) dS + Qs^T dO - W^T dU (in place: each block reads only its own
+        // dS entries); dW = -dU S^T; dV = T^T dU
         for (int tl = warp; tl < nS + nQ + nU; tl += kWarps) {
             float d[4] = {0.f, 0.f, 0.f, 0.f};
             if (tl < nS) {
@@ -469,7 +517,7 @@ __device__ void bwd_body(float *sm, const Tin *q, const Tin *k, const Tin *v, co
                                  [&](int kk, int n) { return s.dO[kk * NP + n]; }, m0, j0, 0, kC);
                 tile_mma<kSplit>(d, [&](int m, int kk) { return -s.W[kk * LD + m]; },
                                  [&](int kk, int n) { return s.dU[kk * NP + n]; }, m0, j0, 0, kC);
-                tile_each(d, m0, j0, [&](int r, int c, float &x) { s.dSn[r * NP + c] = x; });
+                tile_each(d, m0, j0, [&](int r, int c, float &x) { s.dS[r * NP + c] = x; });
             } else if (tl < nS + nQ) {
                 const int c0 = (tl - nS) * 8;
                 tile_mma<kSplit>(d, [&](int m, int kk) { return -s.dU[m * NP + kk]; },
@@ -486,36 +534,35 @@ __device__ void bwd_body(float *sm, const Tin *q, const Tin *k, const Tin *v, co
             }
         }
         __syncthreads();
-        {   // the state gradient moves one chunk back
-            float *t = s.dS;
-            s.dS = s.dSn;
-            s.dSn = t;
-        }
-        // dT = dW Ks^T + dU V^T (lower incl. diagonal), dKs = T^T dW
-        for (int tl = warp; tl < 2 + nQ; tl += kWarps) {
+        // dT = dW Ks^T + dU V^T (depth split in four; its upper triangle is masked where
+        // it is read), dKs = T^T dW; W (read for the last time above) is zeroed for Cc
+        for (int e = tid; e < kC * LD; e += kThreads) s.W[e] = 0.f;
+        for (int tl = warp; tl < 8 + nQ; tl += kWarps) {
             float d[4] = {0.f, 0.f, 0.f, 0.f};
-            if (tl < 2) {
-                const int j0 = tl * 8;
+            if (tl < 8) {
+                const int part = tl >> 1, j0 = (tl & 1) * 8;
                 tile_mma<kSplit>(d, [&](int m, int kk) { return s.dW[m * LD + kk]; },
-                                 [&](int kk, int j) { return s.Ks[j * LD + kk]; }, 0, j0, 0, dkp);
-                tile_mma<kSplit>(d, [&](int m, int kk) { return s.dU[m * NP + kk]; },
-                                 [&](int kk, int j) { return s.V[j * NP + kk]; }, 0, j0, 0, NV);
-                tile_each(d, 0, j0, [&](int r, int c, float &x) { s.dT[r * LC + c] = c <= r ? x : 0.f; });
+                                 [&](int kk, int j) { return s.Ks[j * LD + kk]; }, 0, j0,
+                                 depth_lo(part, dkp / 8), depth_lo(part + 1, dkp / 8));
+                if (part == 0)
+                    tile_mma<kSplit>(d, [&](int m, int kk) { return s.dU[m * NP + kk]; },
+                                     [&](int kk, int j) { return s.V[j * NP + kk]; }, 0, j0, 0, NV);
+                tile_each(d, 0, j0, [&](int r, int c, float &x) { atomicAdd(&s.dT[r * LC + c], x); });
             } else {
-                const int c0 = (tl - 2) * 8;
+                const int c0 = (tl - 8) * 8;
                 tile_mma<kSplit>(d, [&](int m, int kk) { return s.Tm[kk * LC + m]; },
                                  [&](int kk, int c) { return s.dW[kk * LD + c]; }, 0, c0, 0, kC);
                 tile_each(d, 0, c0, [&](int r, int c, float &x) { s.dKs[r * LD + c] = x; });
             }
         }
         __syncthreads();
-        // Z = X^T dX with dX = dT Diag(beta) (kept in dA), and dbeta's T part
+        // Z = X^T dX with dX = lower(dT) Diag(beta) (kept in dA), and dbeta's T part
         for (int e = tid; e < kC * kC + kC; e += kThreads) {
             if (e < kC * kC) {
                 const int i = e / kC, bcol = e - i * kC;
                 float acc = 0.f;
-                for (int a = i; a < kC; ++a) acc = fmaf(s.X[a * LC + i], s.dT[a * LC + bcol] * s.bt[bcol], acc);
-                s.dA[i * LC + bcol] = acc;
+                for (int a = max(i, bcol); a < kC; ++a) acc = fmaf(s.X[a * LC + i], s.dT[a * LC + bcol], acc);
+                s.dA[i * LC + bcol] = acc * s.bt[bcol];
             } else {
                 const int j = e - kC * kC;
                 float acc = 0.f;
@@ -524,25 +571,21 @@ __device__ void bwd_body(float *sm, const Tin *q, const Tin *k, const Tin *v, co
             }
         }
         __syncthreads();
-        // dA = -strict_lower(Z X^T) (into dT, whose values are no longer needed)
-        for (int e = tid; e < kC * kC; e += kThreads) {
-            const int i = e / kC, j = e - i * kC;
+        // dA = -strict_lower(Z X^T); dbeta's A part (row sums of dA o At, over the 16
+        // lanes that hold a row); dAt = Diag(beta) dA, into dT
+        static_assert(kC == 16 && kThreads >= kC * kC, "a row of dA per half warp");
+        if (tid < kC * kC) {
+            const int i = tid / kC, j = tid - i * kC;
             float acc = 0.f;
             if (j < i)
                 for (int bcol = 0; bcol <= j; ++bcol) acc = fmaf(s.dA[i * LC + bcol], s.X[j * LC + bcol], acc);
-            s.dT[i * LC + j] = -acc;
-        }
-        __syncthreads();
-        // dbeta's A part; dAt = Diag(beta) dA (in dT)
-        for (int i = tid; i < kC; i += kThreads) {
-            float acc = 0.f;
-            for (int j = 0; j < i; ++j) acc = fmaf(s.dT[i * LC + j], s.At[i * LC + j], acc);
-            s.dbt[i] += acc;
-        }
-        __syncthreads();
-        for (int e = tid; e < kC * kC; e += kThreads) {
-            const int i = e / kC;
-            s.dT[(i)*LC + (e - i * kC)] *= s.bt[i];
+            float r = -acc * s.At[i * LC + j];
+            r += __shfl_xor_sync(0xffffffffu, r, 8);
+            r += __shfl_xor_sync(0xffffffffu, r, 4);
+            r += __shfl_xor_sync(0xffffffffu, r, 2);
+            r += __shfl_xor_sync(0xffffffffu, r, 1);
+            if (j == 0) s.dbt[i] += r;
+            s.dT[i * LC + j] = -acc * s.bt[i];
         }
         __syncthreads();
         // The intra-chunk products, term by term (E_ij = e^{g_i - g_j} per channel):
@@ -550,36 +593,39 @@ __device__ void bwd_body(float *sm, const Tin *q, const Tin *k, const Tin *v, co
         //   Cc_j = sum_{i>j}  dAt_ij k_i E_ij
         //        + sum_{i>=j} dP_ij  q_i E_ij             (column side,     into W)
         //   Rq_i = sum_{j<=i} dP_ij  k_j E_ij             (row side of P,   into dQt)
-        // One thread per channel walks every pair j < i once, so each decay is computed
-        // once for the three sums; the diagonal (E = 1) starts Cc and Rq.
-        for (int c = tid; c < dkp; c += kThreads) {
-            float g[kC], kk[kC], qq[kC], R[kC], Cc[kC], Rq[kC];
+        // Each decay is computed once for the three sums: a warp takes the rows i of one
+        // residue mod 4 and 32 channels (a lane per channel), walks the pairs j < i of its
+        // rows, writes R and Rq of those rows and adds its Cc parts into W (zeroed);
+        // the diagonal (E = 1) starts Rq and Cc.
+        {
+            const int part = warp & 3, c = (warp >> 2) * 32 + (tid & 31);
+            static_assert(kWarps == 16, "four residues x four groups of 32 channels");
+            if (c < dkp) {
+                float g[kC], kk[kC], qq[kC], Cc[kC];
 #pragma unroll
-            for (int i = 0; i < kC; ++i) {
-                g[i] = s.G[i * LD + c];
-                kk[i] = s.Kt[i * LD + c];
-                qq[i] = s.Qt[i * LD + c];
-                const float pd = s.dP[i * LC + i];
-                R[i] = 0.f;
-                Cc[i] = pd * qq[i];
-                Rq[i] = pd * kk[i];
-            }
-#pragma unroll
-            for (int i = 1; i < kC; ++i) {
-#pragma unroll
-                for (int j = 0; j < i; ++j) {
-                    const float E = tc::ex2(g[i] - g[j]);
-                    const float a = s.dT[i * LC + j], p = s.dP[i * LC + j];
-                    R[i] = fmaf(a * kk[j], E, R[i]);
-                    Rq[i] = fmaf(p * kk[j], E, Rq[i]);
-                    Cc[j] = fmaf(fmaf(a, kk[i], p * qq[i]), E, Cc[j]);
+                for (int i = 0; i < kC; ++i) {
+                    g[i] = s.G[i * LD + c];
+                    kk[i] = s.Kt[i * LD + c];
+                    qq[i] = s.Qt[i * LD + c];
+                    Cc[i] = (i & 3) == part ? s.dP[i * LC + i] * qq[i] : 0.f;
                 }
-            }
 #pragma unroll
-            for (int i = 0; i < kC; ++i) {
-                s.dW[i * LD + c] = R[i];
-                s.W[i * LD + c] = Cc[i];
-                s.dQt[i * LD + c] = Rq[i];
+                for (int i = 0; i < kC; ++i) {
+                    if ((i & 3) != part) continue;
+                    float R = 0.f, Rq = s.dP[i * LC + i] * kk[i];
+#pragma unroll
+                    for (int j = 0; j < i; ++j) {
+                        const float E = tc::ex2(g[i] - g[j]);
+                        const float a = s.dT[i * LC + j], p = s.dP[i * LC + j];
+                        R = fmaf(a * kk[j], E, R);
+                        Rq = fmaf(p * kk[j], E, Rq);
+                        Cc[j] = fmaf(fmaf(a, kk[i], p * qq[i]), E, Cc[j]);
+                    }
+                    s.dW[i * LD + c] = R;
+                    s.dQt[i * LD + c] = Rq;
+                }
+#pragma unroll
+                for (int j = 0; j < kC; ++j) atomicAdd(&s.W[j * LD + c], Cc[j]);
             }
         }
         __syncthreads();
@@ -603,14 +649,34 @@ __device__ void bwd_body(float *sm, const Tin *q, const Tin *k, const Tin *v, co
             }
         }
         __syncthreads();
-        for (int c = tid; c < dk; c += kThreads) {   // g_C's own terms, then the in-chunk suffix sums
-            float gc = s.dgam[c];
-            for (int t = 0; t < kC; ++t) gc = fmaf(s.dKb[t * LD + c], s.Kh[t * LD + c], gc);
-            float acc = gc;
-            for (int t = kC - 1; t >= 0; --t) {
-                acc += s.dKs[t * LD + c];
-                if (t < valid)
-                    atomicAdd(dlog_alpha + ((static_cast<long>(b) * T + t0 + t) * H + h) * dk + c, acc);
+        static_assert(kThreads >= 4 * 128, "four threads per channel");
+        {   // g_C's own terms, then the in-chunk suffix sums: four threads per channel, four
+            // tokens each, the parts' totals combined across the four lanes
+            const int c = tid >> 2, part = tid & 3;
+            float gc = 0.f, loc = 0.f, sfx[4];
+            if (c < dkp) {
+#pragma unroll
+                for (int u = 3; u >= 0; --u) {
+                    const int t = 4 * part + u;
+                    gc = fmaf(s.dKb[t * LD + c], s.Kh[t * LD + c], gc);
+                    loc += s.dKs[t * LD + c];
+                    sfx[u] = loc;
+                }
+            }
+            gc += __shfl_xor_sync(0xffffffffu, gc, 1);
+            gc += __shfl_xor_sync(0xffffffffu, gc, 2);
+            // tokens after this part's: the totals of the higher parts
+            const float t1 = __shfl_down_sync(0xffffffffu, loc, 1), t2 = __shfl_down_sync(0xffffffffu, loc, 2),
+                        t3 = __shfl_down_sync(0xffffffffu, loc, 3);
+            const float after = (part < 3 ? t1 : 0.f) + (part < 2 ? t2 : 0.f) + (part < 1 ? t3 : 0.f);
+            if (c < dk) {
+                const float base = (c < dkp ? s.dgam[c] : 0.f) + gc + after;
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int t = 4 * part + u;
+                    if (t < valid)
+                        atomicAdd(dlog_alpha + ((static_cast<long>(b) * T + t0 + t) * H + h) * dk + c, base + sfx[u]);
+                }
             }
         }
         for (int t = tid; t < valid; t += kThreads)
