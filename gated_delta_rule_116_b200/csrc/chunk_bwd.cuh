@@ -1,4 +1,4 @@
-// chunk_bwd.cuh -- backward pass of the chunked KDA prefill, fp32 on CUDA cores.
+// chunk_bwd.cuh -- backward pass of the chunked KDA prefill (fp32 state and accumulation).
 //
 // The pages print no backward pass (Kimi Linear summary,
 // es.news.hada.io/topic?id=31936, section "Algoritmo paralelo por chunks",
@@ -32,7 +32,7 @@ namespace kbwd {
 constexpr int kThreads = 512;
 constexpr int kWarps = kThreads / 32;
 constexpr int kC = 16;
-constexpr int kNV = 32;
+constexpr int kNV = 64;
 static_assert(kC * kNV % kThreads == 0 && kC * 128 % kThreads == 0, "whole loads per thread");
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -169,8 +169,11 @@ __device__ __forceinline__ void prefetch_chunk(const Tin *q, const Tin *k, const
         else if (r == 2 * qlines + glines) pf(v + row * dv + n0);
         else pf(dout + row * dv + n0);
     }
-    if (state)
-        for (int c = tid; c < dk; c += kThreads) pf(state + static_cast<long>(c) * dv + n0);
+    if (state)   // a row's slice: kNV floats from column n0, in 128-byte lines
+        for (int e = tid; e < dk * (kNV / 32); e += kThreads) {
+            const int c = e / (kNV / 32), l = e - c * (kNV / 32);
+            if (n0 + 32 * l < dv) pf(state + static_cast<long>(c) * dv + n0 + 32 * l);
+        }
 }
 
 // The state-independent terms of one chunk: g, Qs, Ks, Kb, At, P,

@@ -13,7 +13,7 @@
 // the previous chunk's last state, the WY/UT form, and outputs that add the
 // inter-chunk recurrent part to the intra-chunk parallel part. The chunk terms
 // are those of the backward pass (chunk_bwd.cuh: chunk_terms), 16 tokens long;
-// a CTA owns (sequence, head, 32 value columns).
+// a CTA owns (sequence, head, 64 value columns).
 #pragma once
 
 namespace kvar {
