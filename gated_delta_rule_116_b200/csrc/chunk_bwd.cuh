@@ -33,6 +33,7 @@ constexpr int kThreads = 512;
 constexpr int kWarps = kThreads / 32;
 constexpr int kC = 16;
 constexpr int kNV = 64;
+static_assert(kNV % 32 == 0, "whole 32-column strips");
 static_assert(kC * kNV % kThreads == 0 && kC * 128 % kThreads == 0, "whole loads per thread");
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -44,9 +45,10 @@ struct Layout {
     int dk, dkp, NV, NP, LD, LC;
     __host__ __device__ Layout(int dk_, int NV_)
         : dk(dk_), dkp((dk_ + 15) & ~15), NV(NV_), NP(NV_ + 4), LD(((dk_ + 15) & ~15) + 4), LC(kC + 4) {}
-    // 12 [C][LD] tiles, 7 [C][LC], 5 [C][NP], 2 [dkp][NP], vectors
+    // 12 [C][LD] tiles, 7 [C][LC], 5 [C][NP], 2 [dkp][NP], vectors, partial sums
     __host__ __device__ size_t floats() const {
-        return 12ull * kC * LD + 7ull * kC * LC + 5ull * kC * NP + 2ull * dkp * NP + 3ull * dkp + 3ull * kC;
+        return 12ull * kC * LD + 7ull * kC * LC + 5ull * kC * NP + 2ull * dkp * NP + 3ull * dkp + 3ull * kC +
+               8ull * kC * kC;
     }
 };
 
@@ -58,7 +60,8 @@ struct Tiles {
     float *V, *Up, *U, *dO, *dU;                                 // [C][NP]
     float *S, *dS;                                               // [dkp][NP]
     float *gam, *dgam, *gsum;                                    // [dkp]; gsum in log2 units
-    float *bt, *dbt, *pad;                                       // [C]
+    float *bt, *dbt;                                             // [C]
+    float *part;   // [8][C][C]: partial sums of At and P (three parts each) and of dT (eight)
     __device__ Tiles(float *sm, const Layout &L) {
         const int CD = kC * L.LD, CC = kC * L.LC, CN = kC * L.NP, DN = L.dkp * L.NP;
         float *p = sm;
@@ -71,7 +74,7 @@ struct Tiles {
         S = p; p += DN; dS = p; p += DN;
         gam = p; p += L.dkp;
         dgam = p; p += L.dkp; gsum = p; p += L.dkp;
-        bt = p; p += kC; dbt = p; p += kC; pad = p;
+        bt = p; p += kC; dbt = p; p += kC; part = p;
     }
 };
 
@@ -147,6 +150,60 @@ __device__ __forceinline__ void tile_each(float (&d)[4], int m0, int n0, const F
     f(m0 + g + 8, n0 + 2 * t + 1, d[3]);
 }
 
+// A strip of NT adjacent blocks (rows m0..m0+15, columns n0..n0+8NT-1) sharing each
+// step's A fragment, whose tf32 split is then done once for the NT products:
+// d[nt] += sum_{k0 <= k < k1} A(m, k) B(k, n) over block nt. Each block keeps its
+// high and low products in separate chains.
+template <bool kSplit, int NT, class FA, class FB>
+__device__ __forceinline__ void strip_mma(float (&d)[NT][4], const FA &A, const FB &B, int m0, int n0,
+                                          int k0, int k1) {
+    const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+    float e[NT][4];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) e[nt][0] = e[nt][1] = e[nt][2] = e[nt][3] = 0.f;
+    for (int k = k0; k < k1; k += 8) {
+        const float a[4] = {A(m0 + g, k + t), A(m0 + g + 8, k + t), A(m0 + g, k + t + 4),
+                            A(m0 + g + 8, k + t + 4)};
+        uint32_t ah[4], al[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            ah[i] = tf32_bits(a[i]);
+            al[i] = kSplit ? tf32_bits(a[i] - __uint_as_float(ah[i])) : 0u;
+        }
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            const float b0 = B(k + t, n0 + 8 * nt + g), b1 = B(k + t + 4, n0 + 8 * nt + g);
+            const uint32_t bh0 = tf32_bits(b0), bh1 = tf32_bits(b1);
+            if constexpr (kSplit) {
+                tc::mma_16x8x8_tf32(e[nt], al, bh0, bh1);
+                tc::mma_16x8x8_tf32(e[nt], ah, tf32_bits(b0 - __uint_as_float(bh0)),
+                                    tf32_bits(b1 - __uint_as_float(bh1)));
+            }
+            tc::mma_16x8x8_tf32(d[nt], ah, bh0, bh1);
+        }
+    }
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) d[nt][i] += e[nt][i];
+}
+
+template <int NT, class F>
+__device__ __forceinline__ void strip_each(float (&d)[NT][4], int m0, int n0, const F &f) {
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) tile_each(d[nt], m0, n0 + 8 * nt, f);
+}
+
+template <int NT>
+__device__ __forceinline__ void strip_zero(float (&d)[NT][4]) {
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) d[nt][0] = d[nt][1] = d[nt][2] = d[nt][3] = 0.f;
+}
+
+// Strip widths: 32 value columns (kNV is a multiple of 32), 16 key channels (dkp
+// is a multiple of 16).
+constexpr int kVS = 4, kKS = 2;
+
 // Brings the rows of chunk [t0, t0 + C) of q, k, log alpha, v (value slice) and, when
 // given, dL/dO (value slice) and a stored state slice into L2 ahead of their loads.
 template <typename Tin>
@@ -178,9 +235,8 @@ __device__ __forceinline__ void prefetch_chunk(const Tin *q, const Tin *k, const
 
 // The state-independent terms of one chunk: g, Qs, Ks, Kb, At, P,
 // X = (I + A)^{-1}, T, W = T Ks, U' = T V. Loads q, k, log alpha, v (slice), beta,
-// and zeroes U, At and P (which split sums accumulate into). While warp 0
-// solves for X, warps 1 and up run other(warp - 1): work of the caller's that needs
-// none of these terms.
+// While warp 0 solves for X, warps 1 and up run other(warp - 1): work of the
+// caller's that needs none of these terms.
 struct NoWork {
     __device__ void operator()(int) const {}
 };
@@ -228,11 +284,6 @@ __device__ void chunk_terms(Tiles &s, const Layout &L, const Tin *q, const Tin *
         s.V[t * NP + n] = vr[u];
     }
     if (tid < kC) s.bt[tid] = br;
-    for (int e = tid; e < kC * NP; e += kThreads) s.U[e] = 0.f;
-    for (int e = tid; e < kC * LC; e += kThreads) {
-        s.At[e] = 0.f;
-        s.P[e] = 0.f;
-    }
     __syncthreads();
     for (int c = tid; c < dkp; c += kThreads) {   // prefix sums (natural log), kept in log2 units
         float acc = 0.f;
@@ -254,7 +305,7 @@ __device__ void chunk_terms(Tiles &s, const Layout &L, const Tin *q, const Tin *
         s.Kh[t * LD + c] = kv * down;
     }
     // At (strict lower) and P (lower): one thread per (pair i >= j, third of the
-    // channels), summed into the zeroed tiles with shared-memory atomics; both sums use
+    // channels), partial sums written apart and added in a fixed order below; both use
     // the same pairwise decays e^{g_i - g_j} <= 1
     {
         constexpr int kPairs = kC * (kC + 1) / 2;
@@ -281,14 +332,31 @@ __device__ void chunk_terms(Tiles &s, const Layout &L, const Tin *q, const Tin *
                 pp[0] = fmaf(q4.x, w0, pp[0]); pp[1] = fmaf(q4.y, w1, pp[1]);
                 pp[2] = fmaf(q4.z, w2, pp[2]); pp[3] = fmaf(q4.w, w3, pp[3]);
             }
-            if (j < i) atomicAdd(&s.At[i * LC + j], (at[0] + at[1]) + (at[2] + at[3]));
-            if (need_p) atomicAdd(&s.P[i * LC + j], (pp[0] + pp[1]) + (pp[2] + pp[3]));
+            float *part_out = s.part + part * 2 * kC * kC + i * kC + j;   // [part][At|P][i][j]
+            part_out[0] = (at[0] + at[1]) + (at[2] + at[3]);
+            part_out[kC * kC] = (pp[0] + pp[1]) + (pp[2] + pp[3]);
         }
     }
     __syncthreads();
+    static_assert(kThreads - 32 >= kC * kC, "P in one pass of warps 1 and up");
+    const auto third = [&](int which, int e) {   // the three partial sums of At or P, in order
+        const float *x = s.part + which * kC * kC + e;
+        return (x[0] + x[2 * kC * kC]) + x[4 * kC * kC];
+    };
     if (warp > 0) {
+        if (tid - 32 < kC * kC) {
+            const int e = tid - 32, i = e / kC, j = e - i * kC;
+            s.P[i * LC + j] = (need_p && j <= i) ? third(1, e) : 0.f;
+        }
         other(warp - 1);
-    } else if (tid < kC) {   // X = (I + A)^{-1}, A = Diag(beta) At: column j by forward substitution
+    } else {
+        for (int e = tid; e < kC * kC; e += 32) {
+            const int i = e / kC, j = e - i * kC;
+            s.At[i * LC + j] = j < i ? third(0, e) : 0.f;
+        }
+        __syncwarp();
+    }
+    if (tid < kC) {   // X = (I + A)^{-1}, A = Diag(beta) At: column j by forward substitution
         const int j = tid;
         float xc[kC];   // column j of X, in registers
 #pragma unroll
@@ -302,45 +370,31 @@ __device__ void chunk_terms(Tiles &s, const Layout &L, const Tin *q, const Tin *
         }
     }
     __syncthreads();
-    {   // W = T Ks (dkp / 8 blocks), U' = T V (NV / 8 blocks); T is lower triangular
-        const int nW = dkp / 8, nU = NV / 8;
+    {   // W = T Ks (16-channel strips), U' = T V (32-column strips); T is lower triangular
+        const int nW = dkp / 16, nU = NV / 32;
+        const auto A = [&](int m, int kk) { return s.Tm[m * LC + kk]; };
         for (int tl = warp; tl < nW + nU; tl += kWarps) {
-            float d[4] = {0.f, 0.f, 0.f, 0.f};
-            const auto A = [&](int m, int kk) { return s.Tm[m * LC + kk]; };
             if (tl < nW) {
-                const int c0 = tl * 8;
-                tile_mma<kSplit>(d, A, [&](int kk, int n) { return s.Ks[kk * LD + n]; }, 0, c0, 0, kC);
-                tile_each(d, 0, c0, [&](int r, int c, float &x) { s.W[r * LD + c] = x; });
+                float d[kKS][4];
+                strip_zero(d);
+                strip_mma<kSplit>(d, A, [&](int kk, int n) { return s.Ks[kk * LD + n]; }, 0, tl * 16, 0, kC);
+                strip_each(d, 0, tl * 16, [&](int r, int c, float &x) { s.W[r * LD + c] = x; });
             } else {
-                const int j0 = (tl - nW) * 8;
-                tile_mma<kSplit>(d, A, [&](int kk, int n) { return s.V[kk * NP + n]; }, 0, j0, 0, kC);
-                tile_each(d, 0, j0, [&](int r, int c, float &x) { s.Up[r * NP + c] = x; });
+                float d[kVS][4];
+                strip_zero(d);
+                const int j0 = (tl - nW) * 32;
+                strip_mma<kSplit>(d, A, [&](int kk, int n) { return s.V[kk * NP + n]; }, 0, j0, 0, kC);
+                strip_each(d, 0, j0, [&](int r, int c, float &x) { s.Up[r * NP + c] = x; });
             }
         }
     }
     __syncthreads();
 }
 
-// Bounds of part p of 4 of a depth of k8 8-deep steps (some parts empty when k8 < 4).
-__device__ __forceinline__ int depth_lo(int p, int k8) { return (p * k8) / 4 * 8; }
+// Bounds of part p of `parts` of a depth of k8 8-deep steps (parts may be empty).
+__device__ __forceinline__ int depth_lo(int p, int k8, int parts) { return (p * k8) / parts * 8; }
 
-// U += U' - W S over all blocks, the depth (dkp) split in four parts on separate
-// warps and summed with shared-memory atomics; U must be zero on entry.
-template <bool kSplit>
-__device__ __forceinline__ void u_split(Tiles &s, const Layout &L) {
-    const int warp = threadIdx.x >> 5, LD = L.LD, NP = L.NP, nU = L.NV / 8, k8 = L.dkp / 8;
-    for (int tl = warp; tl < 4 * nU; tl += kWarps) {
-        const int part = tl / nU, j0 = (tl - part * nU) * 8;
-        float d[4];
-        tile_each(d, 0, j0, [&](int r, int c, float &x) { x = part == 0 ? s.Up[r * NP + c] : 0.f; });
-        tile_mma<kSplit>(d, [&](int m, int kk) { return -s.W[m * LD + kk]; },
-                         [&](int kk, int n) { return s.S[kk * NP + n]; }, 0, j0, depth_lo(part, k8),
-                         depth_lo(part + 1, k8));
-        tile_each(d, 0, j0, [&](int r, int c, float &x) { atomicAdd(&s.U[r * NP + c], x); });
-    }
-}
-
-// U = U' - W S, one warp per 8 value columns (warps NV/8 and up idle).
+// U = U' - W S, full depth, one warp per 8 value columns.
 template <bool kSplit>
 __device__ __forceinline__ void u_block(Tiles &s, const Layout &L, int j0) {
     const int LD = L.LD, NP = L.NP;
@@ -351,17 +405,17 @@ __device__ __forceinline__ void u_block(Tiles &s, const Layout &L, int j0) {
     tile_each(d, 0, j0, [&](int r, int c, float &x) { s.U[r * NP + c] = x; });
 }
 
-// S <- Diag(gamma) S + Kb^T U over all dkp x NV blocks.
+// S <- Diag(gamma) S + Kb^T U over 16-row x 32-column strips.
 template <bool kSplit>
 __device__ __forceinline__ void state_update(Tiles &s, const Layout &L) {
-    const int warp = threadIdx.x >> 5, LD = L.LD, NP = L.NP, nN = L.NV / 8;
+    const int warp = threadIdx.x >> 5, LD = L.LD, NP = L.NP, nN = L.NV / 32;
     for (int tl = warp; tl < (L.dkp / 16) * nN; tl += kWarps) {
-        const int m0 = (tl / nN) * 16, j0 = (tl - (tl / nN) * nN) * 8;
-        float d[4];
-        tile_each(d, m0, j0, [&](int r, int c, float &x) { x = s.gam[r] * s.S[r * NP + c]; });
-        tile_mma<kSplit>(d, [&](int m, int kk) { return s.Kh[kk * LD + m]; },
-                         [&](int kk, int n) { return s.U[kk * NP + n]; }, m0, j0, 0, kC);
-        tile_each(d, m0, j0, [&](int r, int c, float &x) { s.S[r * NP + c] = x; });
+        const int m0 = (tl / nN) * 16, j0 = (tl - (tl / nN) * nN) * 32;
+        float d[kVS][4];
+        strip_each(d, m0, j0, [&](int r, int c, float &x) { x = s.gam[r] * s.S[r * NP + c]; });
+        strip_mma<kSplit>(d, [&](int m, int kk) { return s.Kh[kk * LD + m]; },
+                          [&](int kk, int n) { return s.U[kk * NP + n]; }, m0, j0, 0, kC);
+        strip_each(d, m0, j0, [&](int r, int c, float &x) { s.S[r * NP + c] = x; });
     }
 }
 
@@ -373,7 +427,7 @@ __device__ void states_body(float *sm, const Tin *q, const Tin *k, const Tin *v,
     constexpr bool kSplit = kSplitProducts;
     const Layout L(dk, kNV);
     Tiles s(sm, L);
-    const int tid = threadIdx.x, dkp = L.dkp, NV = L.NV, NP = L.NP;
+    const int tid = threadIdx.x, warp = tid >> 5, dkp = L.dkp, NV = L.NV, NP = L.NP;
     const int bh = blockIdx.x, b = bh / H, h = bh - b * H;
     const int n0 = blockIdx.y * NV, nv = min(NV, dv - n0);
     const int nchunks = (T + kC - 1) / kC;
@@ -393,7 +447,7 @@ __device__ void states_body(float *sm, const Tin *q, const Tin *k, const Tin *v,
                 if (n < nv) dst[static_cast<long>(c) * dv + n0 + n] = s.S[c * NP + n];
             }
         });
-        u_split<kSplit>(s, L);   // U = U' - W S
+        for (int tl = warp; tl < NV / 8; tl += kWarps) u_block<kSplit>(s, L, tl * 8);   // U = U' - W S
         __syncthreads();
         state_update<kSplit>(s, L);   // S <- Diag(gamma) S + Kb^T U
     }
@@ -415,7 +469,7 @@ __device__ void bwd_body(float *sm, const Tin *q, const Tin *k, const Tin *v, co
     const int bh = blockIdx.x, b = bh / H, h = bh - b * H;
     const int n0 = blockIdx.y * NV, nv = min(NV, dv - n0);
     const int nchunks = (T + kC - 1) / kC;
-    const int nU = NV / 8, nQ = dkp / 8, nS = (dkp / 16) * nU;   // block counts
+    const int nU = NV / 32, nQ = dkp / 16, nS = (dkp / 16) * nU;   // strip counts
     for (int e = tid; e < dkp * NV; e += kThreads) {
         const int c = e / NV, n = e - c * NV;
         s.dS[c * NP + n] =
@@ -455,8 +509,6 @@ __device__ void bwd_body(float *sm, const Tin *q, const Tin *k, const Tin *v, co
                 s.dO[t * NP + n] = orr[u];
             }
         }
-        for (int e = tid; e < kC * NP; e += kThreads) s.dU[e] = 0.f;   // split-depth sums
-        for (int e = tid; e < kC * LC; e += kThreads) s.dT[e] = 0.f;
         // While warp 0 solves for X: gamma's gradient (through the state decay, warps 1-4,
         // one state row per thread) and dQs = dO S^T (warps 5 and up)
         chunk_terms(s, L, q, k, v, log_alpha, beta, b, h, T, H, dv, t0, valid, n0, nv, true, [&](int w) {
@@ -474,89 +526,101 @@ __device__ void bwd_body(float *sm, const Tin *q, const Tin *k, const Tin *v, co
                 }
             } else {
                 for (int tl = w - 4; tl < nQ; tl += kWarps - 5) {
-                    const int c0 = tl * 8;
-                    float d[4] = {0.f, 0.f, 0.f, 0.f};
-                    tile_mma<kSplit>(d, [&](int m, int kk) { return s.dO[m * NP + kk]; },
-                                     [&](int kk, int c) { return s.S[c * NP + kk]; }, 0, c0, 0, NV);
-                    tile_each(d, 0, c0, [&](int r, int c, float &x) { s.dQs[r * LD + c] = x; });
+                    const int c0 = tl * 16;
+                    float d[kKS][4];
+                    strip_zero(d);
+                    strip_mma<kSplit>(d, [&](int m, int kk) { return s.dO[m * NP + kk]; },
+                                      [&](int kk, int c) { return s.S[c * NP + kk]; }, 0, c0, 0, NV);
+                    strip_each(d, 0, c0, [&](int r, int c, float &x) { s.dQs[r * LD + c] = x; });
                 }
             }
         });
-        u_split<kSplit>(s, L);   // U = U' - W S
+        for (int tl = warp; tl < NV / 8; tl += kWarps) u_block<kSplit>(s, L, tl * 8);   // U = U' - W S
         __syncthreads();
-        // dU = P^T dO + Kb dS (depth split in four); dKb = U dS^T; dP = lower(dO U^T)
-        for (int tl = warp; tl < 4 * nU + nQ + 2; tl += kWarps) {
-            float d[4] = {0.f, 0.f, 0.f, 0.f};
-            if (tl < 4 * nU) {
-                const int part = tl / nU, j0 = (tl - part * nU) * 8;
-                if (part == 0)
-                    tile_mma<kSplit>(d, [&](int m, int kk) { return s.P[kk * LC + m]; },
-                                     [&](int kk, int n) { return s.dO[kk * NP + n]; }, 0, j0, 0, kC);
+        // dU = P^T dO + Kb dS (full depth, 8-column blocks); dKb = U dS^T
+        for (int tl = warp; tl < NV / 8 + nQ; tl += kWarps) {
+            if (tl < NV / 8) {
+                const int j0 = tl * 8;
+                float d[4] = {0.f, 0.f, 0.f, 0.f};
+                tile_mma<kSplit>(d, [&](int m, int kk) { return s.P[kk * LC + m]; },
+                                 [&](int kk, int n) { return s.dO[kk * NP + n]; }, 0, j0, 0, kC);
                 tile_mma<kSplit>(d, [&](int m, int kk) { return s.Kh[m * LD + kk]; },
-                                 [&](int kk, int n) { return s.dS[kk * NP + n]; }, 0, j0,
-                                 depth_lo(part, dkp / 8), depth_lo(part + 1, dkp / 8));
-                tile_each(d, 0, j0, [&](int r, int c, float &x) { atomicAdd(&s.dU[r * NP + c], x); });
-            } else if (tl < 4 * nU + nQ) {
-                const int c0 = (tl - 4 * nU) * 8;
-                tile_mma<kSplit>(d, [&](int m, int kk) { return s.U[m * NP + kk]; },
-                                 [&](int kk, int c) { return s.dS[c * NP + kk]; }, 0, c0, 0, NV);
-                tile_each(d, 0, c0, [&](int r, int c, float &x) { s.dKb[r * LD + c] = x; });
+                                 [&](int kk, int n) { return s.dS[kk * NP + n]; }, 0, j0, 0, dkp);
+                tile_each(d, 0, j0, [&](int r, int c, float &x) { s.dU[r * NP + c] = x; });
             } else {
-                const int j0 = (tl - 4 * nU - nQ) * 8;
-                tile_mma<kSplit>(d, [&](int m, int kk) { return s.dO[m * NP + kk]; },
-                                 [&](int kk, int j) { return s.U[j * NP + kk]; }, 0, j0, 0, NV);
-                tile_each(d, 0, j0, [&](int r, int c, float &x) { s.dP[r * LC + c] = c <= r ? x : 0.f; });
+                const int c0 = (tl - NV / 8) * 16;
+                float d[kKS][4];
+                strip_zero(d);
+                strip_mma<kSplit>(d, [&](int m, int kk) { return s.U[m * NP + kk]; },
+                                  [&](int kk, int c) { return s.dS[c * NP + kk]; }, 0, c0, 0, NV);
+                strip_each(d, 0, c0, [&](int r, int c, float &x) { s.dKb[r * LD + c] = x; });
             }
         }
         __syncthreads();
-        // dS <- Diag(gamma) dS + Qs^T dO - W^T dU (in place: each block reads only its own
+        // dS <- Diag(gamma) dS + Qs^T dO - W^T dU (in place: each strip reads only its own
         // dS entries); dW = -dU S^T; dV = T^T dU
         for (int tl = warp; tl < nS + nQ + nU; tl += kWarps) {
-            float d[4] = {0.f, 0.f, 0.f, 0.f};
             if (tl < nS) {
-                const int m0 = (tl / nU) * 16, j0 = (tl - (tl / nU) * nU) * 8;
-                tile_each(d, m0, j0, [&](int r, int c, float &x) { x = s.gam[r] * s.dS[r * NP + c]; });
-                tile_mma<kSplit>(d, [&](int m, int kk) { return s.Qs[kk * LD + m]; },
-                                 [&](int kk, int n) { return s.dO[kk * NP + n]; }, m0, j0, 0, kC);
-                tile_mma<kSplit>(d, [&](int m, int kk) { return -s.W[kk * LD + m]; },
-                                 [&](int kk, int n) { return s.dU[kk * NP + n]; }, m0, j0, 0, kC);
-                tile_each(d, m0, j0, [&](int r, int c, float &x) { s.dS[r * NP + c] = x; });
+                const int m0 = (tl / nU) * 16, j0 = (tl - (tl / nU) * nU) * 32;
+                float d[kVS][4];
+                strip_each(d, m0, j0, [&](int r, int c, float &x) { x = s.gam[r] * s.dS[r * NP + c]; });
+                strip_mma<kSplit>(d, [&](int m, int kk) { return s.Qs[kk * LD + m]; },
+                                  [&](int kk, int n) { return s.dO[kk * NP + n]; }, m0, j0, 0, kC);
+                strip_mma<kSplit>(d, [&](int m, int kk) { return -s.W[kk * LD + m]; },
+                                  [&](int kk, int n) { return s.dU[kk * NP + n]; }, m0, j0, 0, kC);
+                strip_each(d, m0, j0, [&](int r, int c, float &x) { s.dS[r * NP + c] = x; });
             } else if (tl < nS + nQ) {
-                const int c0 = (tl - nS) * 8;
-                tile_mma<kSplit>(d, [&](int m, int kk) { return -s.dU[m * NP + kk]; },
-                                 [&](int kk, int c) { return s.S[c * NP + kk]; }, 0, c0, 0, NV);
-                tile_each(d, 0, c0, [&](int r, int c, float &x) { s.dW[r * LD + c] = x; });
+                const int c0 = (tl - nS) * 16;
+                float d[kKS][4];
+                strip_zero(d);
+                strip_mma<kSplit>(d, [&](int m, int kk) { return -s.dU[m * NP + kk]; },
+                                  [&](int kk, int c) { return s.S[c * NP + kk]; }, 0, c0, 0, NV);
+                strip_each(d, 0, c0, [&](int r, int c, float &x) { s.dW[r * LD + c] = x; });
             } else {
-                const int j0 = (tl - nS - nQ) * 8;
-                tile_mma<kSplit>(d, [&](int m, int kk) { return s.Tm[kk * LC + m]; },
-                                 [&](int kk, int n) { return s.dU[kk * NP + n]; }, 0, j0, 0, kC);
-                tile_each(d, 0, j0, [&](int r, int c, float &x) {
+                const int j0 = (tl - nS - nQ) * 32;
+                float d[kVS][4];
+                strip_zero(d);
+                strip_mma<kSplit>(d, [&](int m, int kk) { return s.Tm[kk * LC + m]; },
+                                  [&](int kk, int n) { return s.dU[kk * NP + n]; }, 0, j0, 0, kC);
+                strip_each(d, 0, j0, [&](int r, int c, float &x) {
                     if (r < valid && c < nv)
                         dv_out[((static_cast<long>(b) * T + t0 + r) * H + h) * dv + n0 + c] = from_f32<Tin>(x);
                 });
             }
         }
         __syncthreads();
-        // dT = dW Ks^T + dU V^T (depth split in four; its upper triangle is masked where
-        // it is read), dKs = T^T dW; W (read for the last time above) is zeroed for Cc
-        for (int e = tid; e < kC * LD; e += kThreads) s.W[e] = 0.f;
-        for (int tl = warp; tl < 8 + nQ; tl += kWarps) {
-            float d[4] = {0.f, 0.f, 0.f, 0.f};
+        // dT = dW Ks^T + dU V^T, both depths split in eight parts written apart and summed
+        // in order below; its upper triangle is masked where it is read.
+        // dP = lower(dO U^T); dKs = T^T dW.
+        for (int tl = warp; tl < 9 + nQ; tl += kWarps) {
+            float d[kKS][4];
+            strip_zero(d);
             if (tl < 8) {
-                const int part = tl >> 1, j0 = (tl & 1) * 8;
-                tile_mma<kSplit>(d, [&](int m, int kk) { return s.dW[m * LD + kk]; },
-                                 [&](int kk, int j) { return s.Ks[j * LD + kk]; }, 0, j0,
-                                 depth_lo(part, dkp / 8), depth_lo(part + 1, dkp / 8));
-                if (part == 0)
-                    tile_mma<kSplit>(d, [&](int m, int kk) { return s.dU[m * NP + kk]; },
-                                     [&](int kk, int j) { return s.V[j * NP + kk]; }, 0, j0, 0, NV);
-                tile_each(d, 0, j0, [&](int r, int c, float &x) { atomicAdd(&s.dT[r * LC + c], x); });
+                strip_mma<kSplit>(d, [&](int m, int kk) { return s.dW[m * LD + kk]; },
+                                  [&](int kk, int j) { return s.Ks[j * LD + kk]; }, 0, 0,
+                                  depth_lo(tl, dkp / 8, 8), depth_lo(tl + 1, dkp / 8, 8));
+                strip_mma<kSplit>(d, [&](int m, int kk) { return s.dU[m * NP + kk]; },
+                                  [&](int kk, int j) { return s.V[j * NP + kk]; }, 0, 0,
+                                  depth_lo(tl, NV / 8, 8), depth_lo(tl + 1, NV / 8, 8));
+                strip_each(d, 0, 0, [&](int r, int c, float &x) { s.part[tl * kC * kC + r * kC + c] = x; });
+            } else if (tl == 8) {
+                strip_mma<kSplit>(d, [&](int m, int kk) { return s.dO[m * NP + kk]; },
+                                  [&](int kk, int j) { return s.U[j * NP + kk]; }, 0, 0, 0, NV);
+                strip_each(d, 0, 0, [&](int r, int c, float &x) { s.dP[r * LC + c] = c <= r ? x : 0.f; });
             } else {
-                const int c0 = (tl - 8) * 8;
-                tile_mma<kSplit>(d, [&](int m, int kk) { return s.Tm[kk * LC + m]; },
-                                 [&](int kk, int c) { return s.dW[kk * LD + c]; }, 0, c0, 0, kC);
-                tile_each(d, 0, c0, [&](int r, int c, float &x) { s.dKs[r * LD + c] = x; });
+                const int c0 = (tl - 9) * 16;
+                strip_mma<kSplit>(d, [&](int m, int kk) { return s.Tm[kk * LC + m]; },
+                                  [&](int kk, int c) { return s.dW[kk * LD + c]; }, 0, c0, 0, kC);
+                strip_each(d, 0, c0, [&](int r, int c, float &x) { s.dKs[r * LD + c] = x; });
             }
+        }
+        __syncthreads();
+        for (int e = tid; e < kC * kC; e += kThreads) {
+            const float *x = s.part + e;
+            float a = 0.f;
+#pragma unroll
+            for (int part = 0; part < 8; ++part) a += x[part * kC * kC];
+            s.dT[(e / kC) * LC + e % kC] = a;
         }
         __syncthreads();
         // Z = X^T dX with dX = lower(dT) Diag(beta) (kept in dA), and dbeta's T part
@@ -594,12 +658,13 @@ __device__ void bwd_body(float *sm, const Tin *q, const Tin *k, const Tin *v, co
         // The intra-chunk products, term by term (E_ij = e^{g_i - g_j} per channel):
         //   R_i  = sum_{j<i}  dAt_ij k_j E_ij             (row side of A,   into dW)
         //   Cc_j = sum_{i>j}  dAt_ij k_i E_ij
-        //        + sum_{i>=j} dP_ij  q_i E_ij             (column side,     into W)
+        //        + sum_{i>=j} dP_ij  q_i E_ij             (column side)
         //   Rq_i = sum_{j<=i} dP_ij  k_j E_ij             (row side of P,   into dQt)
         // Each decay is computed once for the three sums: a warp takes the rows i of one
         // residue mod 4 and 32 channels (a lane per channel), walks the pairs j < i of its
-        // rows, writes R and Rq of those rows and adds its Cc parts into W (zeroed);
-        // the diagonal (E = 1) starts Rq and Cc.
+        // rows, writes R and Rq of those rows and writes its part of every Cc into the
+        // S tile (S is not read again in this chunk); the four parts are added in order
+        // where Cc is used. The diagonal (E = 1) starts Rq and Cc.
         {
             const int part = warp & 3, c = (warp >> 2) * 32 + (tid & 31);
             static_assert(kWarps == 16, "four residues x four groups of 32 channels");
@@ -628,7 +693,7 @@ __device__ void bwd_body(float *sm, const Tin *q, const Tin *k, const Tin *v, co
                     s.dQt[i * LD + c] = Rq;
                 }
 #pragma unroll
-                for (int j = 0; j < kC; ++j) atomicAdd(&s.W[j * LD + c], Cc[j]);
+                for (int j = 0; j < kC; ++j) s.S[(part * kC + j) * dkp + c] = Cc[j];
             }
         }
         __syncthreads();
@@ -638,7 +703,9 @@ __device__ void bwd_body(float *sm, const Tin *q, const Tin *k, const Tin *v, co
             const float gv = s.G[t * LD + c];
             const float up = tc::ex2(gv), down = tc::ex2(s.gsum[c] - gv);
             const float kv = s.Kt[t * LD + c], qv = s.Qt[t * LD + c];
-            const float rk = s.dW[t * LD + c], cc = s.W[t * LD + c], rq = s.dQt[t * LD + c];
+            const float *ccp = s.S + t * dkp + c;   // the four parts of Cc, in order
+            const float cc = ((ccp[0] + ccp[kC * dkp]) + ccp[2 * kC * dkp]) + ccp[3 * kC * dkp];
+            const float rk = s.dW[t * LD + c], rq = s.dQt[t * LD + c];
             const float dks = s.dKs[t * LD + c], dkb = s.dKb[t * LD + c], dqs = s.dQs[t * LD + c];
             const float dk_v = rk + cc + dks * up + dkb * down;
             const float dq_v = rq + dqs * up;
