@@ -23,8 +23,9 @@
 // dense products run on the tensor cores as warp-level tf32 tiles; the terms
 // with a pairwise decay e^{g_i - g_j} (At, P and their gradients) and the 16 x 16
 // triangular algebra stay on the CUDA cores, so no decay factor is ever split
-// into a growing and a shrinking part. The kernels, their launch and the fp32 ->
-// dtype casts are in chunk_bwd.cu.
+// into a growing and a shrinking part. Products split over warps write their parts
+// to separate buffers that are added in a fixed order (no shared-memory atomics).
+// The kernels, their launch and the fp32 -> dtype casts are in chunk_bwd.cu.
 #pragma once
 
 namespace kbwd {

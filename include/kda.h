@@ -185,9 +185,9 @@ int kda_recurrent_step(const void *q, const void *k, const void *v,
  * kda_recurrent_step continues from the same rows (the serving path: packed
  * prompts prefill the decode step's cache "without modifying the cache or
  * scheduling interfaces", Kimi Linear summary, section "Uso de NoPE y
- * resultados de evaluacion"). This entry computes in fp32 on CUDA cores with
- * 16-token chunks; kda_chunk_fwd_varlen_engine below also runs the tensor-core
- * engine.
+ * resultados de evaluacion"). This entry runs the 16-token engine: fp32 state,
+ * dense products as warp-level tensor-core tiles in the 3xTF32 form (about fp32
+ * accuracy); kda_chunk_fwd_varlen_engine below also runs the tcgen05 engine.
  *
  *   q, k       [total_T,H,dk]  dtype     (packed over sequences)
  *   v          [total_T,H,dv]  dtype
@@ -229,18 +229,18 @@ size_t kda_varlen_workspace_bytes(int N, int H, int dk, int dv, int dtype);
 /*
  * kda_chunk_fwd_varlen with a choice of engine. Arguments, layouts, results
  * and limits as kda_chunk_fwd_varlen, plus:
- *   engine     KDA_ENGINE_GENERIC: the fp32 CUDA-core kernel (16-token chunks);
+ *   engine     KDA_ENGINE_GENERIC: the 16-token engine of kda_chunk_fwd_varlen;
  *              KDA_ENGINE_TC_CLUSTER: the tensor-core engine of kda_chunk_fwd
  *              (bf16, dk = dv = 128, chunk 64), one 4-CTA cluster per
  *              (sequence, head) over the same packed tensors; anything else
  *              returns KDA_ERR_UNSUPPORTED, a missing or small workspace
  *              KDA_ERR_WORKSPACE;
  *              KDA_ENGINE_AUTO: the tensor-core engine when it supports the
- *              shape and the workspace is large enough, else the CUDA-core one.
+ *              shape and the workspace is large enough, else the 16-token one.
  *   workspace  device scratch, 16-byte aligned, kda_varlen_workspace_bytes(...)
  *              bytes (the caller owns it; not kept after the call; one call at
  *              a time per workspace). May be NULL for KDA_ENGINE_GENERIC.
- * Calls with total_T = 0 only move the states and run the CUDA-core kernel.
+ * Calls with total_T = 0 only move the states and run the 16-token kernel.
  * A bounded device wait that gives up on the tensor-core engine is reported by
  * kda_device_status as KDA_ERR_DEVICE_TIMEOUT, as for kda_chunk_fwd.
  */
@@ -337,7 +337,12 @@ int kda_short_conv_swish(const void *x, const float *weight, const int32_t *cu_s
  *                                       kda_bwd_workspace_bytes(...) bytes: the
  *                                       entry state of every 16-token chunk plus
  *                                       fp32 accumulators for grad_q and grad_k
- * Outputs must not alias inputs. Computes in fp32 on CUDA cores.
+ * Outputs must not alias inputs. Computes with fp32 states and accumulation:
+ * dense products as warp-level tensor-core tiles in the 3xTF32 form, terms with
+ * a pairwise decay on CUDA cores. Sums inside a CTA are in a fixed order; the
+ * key-side gradients of the two 64-column value slices meet in fp32 atomics, so
+ * grad_q, grad_k, grad_log_alpha and grad_beta may differ in the last bits
+ * between runs.
  * T = 0 copies grad_S_T (or zeros) to grad_S0. B = 0 or H = 0 is a no-op.
  * Supported: dtype KDA_BF16 or KDA_F32, dk and dv in [1,128]; the same B*T and
  * B*H limits as kda_chunk_fwd.
