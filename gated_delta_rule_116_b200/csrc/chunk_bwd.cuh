@@ -88,11 +88,16 @@ struct Tiles {
 // terms much larger than themselves (the gradient of k sums four such terms), and
 // single tf32 products (11 bits) left errors of 6 % of a gradient element.
 constexpr bool kSplitProducts = true;
+// bf16 inputs (dL/dO, v) reach the products unchanged and are exact in tf32.
+template <typename T> struct ExactInTf32 { static constexpr bool value = false; };
+template <> struct ExactInTf32<__nv_bfloat16> { static constexpr bool value = true; };
 
 __device__ __forceinline__ uint32_t tf32_bits(float x) { return tc::to_tf32(x) & 0xFFFFE000u; }
 
 // d += A B for one 8-deep step; the low-part products go to e (a separate chain).
-template <bool kSplit>
+// kAExact / kBExact: that operand holds bf16 values, which tf32 represents exactly
+// (its low part is zero), so its low-part product is skipped.
+template <bool kSplit, bool kAExact = false, bool kBExact = false>
 __device__ __forceinline__ void mma_step(float (&d)[4], float (&e)[4], const float (&a)[4],
                                          const float (&b)[2]) {
     uint32_t ah[4], bh[2];
@@ -106,8 +111,8 @@ __device__ __forceinline__ void mma_step(float (&d)[4], float (&e)[4], const flo
         for (int i = 0; i < 4; ++i) al[i] = tf32_bits(a[i] - __uint_as_float(ah[i]));
         const uint32_t bl0 = tf32_bits(b[0] - __uint_as_float(bh[0]));
         const uint32_t bl1 = tf32_bits(b[1] - __uint_as_float(bh[1]));
-        tc::mma_16x8x8_tf32(e, al, bh[0], bh[1]);
-        tc::mma_16x8x8_tf32(e, ah, bl0, bl1);
+        if constexpr (!kAExact) tc::mma_16x8x8_tf32(e, al, bh[0], bh[1]);
+        if constexpr (!kBExact) tc::mma_16x8x8_tf32(e, ah, bl0, bl1);
     }
     tc::mma_16x8x8_tf32(d, ah, bh[0], bh[1]);
 }
@@ -115,7 +120,7 @@ __device__ __forceinline__ void mma_step(float (&d)[4], float (&e)[4], const flo
 // d += sum_{k0 <= k < k1} A(m, k) B(k, n) over the block at rows m0..m0+15, columns
 // n0..n0+7; k1 - k0 is a multiple of 8. A and B read shared memory. Even and odd
 // 8-deep steps, and the high and low parts, accumulate in separate chains.
-template <bool kSplit, class FA, class FB>
+template <bool kSplit, bool kAExact = false, bool kBExact = false, class FA, class FB>
 __device__ __forceinline__ void tile_mma(float (&d)[4], const FA &A, const FB &B, int m0, int n0, int k0,
                                          int k1) {
     const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
@@ -128,14 +133,14 @@ __device__ __forceinline__ void tile_mma(float (&d)[4], const FA &A, const FB &B
         const float a1[4] = {A(m0 + g, k + 8 + t), A(m0 + g + 8, k + 8 + t), A(m0 + g, k + 12 + t),
                              A(m0 + g + 8, k + 12 + t)};
         const float b1[2] = {B(k + 8 + t, n0 + g), B(k + 12 + t, n0 + g)};
-        mma_step<kSplit>(d, e0, a0, b0);
-        mma_step<kSplit>(d1, e1, a1, b1);
+        mma_step<kSplit, kAExact, kBExact>(d, e0, a0, b0);
+        mma_step<kSplit, kAExact, kBExact>(d1, e1, a1, b1);
     }
     if (k < k1) {
         const float a0[4] = {A(m0 + g, k + t), A(m0 + g + 8, k + t), A(m0 + g, k + t + 4),
                              A(m0 + g + 8, k + t + 4)};
         const float b0[2] = {B(k + t, n0 + g), B(k + t + 4, n0 + g)};
-        mma_step<kSplit>(d, e0, a0, b0);
+        mma_step<kSplit, kAExact, kBExact>(d, e0, a0, b0);
     }
 #pragma unroll
     for (int i = 0; i < 4; ++i) d[i] += d1[i] + (e0[i] + e1[i]);
@@ -155,7 +160,7 @@ __device__ __forceinline__ void tile_each(float (&d)[4], int m0, int n0, const F
 // step's A fragment, whose tf32 split is then done once for the NT products:
 // d[nt] += sum_{k0 <= k < k1} A(m, k) B(k, n) over block nt. Each block keeps its
 // high and low products in separate chains.
-template <bool kSplit, int NT, class FA, class FB>
+template <bool kSplit, bool kAExact = false, bool kBExact = false, int NT, class FA, class FB>
 __device__ __forceinline__ void strip_mma(float (&d)[NT][4], const FA &A, const FB &B, int m0, int n0,
                                           int k0, int k1) {
     const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
@@ -175,11 +180,10 @@ __device__ __forceinline__ void strip_mma(float (&d)[NT][4], const FA &A, const 
         for (int nt = 0; nt < NT; ++nt) {
             const float b0 = B(k + t, n0 + 8 * nt + g), b1 = B(k + t + 4, n0 + 8 * nt + g);
             const uint32_t bh0 = tf32_bits(b0), bh1 = tf32_bits(b1);
-            if constexpr (kSplit) {
-                tc::mma_16x8x8_tf32(e[nt], al, bh0, bh1);
+            if constexpr (kSplit && !kAExact) tc::mma_16x8x8_tf32(e[nt], al, bh0, bh1);
+            if constexpr (kSplit && !kBExact)
                 tc::mma_16x8x8_tf32(e[nt], ah, tf32_bits(b0 - __uint_as_float(bh0)),
                                     tf32_bits(b1 - __uint_as_float(bh1)));
-            }
             tc::mma_16x8x8_tf32(d[nt], ah, bh0, bh1);
         }
     }
@@ -324,14 +328,25 @@ __device__ void chunk_terms(Tiles &s, const Layout &L, const Tin *q, const Tin *
             const float4 *gi = reinterpret_cast<const float4 *>(s.G + i * LD);
             const float4 *gj = reinterpret_cast<const float4 *>(s.G + j * LD);
             float at[4] = {0.f, 0.f, 0.f, 0.f}, pp[4] = {0.f, 0.f, 0.f, 0.f};
-            for (int c4 = part * n4 / 3; c4 < (part + 1) * n4 / 3; ++c4) {
-                const float4 a = ki[c4], bj = kj[c4], q4 = qi[c4], x = gi[c4], y = gj[c4];
-                const float w0 = bj.x * tc::ex2(x.x - y.x), w1 = bj.y * tc::ex2(x.y - y.y);
-                const float w2 = bj.z * tc::ex2(x.z - y.z), w3 = bj.w * tc::ex2(x.w - y.w);
-                at[0] = fmaf(a.x, w0, at[0]); at[1] = fmaf(a.y, w1, at[1]);
-                at[2] = fmaf(a.z, w2, at[2]); at[3] = fmaf(a.w, w3, at[3]);
-                pp[0] = fmaf(q4.x, w0, pp[0]); pp[1] = fmaf(q4.y, w1, pp[1]);
-                pp[2] = fmaf(q4.z, w2, pp[2]); pp[3] = fmaf(q4.w, w3, pp[3]);
+            const int c4a = part * n4 / 3, c4b = (part + 1) * n4 / 3;
+            if (need_p) {
+                for (int c4 = c4a; c4 < c4b; ++c4) {
+                    const float4 a = ki[c4], bj = kj[c4], q4 = qi[c4], x = gi[c4], y = gj[c4];
+                    const float w0 = bj.x * tc::ex2(x.x - y.x), w1 = bj.y * tc::ex2(x.y - y.y);
+                    const float w2 = bj.z * tc::ex2(x.z - y.z), w3 = bj.w * tc::ex2(x.w - y.w);
+                    at[0] = fmaf(a.x, w0, at[0]); at[1] = fmaf(a.y, w1, at[1]);
+                    at[2] = fmaf(a.z, w2, at[2]); at[3] = fmaf(a.w, w3, at[3]);
+                    pp[0] = fmaf(q4.x, w0, pp[0]); pp[1] = fmaf(q4.y, w1, pp[1]);
+                    pp[2] = fmaf(q4.z, w2, pp[2]); pp[3] = fmaf(q4.w, w3, pp[3]);
+                }
+            } else {
+                for (int c4 = c4a; c4 < c4b; ++c4) {
+                    const float4 a = ki[c4], bj = kj[c4], x = gi[c4], y = gj[c4];
+                    at[0] = fmaf(a.x, bj.x * tc::ex2(x.x - y.x), at[0]);
+                    at[1] = fmaf(a.y, bj.y * tc::ex2(x.y - y.y), at[1]);
+                    at[2] = fmaf(a.z, bj.z * tc::ex2(x.z - y.z), at[2]);
+                    at[3] = fmaf(a.w, bj.w * tc::ex2(x.w - y.w), at[3]);
+                }
             }
             float *part_out = s.part + part * 2 * kC * kC + i * kC + j;   // [part][At|P][i][j]
             part_out[0] = (at[0] + at[1]) + (at[2] + at[3]);
@@ -357,17 +372,46 @@ __device__ void chunk_terms(Tiles &s, const Layout &L, const Tin *q, const Tin *
         }
         __syncwarp();
     }
-    if (tid < kC) {   // X = (I + A)^{-1}, A = Diag(beta) At: column j by forward substitution
-        const int j = tid;
-        float xc[kC];   // column j of X, in registers
+    if (warp == 0) {
+        // X = (I + A)^{-1}, A = Diag(beta) At, in 8 x 8 blocks: the two diagonal blocks
+        // X00 = (I + A00)^{-1} and X11 = (I + A11)^{-1} by forward substitution (lane l < 16
+        // takes column l % 8 of block l / 8), then X10 = -X11 (A10 X00) through dA, which
+        // is free until the gradient terms; X01 = 0. T = X Diag(beta).
+        static_assert(kC == 16, "two 8 x 8 diagonal blocks");
+        const int lane = tid & 31;
+        if (lane < kC) {
+            const int o = (lane >> 3) * 8, jj = lane & 7;
+            float xc[8];   // column jj of the diagonal block, in registers
 #pragma unroll
-        for (int i = 0; i < kC; ++i) {
+            for (int ii = 0; ii < 8; ++ii) {
+                float acc = 0.f;
+#pragma unroll
+                for (int mm = 0; mm < ii; ++mm) acc = fmaf(s.At[(o + ii) * LC + o + mm], xc[mm], acc);
+                xc[ii] = ii == jj ? 1.f : (ii > jj ? -s.bt[o + ii] * acc : 0.f);   // xc[mm] = 0 for mm < jj
+                s.X[(o + ii) * LC + o + jj] = xc[ii];
+                if (o == 8) s.X[ii * LC + 8 + jj] = 0.f;   // X01 = 0
+            }
+        }
+        __syncwarp();
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {   // Y = A10 X00 = Diag(beta_8..15) At[8..15][0..7] X00
+            const int e = lane + 32 * r, m = e >> 3, j = e & 7;
             float acc = 0.f;
+            for (int n = j; n < 8; ++n) acc = fmaf(s.At[(8 + m) * LC + n], s.X[n * LC + j], acc);
+            s.dA[m * LC + j] = s.bt[8 + m] * acc;
+        }
+        __syncwarp();
 #pragma unroll
-            for (int m = 0; m < i; ++m) acc = fmaf(s.At[i * LC + m], xc[m], acc);   // xc[m] = 0 for m < j
-            xc[i] = i == j ? 1.f : (i > j ? -s.bt[i] * acc : 0.f);
-            s.X[i * LC + j] = xc[i];
-            s.Tm[i * LC + j] = xc[i] * s.bt[j];
+        for (int r = 0; r < 2; ++r) {   // X10 = -X11 Y
+            const int e = lane + 32 * r, i = e >> 3, j = e & 7;
+            float acc = 0.f;
+            for (int m = 0; m <= i; ++m) acc = fmaf(s.X[(8 + i) * LC + 8 + m], s.dA[m * LC + j], acc);
+            s.X[(8 + i) * LC + j] = -acc;
+        }
+        __syncwarp();
+        for (int e = lane; e < kC * kC; e += 32) {
+            const int i = e / kC, j = e - i * kC;
+            s.Tm[i * LC + j] = s.X[i * LC + j] * s.bt[j];
         }
     }
     __syncthreads();
@@ -384,7 +428,8 @@ __device__ void chunk_terms(Tiles &s, const Layout &L, const Tin *q, const Tin *
                 float d[kVS][4];
                 strip_zero(d);
                 const int j0 = (tl - nW) * 32;
-                strip_mma<kSplit>(d, A, [&](int kk, int n) { return s.V[kk * NP + n]; }, 0, j0, 0, kC);
+                strip_mma<kSplit, false, ExactInTf32<Tin>::value>(
+                    d, A, [&](int kk, int n) { return s.V[kk * NP + n]; }, 0, j0, 0, kC);
                 strip_each(d, 0, j0, [&](int r, int c, float &x) { s.Up[r * NP + c] = x; });
             }
         }
@@ -530,7 +575,7 @@ __device__ void bwd_body(float *sm, const Tin *q, const Tin *k, const Tin *v, co
                     const int c0 = tl * 16;
                     float d[kKS][4];
                     strip_zero(d);
-                    strip_mma<kSplit>(d, [&](int m, int kk) { return s.dO[m * NP + kk]; },
+                    strip_mma<kSplit, ExactInTf32<Tin>::value>(d, [&](int m, int kk) { return s.dO[m * NP + kk]; },
                                       [&](int kk, int c) { return s.S[c * NP + kk]; }, 0, c0, 0, NV);
                     strip_each(d, 0, c0, [&](int r, int c, float &x) { s.dQs[r * LD + c] = x; });
                 }
@@ -543,7 +588,7 @@ __device__ void bwd_body(float *sm, const Tin *q, const Tin *k, const Tin *v, co
             if (tl < NV / 8) {
                 const int j0 = tl * 8;
                 float d[4] = {0.f, 0.f, 0.f, 0.f};
-                tile_mma<kSplit>(d, [&](int m, int kk) { return s.P[kk * LC + m]; },
+                tile_mma<kSplit, false, ExactInTf32<Tin>::value>(d, [&](int m, int kk) { return s.P[kk * LC + m]; },
                                  [&](int kk, int n) { return s.dO[kk * NP + n]; }, 0, j0, 0, kC);
                 tile_mma<kSplit>(d, [&](int m, int kk) { return s.Kh[m * LD + kk]; },
                                  [&](int kk, int n) { return s.dS[kk * NP + n]; }, 0, j0, 0, dkp);
@@ -565,7 +610,7 @@ __device__ void bwd_body(float *sm, const Tin *q, const Tin *k, const Tin *v, co
                 const int m0 = (tl / nU) * 16, j0 = (tl - (tl / nU) * nU) * 32;
                 float d[kVS][4];
                 strip_each(d, m0, j0, [&](int r, int c, float &x) { x = s.gam[r] * s.dS[r * NP + c]; });
-                strip_mma<kSplit>(d, [&](int m, int kk) { return s.Qs[kk * LD + m]; },
+                strip_mma<kSplit, false, ExactInTf32<Tin>::value>(d, [&](int m, int kk) { return s.Qs[kk * LD + m]; },
                                   [&](int kk, int n) { return s.dO[kk * NP + n]; }, m0, j0, 0, kC);
                 strip_mma<kSplit>(d, [&](int m, int kk) { return -s.W[kk * LD + m]; },
                                   [&](int kk, int n) { return s.dU[kk * NP + n]; }, m0, j0, 0, kC);
@@ -600,12 +645,12 @@ __device__ void bwd_body(float *sm, const Tin *q, const Tin *k, const Tin *v, co
                 strip_mma<kSplit>(d, [&](int m, int kk) { return s.dW[m * LD + kk]; },
                                   [&](int kk, int j) { return s.Ks[j * LD + kk]; }, 0, 0,
                                   depth_lo(tl, dkp / 8, 8), depth_lo(tl + 1, dkp / 8, 8));
-                strip_mma<kSplit>(d, [&](int m, int kk) { return s.dU[m * NP + kk]; },
+                strip_mma<kSplit, false, ExactInTf32<Tin>::value>(d, [&](int m, int kk) { return s.dU[m * NP + kk]; },
                                   [&](int kk, int j) { return s.V[j * NP + kk]; }, 0, 0,
                                   depth_lo(tl, NV / 8, 8), depth_lo(tl + 1, NV / 8, 8));
                 strip_each(d, 0, 0, [&](int r, int c, float &x) { s.part[tl * kC * kC + r * kC + c] = x; });
             } else if (tl == 8) {
-                strip_mma<kSplit>(d, [&](int m, int kk) { return s.dO[m * NP + kk]; },
+                strip_mma<kSplit, ExactInTf32<Tin>::value>(d, [&](int m, int kk) { return s.dO[m * NP + kk]; },
                                   [&](int kk, int j) { return s.U[j * NP + kk]; }, 0, 0, 0, NV);
                 strip_each(d, 0, 0, [&](int r, int c, float &x) { s.dP[r * LC + c] = c <= r ? x : 0.f; });
             } else {
