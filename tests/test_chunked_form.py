@@ -145,6 +145,26 @@ def test_forward_substitution_inverts():
     np.testing.assert_allclose(unit_lower_inverse(A) @ (np.eye(20) + A), np.eye(20), atol=1e-10)
 
 
+def test_blocked_inverse_of_the_16_token_chunk():
+    """The 16-token kernels solve (I + A)^{-1}, A = Diag(beta) At, in 8 x 8 blocks: the
+    diagonal blocks by forward substitution, X10 = -X11 (A10 X00), X01 = 0. The same
+    steps in NumPy, on the At of real chunks (strong and weak gates), equal the dense
+    inverse."""
+    rng = np.random.default_rng(3)
+    for gate_scale in (0.05, 1.0, 4.0):
+        kc = rng.standard_normal((16, 8))
+        kc /= np.linalg.norm(kc, axis=1, keepdims=True)
+        lc = -gate_scale * np.log1p(np.exp(rng.standard_normal((16, 8))))
+        bc = 1.0 / (1.0 + np.exp(-rng.standard_normal(16)))
+        At = chunk_terms(kc, kc, kc, lc, bc)["At"]
+        X00 = unit_lower_inverse(bc[:8, None] * At[:8, :8])
+        X11 = unit_lower_inverse(bc[8:, None] * At[8:, 8:])
+        Y = (bc[8:, None] * At[8:, :8]) @ X00
+        X = np.zeros((16, 16))
+        X[:8, :8], X[8:, 8:], X[8:, :8] = X00, X11, -X11 @ Y
+        np.testing.assert_allclose(X, np.linalg.inv(np.eye(16) + bc[:, None] * At), rtol=1e-12, atol=1e-13)
+
+
 def chunked_chain(q, k, v, la, be, S_init, C):
     """The chunked chain from S_init; returns outputs and final state (columns of
     S_init evolve independently, so S_init may be any d x n matrix)."""
